@@ -1,0 +1,185 @@
+"""fp64 CPU oracle for the LongCat Sparse Attention (LSA) hot path.
+
+TEST INFRASTRUCTURE ONLY. Only ``tests/``, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this module. The product path (the
+CUDA library and its Python binding) never calls it and shares no code with it.
+
+Plain numpy float64, one query row at a time, in the order the pages state the
+method. Sources (web pages; cited by title and section):
+
+* [Lite-Sparse] "MLX-VLM 的 LongCat-Flash-Lite-Sparse 支持：LSA 稀疏注意力、
+  n-gram 融合与预填充优化解析" (lmnt.cn). Sections used: "架构总览"
+  (MLA dimensions), "LSA（LongCat 稀疏注意力）" (indexer, forcing, top-k,
+  dense fallback, cross-layer reuse, gather vs mask), "预填充优化" (the
+  ReLU-weighted head sum written as ``acc += max(g, 0) * w[h]``, and the
+  unfused ``maximum(q k^T, 0)`` weighted-sum form), "测试与验证" (tiny
+  config 8/2/4, absorbed == non-absorbed MLA).
+* [LSA-2.0] "LongCat Sparse Attention技术深度解析：为什么它能提升100万上下文
+  处理效率" (wmrh.cn). Sections used: "模型架构配置" (index_n_heads 32,
+  index_head_dim 128, index_topk 2048, index_local_tokens 1024,
+  index_init_tokens 16, cli_factor 2), "跨层索引" (one index pass serves
+  consecutive layers).
+
+Readings taken where the pages are silent or garbled (each is also listed in
+the design notes):
+* The fallback comparison lost its operator in the scrape; it is read as
+  "cached length <= index_topk", applied per query row.
+* No extra scale in the index score; any scale lives in w.
+* The local window is relative to each row: columns p-n_loc+1 .. p.
+* Masking precedes forcing: columns after the query stay -inf.
+* The query sees its own key (the cache is appended before indexing).
+* Top-k is a set; ties are broken by the lower column index.
+* Attention is MLA in absorbed form: logits use all 576 latent dims
+  (512 c_kv + 64 rope), values are the first 512, scale 1/sqrt(128 + 64).
+
+Parity pins for every function live in tests/test_oracle.py.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+
+@dataclass(frozen=True)
+class LsaConfig:
+    """Constants of the method ([LSA-2.0] 模型架构配置; [Lite-Sparse] 架构总览)."""
+
+    index_topk: int = 2048
+    index_init_tokens: int = 16
+    index_local_tokens: int = 1024
+    cli_factor: int = 2
+    kv_lora_rank: int = 512          # value part of a latent row
+    qk_rope_head_dim: int = 64
+    qk_nope_head_dim: int = 128
+
+    @property
+    def softmax_scale(self) -> float:
+        return 1.0 / np.sqrt(self.qk_nope_head_dim + self.qk_rope_head_dim)
+
+
+PAGES = LsaConfig()
+# The tiny configuration of the pages' language-model test ([Lite-Sparse] 测试与验证).
+TINY = LsaConfig(index_topk=8, index_init_tokens=2, index_local_tokens=4, cli_factor=2)
+
+
+def score_row(q: np.ndarray, w: np.ndarray, k: np.ndarray) -> np.ndarray:
+    """Lightning-indexer scores of one query against keys k.
+
+    [Lite-Sparse] LSA section: q k per index head, then ReLU, then the sum over
+    heads weighted by the per-head scalar; 预填充优化 gives the unfused form
+    ``maximum(q k^T, 0)`` weighted sum, which is what this computes.
+
+    q [Hi, d], w [Hi], k [n, d]  ->  s [n] with s[j] = sum_h w[h] * max(q[h].k[j], 0).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    w = np.asarray(w, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    g = q @ k.T                       # [Hi, n]: one dot product per head and key
+    return w @ np.maximum(g, 0.0)     # ReLU, then head-weighted sum
+
+
+def mask_and_force(s_vis: np.ndarray, p: int, length: int, cfg: LsaConfig) -> np.ndarray:
+    """Causal mask and streaming-aware forcing on one row of length ``length``.
+
+    s_vis holds the scores of the visible columns 0..p. Columns after p become
+    -inf (a query sees keys at positions <= its own). Of the visible columns,
+    the first index_init_tokens (sink) and the last index_local_tokens (local
+    window p-n_loc+1 .. p) become +inf ([Lite-Sparse] LSA section, streaming-
+    aware indexing; [LSA-2.0] 模型架构配置).
+    """
+    out = np.full(length, -np.inf)
+    out[: p + 1] = s_vis[: p + 1]
+    j = np.arange(p + 1)
+    forced = (j < cfg.index_init_tokens) | (j >= p + 1 - cfg.index_local_tokens)
+    out[: p + 1][forced] = np.inf
+    return out
+
+
+def select_topk(s_row: np.ndarray, p: int, cfg: LsaConfig):
+    """Top-k selection with the dense fallback ([Lite-Sparse] LSA section).
+
+    If the query sees n = p+1 <= index_topk keys, the indexer returns nothing
+    and attention is dense over all visible keys: returns (arange(n), True).
+    Otherwise returns (the index_topk visible columns of highest score, ties to
+    the lower index, False). The result is a set; its order carries no meaning.
+    """
+    n = p + 1
+    if n <= cfg.index_topk:
+        return np.arange(n, dtype=np.int64), True
+    order = np.argsort(-s_row[:n], kind="stable")
+    return np.sort(order[: cfg.index_topk]).astype(np.int64), False
+
+
+def mla(q_abs: np.ndarray, c_sel: np.ndarray, cfg: LsaConfig):
+    """Absorbed-latent MLA of one query over the selected latent rows.
+
+    [Lite-Sparse] 架构总览 and LSA section: attention runs in the kv-LoRA latent
+    space; keys are whole latent rows (c_kv 512 + rope 64), values are c_kv.
+    q_abs [H, 576], c_sel [n, 576]  ->  o [H, 512], lse [H] (natural log).
+    """
+    q = np.asarray(q_abs, dtype=np.float64)
+    c = np.asarray(c_sel, dtype=np.float64)
+    x = cfg.softmax_scale * (q @ c.T)                 # [H, n] logits
+    m = x.max(axis=1, keepdims=True)
+    e = np.exp(x - m)
+    l = e.sum(axis=1, keepdims=True)
+    o = (e / l) @ c[:, : cfg.kv_lora_rank]
+    lse = (m + np.log(l))[:, 0]
+    return o, lse
+
+
+def lsa_row(q_idx, w, k_seq, p, q_abs_list, latent_list, cfg: LsaConfig = PAGES):
+    """One query row through the whole path: index -> top-k -> cli_factor x MLA.
+
+    k_seq [L, 128] and each latent [L, 576] hold the row's own sequence, with
+    the current token already appended (the pages order the cache update before
+    the gather). The index pass runs once and every sub-block reuses its
+    selection ([Lite-Sparse] LSA section, cross-layer index reuse; [LSA-2.0]
+    跨层索引). Returns (selected, dense, [(o, lse) per sub-block]).
+    """
+    L = k_seq.shape[0]
+    n = p + 1
+    if n <= cfg.index_topk:
+        sel, dense = np.arange(n, dtype=np.int64), True     # the indexer is not run
+    else:
+        s = mask_and_force(score_row(q_idx, w, k_seq[:n]), p, L, cfg)
+        sel, dense = select_topk(s, p, cfg)
+    outs = [mla(qa, lat[sel], cfg) for qa, lat in zip(q_abs_list, latent_list)]
+    return sel, dense, outs
+
+
+def dense_mla_row(q_abs, latent, p, cfg: LsaConfig = PAGES):
+    """Plain dense MLA over every visible key (attention_method MLA)."""
+    return mla(q_abs, latent[: p + 1], cfg)
+
+
+def explicit_mla(q_nope, q_rope, c_kv, k_rope, w_uk, w_uv, cfg: LsaConfig = PAGES):
+    """Non-absorbed MLA, per head, for the absorbed == explicit self-check.
+
+    k_h[i] = [W_UK[h] c[i] ; k_rope[i]], v_h[i] = W_UV[h] c[i]; softmax over i of
+    scale * [q_nope[h]; q_rope[h]] . k_h[i]. ([Lite-Sparse] 测试与验证: the
+    absorbed embed_q / unembed_out form must equal this.)
+    q_nope [H,128], q_rope [H,64], c_kv [n,512], k_rope [n,64],
+    w_uk [H,128,512], w_uv [H,128,512]  ->  out [H,128].
+    """
+    H = q_nope.shape[0]
+    out = np.zeros((H, w_uv.shape[1]))
+    for h in range(H):
+        k = np.concatenate([c_kv @ w_uk[h].T, k_rope], axis=1)      # [n, 192]
+        v = c_kv @ w_uv[h].T                                          # [n, 128]
+        x = cfg.softmax_scale * (k @ np.concatenate([q_nope[h], q_rope[h]]))
+        e = np.exp(x - x.max())
+        out[h] = (e / e.sum()) @ v
+    return out
+
+
+def absorb_query(q_nope, q_rope, w_uk):
+    """embed_q: fold W_UK into the query, q_abs[h] = [W_UK[h]^T q_nope[h] ; q_rope[h]]."""
+    H = q_nope.shape[0]
+    return np.stack([np.concatenate([w_uk[h].T @ q_nope[h], q_rope[h]]) for h in range(H)])
+
+
+def unembed_out(o_lat, w_uv):
+    """unembed_out: map each head's 512-d latent output back, out[h] = W_UV[h] o_lat[h]."""
+    return np.stack([w_uv[h] @ o_lat[h] for h in range(o_lat.shape[0])])

@@ -1,0 +1,326 @@
+"""Pins for the fp64 oracle (CPU only).
+
+Each test ties one oracle function to something other than itself: a closed
+form, an identity of the mathematics, a brute-force enumeration, or an
+independent library routine (torch's scaled_dot_product_attention). A
+plausible slip in the oracle (dropped ReLU, wrong head index, sign error,
+off-by-one in the window, wrong scale, values taken from the wrong dims) fails
+at least one of them.
+"""
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import lsa_ref as R
+from oracle.lsa_ref import PAGES, TINY, LsaConfig
+
+rng = np.random.default_rng(1234)
+
+
+# --------------------------------------------------------------------------
+# Index scores
+# --------------------------------------------------------------------------
+def test_score_closed_form_one_head():
+    # One head, w = 1, q = e0, keys c * e0: s = ReLU(c).
+    c = np.array([-2.0, -0.5, 0.0, 0.25, 3.0])
+    q = np.zeros((1, 8)); q[0, 0] = 1.0
+    k = np.zeros((5, 8)); k[:, 0] = c
+    np.testing.assert_array_equal(R.score_row(q, np.array([1.0]), k), np.maximum(c, 0))
+    # negative weight flips the sign of the ReLU'd value
+    np.testing.assert_array_equal(R.score_row(q, np.array([-2.0]), k), -2.0 * np.maximum(c, 0))
+
+
+def test_score_heads_weighted_independently():
+    # Two heads looking at different coordinates with different weights.
+    q = np.zeros((2, 4)); q[0, 0] = 1.0; q[1, 1] = 1.0
+    k = np.array([[1.0, -1.0, 0, 0], [-3.0, 2.0, 0, 0], [0.5, 0.5, 0, 0]])
+    w = np.array([0.25, 4.0])
+    expect = np.array([0.25 * 1.0 + 0.0, 0.0 + 4.0 * 2.0, 0.25 * 0.5 + 4.0 * 0.5])
+    np.testing.assert_allclose(R.score_row(q, w, k), expect, rtol=0, atol=1e-15)
+
+
+def test_score_odd_part_is_linear():
+    # ReLU(x) - ReLU(-x) = x, so s(q) - s(-q) = (sum_h w_h q_h) . k, a plain matmul.
+    q = rng.standard_normal((32, 128)); w = rng.standard_normal(32); k = rng.standard_normal((300, 128))
+    lhs = R.score_row(q, w, k) - R.score_row(-q, w, k)
+    rhs = k @ (w @ q)
+    np.testing.assert_allclose(lhs, rhs, rtol=1e-12, atol=1e-10)
+
+
+def test_score_even_part_is_weighted_abs():
+    # ReLU(x) + ReLU(-x) = |x|.
+    q = rng.standard_normal((32, 128)); w = rng.standard_normal(32); k = rng.standard_normal((200, 128))
+    lhs = R.score_row(q, w, k) + R.score_row(-q, w, k)
+    rhs = np.abs(k @ q.T) @ w
+    np.testing.assert_allclose(lhs, rhs, rtol=1e-12, atol=1e-10)
+
+
+def test_score_homogeneity():
+    q = rng.standard_normal((32, 128)); w = rng.standard_normal(32); k = rng.standard_normal((64, 128))
+    s = R.score_row(q, w, k)
+    np.testing.assert_allclose(R.score_row(3.0 * q, w, k), 3.0 * s, rtol=1e-12, atol=1e-10)
+    np.testing.assert_allclose(R.score_row(q, -0.5 * w, k), -0.5 * s, rtol=1e-12, atol=1e-10)
+
+
+# --------------------------------------------------------------------------
+# Mask and forcing
+# --------------------------------------------------------------------------
+@pytest.mark.parametrize("p", [0, 5, 15, 16, 1039, 1040, 2047, 2048, 5000])
+def test_mask_and_force_pages_constants(p):
+    L = p + 7
+    s = mask_and_force_input = np.arange(p + 1, dtype=np.float64)
+    out = R.mask_and_force(s, p, L, PAGES)
+    assert np.all(np.isneginf(out[p + 1:]))
+    forced = set(range(min(16, p + 1))) | set(range(max(0, p + 1 - 1024), p + 1))
+    got = set(np.flatnonzero(np.isposinf(out)).tolist())
+    assert got == forced
+    rest = sorted(set(range(p + 1)) - forced)
+    np.testing.assert_array_equal(out[rest], mask_and_force_input[rest])
+
+
+def test_mask_and_force_tiny():
+    out = R.mask_and_force(np.arange(10.0), 9, 12, TINY)
+    # sink {0,1}, local {6,7,8,9}, masked {10,11}
+    assert np.isposinf(out[[0, 1, 6, 7, 8, 9]]).all()
+    np.testing.assert_array_equal(out[2:6], [2.0, 3.0, 4.0, 5.0])
+    assert np.isneginf(out[10:]).all()
+
+
+# --------------------------------------------------------------------------
+# Top-k
+# --------------------------------------------------------------------------
+def _brute_force_topk(s, n, k):
+    """The unique k-subset S of 0..n-1 such that every chosen i beats every
+    unchosen j: s_i > s_j, or s_i == s_j and i < j. Found by enumeration."""
+    found = []
+    for sub in itertools.combinations(range(n), k):
+        chosen = set(sub)
+        ok = all((s[i] > s[j]) or (s[i] == s[j] and i < j)
+                 for i in chosen for j in range(n) if j not in chosen)
+        if ok:
+            found.append(sub)
+    assert len(found) == 1
+    return np.array(found[0])
+
+
+@pytest.mark.parametrize("trial", range(12))
+def test_topk_brute_force_tiny(trial):
+    r = np.random.default_rng(100 + trial)
+    n = int(r.integers(9, 13))
+    p = n - 1
+    # coarse values so that exact ties occur
+    s = r.integers(-3, 4, size=n).astype(np.float64)
+    row = R.mask_and_force(s, p, n + 3, TINY)
+    sel, dense = R.select_topk(row, p, TINY)
+    assert not dense
+    np.testing.assert_array_equal(sel, _brute_force_topk(row, n, TINY.index_topk))
+
+
+def test_topk_dense_fallback_boundary():
+    for n in (1, 7, 8):
+        sel, dense = R.select_topk(np.zeros(n + 2), n - 1, TINY)
+        assert dense and np.array_equal(sel, np.arange(n))
+    sel, dense = R.select_topk(np.zeros(12), 8, TINY)
+    assert not dense and len(sel) == 8
+
+
+def test_topk_planted_pages_constants():
+    # 1008 planted middle columns with the largest finite scores are chosen
+    # together with the 16 + 1024 forced columns.
+    p = 6000
+    r = np.random.default_rng(7)
+    s = r.uniform(-1.0, 1.0, p + 1)
+    middle = np.arange(16, p + 1 - 1024)
+    planted = np.sort(r.choice(middle, 1008, replace=False))
+    s[planted] = 10.0 + r.uniform(0, 1, 1008)
+    row = R.mask_and_force(s, p, p + 100, PAGES)
+    sel, dense = R.select_topk(row, p, PAGES)
+    expect = np.sort(np.concatenate([np.arange(16), planted, np.arange(p + 1 - 1024, p + 1)]))
+    assert not dense
+    np.testing.assert_array_equal(sel, expect)
+
+
+def test_topk_all_equal_takes_lowest_indices():
+    p = 4000
+    row = R.mask_and_force(np.zeros(p + 1), p, p + 1, PAGES)
+    sel, _ = R.select_topk(row, p, PAGES)
+    expect = np.concatenate([np.arange(16), np.arange(16, 16 + 1008), np.arange(p + 1 - 1024, p + 1)])
+    np.testing.assert_array_equal(sel, np.sort(expect))
+
+
+def test_topk_through_scores_planted():
+    # Plant through the indexer itself: keys aligned with every head's query
+    # score high, keys anti-aligned score 0 (all weights positive).
+    p, d = 3500, 128
+    r = np.random.default_rng(3)
+    u = r.standard_normal(d); u /= np.linalg.norm(u)
+    q = np.tile(u, (32, 1)) + 0.01 * r.standard_normal((32, d))
+    w = np.abs(r.standard_normal(32)) + 0.1
+    k = -np.abs(r.standard_normal((p + 1, 1))) * u + 0.001 * r.standard_normal((p + 1, d))
+    planted = np.sort(r.choice(np.arange(16, p + 1 - 1024), 1008, replace=False))
+    k[planted] = (5.0 + r.uniform(0, 1, (1008, 1))) * u
+    s = R.mask_and_force(R.score_row(q, w, k), p, p + 1, PAGES)
+    sel, _ = R.select_topk(s, p, PAGES)
+    expect = np.sort(np.concatenate([np.arange(16), planted, np.arange(p + 1 - 1024, p + 1)]))
+    np.testing.assert_array_equal(sel, expect)
+
+
+# --------------------------------------------------------------------------
+# Attention
+# --------------------------------------------------------------------------
+def test_softmax_scale_from_dims():
+    assert PAGES.softmax_scale == pytest.approx(1.0 / math.sqrt(192.0), rel=0, abs=1e-16)
+
+
+def test_mla_zero_query_is_mean_of_values():
+    c = rng.standard_normal((37, 576))
+    o, lse = R.mla(np.zeros((32, 576)), c, PAGES)
+    np.testing.assert_allclose(o, np.tile(c[:, :512].mean(axis=0), (32, 1)), rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(lse, np.full(32, math.log(37)), rtol=1e-14)
+
+
+def test_mla_single_key():
+    c = rng.standard_normal((1, 576)); q = rng.standard_normal((32, 576))
+    o, lse = R.mla(q, c, PAGES)
+    np.testing.assert_allclose(o, np.tile(c[0, :512], (32, 1)), rtol=1e-14)
+    np.testing.assert_allclose(lse, PAGES.softmax_scale * (q @ c[0]), rtol=1e-13)
+
+
+def test_mla_two_keys_sigmoid():
+    c = rng.standard_normal((2, 576)); q = rng.standard_normal((32, 576))
+    o, _ = R.mla(q, c, PAGES)
+    d = PAGES.softmax_scale * (q @ (c[0] - c[1]))
+    a = 1.0 / (1.0 + np.exp(-d))
+    np.testing.assert_allclose(o, a[:, None] * c[0, :512] + (1 - a[:, None]) * c[1, :512], rtol=1e-12, atol=1e-13)
+
+
+def test_mla_one_hot_values_reveal_selection():
+    # q = 0 and V[i] = e_{i mod 512}: the output shows exactly which rows were used.
+    n = 700
+    c = np.zeros((n, 576))
+    c[np.arange(n), np.arange(n) % 512] = 1.0
+    sel = np.sort(rng.choice(n, 300, replace=False))
+    o, _ = R.mla(np.zeros((4, 576)), c[sel], PAGES)
+    expect = np.zeros(512)
+    np.add.at(expect, sel % 512, 1.0 / 300)
+    np.testing.assert_allclose(o[0], expect, atol=1e-15)
+
+
+def test_mla_matches_torch_sdpa():
+    q = rng.standard_normal((32, 576)); c = rng.standard_normal((513, 576))
+    o, lse = R.mla(q, c, PAGES)
+    tq = torch.from_numpy(q)[None, :, None, :]
+    tk = torch.from_numpy(c)[None, None].expand(1, 32, -1, -1)
+    tv = torch.from_numpy(c[:, :512])[None, None].expand(1, 32, -1, -1)
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=PAGES.softmax_scale)
+    np.testing.assert_allclose(o, ref[0, :, 0].numpy(), rtol=1e-12, atol=1e-12)
+    ref_lse = torch.logsumexp(PAGES.softmax_scale * (torch.from_numpy(q) @ torch.from_numpy(c).T), dim=1)
+    np.testing.assert_allclose(lse, ref_lse.numpy(), rtol=1e-13)
+
+
+def test_absorbed_equals_explicit_mla():
+    # The pages' absorbed-attention test: embed_q / unembed_out == explicit heads.
+    H, n = 4, 50
+    q_nope = rng.standard_normal((H, 128)); q_rope = rng.standard_normal((H, 64))
+    c_kv = rng.standard_normal((n, 512)); k_rope = rng.standard_normal((n, 64))
+    w_uk = rng.standard_normal((H, 128, 512)) / 20; w_uv = rng.standard_normal((H, 128, 512)) / 20
+    q_abs = R.absorb_query(q_nope, q_rope, w_uk)
+    o_lat, _ = R.mla(q_abs, np.concatenate([c_kv, k_rope], axis=1), PAGES)
+    absorbed = R.unembed_out(o_lat, w_uv)
+    explicit = R.explicit_mla(q_nope, q_rope, c_kv, k_rope, w_uk, w_uv, PAGES)
+    np.testing.assert_allclose(absorbed, explicit, rtol=1e-10, atol=1e-12)
+    # and the explicit heads against torch's attention on the explicit tensors
+    for h in range(H):
+        k = np.concatenate([c_kv @ w_uk[h].T, k_rope], axis=1)
+        v = c_kv @ w_uv[h].T
+        qq = np.concatenate([q_nope[h], q_rope[h]])
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qq)[None, None], torch.from_numpy(k)[None], torch.from_numpy(v)[None],
+            scale=PAGES.softmax_scale)
+        np.testing.assert_allclose(explicit[h], ref[0, 0].numpy(), rtol=1e-10, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Whole row: invariants from the pages
+# --------------------------------------------------------------------------
+def _row_inputs(L, d_idx=128, seed=0):
+    r = np.random.default_rng(seed)
+    return (r.standard_normal((32, d_idx)), r.standard_normal(32) / math.sqrt(32),
+            r.standard_normal((L, d_idx)), [r.standard_normal((32, 576)) for _ in range(2)],
+            [r.standard_normal((L, 576)) for _ in range(2)])
+
+
+def test_dense_fallback_equals_dense_mla():
+    # (a) cached length <= 2048: the result is dense MLA.
+    q, w, k, qa, lat = _row_inputs(2048)
+    sel, dense, outs = R.lsa_row(q, w, k, 2047, qa, lat, PAGES)
+    assert dense and len(sel) == 2048
+    for z in range(2):
+        o, lse = R.dense_mla_row(qa[z], lat[z], 2047)
+        np.testing.assert_array_equal(outs[z][0], o)
+
+
+def test_topk_at_least_length_equals_dense():
+    # (b) topk >= cached length in a generic config: sparse == dense.
+    cfg = LsaConfig(index_topk=64, index_init_tokens=2, index_local_tokens=4)
+    q, w, k, qa, lat = _row_inputs(60)
+    _, dense, outs = R.lsa_row(q, w, k, 59, qa, lat, cfg)
+    assert dense
+    # force the sparse branch with topk == n explicitly
+    s = R.mask_and_force(R.score_row(q, w, k), 59, 60, cfg)
+    sel = np.argsort(-s, kind="stable")[:60]
+    o, _ = R.mla(qa[0], lat[0][np.sort(sel)], cfg)
+    np.testing.assert_allclose(outs[0][0], o, rtol=1e-13, atol=1e-13)
+
+
+def test_sink_and_local_always_selected():
+    # (c) even when their scores are the lowest possible.
+    p = 3000
+    q, w, k, qa, lat = _row_inputs(p + 1, seed=5)
+    w = np.abs(w)
+    k[:16] = -10 * q.mean(axis=0)               # sinks score ~0
+    k[p + 1 - 1024:] = -10 * q.mean(axis=0)      # local window scores ~0
+    sel, dense, _ = R.lsa_row(q, w, k, p, qa, lat, PAGES)
+    assert not dense and len(sel) == 2048
+    assert set(range(16)) <= set(sel.tolist())
+    assert set(range(p + 1 - 1024, p + 1)) <= set(sel.tolist())
+
+
+def test_cli_sharing_equals_two_passes():
+    # (e) two sub-blocks sharing one index pass == two passes on the same indices.
+    p = 2600
+    q, w, k, qa, lat = _row_inputs(p + 1, seed=9)
+    sel, _, outs = R.lsa_row(q, w, k, p, qa, lat, PAGES)
+    for z in range(2):
+        sel_z, _, outs_z = R.lsa_row(q, w, k, p, [qa[z]], [lat[z]], PAGES)
+        np.testing.assert_array_equal(sel_z, sel)
+        np.testing.assert_array_equal(outs_z[0][0], outs[z][0])
+
+
+def test_decode_equals_prefill_row():
+    # Cached decode at length p+1 equals row p of a prefill over the same cache.
+    L = 2300
+    q, w, k, qa, lat = _row_inputs(L, seed=11)
+    for p in (100, 2047, 2048, 2299):
+        sel_d, _, outs_d = R.lsa_row(q, w, k[: p + 1], p, qa, [x[: p + 1] for x in lat], PAGES)
+        sel_p, _, outs_p = R.lsa_row(q, w, k, p, qa, lat, PAGES)
+        np.testing.assert_array_equal(sel_d, sel_p)
+        np.testing.assert_array_equal(outs_d[1][0], outs_p[1][0])
+
+
+def test_tiny_config_whole_row():
+    # The pages' tiny LSA config (topk 8, init 2, local 4) end to end.
+    L = 20
+    q, w, k, qa, lat = _row_inputs(L, seed=13)
+    for p in range(L):
+        sel, dense, outs = R.lsa_row(q, w, k, p, qa, lat, TINY)
+        n = p + 1
+        assert dense == (n <= 8)
+        assert len(sel) == min(n, 8) and len(set(sel.tolist())) == len(sel)
+        assert sel.max() <= p
+        if not dense:
+            assert {0, 1, p - 3, p - 2, p - 1, p} <= set(sel.tolist())
+        assert np.isfinite(outs[0][0]).all()
