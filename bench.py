@@ -1,0 +1,474 @@
+#!/usr/bin/env python
+"""LSA hot-path benchmark on B200.
+
+Headline: LSA decode tokens/s/layer at 128K context. Workload: batch 16, every
+sequence at cached length 131072, 14 layers, each layer one index pass
+(lightning indexer over all 131072 keys, top-2048 with 16 sink + 1024 local
+forced) feeding two attention sub-blocks of sparse absorbed-latent MLA over
+independent latent caches. One step = one decode token for every sequence
+through all 14 layers. tokens/s/layer = batch * 14 / step time. Per step the
+caches read are ~8.6 GB (> L2), so no L2 flush is needed between steps.
+
+Also reported: prefill tok/s of one 16384-token causal sequence (same path in
+prefill form), the roofline fraction of the dominant kernel, the fp64 CPU
+oracle on a bounded sample, and an end-to-end number through lsa_forward with
+pinned host buffers and host<->device copies inside the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
+Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
+collective on the data path); rank 0 prints the aggregate.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import lsa_synth as S  # noqa: E402
+
+METRIC = "LSA decode tokens/s/layer at 128K ctx"
+DECODE = dict(batch=16, ctx=131072, layers=14, cli=2)
+PREFILL = dict(seq=16384)
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# multi-process plumbing
+# ---------------------------------------------------------------------------
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def dist_init(world, backend):
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        from datetime import timedelta
+        dist.init_process_group(backend=backend, timeout=timedelta(seconds=120))
+
+
+def reduce_max(x: float, world: int, device=None) -> float:
+    if world <= 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def aggregate(units_per_rank: float, seconds_per_rank: float, world: int, device=None):
+    """Whole-job throughput: units of all ranks / the slowest rank's time."""
+    t = reduce_max(seconds_per_rank, world, device)
+    return units_per_rank * world / t, t
+
+
+# ---------------------------------------------------------------------------
+# clocks
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.idx = device_index
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.idx), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                self.out, _ = self.proc.communicate()
+
+    def summary(self):
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in (self.out or "").strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 7:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx.append(float(parts[1]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[3:7]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return PEAKS_FALLBACK, "fallback"
+
+
+def kernel_traffic(kernel: str, src: str):
+    """dram bytes per launch from the committed ncu summary, if it was taken on this source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel)
+    if not d:
+        return None
+    h = hashlib.sha256(open(os.path.join(ROOT, "sparse_attention_03_b200", "csrc", src), "rb").read()).hexdigest()
+    return d["bytes_per_launch"] if d.get("source_sha256") == h else None
+
+
+# ---------------------------------------------------------------------------
+# the CPU oracle on a bounded sample (rank 0, N=1 only; also the reference arm)
+# ---------------------------------------------------------------------------
+class OracleSample:
+    """Host inputs for a few decode rows of the 128K workload (drawn untimed)."""
+
+    def __init__(self, n_rows: int, layer: int = 0):
+        ctx = DECODE["ctx"]
+        self.rows = []
+        f = S.bf16_bits_to_f64
+        for b in range(n_rows):
+            q = f(S.normal_bf16(0, S.tid(layer, S.Q_IDX), b * 4096, 4096)).reshape(32, 128)
+            w = S.normal_f32(0, S.tid(layer, S.W), b * 32, 32, S.W_SIGMA).astype(np.float64)
+            k = f(S.rms_rows_bf16(0, S.tid(layer, S.K_IDX), b * ctx, ctx, 128))
+            qa = [f(S.normal_bf16(0, S.tid(layer, S.q_abs_kind(z)), b * 32 * 576, 32 * 576)).reshape(32, 576)
+                  for z in range(2)]
+            self.rows.append((q, w, k, qa, b))
+        self.layer = layer
+
+    def unit(self, i):
+        """One decode token of one sequence through one layer, as the oracle computes it."""
+        from oracle import lsa_ref as R
+        q, w, k, qa, b = self.rows[i % len(self.rows)]
+        p = DECODE["ctx"] - 1
+        s = R.mask_and_force(R.score_row(q, w, k), p, DECODE["ctx"], R.PAGES)
+        sel, _ = R.select_topk(s, p, R.PAGES)
+        for z in range(2):
+            c = S.bf16_bits_to_f64(S.normal_bf16_rows(0, S.tid(self.layer, S.lat_kind(z)),
+                                                      b * DECODE["ctx"] + sel, 576))
+            R.mla(qa[z], c, R.PAGES)
+
+
+def oracle_rate(sample: OracleSample, budget_s: float):
+    n, t0 = 0, time.perf_counter()
+    while True:
+        sample.unit(n)
+        n += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    return n, time.perf_counter() - t0
+
+
+def host_cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count()
+
+
+def cpu_baseline(budget_s: float = 12.0):
+    sample = OracleSample(2)
+    sample.unit(0)  # warm BLAS
+    n, t = oracle_rate(sample, budget_s)
+    return {"value": n / t, "unit": "tokens/s/layer", "cores": host_cores(), "kind": "oracle",
+            "sample": f"{n} decode tokens (one sequence through one layer each: indexer over 131072 keys, "
+                      f"top-2048, 2 sub-blocks of sparse MLA) of the 128K workload, fp64 numpy, {t:.1f} s"}
+
+
+def reference_arm(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    sample = OracleSample(2)
+    sample.unit(0)
+    for _ in range(args.warmup):
+        sample.unit(1)
+    per_step = 4
+    t0 = time.perf_counter()
+    for s in range(args.steps):
+        for u in range(per_step):
+            sample.unit(s * per_step + u)
+    t = time.perf_counter() - t0
+    units = args.steps * per_step
+    v = units / t
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s/layer", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": "decode_b16_ctx131072_14layers_cli2",
+                                            "sample": f"{per_step} decode tokens per step"},
+            "cpu_baseline": {"value": v, "unit": "tokens/s/layer", "cores": host_cores(), "kind": "oracle",
+                             "sample": f"{units} decode tokens of the 128K workload, fp64 numpy"},
+            "e2e": {"value": v, "unit": "tokens/s/layer", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# GPU arm
+# ---------------------------------------------------------------------------
+def build_decode(device):
+    import torch
+    from sparse_attention_03_b200 import lsa
+    from sparse_attention_03_b200.device_inputs import DeviceWorkload
+    B, ctx, nl = DECODE["batch"], DECODE["ctx"], DECODE["layers"]
+    lengths = np.full(B, ctx, dtype=np.int64)
+    layers = [DeviceWorkload(0, l, lengths, device=device) for l in range(nl)]
+    # per-step inputs and outputs of all layers in single buffers (one copy each way)
+    q_idx = torch.stack([l.q_idx for l in layers]).contiguous()
+    w = torch.stack([l.w for l in layers]).contiguous()
+    q_abs = torch.stack([torch.stack(l.q_abs) for l in layers]).contiguous()
+    for i, l in enumerate(layers):
+        l.q_idx, l.w, l.q_abs = q_idx[i], w[i], [q_abs[i, 0], q_abs[i, 1]]
+    out = torch.empty((nl, 2, B, 32, 512), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((nl, 2, B, 32), dtype=torch.float32, device=device)
+    cfg = lsa.LsaConfig()
+    ws = lsa.workspace(cfg, lsa.OP_FORWARD_DECODE, B, B, ctx, device=device)
+    scores = torch.empty((B, ctx), dtype=torch.float32, device=device)
+    idx = torch.empty((B, 2048), dtype=torch.int32, device=device)
+    cnt = torch.empty((B,), dtype=torch.int32, device=device)
+    tk_ws = lsa.workspace(cfg, lsa.OP_TOPK, B, B, ctx, device=device)
+    mla_ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE, B, B, ctx, device=device)
+    return dict(layers=layers, q_idx=q_idx, w=w, q_abs=q_abs, out=out, lse=lse, cfg=cfg, ws=ws, scores=scores,
+                idx=idx, cnt=cnt, tk_ws=tk_ws, mla_ws=mla_ws, ctx=ctx)
+
+
+def decode_step(D, ev=None):
+    """One decode step through every layer via the C-ABI entry points. If `ev`
+    is given, records events around each indexer launch."""
+    from sparse_attention_03_b200 import lsa
+    cfg, ctx = D["cfg"], D["ctx"]
+    for i, l in enumerate(D["layers"]):
+        if ev is not None:
+            ev[i][0].record()
+        lsa.index_scores(cfg, l.seq_of_row, l.pos, l.q_idx, l.w, l.k_idx, l.k_off, ctx, D["scores"])
+        if ev is not None:
+            ev[i][1].record()
+        lsa.topk(cfg, l.pos, ctx, D["scores"], D["idx"], D["cnt"], D["tk_ws"])
+        for z in range(2):
+            lsa.sparse_mla_decode(cfg, l.q_abs[z], l.latent[z], l.k_off, D["idx"], D["cnt"], ctx,
+                                  D["out"][i, z], D["lse"][i, z], D["mla_ws"])
+
+
+def decode_forward_e2e(D, h_in, h_out):
+    """One step through lsa_forward with the per-step inputs copied from pinned host
+    memory and the outputs copied back."""
+    from sparse_attention_03_b200 import lsa
+    D["q_idx"].copy_(h_in[0], non_blocking=True)
+    D["w"].copy_(h_in[1], non_blocking=True)
+    D["q_abs"].copy_(h_in[2], non_blocking=True)
+    cfg, ctx = D["cfg"], D["ctx"]
+    for i, l in enumerate(D["layers"]):
+        lsa.forward(cfg, 0, l.seq_of_row, l.pos, ctx, l.q_idx, l.w, l.k_idx, l.k_off, l.q_abs, l.latent,
+                    [D["out"][i, 0], D["out"][i, 1]], [D["lse"][i, 0], D["lse"][i, 1]], D["ws"])
+    h_out.copy_(D["out"], non_blocking=True)
+
+
+def time_region(fn, steps, world, device):
+    import torch
+    barrier(world)
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record()
+    for s in range(steps):
+        fn(s)
+    b.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return a.elapsed_time(b) / 1e3
+
+
+def run_prefill(device, steps, warmup):
+    import torch
+    from sparse_attention_03_b200 import lsa
+    from sparse_attention_03_b200.device_inputs import DeviceWorkload
+    n = PREFILL["seq"]
+    wl = DeviceWorkload(0, 100, [n], n_rows=n, q_start=0, device=device)
+    cfg = lsa.LsaConfig()
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    lses = [torch.empty((n, 32), device=device) for _ in range(2)]
+    ws = lsa.workspace(cfg, lsa.OP_FORWARD_PREFILL, n, 1, n, device=device)
+    scores = torch.empty((n, n), device=device)
+    idx = torch.empty((n, 2048), dtype=torch.int32, device=device)
+    cnt = torch.empty((n,), dtype=torch.int32, device=device)
+    tk_ws = lsa.workspace(cfg, lsa.OP_TOPK, n, 1, n, device=device)
+    mla_ws = lsa.workspace(cfg, lsa.OP_MLA_PREFILL, n, 1, n, device=device)
+    ev = []
+
+    def step(record):
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lsa.index_scores(cfg, None, wl.pos, wl.q_idx, wl.w, wl.k_idx, None, n, scores)
+        e1.record()
+        if record:
+            ev.append((e0, e1))
+        lsa.topk(cfg, wl.pos, n, scores, idx, cnt, tk_ws)
+        for z in range(2):
+            lsa.sparse_mla_prefill(cfg, wl.pos, wl.q_abs[z], wl.latent[z], idx, cnt, outs[z], lses[z], mla_ws)
+
+    for _ in range(warmup):
+        step(False)
+    t = time_region(lambda s: step(True), steps, 1, device)
+    idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
+    flops = 2.0 * 32 * 128 * (n * (n + 1) / 2)  # visible (row, key) pairs
+    pk, src = peaks()
+    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    achieved = flops / (idx_ms / 1e3) / 1e12
+    del wl, scores
+    torch.cuda.empty_cache()
+    return {"value": n * steps / t, "unit": "tok/s", "ms_per_step": 1e3 * t / steps,
+            "config": {"workload": "prefill_causal_16384", "seq_len": n},
+            "roofline": {"kernel": "index_decode_kernel (indexer, prefill rows)", "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{src} bf16_tflops_sustained", "traffic": None}}
+
+
+def gpu_arm(args):
+    import torch
+    from sparse_attention_03_b200 import lsa
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    lsa.load()
+    D = build_decode(device)
+    nl, B = DECODE["layers"], DECODE["batch"]
+
+    def events():
+        return [[torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)] for _ in range(nl)]
+
+    for _ in range(args.warmup):
+        decode_step(D)
+    torch.cuda.synchronize()
+    assert lsa.device_error() == 0
+
+    # kernel-level timed region (inputs resident in HBM); events on the launching
+    # (current) stream bracket every indexer launch
+    ev = [events() for _ in range(args.steps)]
+    with ClockSampler(local) as clk:
+        l0 = lsa.launch_count()
+        barrier(world)
+        torch.cuda.synchronize()
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record()
+        for s in range(args.steps):
+            decode_step(D, ev[s])
+        t1.record()
+        torch.cuda.synchronize()
+        barrier(world)
+        launches = lsa.launch_count() - l0
+    t = t0.elapsed_time(t1) / 1e3
+    idx_ms = [a.elapsed_time(b) for step_ev in ev for a, b in step_ev]
+    units = B * nl * args.steps
+    value, tmax = aggregate(units, t, world, device)
+
+    # roofline of the dominant kernel (the indexer: 256 B of k_idx + 4 B of score per key)
+    keys = B * DECODE["ctx"]
+    alg_bytes = keys * (256 + 4) + B * (32 * 128 * 2 + 32 * 4)
+    pk, psrc = peaks()
+    peak = pk["hbm_gbs"]
+    achieved = alg_bytes / (statistics.mean(idx_ms) / 1e3) / 1e9
+
+    # end-to-end through lsa_forward with pinned host buffers
+    h_in = [D["q_idx"].cpu().pin_memory(), D["w"].cpu().pin_memory(), D["q_abs"].cpu().pin_memory()]
+    h_out = torch.empty(D["out"].shape, dtype=D["out"].dtype).pin_memory()
+    for _ in range(max(3, args.warmup // 2)):
+        decode_forward_e2e(D, h_in, h_out)
+    torch.cuda.synchronize()
+    e2e_steps = max(5, args.steps // 2)
+    te = time_region(lambda s: decode_forward_e2e(D, h_in, h_out), e2e_steps, world, device)
+    e2e_value, _ = aggregate(B * nl * e2e_steps, te, world, device)
+    h2d = sum(x.numel() * x.element_size() for x in h_in)
+    d2h = h_out.numel() * h_out.element_size()
+    assert lsa.device_error() == 0
+
+    del D
+    torch.cuda.empty_cache()
+    prefill = None
+    if not args.no_prefill:
+        prefill = run_prefill(device, max(3, args.steps // 20), 3)
+
+    clocks = clk.summary()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s/layer", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * tmax / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "decode_b16_ctx131072_14layers_cli2", "batch": B, "ctx": DECODE["ctx"],
+                   "layers": nl, "cli_factor": 2, "index_topk": 2048, "parallelism": f"replicas x{world}",
+                   "l2": "inputs larger than L2 (8.6 GB of caches read per step), no flush"},
+        "roofline": {"kernel": "index_decode_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{psrc} hbm_gbs",
+                     "traffic": kernel_traffic("index_decode_kernel", "index_decode.cu"),
+                     "alg_bytes_per_launch": alg_bytes, "avg_launch_ms": statistics.mean(idx_ms)},
+        "e2e": {"value": e2e_value, "unit": "tokens/s/layer", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": launches,
+        "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+    }
+    if prefill:
+        line["prefill"] = prefill
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline()
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["lsa", "reference"], default="lsa")
+    ap.add_argument("--no-prefill", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        reference_arm(args)
+        return
+    gpu_arm(args)
+    rank, world, _ = dist_env()
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

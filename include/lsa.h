@@ -1,0 +1,255 @@
+/*
+ * lsa.h - C-ABI of liblsa.so, the B200 (sm_100a) hot path of LongCat Sparse
+ * Attention (LSA): lightning indexer -> top-k with forced sink/local columns
+ * and a dense fallback -> absorbed-latent MLA over the selected keys, with one
+ * index pass shared by a layer's attention sub-blocks.
+ *
+ * Sources (web pages, cited by title and section):
+ *   [Lite-Sparse] "MLX-VLM 的 LongCat-Flash-Lite-Sparse 支持：LSA 稀疏注意力、
+ *     n-gram 融合与预填充优化解析", sections "架构总览",
+ *     "LSA（LongCat 稀疏注意力）", "预填充优化", "测试与验证".
+ *   [LSA-2.0] "LongCat Sparse Attention技术深度解析：为什么它能提升100万上下文
+ *     处理效率", sections "流式感知索引", "跨层索引", "模型架构配置".
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Every array argument is DEVICE memory owned by the caller, unless stated
+ *   otherwise. The library never allocates, frees or synchronises (except the
+ *   two debugging calls marked "synchronising"). All work is enqueued on
+ *   `stream` (a cudaStream_t passed as void*; NULL = the legacy default stream).
+ * - lsa_bf16 is the raw 16-bit pattern of a bfloat16 value.
+ * - Row-major layouts. Index vectors: 128 bf16 = 256 B per key. Latent rows:
+ *   576 bf16 = 1152 B (512 c_kv then 64 rope). Bases of bf16 arrays must be
+ *   16-byte aligned.
+ * - Sequences: the keys of sequence b are rows [k_off[b], k_off[b+1]) of the
+ *   packed caches (k_off: int64 [n_seq+1], device). Query row r belongs to
+ *   sequence seq_of_row[r] and sits at absolute position pos[r] inside it; it
+ *   sees keys 0..pos[r] (its own key included: the caller appends the current
+ *   token's cache rows before calling, as the pages order the cache update
+ *   before the gather).
+ * - Errors: host-detectable errors return at once and enqueue nothing
+ *   (LSA_ERR_INVALID, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE); a failed launch
+ *   returns LSA_ERR_CUDA. Device-detected errors (a position past its
+ *   sequence, an index out of range) never fault: the kernel clamps or skips
+ *   the bad item and sets a sticky flag read by lsa_device_error().
+ *   lsa_last_error() gives a message for the last failing call on the thread.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define LSA_API __attribute__((visibility("default")))
+#else
+#define LSA_API
+#endif
+
+typedef uint16_t lsa_bf16;
+
+typedef enum lsa_status {
+  LSA_OK = 0,
+  LSA_DENSE = 1,             /* lsa_topk: every row is dense (no selection needed) */
+  LSA_ERR_INVALID = -1,      /* null pointer, bad size, misalignment */
+  LSA_ERR_UNSUPPORTED = -2,  /* configuration the kernels do not implement */
+  LSA_ERR_WORKSPACE = -3,    /* ws_bytes below the minimum */
+  LSA_ERR_CUDA = -4,         /* a CUDA call or launch failed */
+  LSA_ERR_DEVICE = -5        /* lsa_device_error() found a device-side flag */
+} lsa_status;
+
+/* Device-side error flags (lsa_device_error). */
+#define LSA_DEVERR_POS 1     /* pos[r] < 0 or beyond its sequence or max_len */
+#define LSA_DEVERR_INDEX 2   /* a selected index outside the row's visible keys */
+#define LSA_DEVERR_COUNT 4   /* count[r] outside [0, index_topk] */
+#define LSA_DEVERR_SEQ 8     /* seq_of_row[r] outside [0, n_seq) */
+
+/*
+ * Method constants, under the pages' config key names ([LSA-2.0] 模型架构配置;
+ * [Lite-Sparse] 架构总览). Supported: index_n_heads 32, index_head_dim 128,
+ * n_heads 32, kv_lora_rank 512, qk_rope_head_dim 64, cli_factor 1 or 2,
+ * 0 <= index_init_tokens, 0 <= index_local_tokens,
+ * index_init_tokens + index_local_tokens < index_topk <= 2048.
+ */
+typedef struct lsa_config {
+  int32_t index_n_heads;      /* 32 */
+  int32_t index_head_dim;     /* 128 */
+  int32_t index_topk;         /* 2048 */
+  int32_t index_init_tokens;  /* 16: sink columns forced into the selection */
+  int32_t index_local_tokens; /* 1024: local-window columns forced in */
+  int32_t cli_factor;         /* 2: attention sub-blocks sharing one index pass */
+  int32_t n_heads;            /* 32 MLA heads */
+  int32_t kv_lora_rank;       /* 512: value part of a latent row */
+  int32_t qk_rope_head_dim;   /* 64: rope part of a latent row */
+  float softmax_scale;        /* 1/sqrt(qk_nope 128 + qk_rope 64) */
+} lsa_config;
+
+/* Fills the pages' constants (the values in the comments above). */
+LSA_API void lsa_config_default(lsa_config* cfg);
+
+/* Operation codes for lsa_workspace_size. */
+#define LSA_OP_TOPK 1
+#define LSA_OP_MLA_DECODE 2
+#define LSA_OP_MLA_PREFILL 3
+#define LSA_OP_FORWARD_DECODE 4
+#define LSA_OP_FORWARD_PREFILL 5
+
+/*
+ * Bytes of workspace the operation uses at full speed for these sizes (host
+ * only, no CUDA call). Smaller workspaces are accepted down to a minimum
+ * (one row block for top-k and forward; zero for the MLA calls, which then
+ * run without split-K); below it the call returns LSA_ERR_WORKSPACE.
+ * Returns 0 on invalid arguments.
+ */
+LSA_API size_t lsa_workspace_size(const lsa_config* cfg, int32_t op, int32_t n_rows, int32_t n_seq,
+                          int64_t max_len);
+
+/*
+ * Lightning-indexer scores, mask and forcing ([Lite-Sparse] LSA section: q k
+ * per index head, ReLU, head-weighted sum; streaming-aware forcing; 预填充优化:
+ * the fused ReLU-weighted epilogue that never materialises the per-head
+ * tensor).
+ *
+ *   scores[r, j] = sum_h w[r,h] * max(q_idx[r,h,:] . k_idx[k_off[b] + j, :], 0)
+ *                  for j <= pos[r], b = seq_of_row[r];
+ *                = +inf  if j <= pos[r] and (j < index_init_tokens or
+ *                        j > pos[r] - index_local_tokens)   (forced columns);
+ *                = -inf  for pos[r] < j < max_len            (causal mask).
+ * Entries at j >= max_len are not written.
+ *
+ * q_idx   bf16 [n_rows, 32, 128]     w  fp32 [n_rows, 32]
+ * k_idx   bf16 [sum L_b, 128]        k_off int64 [n_seq+1], or NULL: one
+ *         sequence of max_len keys at row 0 (then n_seq must be 1)
+ * seq_of_row int32 [n_rows] or NULL (every row in sequence 0)
+ * pos     int32 [n_rows]             scores fp32 [n_rows, ld], ld >= max_len
+ * max_len host bound: every pos[r] < max_len.
+ * Products bf16 x bf16 exact in fp32, fp32 accumulation.
+ */
+LSA_API lsa_status lsa_index_scores(const lsa_config* cfg, int32_t n_rows, int32_t n_seq,
+                            const int32_t* seq_of_row, const int32_t* pos, const lsa_bf16* q_idx,
+                            const float* w, const lsa_bf16* k_idx, const int64_t* k_off,
+                            int64_t max_len, float* scores, int64_t ld, void* stream);
+
+/*
+ * Top-k selection with the dense fallback ([Lite-Sparse] LSA section: the
+ * index_topk columns of highest score; the forced columns always enter; when
+ * the cached length is <= index_topk the indexer yields nothing and attention
+ * is dense).
+ *
+ * Row r with n = pos[r]+1 visible columns:
+ *   n <= index_topk: idx[r, :n] = 0..n-1, idx[r, n:] = -1, count[r] = n;
+ *   otherwise: count[r] = index_topk and idx[r, :] holds, unordered, the
+ *   index_init_tokens sink columns, the index_local_tokens local columns and
+ *   the remaining columns of highest score (ties to the lower index).
+ * scores fp32 [n_rows, ld] as written by lsa_index_scores (only columns
+ * 0..pos[r] are read). idx int32 [n_rows, index_topk], count int32 [n_rows].
+ * max_len (host): every pos[r] < max_len. Returns LSA_DENSE when
+ * max_len <= index_topk (every row dense; idx/count still written).
+ * Workspace: lsa_workspace_size(LSA_OP_TOPK, ...); rows are processed in
+ * blocks that fit (minimum one row, 40992 B).
+ */
+LSA_API lsa_status lsa_topk(const lsa_config* cfg, int32_t n_rows, const int32_t* pos, int64_t max_len,
+                    const float* scores, int64_t ld, int32_t* idx, int32_t* count, void* ws,
+                    size_t ws_bytes, void* stream);
+
+/*
+ * Sparse absorbed-latent MLA, decode ([Lite-Sparse] LSA section: at decode
+ * the latent rows are gathered by the top-k indices; 架构总览: kv_lora_rank 512,
+ * qk_rope_head_dim 64, 32 heads).
+ *
+ * Row b (one query of sequence b) attends over the latent rows
+ * latent[k_off[b] + idx[b, i]], i < count[b]:
+ *   x_i = softmax_scale * (q_abs[b,h,:] . latent[., :576])
+ *   out[b,h,:] = sum_i softmax(x)_i * latent[., :512];  lse[b,h] = log sum_i exp(x_i)
+ * idx == NULL: dense over all L_b = k_off[b+1]-k_off[b] keys (count unused).
+ * q_abs bf16 [batch, 32, 576]; latent bf16 [sum L_b, 576]; idx int32
+ * [batch, index_topk]; count int32 [batch]; out bf16 [batch, 32, 512];
+ * lse fp32 [batch, 32] or NULL. max_len (host) >= every L_b (sizes split-K).
+ * Workspace optional (split-K partials): lsa_workspace_size(LSA_OP_MLA_DECODE).
+ */
+LSA_API lsa_status lsa_sparse_mla_decode(const lsa_config* cfg, int32_t batch, const lsa_bf16* q_abs,
+                                 const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
+                                 const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,
+                                 void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Sparse absorbed-latent MLA, prefill ([Lite-Sparse] LSA section: at prefill
+ * a sparse boolean mask built from the indices enters attention). Row r
+ * attends over {idx[r, i] : i < count[r]}, which is the set that mask keeps,
+ * gathered instead of masked; idx == NULL: dense causal over 0..pos[r].
+ * One sequence: latent bf16 [n_keys, 576], every pos[r] < n_keys.
+ * Shapes otherwise as lsa_sparse_mla_decode, with n_rows query rows.
+ */
+LSA_API lsa_status lsa_sparse_mla_prefill(const lsa_config* cfg, int32_t n_rows, const int32_t* pos,
+                                  const lsa_bf16* q_abs, const lsa_bf16* latent, int64_t n_keys,
+                                  const int32_t* idx, const int32_t* count, lsa_bf16* out,
+                                  float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The whole layer: one index pass and top-k, then cli_factor attention
+ * sub-blocks over the same selection ([Lite-Sparse] LSA section, cross-layer
+ * index reuse: only the first sub-block owns an indexer; [LSA-2.0] 跨层索引).
+ * When max_len <= index_topk the indexer is not run and every sub-block is
+ * dense MLA, as the pages' fallback does.
+ *
+ * mode 0 = decode (rows are queries of sequences given by seq_of_row/k_off;
+ *          seq_of_row NULL means row b is the query of sequence b;
+ *          each sub-block's latent cache is packed like k_idx);
+ * mode 1 = prefill (one sequence, k_off NULL; max_len = keys in the caches).
+ * q_abs, latent, out, lse: HOST arrays of cli_factor DEVICE pointers
+ *   (lse entries may be NULL; lse itself may be NULL).
+ * idx_out int32 [n_rows, index_topk] and count_out int32 [n_rows]: optional
+ *   (NULL = keep the selection in the workspace). Unwritten when dense.
+ * Workspace: lsa_workspace_size(LSA_OP_FORWARD_*); prefill rows are processed
+ * in blocks that fit.
+ */
+LSA_API lsa_status lsa_forward(const lsa_config* cfg, int32_t mode, int32_t n_rows, int32_t n_seq,
+                       const int32_t* seq_of_row, const int32_t* pos, int64_t max_len,
+                       const lsa_bf16* q_idx, const float* w, const lsa_bf16* k_idx,
+                       const int64_t* k_off, const lsa_bf16* const* q_abs,
+                       const lsa_bf16* const* latent, lsa_bf16* const* out, float* const* lse,
+                       int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                       void* stream);
+
+/* Message for the last non-OK status returned on this thread ("" if none). */
+LSA_API const char* lsa_last_error(void);
+
+/* Synchronising: waits for the current device, returns and clears the sticky
+ * device-side flags (LSA_DEVERR_*) in *flags. LSA_ERR_DEVICE if any was set. */
+LSA_API lsa_status lsa_device_error(int32_t* flags);
+
+/* Number of kernels this library has launched in the process so far (host
+ * counter, no CUDA call). Used to count the launches inside a timed region. */
+LSA_API int64_t lsa_launch_count(void);
+
+/* ABI version of this header (1). */
+LSA_API int32_t lsa_abi_version(void);
+
+/*
+ * Synthetic inputs (tests and benchmarks; not part of the attention path).
+ * Counter-based SplitMix64 (Steele, Lea, Flood, OOPSLA 2014): the stream of
+ * tensor `tid` under `seed` starts at key = mix64(seed ^ tid*0xD1B54A32D192ED03)
+ * and element i is mix64(key + (i+1)*0x9E3779B97F4A7C15). A normal draw is
+ * (sum of the four 16-bit fields - 131070) * fp32(sigma/sqrt((2^32-1)/3)),
+ * one fp32 multiply; bf16 outputs round to nearest even. Elements
+ * first .. first+n-1 are written to dst[0 .. n-1].
+ * lsa_synth_rms_rows_bf16 draws n_rows rows of d values, rounds them to bf16,
+ * divides each row by sqrt(sum x^2 / d + 1e-6) in fp64, then rounds to fp32
+ * and to bf16 (row first_row+i of the stream goes to dst row i).
+ */
+LSA_API lsa_status lsa_synth_normal_bf16(lsa_bf16* dst, int64_t n, uint64_t seed, uint64_t tid,
+                                 int64_t first, double sigma, void* stream);
+LSA_API lsa_status lsa_synth_normal_f32(float* dst, int64_t n, uint64_t seed, uint64_t tid, int64_t first,
+                                double sigma, void* stream);
+LSA_API lsa_status lsa_synth_rms_rows_bf16(lsa_bf16* dst, int64_t n_rows, int32_t d, uint64_t seed,
+                                   uint64_t tid, int64_t first_row, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

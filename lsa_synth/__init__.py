@@ -68,12 +68,35 @@ def normal_scale(sigma: float) -> np.float32:
     return np.float32(float(sigma) / np.sqrt(IH_VAR))
 
 
-def normal_f32(seed: int, tid: int, first: int, n: int, sigma: float = 1.0) -> np.ndarray:
-    h = hash_range(seed, tid, first, n)
+def hash_at(seed: int, tid: int, index: np.ndarray) -> np.ndarray:
+    """uint64 words for arbitrary element indices of stream (seed, tid)."""
+    key = _U(stream_key(seed, tid))
+    i = np.asarray(index, dtype=np.uint64) + _U(1)
+    with np.errstate(over="ignore"):
+        z = key + i * _U(GOLDEN)
+    return mix64(z)
+
+
+def _irwin_hall(h: np.ndarray, sigma: float) -> np.ndarray:
     m = _U(0xFFFF)
     s = (h & m) + ((h >> _U(16)) & m) + ((h >> _U(32)) & m) + ((h >> _U(48)) & m)
     centred = s.astype(np.int64) - IH_CENTRE
     return centred.astype(np.float32) * normal_scale(sigma)
+
+
+def normal_f32_at(seed: int, tid: int, index: np.ndarray, sigma: float = 1.0) -> np.ndarray:
+    return _irwin_hall(hash_at(seed, tid, index), sigma)
+
+
+def normal_bf16_rows(seed: int, tid: int, rows: np.ndarray, d: int) -> np.ndarray:
+    """bf16 bits [len(rows), d] of the given rows of a [*, d] normal tensor."""
+    rows = np.asarray(rows, dtype=np.int64)
+    index = rows[:, None] * d + np.arange(d, dtype=np.int64)[None, :]
+    return f32_to_bf16_bits(normal_f32_at(seed, tid, index.ravel())).reshape(len(rows), d)
+
+
+def normal_f32(seed: int, tid: int, first: int, n: int, sigma: float = 1.0) -> np.ndarray:
+    return _irwin_hall(hash_range(seed, tid, first, n), sigma)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -1,0 +1,192 @@
+// Lightning indexer, streaming form (decode and any row set that does not share keys).
+//
+// [Lite-Sparse] "LSA（LongCat 稀疏注意力）": per index head q.k, ReLU, then the
+// head-weighted sum; sink and local-window columns forced to +inf.
+// [Lite-Sparse] "预填充优化": the ReLU-weighted head sum is fused into the
+// epilogue so the per-head [heads x keys] tensor is never written.
+// [LSA-2.0] "流式感知索引": the key stream is read as contiguous, coalesced HBM
+// traffic.
+//
+// Design. The per-key work is a [32 heads x 128] x [128] contraction (8192 flop
+// per 256-byte key row), too much for the FP32 pipes at HBM speed, so the keys
+// go through the tensor cores: a warp takes 16 keys as the M dimension of
+// mma.m16n8k16 (bf16 in, fp32 accumulate), the 32 heads as four n8 tiles, and
+// the 128 dims as eight k16 steps. The query's B fragments stay in registers for
+// the whole CTA. Each lane loads its A fragments straight from HBM with 16-byte
+// non-allocating loads: the contraction dimension is permuted (identically for
+// q and k, which leaves every dot product unchanged) so that one lane's eight
+// bf16 pairs of a key row are four contiguous 16-byte chunks, and the four lanes
+// of a quad read 64 contiguous bytes per instruction. The ReLU-weighted head sum
+// runs on the accumulators in registers, then two quad shuffles finish it.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lsa {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = kWarps * 32;
+constexpr int kKeysPerWarpTile = 16;
+
+struct KeyFrag {
+  uint4 lo[4];  // key g:   physical dims 8*(4c+t) .. +7, c = 0..3
+  uint4 hi[4];  // key g+8
+};
+
+__device__ __forceinline__ void load_keys(KeyFrag& f, const uint16_t* __restrict__ kb, int64_t ja,
+                                          int64_t jend, int t) {
+  const int64_t jb = ja + 8;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    f.lo[c] = (ja < jend) ? ld_stream_v4(kb + ja * kDi + 8 * (4 * c + t)) : make_uint4(0, 0, 0, 0);
+    f.hi[c] = (jb < jend) ? ld_stream_v4(kb + jb * kDi + 8 * (4 * c + t)) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+// Scores of keys g and g+8 of the tile (valid in every lane of the quad).
+__device__ __forceinline__ void score_tile(const KeyFrag& f, const uint4 (&qf)[4][4],
+                                           const float (&wf)[4][2], float& sa, float& sb) {
+  float acc[4][4];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[nt][i] = 0.f;
+#pragma unroll
+  for (int s = 0; s < 8; ++s) {
+    const int c = s >> 1;
+    const bool h = (s & 1) != 0;
+    // logical k (2t, 2t+1) -> physical elements {0,1} or {4,5} of chunk c;
+    // logical k (2t+8, 2t+9) -> physical {2,3} or {6,7}.
+    const uint32_t a0 = h ? f.lo[c].z : f.lo[c].x;
+    const uint32_t a1 = h ? f.hi[c].z : f.hi[c].x;
+    const uint32_t a2 = h ? f.lo[c].w : f.lo[c].y;
+    const uint32_t a3 = h ? f.hi[c].w : f.hi[c].y;
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const uint32_t b0 = h ? qf[nt][c].z : qf[nt][c].x;
+      const uint32_t b1 = h ? qf[nt][c].w : qf[nt][c].y;
+      mma_16816(acc[nt], a0, a1, a2, a3, b0, b1);
+    }
+  }
+  // acc[nt][e] = (key g, head 8nt+2t+e); acc[nt][2+e] = (key g+8, same head).
+  float x = 0.f, y = 0.f;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      x = fmaf(wf[nt][e], fmaxf(acc[nt][e], 0.f), x);
+      y = fmaf(wf[nt][e], fmaxf(acc[nt][2 + e], 0.f), y);
+    }
+  x += __shfl_xor_sync(0xffffffffu, x, 1);
+  x += __shfl_xor_sync(0xffffffffu, x, 2);
+  y += __shfl_xor_sync(0xffffffffu, y, 1);
+  y += __shfl_xor_sync(0xffffffffu, y, 2);
+  sa = x;
+  sb = y;
+}
+
+__global__ void __launch_bounds__(kThreads, 3)
+    index_decode_kernel(IndexArgs a, int keys_per_cta, int row0) {
+  const int r = row0 + blockIdx.y;
+  const int64_t j0 = (int64_t)blockIdx.x * keys_per_cta;
+  if (j0 >= a.max_len) return;
+  const int64_t j1 = min(j0 + (int64_t)keys_per_cta, a.max_len);
+
+  // Row geometry, with every out-of-range input clamped and flagged.
+  const int seq = a.seq_of_row ? a.seq_of_row[r] : (a.seq_identity ? r : 0);
+  int64_t kbase = 0, klen = a.max_len;
+  bool ok = true;
+  if (seq < 0 || seq >= a.n_seq) {
+    ok = false;
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(a.err, LSA_DEVERR_SEQ);
+  } else if (a.k_off) {
+    kbase = a.k_off[seq];
+    klen = a.k_off[seq + 1] - kbase;
+  }
+  const int64_t p = a.pos[r];
+  int64_t nvis = p + 1;
+  if (ok && (p < 0 || nvis > klen || nvis > a.max_len)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(a.err, LSA_DEVERR_POS);
+    nvis = max64(0, min(nvis, min(klen, a.max_len)));
+  }
+  if (!ok) nvis = 0;
+
+  float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
+  for (int64_t j = max(j0, nvis) + threadIdx.x; j < j1; j += kThreads) srow[j] = -INFINITY;
+  const int64_t jend = min(j1, nvis);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  int64_t tile = j0 + warp * kKeysPerWarpTile;
+  if (tile >= jend) return;
+
+  // Query B fragments (head 8nt+g, physical chunk 4c+t) and head weights.
+  uint4 qf[4][4];
+  const uint16_t* __restrict__ qr = a.q_idx + (int64_t)r * kHi * kDi;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      qf[nt][c] = __ldg(reinterpret_cast<const uint4*>(qr + (8 * nt + g) * kDi + 8 * (4 * c + t)));
+  float wf[4][2];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) wf[nt][e] = __ldg(a.w + (int64_t)r * kHi + 8 * nt + 2 * t + e);
+
+  const uint16_t* __restrict__ kb = a.k_idx + kbase * kDi;
+  const int64_t step = kWarps * kKeysPerWarpTile;
+  const int64_t lo_force = a.n_init, hi_force = p + 1 - a.n_loc;
+
+  auto put = [&](int64_t tl, float sa, float sb) {
+    if (t < 2) {
+      const int64_t j = tl + g + (t == 1 ? 8 : 0);
+      if (j < jend) {
+        const bool forced = (j < lo_force) || (j >= hi_force);
+        srow[j] = forced ? INFINITY : (t == 1 ? sb : sa);
+      }
+    }
+  };
+
+  // Two register sets: the next tile's loads are in flight while this one computes.
+  KeyFrag f0, f1;
+  load_keys(f0, kb, tile + g, jend, t);
+  while (true) {
+    int64_t nxt = tile + step;
+    if (nxt < jend) load_keys(f1, kb, nxt + g, jend, t);
+    float sa, sb;
+    score_tile(f0, qf, wf, sa, sb);
+    put(tile, sa, sb);
+    if (nxt >= jend) break;
+    tile = nxt;
+    nxt = tile + step;
+    if (nxt < jend) load_keys(f0, kb, nxt + g, jend, t);
+    score_tile(f1, qf, wf, sa, sb);
+    put(tile, sa, sb);
+    if (nxt >= jend) break;
+    tile = nxt;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st) {
+  if (a.n_rows <= 0) return cudaSuccess;
+  // Keys per CTA: a multiple of one CTA pass (64 keys), large enough to amortise
+  // the query-fragment load, small enough to give every SM several CTAs.
+  int sms = 148;
+  int dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t target_ctas = (int64_t)sms * 6;
+  int64_t kpc = (a.max_len * a.n_rows + target_ctas - 1) / target_ctas;
+  kpc = ((kpc + 255) / 256) * 256;
+  kpc = max64(256, min64(kpc, 8192));
+  const int64_t nx = (a.max_len + kpc - 1) / kpc;
+  for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
+    const int ny = min(65535, a.n_rows - row0);
+    index_decode_kernel<<<dim3((unsigned)nx, (unsigned)ny), kThreads, 0, st>>>(a, (int)kpc, row0);
+    count_launches(1);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace lsa

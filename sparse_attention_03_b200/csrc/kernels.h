@@ -1,0 +1,78 @@
+// Internal launchers of the LSA kernels (host side). Not part of the C-ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "lsa.h"
+
+namespace lsa {
+
+// Records the message for lsa_last_error() and returns `st`.
+lsa_status set_error(lsa_status st, const char* fmt, ...);
+// Address of this device's sticky error word (device memory).
+int* device_error_word();
+// Adds n to the process-wide launch counter (lsa_launch_count).
+void count_launches(int64_t n);
+
+struct IndexArgs {
+  const uint16_t* q_idx;   // [n_rows, 32, 128]
+  const float* w;          // [n_rows, 32]
+  const uint16_t* k_idx;   // packed [sum L, 128]
+  const int64_t* k_off;    // [n_seq+1] or null
+  const int32_t* seq_of_row;  // null: sequence r (seq_identity) or sequence 0
+  int seq_identity;
+  const int32_t* pos;
+  int n_rows, n_seq;
+  int64_t max_len;
+  int n_init, n_loc;
+  float* scores;
+  int64_t ld;
+  int* err;
+};
+
+// Streaming indexer: each CTA scores a run of keys of one row (decode shape).
+cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st);
+
+struct TopkArgs {
+  const float* scores;
+  int64_t ld;
+  const int32_t* pos;
+  int n_rows;
+  int64_t max_len;
+  int topk, n_init, n_loc;
+  int32_t* idx;
+  int32_t* count;
+  void* ws;
+  size_t ws_bytes;
+};
+constexpr int kTopkCap = 4096;                              // candidates kept per row
+constexpr size_t kTopkRowBytes = 2048 * 4 + 32 + kTopkCap * 8;  // hist + ctl + candidates
+cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
+cudaError_t launch_topk_dense(const TopkArgs& a, cudaStream_t st);
+
+struct MlaArgs {
+  const uint16_t* q[2];
+  const uint16_t* lat[2];
+  uint16_t* out[2];
+  float* lse[2];
+  const int64_t* k_off;      // decode: [n_seq+1]
+  const int32_t* seq_of_row; // decode: row -> sequence (null: identity)
+  const int32_t* pos;        // prefill: required; decode: optional (null: the whole sequence)
+  const int32_t* idx;        // [n_rows, topk] or null (dense)
+  const int32_t* count;
+  int n_rows, n_seq, topk, decode, cli;
+  int64_t n_keys;            // prefill: rows in latent
+  int64_t max_list;          // host bound on keys per row (sizes split-K)
+  float scale;
+  void* ws;
+  size_t ws_bytes;
+  int* err;
+};
+// Split-K partial bytes for a given split count.
+size_t mla_ws_bytes(int n_rows, int cli, int n_split);
+int mla_choose_splits(int n_rows, int cli, int64_t max_list);
+cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st);
+
+}  // namespace lsa

@@ -1,0 +1,419 @@
+// C-ABI of liblsa.so: argument checks, workspace carving and kernel dispatch.
+// The operations themselves are defined (with their sources) in include/lsa.h.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+
+#include <algorithm>
+#include <atomic>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lsa {
+
+static thread_local char g_msg[1024];
+__device__ int g_dev_err;
+
+lsa_status set_error(lsa_status st, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_msg, sizeof(g_msg), fmt, ap);
+  va_end(ap);
+  return st;
+}
+
+static std::atomic<int64_t> g_launches{0};
+void count_launches(int64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+
+int* device_error_word() {
+  static int* ptrs[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_dev_err) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kTopkPreferredRows = 4096;
+constexpr size_t kPrefillScoreBudget = size_t(4) << 30;  // bytes of scores per prefill block
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lsa_status check_cfg(const lsa_config* c, const char* fn) {
+  if (!c) return set_error(LSA_ERR_INVALID, "%s: cfg is NULL", fn);
+  if (c->index_n_heads != kHi || c->index_head_dim != kDi || c->n_heads != kH ||
+      c->kv_lora_rank != kDV || c->qk_rope_head_dim != kDLat - kDV)
+    return set_error(LSA_ERR_UNSUPPORTED,
+                     "%s: kernels implement index heads 32x128 and MLA 32 heads x (512+64) only", fn);
+  if (c->cli_factor < 1 || c->cli_factor > 2)
+    return set_error(LSA_ERR_UNSUPPORTED, "%s: cli_factor must be 1 or 2", fn);
+  if (c->index_topk < 1 || c->index_topk > kMaxTopk || c->index_init_tokens < 0 ||
+      c->index_local_tokens < 0 ||
+      (int64_t)c->index_init_tokens + c->index_local_tokens >= c->index_topk)
+    return set_error(LSA_ERR_UNSUPPORTED,
+                     "%s: need 0 <= init, 0 <= local, init + local < topk <= 2048", fn);
+  if (!(c->softmax_scale > 0.f) || !isfinite(c->softmax_scale))
+    return set_error(LSA_ERR_INVALID, "%s: softmax_scale must be finite and > 0", fn);
+  return LSA_OK;
+}
+
+lsa_status cuda_status(cudaError_t e, const char* fn) {
+  if (e == cudaSuccess) return LSA_OK;
+  return set_error(LSA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
+}
+
+size_t topk_ws(int n_rows) {
+  return (size_t)std::min(n_rows, kTopkPreferredRows) * kTopkRowBytes + kAlign;
+}
+
+size_t mla_ws(int n_rows, int cli, int64_t max_list) {
+  return mla_ws_bytes(n_rows, cli, mla_choose_splits(n_rows, cli, max_list));
+}
+
+// Workspace of one forward block of R rows (sparse path).
+size_t forward_block_ws(const lsa_config* c, int R, int64_t max_len) {
+  return align_up((size_t)R * max_len * sizeof(float)) +
+         align_up((size_t)R * c->index_topk * sizeof(int32_t)) +
+         align_up((size_t)R * sizeof(int32_t)) + topk_ws(R) + mla_ws(R, c->cli_factor, c->index_topk);
+}
+
+int prefill_block_rows(int n_rows, int64_t max_len) {
+  int64_t r = (int64_t)(kPrefillScoreBudget / ((size_t)max_len * sizeof(float)));
+  r = std::max<int64_t>(64, r / 64 * 64);
+  return (int)std::min<int64_t>(r, n_rows);
+}
+
+lsa_status run_index_scores(const lsa_config* c, int n_rows, int n_seq, const int32_t* seq_of_row,
+                            int seq_identity, const int32_t* pos, const lsa_bf16* q_idx, const float* w,
+                            const lsa_bf16* k_idx, const int64_t* k_off, int64_t max_len,
+                            float* scores, int64_t ld, cudaStream_t st) {
+  IndexArgs a;
+  a.q_idx = q_idx;
+  a.w = w;
+  a.k_idx = k_idx;
+  a.k_off = k_off;
+  a.seq_of_row = seq_of_row;
+  a.seq_identity = seq_identity;
+  a.pos = pos;
+  a.n_rows = n_rows;
+  a.n_seq = n_seq;
+  a.max_len = max_len;
+  a.n_init = c->index_init_tokens;
+  a.n_loc = c->index_local_tokens;
+  a.scores = scores;
+  a.ld = ld;
+  a.err = device_error_word();
+  return cuda_status(launch_index_decode(a, st), "lsa_index_scores");
+}
+
+lsa_status run_topk(const lsa_config* c, int n_rows, const int32_t* pos, int64_t max_len,
+                    const float* scores, int64_t ld, int32_t* idx, int32_t* count, void* ws,
+                    size_t ws_bytes, cudaStream_t st) {
+  TopkArgs a;
+  a.scores = scores;
+  a.ld = ld;
+  a.pos = pos;
+  a.n_rows = n_rows;
+  a.max_len = max_len;
+  a.topk = c->index_topk;
+  a.n_init = c->index_init_tokens;
+  a.n_loc = c->index_local_tokens;
+  a.idx = idx;
+  a.count = count;
+  uintptr_t p = (reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~uintptr_t(kAlign - 1);
+  a.ws = reinterpret_cast<void*>(p);
+  const size_t slack = ws ? p - reinterpret_cast<uintptr_t>(ws) : 0;
+  a.ws_bytes = ws_bytes > slack ? ws_bytes - slack : 0;
+  if (max_len > c->index_topk && a.ws_bytes < kTopkRowBytes)
+    return set_error(LSA_ERR_WORKSPACE, "lsa_topk: workspace below one row (%zu bytes)",
+                     (size_t)kTopkRowBytes);
+  const lsa_status st2 = cuda_status(launch_topk(a, st), "lsa_topk");
+  if (st2 != LSA_OK) return st2;
+  return max_len <= c->index_topk ? LSA_DENSE : LSA_OK;
+}
+
+MlaArgs mla_args(const lsa_config* c, int cli, int n_rows, int decode) {
+  MlaArgs a = {};
+  a.n_rows = n_rows;
+  a.cli = cli;
+  a.decode = decode;
+  a.topk = c->index_topk;
+  a.scale = c->softmax_scale;
+  a.err = device_error_word();
+  return a;
+}
+
+}  // namespace
+}  // namespace lsa
+
+using namespace lsa;
+
+extern "C" {
+
+int32_t lsa_abi_version(void) { return 1; }
+
+int64_t lsa_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char* lsa_last_error(void) { return g_msg; }
+
+void lsa_config_default(lsa_config* c) {
+  if (!c) return;
+  c->index_n_heads = 32;
+  c->index_head_dim = 128;
+  c->index_topk = 2048;
+  c->index_init_tokens = 16;
+  c->index_local_tokens = 1024;
+  c->cli_factor = 2;
+  c->n_heads = 32;
+  c->kv_lora_rank = 512;
+  c->qk_rope_head_dim = 64;
+  c->softmax_scale = (float)(1.0 / sqrt(128.0 + 64.0));
+}
+
+size_t lsa_workspace_size(const lsa_config* c, int32_t op, int32_t n_rows, int32_t n_seq,
+                          int64_t max_len) {
+  (void)n_seq;
+  if (check_cfg(c, "lsa_workspace_size") != LSA_OK || n_rows < 0 || max_len < 1) return 0;
+  if (n_rows == 0) return kAlign;
+  const int64_t list = std::min<int64_t>(max_len, c->index_topk);
+  switch (op) {
+    case LSA_OP_TOPK:
+      return max_len <= c->index_topk ? kAlign : topk_ws(n_rows);
+    case LSA_OP_MLA_DECODE:
+    case LSA_OP_MLA_PREFILL:
+      return std::max(mla_ws(n_rows, 1, max_len), mla_ws(n_rows, 1, list)) + kAlign;
+    case LSA_OP_FORWARD_DECODE:
+      if (max_len <= c->index_topk) return mla_ws(n_rows, c->cli_factor, max_len) + kAlign;
+      return forward_block_ws(c, n_rows, max_len) + kAlign;
+    case LSA_OP_FORWARD_PREFILL:
+      if (max_len <= c->index_topk) return mla_ws(n_rows, c->cli_factor, max_len) + kAlign;
+      return forward_block_ws(c, prefill_block_rows(n_rows, max_len), max_len) + kAlign;
+    default:
+      return 0;
+  }
+}
+
+lsa_status lsa_device_error(int32_t* flags) {
+  int* p = device_error_word();
+  if (!p) return set_error(LSA_ERR_CUDA, "lsa_device_error: no device error word");
+  cudaError_t e = cudaDeviceSynchronize();
+  if (e != cudaSuccess) return cuda_status(e, "lsa_device_error");
+  int v = 0;
+  e = cudaMemcpy(&v, p, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e == cudaSuccess) e = cudaMemset(p, 0, sizeof(int));
+  if (e != cudaSuccess) return cuda_status(e, "lsa_device_error");
+  if (flags) *flags = v;
+  if (v) return set_error(LSA_ERR_DEVICE, "lsa_device_error: device flags 0x%x", v);
+  return LSA_OK;
+}
+
+lsa_status lsa_index_scores(const lsa_config* c, int32_t n_rows, int32_t n_seq,
+                            const int32_t* seq_of_row, const int32_t* pos, const lsa_bf16* q_idx,
+                            const float* w, const lsa_bf16* k_idx, const int64_t* k_off,
+                            int64_t max_len, float* scores, int64_t ld, void* stream) {
+  const char* fn = "lsa_index_scores";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (n_rows < 0 || n_seq < 1 || max_len < 1 || ld < max_len)
+    return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0, n_seq >= 1, 1 <= max_len <= ld", fn);
+  if (!k_off && n_seq != 1) return set_error(LSA_ERR_INVALID, "%s: k_off is NULL with n_seq > 1", fn);
+  if (n_rows == 0) return LSA_OK;
+  if (!pos || !q_idx || !w || !k_idx || !scores)
+    return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (!aligned16(q_idx) || !aligned16(k_idx))
+    return set_error(LSA_ERR_INVALID, "%s: q_idx and k_idx must be 16-byte aligned", fn);
+  return run_index_scores(c, n_rows, n_seq, seq_of_row, 0, pos, q_idx, w, k_idx, k_off, max_len,
+                          scores, ld, (cudaStream_t)stream);
+}
+
+lsa_status lsa_topk(const lsa_config* c, int32_t n_rows, const int32_t* pos, int64_t max_len,
+                    const float* scores, int64_t ld, int32_t* idx, int32_t* count, void* ws,
+                    size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_topk";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (n_rows < 0 || max_len < 1 || ld < max_len)
+    return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0 and 1 <= max_len <= ld", fn);
+  if (n_rows == 0) return max_len <= c->index_topk ? LSA_DENSE : LSA_OK;
+  if (!pos || !scores || !idx || !count) return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (max_len > c->index_topk && !ws) return set_error(LSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
+  return run_topk(c, n_rows, pos, max_len, scores, ld, idx, count, ws, ws_bytes, (cudaStream_t)stream);
+}
+
+lsa_status lsa_sparse_mla_decode(const lsa_config* c, int32_t batch, const lsa_bf16* q_abs,
+                                 const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
+                                 const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_sparse_mla_decode";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (batch < 0 || max_len < 1) return set_error(LSA_ERR_INVALID, "%s: need batch >= 0, max_len >= 1", fn);
+  if (batch == 0) return LSA_OK;
+  if (!q_abs || !latent || !k_off || !out || (idx && !count))
+    return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (!aligned16(q_abs) || !aligned16(latent) || !aligned16(out))
+    return set_error(LSA_ERR_INVALID, "%s: q_abs, latent and out must be 16-byte aligned", fn);
+  MlaArgs a = mla_args(c, 1, batch, 1);
+  a.q[0] = q_abs;
+  a.lat[0] = latent;
+  a.out[0] = out;
+  a.lse[0] = lse;
+  a.k_off = k_off;
+  a.n_seq = batch;
+  a.idx = idx;
+  a.count = count;
+  a.max_list = idx ? c->index_topk : max_len;
+  a.ws = ws;
+  a.ws_bytes = ws ? ws_bytes : 0;
+  return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
+}
+
+lsa_status lsa_sparse_mla_prefill(const lsa_config* c, int32_t n_rows, const int32_t* pos,
+                                  const lsa_bf16* q_abs, const lsa_bf16* latent, int64_t n_keys,
+                                  const int32_t* idx, const int32_t* count, lsa_bf16* out,
+                                  float* lse, void* ws, size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_sparse_mla_prefill";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (n_rows < 0 || n_keys < 1) return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0, n_keys >= 1", fn);
+  if (n_rows == 0) return LSA_OK;
+  if (!pos || !q_abs || !latent || !out || (idx && !count))
+    return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (!aligned16(q_abs) || !aligned16(latent) || !aligned16(out))
+    return set_error(LSA_ERR_INVALID, "%s: q_abs, latent and out must be 16-byte aligned", fn);
+  MlaArgs a = mla_args(c, 1, n_rows, 0);
+  a.q[0] = q_abs;
+  a.lat[0] = latent;
+  a.out[0] = out;
+  a.lse[0] = lse;
+  a.pos = pos;
+  a.n_keys = n_keys;
+  a.idx = idx;
+  a.count = count;
+  a.max_list = idx ? c->index_topk : n_keys;
+  a.ws = ws;
+  a.ws_bytes = ws ? ws_bytes : 0;
+  return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
+}
+
+lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_t n_seq,
+                       const int32_t* seq_of_row, const int32_t* pos, int64_t max_len,
+                       const lsa_bf16* q_idx, const float* w, const lsa_bf16* k_idx,
+                       const int64_t* k_off, const lsa_bf16* const* q_abs,
+                       const lsa_bf16* const* latent, lsa_bf16* const* out, float* const* lse,
+                       int32_t* idx_out, int32_t* count_out, void* ws, size_t ws_bytes,
+                       void* stream) {
+  const char* fn = "lsa_forward";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  const cudaStream_t st = (cudaStream_t)stream;
+  const int cli = c->cli_factor;
+  if ((mode != 0 && mode != 1) || n_rows < 0 || n_seq < 1 || max_len < 1)
+    return set_error(LSA_ERR_INVALID, "%s: need mode 0/1, n_rows >= 0, n_seq >= 1, max_len >= 1", fn);
+  if (mode == 0 && !k_off) return set_error(LSA_ERR_INVALID, "%s: decode needs k_off", fn);
+  if (mode == 1 && n_seq != 1) return set_error(LSA_ERR_INVALID, "%s: prefill takes one sequence", fn);
+  if (n_rows == 0) return LSA_OK;
+  if (!pos || !q_abs || !latent || !out) return set_error(LSA_ERR_INVALID, "%s: NULL argument", fn);
+  for (int z = 0; z < cli; ++z) {
+    if (!q_abs[z] || !latent[z] || !out[z])
+      return set_error(LSA_ERR_INVALID, "%s: NULL sub-block pointer %d", fn, z);
+    if (!aligned16(q_abs[z]) || !aligned16(latent[z]) || !aligned16(out[z]))
+      return set_error(LSA_ERR_INVALID, "%s: sub-block %d arrays must be 16-byte aligned", fn, z);
+  }
+  const bool dense = max_len <= c->index_topk;
+  if (!dense) {
+    if (!q_idx || !w || !k_idx) return set_error(LSA_ERR_INVALID, "%s: NULL indexer argument", fn);
+    if (!aligned16(q_idx) || !aligned16(k_idx))
+      return set_error(LSA_ERR_INVALID, "%s: q_idx and k_idx must be 16-byte aligned", fn);
+    if (!ws) return set_error(LSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
+  }
+
+  // Carve the workspace.
+  uintptr_t base = (reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~uintptr_t(kAlign - 1);
+  size_t avail = ws ? ws_bytes - std::min(ws_bytes, (size_t)(base - reinterpret_cast<uintptr_t>(ws))) : 0;
+
+  MlaArgs m = mla_args(c, cli, n_rows, mode == 0 ? 1 : 0);
+  for (int z = 0; z < cli; ++z) {
+    m.q[z] = q_abs[z];
+    m.lat[z] = latent[z];
+    m.out[z] = out[z];
+    m.lse[z] = lse ? lse[z] : nullptr;
+  }
+  m.k_off = mode == 0 ? k_off : nullptr;
+  m.seq_of_row = mode == 0 ? seq_of_row : nullptr;
+  m.n_seq = n_seq;
+  m.pos = pos;
+  m.n_keys = max_len;
+
+  if (dense) {
+    // The pages' fallback: no index pass, dense MLA in every sub-block.
+    m.idx = nullptr;
+    m.count = nullptr;
+    m.max_list = max_len;
+    m.ws = reinterpret_cast<void*>(base);
+    m.ws_bytes = avail;
+    return cuda_status(launch_mla(m, st), fn);
+  }
+
+  int R = n_rows;
+  if (mode == 1) R = prefill_block_rows(n_rows, max_len);
+  while (R > 1 && forward_block_ws(c, R, max_len) > avail) R = R > 64 ? R / 64 * 32 : R / 2;
+  if (forward_block_ws(c, R, max_len) > avail)
+    return set_error(LSA_ERR_WORKSPACE, "%s: workspace %zu below the minimum %zu", fn, ws_bytes,
+                     forward_block_ws(c, 1, max_len) + kAlign);
+  if (mode == 0 && R < n_rows)
+    return set_error(LSA_ERR_WORKSPACE, "%s: decode needs lsa_workspace_size(LSA_OP_FORWARD_DECODE)", fn);
+
+  char* p = reinterpret_cast<char*>(base);
+  float* scores = reinterpret_cast<float*>(p);
+  p += align_up((size_t)R * max_len * sizeof(float));
+  int32_t* idx_ws = reinterpret_cast<int32_t*>(p);
+  p += align_up((size_t)R * c->index_topk * sizeof(int32_t));
+  int32_t* cnt_ws = reinterpret_cast<int32_t*>(p);
+  p += align_up((size_t)R * sizeof(int32_t));
+  void* topk_w = p;
+  const size_t topk_bytes = topk_ws(R);
+  p += topk_bytes;
+  void* mla_w = p;
+  const size_t mla_bytes = mla_ws(R, cli, c->index_topk);
+
+  for (int r0 = 0; r0 < n_rows; r0 += R) {
+    const int nr = std::min(R, n_rows - r0);
+    int32_t* idx_b = idx_out ? idx_out + (int64_t)r0 * c->index_topk : idx_ws;
+    int32_t* cnt_b = count_out ? count_out + r0 : cnt_ws;
+    s = run_index_scores(c, nr, n_seq, seq_of_row ? seq_of_row + r0 : nullptr, mode == 0, pos + r0,
+                         q_idx + (int64_t)r0 * kHi * kDi, w + (int64_t)r0 * kHi, k_idx, k_off,
+                         max_len, scores, max_len, st);
+    if (s != LSA_OK) return s;
+    s = run_topk(c, nr, pos + r0, max_len, scores, max_len, idx_b, cnt_b, topk_w, topk_bytes, st);
+    if (s != LSA_OK && s != LSA_DENSE) return s;
+    MlaArgs b = m;
+    b.n_rows = nr;
+    for (int z = 0; z < cli; ++z) {
+      b.q[z] = q_abs[z] + (int64_t)r0 * kH * kDLat;
+      b.out[z] = out[z] + (int64_t)r0 * kH * kDV;
+      b.lse[z] = m.lse[z] ? m.lse[z] + (int64_t)r0 * kH : nullptr;
+    }
+    if (b.seq_of_row) b.seq_of_row += r0;
+    else if (mode == 0 && r0 > 0) return set_error(LSA_ERR_INVALID, "%s: internal row split", fn);
+    b.pos = pos + r0;
+    b.idx = idx_b;
+    b.count = cnt_b;
+    b.max_list = c->index_topk;
+    b.ws = mla_w;
+    b.ws_bytes = mla_bytes;
+    s = cuda_status(launch_mla(b, st), fn);
+    if (s != LSA_OK) return s;
+  }
+  return LSA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,242 @@
+"""Python binding of liblsa.so (argument marshalling only).
+
+Every function here takes torch tensors that live on a CUDA device, checks
+their dtype, shape and contiguity, and passes raw pointers to the C entry point
+of the same name (declared in include/lsa.h). All work runs in the library's
+CUDA kernels on the current torch stream; there is no other implementation
+behind these names. If the library is missing, load() raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblsa.so")
+
+LSA_OK, LSA_DENSE = 0, 1
+LSA_ERR_INVALID, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_DEVICE = -1, -2, -3, -4, -5
+OP_TOPK, OP_MLA_DECODE, OP_MLA_PREFILL, OP_FORWARD_DECODE, OP_FORWARD_PREFILL = 1, 2, 3, 4, 5
+DEVERR_POS, DEVERR_INDEX, DEVERR_COUNT, DEVERR_SEQ = 1, 2, 4, 8
+
+EXPORTS = (
+    "lsa_config_default", "lsa_workspace_size", "lsa_index_scores", "lsa_topk",
+    "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill", "lsa_forward", "lsa_last_error",
+    "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16", "lsa_synth_normal_f32",
+    "lsa_synth_rms_rows_bf16", "lsa_launch_count",
+)
+
+
+class LsaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"status {status}: {msg}")
+        self.status = status
+
+
+class Config(ctypes.Structure):
+    _fields_ = [
+        ("index_n_heads", ctypes.c_int32),
+        ("index_head_dim", ctypes.c_int32),
+        ("index_topk", ctypes.c_int32),
+        ("index_init_tokens", ctypes.c_int32),
+        ("index_local_tokens", ctypes.c_int32),
+        ("cli_factor", ctypes.c_int32),
+        ("n_heads", ctypes.c_int32),
+        ("kv_lora_rank", ctypes.c_int32),
+        ("qk_rope_head_dim", ctypes.c_int32),
+        ("softmax_scale", ctypes.c_float),
+    ]
+
+
+_lib = None
+_P = ctypes.c_void_p
+_I32, _I64, _U64, _SZ = ctypes.c_int32, ctypes.c_int64, ctypes.c_uint64, ctypes.c_size_t
+
+
+def load():
+    """Loads liblsa.so once. Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with `python -m sparse_attention_03_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.lsa_config_default.argtypes = [ctypes.POINTER(Config)]
+    lib.lsa_config_default.restype = None
+    lib.lsa_workspace_size.argtypes = [ctypes.POINTER(Config), _I32, _I32, _I32, _I64]
+    lib.lsa_workspace_size.restype = _SZ
+    lib.lsa_index_scores.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P]
+    lib.lsa_topk.argtypes = [ctypes.POINTER(Config), _I32, _P, _I64, _P, _I64, _P, _P, _P, _SZ, _P]
+    lib.lsa_sparse_mla_decode.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]
+    lib.lsa_sparse_mla_prefill.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.lsa_forward.argtypes = [ctypes.POINTER(Config), _I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P,
+                                ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
+                                _P, _P, _P, _SZ, _P]
+    lib.lsa_last_error.argtypes = []
+    lib.lsa_last_error.restype = ctypes.c_char_p
+    lib.lsa_device_error.argtypes = [ctypes.POINTER(_I32)]
+    lib.lsa_abi_version.argtypes = []
+    lib.lsa_launch_count.argtypes = []
+    lib.lsa_launch_count.restype = _I64
+    lib.lsa_synth_normal_bf16.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
+    lib.lsa_synth_normal_f32.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
+    lib.lsa_synth_rms_rows_bf16.argtypes = [_P, _I64, _I32, _U64, _U64, _I64, _P]
+    for name in ("lsa_index_scores", "lsa_topk", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
+                 "lsa_forward", "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16",
+                 "lsa_synth_normal_f32", "lsa_synth_rms_rows_bf16"):
+        getattr(lib, name).restype = _I32
+    _lib = lib
+    return lib
+
+
+@dataclass
+class LsaConfig:
+    index_topk: int = 2048
+    index_init_tokens: int = 16
+    index_local_tokens: int = 1024
+    cli_factor: int = 2
+    softmax_scale: float = 1.0 / (192.0 ** 0.5)
+
+    def c(self) -> Config:
+        cfg = Config()
+        load().lsa_config_default(ctypes.byref(cfg))
+        cfg.index_topk = self.index_topk
+        cfg.index_init_tokens = self.index_init_tokens
+        cfg.index_local_tokens = self.index_local_tokens
+        cfg.cli_factor = self.cli_factor
+        cfg.softmax_scale = self.softmax_scale
+        return cfg
+
+
+def _check(status: int, allow_dense: bool = False) -> int:
+    if status < 0 or (status == LSA_DENSE and not allow_dense):
+        raise LsaError(status, load().lsa_last_error().decode())
+    return status
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t, dtype, name):
+    if t is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _stream(stream):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def workspace_size(cfg: LsaConfig, op: int, n_rows: int, n_seq: int, max_len: int) -> int:
+    return int(load().lsa_workspace_size(ctypes.byref(cfg.c()), op, n_rows, n_seq, max_len))
+
+
+def workspace(cfg: LsaConfig, op: int, n_rows: int, n_seq: int, max_len: int, device=None) -> torch.Tensor:
+    n = workspace_size(cfg, op, n_rows, n_seq, max_len)
+    return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
+
+
+def index_scores(cfg, seq_of_row, pos, q_idx, w, k_idx, k_off, max_len, scores, n_seq=None, stream=None):
+    _dt(q_idx, torch.bfloat16, "q_idx"); _dt(k_idx, torch.bfloat16, "k_idx"); _dt(w, torch.float32, "w")
+    _dt(pos, torch.int32, "pos"); _dt(seq_of_row, torch.int32, "seq_of_row"); _dt(k_off, torch.int64, "k_off")
+    _dt(scores, torch.float32, "scores")
+    n_rows = pos.shape[0]
+    if n_seq is None:
+        n_seq = 1 if k_off is None else k_off.shape[0] - 1
+    return _check(load().lsa_index_scores(
+        ctypes.byref(cfg.c()), n_rows, n_seq, _ptr(seq_of_row), _ptr(pos), _ptr(q_idx), _ptr(w),
+        _ptr(k_idx), _ptr(k_off), int(max_len), _ptr(scores), scores.shape[1], _stream(stream)))
+
+
+def topk(cfg, pos, max_len, scores, idx, count, ws, stream=None):
+    _dt(scores, torch.float32, "scores"); _dt(pos, torch.int32, "pos")
+    _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
+    return _check(load().lsa_topk(
+        ctypes.byref(cfg.c()), pos.shape[0], _ptr(pos), int(max_len), _ptr(scores), scores.shape[1],
+        _ptr(idx), _ptr(count), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)), allow_dense=True)
+
+
+def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None):
+    for t, n in ((q_abs, "q_abs"), (latent, "latent"), (out, "out")):
+        _dt(t, torch.bfloat16, n)
+    _dt(k_off, torch.int64, "k_off"); _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
+    _dt(lse, torch.float32, "lse")
+    return _check(load().lsa_sparse_mla_decode(
+        ctypes.byref(cfg.c()), q_abs.shape[0], _ptr(q_abs), _ptr(latent), _ptr(k_off), _ptr(idx),
+        _ptr(count), int(max_len), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)))
+
+
+def sparse_mla_prefill(cfg, pos, q_abs, latent, idx, count, out, lse, ws, stream=None):
+    for t, n in ((q_abs, "q_abs"), (latent, "latent"), (out, "out")):
+        _dt(t, torch.bfloat16, n)
+    _dt(pos, torch.int32, "pos"); _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
+    _dt(lse, torch.float32, "lse")
+    return _check(load().lsa_sparse_mla_prefill(
+        ctypes.byref(cfg.c()), pos.shape[0], _ptr(pos), _ptr(q_abs), _ptr(latent), latent.shape[0],
+        _ptr(idx), _ptr(count), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)))
+
+
+def _ptr_array(ts):
+    arr = (ctypes.c_void_p * len(ts))()
+    for i, t in enumerate(ts):
+        arr[i] = None if t is None else t.data_ptr()
+    return arr
+
+
+def forward(cfg, mode, seq_of_row, pos, max_len, q_idx, w, k_idx, k_off, q_abs, latent, out, lse,
+            ws, idx_out=None, count_out=None, n_seq=None, stream=None):
+    """mode 0 decode / 1 prefill; q_abs, latent, out, lse: lists of cli_factor tensors."""
+    for t in list(q_abs) + list(latent) + list(out):
+        _dt(t, torch.bfloat16, "q_abs/latent/out")
+        _ptr(t)
+    for t in (lse or []):
+        _dt(t, torch.float32, "lse")
+        if t is not None:
+            _ptr(t)
+    if n_seq is None:
+        n_seq = 1 if k_off is None else k_off.shape[0] - 1
+    keep = (_ptr_array(q_abs), _ptr_array(latent), _ptr_array(out), _ptr_array(lse) if lse else None)
+    return _check(load().lsa_forward(
+        ctypes.byref(cfg.c()), int(mode), pos.shape[0], n_seq, _ptr(seq_of_row), _ptr(pos), int(max_len),
+        _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_off), keep[0], keep[1], keep[2], keep[3],
+        _ptr(idx_out), _ptr(count_out), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+
+
+def launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(load().lsa_launch_count())
+
+
+def device_error() -> int:
+    """Synchronises, returns and clears the sticky device-side error flags."""
+    flags = ctypes.c_int32(0)
+    load().lsa_device_error(ctypes.byref(flags))
+    return int(flags.value)
+
+
+def synth_normal_bf16(dst, seed, tid, first=0, sigma=1.0, stream=None):
+    _dt(dst, torch.bfloat16, "dst")
+    return _check(load().lsa_synth_normal_bf16(_ptr(dst), dst.numel(), seed, tid, first, sigma, _stream(stream)))
+
+
+def synth_normal_f32(dst, seed, tid, first=0, sigma=1.0, stream=None):
+    _dt(dst, torch.float32, "dst")
+    return _check(load().lsa_synth_normal_f32(_ptr(dst), dst.numel(), seed, tid, first, sigma, _stream(stream)))
+
+
+def synth_rms_rows_bf16(dst, seed, tid, first_row=0, stream=None):
+    _dt(dst, torch.bfloat16, "dst")
+    n_rows, d = dst.shape
+    return _check(load().lsa_synth_rms_rows_bf16(_ptr(dst), n_rows, d, seed, tid, first_row, _stream(stream)))

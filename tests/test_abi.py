@@ -1,0 +1,108 @@
+"""The C-ABI library loads, exports every symbol include/lsa.h declares, and its
+host-side checks reject bad arguments before any CUDA call (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_attention_03_b200 import lsa
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "lsa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return lsa.load()
+
+
+def _declared():
+    txt = open(HEADER).read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(lsa_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("lsa_index_scores", "lsa_topk", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
+                     "lsa_forward"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared():
+        assert hasattr(lib, name), f"{name} declared in lsa.h but not exported"
+    assert set(lsa.EXPORTS) <= set(_declared())
+
+
+def test_abi_version_and_defaults(lib):
+    assert lib.lsa_abi_version() == 1
+    c = lsa.Config()
+    lib.lsa_config_default(ctypes.byref(c))
+    assert (c.index_n_heads, c.index_head_dim, c.index_topk, c.index_init_tokens, c.index_local_tokens,
+            c.cli_factor, c.n_heads, c.kv_lora_rank, c.qk_rope_head_dim) == (32, 128, 2048, 16, 1024, 2, 32, 512, 64)
+    assert abs(c.softmax_scale - 192 ** -0.5) < 1e-7
+
+
+def test_workspace_sizes(lib):
+    cfg = lsa.LsaConfig()
+    assert lsa.workspace_size(cfg, lsa.OP_TOPK, 64, 64, 1000) <= 256      # dense: nothing needed
+    assert lsa.workspace_size(cfg, lsa.OP_TOPK, 64, 64, 32768) >= 64 * 40992
+    big = lsa.workspace_size(cfg, lsa.OP_FORWARD_DECODE, 16, 16, 131072)
+    assert big >= 16 * 131072 * 4        # the score rows
+    pre = lsa.workspace_size(cfg, lsa.OP_FORWARD_PREFILL, 16384, 1, 16384)
+    assert pre >= 16384 * 16384 * 4
+    bad = lsa.LsaConfig(index_topk=10, index_init_tokens=5, index_local_tokens=5)
+    assert lsa.workspace_size(bad, lsa.OP_TOPK, 4, 4, 100) == 0
+
+
+def _fake(n=1):
+    return ctypes.c_void_p(0x10000 * n)  # aligned, never dereferenced by the host checks
+
+
+def test_rejects_bad_config(lib):
+    c = lsa.LsaConfig().c()
+    c.index_n_heads = 16
+    st = lib.lsa_index_scores(ctypes.byref(c), 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100,
+                              _fake(), 100, None)
+    assert st == lsa.LSA_ERR_UNSUPPORTED
+    assert b"32x128" in lib.lsa_last_error()
+    st = lib.lsa_index_scores(None, 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100, _fake(), 100, None)
+    assert st == lsa.LSA_ERR_INVALID
+
+
+def test_rejects_bad_arguments(lib):
+    c = lsa.LsaConfig().c()
+    # ld < max_len
+    assert lib.lsa_index_scores(ctypes.byref(c), 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100,
+                                _fake(), 50, None) == lsa.LSA_ERR_INVALID
+    # misaligned q_idx
+    assert lib.lsa_index_scores(ctypes.byref(c), 4, 1, None, _fake(), ctypes.c_void_p(0x10002), _fake(),
+                                _fake(), None, 100, _fake(), 100, None) == lsa.LSA_ERR_INVALID
+    # several sequences without offsets
+    assert lib.lsa_index_scores(ctypes.byref(c), 4, 3, None, _fake(), _fake(), _fake(), _fake(), None, 100,
+                                _fake(), 100, None) == lsa.LSA_ERR_INVALID
+    # top-k without a workspace on a sparse length
+    assert lib.lsa_topk(ctypes.byref(c), 4, _fake(), 5000, _fake(), 5000, _fake(), _fake(), None, 0,
+                        None) == lsa.LSA_ERR_WORKSPACE
+    # decode MLA without offsets
+    assert lib.lsa_sparse_mla_decode(ctypes.byref(c), 2, _fake(), _fake(), None, None, None, 10, _fake(),
+                                     None, None, 0, None) == lsa.LSA_ERR_INVALID
+    # forward: bad mode, prefill with several sequences
+    arr = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    assert lib.lsa_forward(ctypes.byref(c), 2, 1, 1, None, _fake(), 10, _fake(), _fake(), _fake(), _fake(),
+                           arr, arr, arr, None, None, None, None, 0, None) == lsa.LSA_ERR_INVALID
+    assert lib.lsa_forward(ctypes.byref(c), 1, 1, 2, None, _fake(), 10, _fake(), _fake(), _fake(), None,
+                           arr, arr, arr, None, None, None, None, 0, None) == lsa.LSA_ERR_INVALID
+    # sparse forward without workspace
+    assert lib.lsa_forward(ctypes.byref(c), 0, 1, 1, None, _fake(), 5000, _fake(), _fake(), _fake(), _fake(),
+                           arr, arr, arr, None, None, None, None, 0, None) == lsa.LSA_ERR_WORKSPACE
+
+
+def test_empty_inputs_are_noops(lib):
+    c = lsa.LsaConfig().c()
+    assert lib.lsa_index_scores(ctypes.byref(c), 0, 1, None, None, None, None, None, None, 10, None, 10,
+                                None) == lsa.LSA_OK
+    assert lib.lsa_topk(ctypes.byref(c), 0, None, 10, None, 10, None, None, None, 0, None) == lsa.LSA_DENSE
+    assert lib.lsa_sparse_mla_prefill(ctypes.byref(c), 0, None, None, None, 5, None, None, None, None, None,
+                                      0, None) == lsa.LSA_OK

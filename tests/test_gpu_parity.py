@@ -1,0 +1,504 @@
+"""GPU parity: every C-ABI entry point against the fp64 oracle on seeded inputs.
+
+Inputs come from the host generator (lsa_synth) and are uploaded, or, for the
+full-size workloads, are drawn on the device and the sampled rows re-drawn on
+the host; no oracle input or expected value comes from the CUDA path.
+"""
+import numpy as np
+import pytest
+import torch
+
+import lsa_synth as S
+from lsa_testutil import (assert_attention, assert_scores, bf16_dev, bf16_host_f64, check_selection,
+                          f32_dev, host_rows, i32_dev, i64_dev, oracle_cfg)
+from oracle import lsa_ref as R
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def L():
+    from sparse_attention_03_b200 import lsa
+    lsa.load()
+    assert torch.cuda.is_available()
+    return lsa
+
+
+def _upload(wl: S.Workload):
+    d = {}
+    d["q_idx"] = bf16_dev(wl.q_idx)
+    d["w"] = f32_dev(wl.w)
+    d["k_idx"] = bf16_dev(wl.k_idx)
+    d["q_abs"] = [bf16_dev(q) for q in wl.q_abs]
+    d["latent"] = [bf16_dev(c) for c in wl.latent]
+    d["pos"] = i32_dev(wl.pos)
+    d["seq_of_row"] = i32_dev(wl.seq_of_row)
+    d["k_off"] = i64_dev(wl.k_off)
+    return d
+
+
+# --------------------------------------------------------------------------
+# Generator: the device kernels reproduce the host definition bit for bit.
+# --------------------------------------------------------------------------
+def test_device_generator_matches_host(L):
+    x = torch.empty(100003, dtype=torch.bfloat16, device="cuda")
+    L.synth_normal_bf16(x, 7, 21, first=12345)
+    host = S.normal_bf16(7, 21, 12345, 100003)
+    np.testing.assert_array_equal(x.view(torch.int16).cpu().numpy().view(np.uint16), host)
+    y = torch.empty(5001, dtype=torch.float32, device="cuda")
+    L.synth_normal_f32(y, 3, 4, first=99, sigma=float(S.W_SIGMA))
+    np.testing.assert_array_equal(y.cpu().numpy(), S.normal_f32(3, 4, 99, 5001, S.W_SIGMA))
+    k = torch.empty((777, 128), dtype=torch.bfloat16, device="cuda")
+    L.synth_rms_rows_bf16(k, 0, 2, first_row=1000)
+    np.testing.assert_array_equal(k.view(torch.int16).cpu().numpy().view(np.uint16),
+                                  S.rms_rows_bf16(0, 2, 1000, 777, 128))
+
+
+# --------------------------------------------------------------------------
+# Indexer
+# --------------------------------------------------------------------------
+DECODE_LENGTHS = [1, 17, 1040, 1041, 2047, 2048, 2049, 3001, 5000, 8191, 12345]
+
+
+def test_index_scores_decode_varlen(L):
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    wl = S.Workload(0, 0, DECODE_LENGTHS, cli=1)
+    d = _upload(wl)
+    max_len = int(max(DECODE_LENGTHS)) + 3
+    ld = max_len + 5
+    scores = torch.full((wl.n_rows, ld), float("nan"), device="cuda")
+    L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], max_len, scores)
+    assert L.device_error() == 0
+    got = scores.cpu().numpy().astype(np.float64)
+    for r in range(wl.n_rows):
+        q, w, k, _, _ = host_rows(wl, r)
+        assert_scores(got[r, :max_len], q, w, k, int(wl.pos[r]), ocfg, where=f"row {r}")
+        assert np.isnan(got[r, max_len:]).all(), "columns past max_len must be untouched"
+
+
+def test_index_scores_prefill_rows(L):
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    n = 3000
+    wl = S.Workload(1, 0, [n], n_rows=n, q_start=0, cli=1)
+    d = _upload(wl)
+    scores = torch.empty((n, n), device="cuda")
+    L.index_scores(cfg, None, d["pos"], d["q_idx"], d["w"], d["k_idx"], None, n, scores)
+    assert L.device_error() == 0
+    got = scores.cpu().numpy().astype(np.float64)
+    rng = np.random.default_rng(0)
+    rows = sorted({0, 1, 15, 16, 1023, 1024, 2047, 2048, 2999} | set(rng.integers(0, n, 20).tolist()))
+    for r in rows:
+        q, w, k, _, _ = host_rows(wl, r)
+        assert_scores(got[r], q, w, k, r, ocfg, where=f"row {r}")
+
+
+def test_index_scores_tiny_config_forcing(L):
+    cfg = L.LsaConfig(index_topk=8, index_init_tokens=2, index_local_tokens=4)
+    ocfg = oracle_cfg(cfg)
+    wl = S.Workload(2, 0, [1, 3, 7, 8, 9, 20, 33], cli=1)
+    d = _upload(wl)
+    scores = torch.empty((wl.n_rows, 33), device="cuda")
+    L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], 33, scores)
+    got = scores.cpu().numpy().astype(np.float64)
+    for r in range(wl.n_rows):
+        q, w, k, _, _ = host_rows(wl, r)
+        assert_scores(got[r], q, w, k, int(wl.pos[r]), ocfg, where=f"row {r}")
+
+
+def test_index_scores_many_rows_grid_chunks(L):
+    # more than 65535 rows: exercises the row-chunked launch
+    cfg = L.LsaConfig()
+    n_rows, n_keys = 70000, 40
+    wl_q = S.normal_bf16(3, 0, 0, n_rows * 32 * 128).reshape(n_rows, 32, 128)
+    w = S.normal_f32(3, 1, 0, n_rows * 32, S.W_SIGMA).reshape(n_rows, 32)
+    k = S.rms_rows_bf16(3, 2, 0, n_keys, 128)
+    pos = (np.arange(n_rows) % n_keys).astype(np.int32)
+    scores = torch.empty((n_rows, n_keys), device="cuda")
+    L.index_scores(cfg, None, i32_dev(pos), bf16_dev(wl_q), f32_dev(w), bf16_dev(k), None, n_keys, scores)
+    got = scores.cpu().numpy().astype(np.float64)
+    f = S.bf16_bits_to_f64
+    for r in (0, 39, 65535, 65536, 69999):
+        assert_scores(got[r], f(wl_q[r]), w[r].astype(np.float64), f(k), int(pos[r]), oracle_cfg(cfg))
+
+
+# --------------------------------------------------------------------------
+# Top-k on given fp32 scores: the decision is taken in fp32 on both sides, so
+# the selection must match the oracle's exactly, ties included.
+# --------------------------------------------------------------------------
+def _topk_case(L, cfg, s_rows, pos, max_len):
+    n_rows = len(pos)
+    ld = max_len + 3
+    s = np.full((n_rows, ld), np.nan, dtype=np.float32)
+    for r in range(n_rows):
+        s[r, : pos[r] + 1] = s_rows[r][: pos[r] + 1]
+        s[r, pos[r] + 1:max_len] = -np.inf
+    ws = L.workspace(cfg, L.OP_TOPK, n_rows, 1, max_len)
+    idx = torch.full((n_rows, cfg.index_topk), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((n_rows,), -7, dtype=torch.int32, device="cuda")
+    st = L.topk(cfg, i32_dev(pos), max_len, f32_dev(s), idx, cnt, ws)
+    return st, idx.cpu().numpy(), cnt.cpu().numpy()
+
+
+def test_topk_exact_on_fp32_scores(L):
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(5)
+    pos = np.array([0, 100, 2047, 2048, 2049, 3000, 20000, 70000, 250000, 9000], dtype=np.int64)
+    max_len = int(pos.max()) + 1
+    rows = []
+    for i, p in enumerate(pos):
+        if i == 7:
+            v = rng.integers(-20, 20, p + 1).astype(np.float32)          # heavy ties
+        elif i == 9:
+            v = np.where(rng.random(p + 1) < 0.5, -0.0, 0.0).astype(np.float32)  # signed zeros
+        else:
+            v = rng.standard_normal(p + 1).astype(np.float32) * 8
+        rows.append(v)
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, max_len)
+    assert st == L.LSA_OK
+    for r, p in enumerate(pos):
+        s64 = R.mask_and_force(rows[r].astype(np.float64), int(p), max_len, ocfg)
+        exp, dense = R.select_topk(s64, int(p), ocfg)
+        n = int(p) + 1
+        if dense:
+            assert cnt[r] == n and np.array_equal(np.sort(idx[r, :n]), exp) and np.all(idx[r, n:] == -1)
+        else:
+            assert cnt[r] == cfg.index_topk
+            np.testing.assert_array_equal(np.sort(idx[r]), exp, err_msg=f"row {r}")
+
+
+def test_topk_all_equal_overflow_path(L):
+    # all-equal scores overflow the candidate buffer and take the rescan path;
+    # ties go to the lowest indices.
+    cfg = L.LsaConfig()
+    pos = np.array([150000, 4096], dtype=np.int64)
+    rows = [np.full(p + 1, 1.5, dtype=np.float32) for p in pos]
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, int(pos.max()) + 1)
+    for r, p in enumerate(pos):
+        exp = np.sort(np.concatenate([np.arange(16), np.arange(16, 16 + 1008), np.arange(p + 1 - 1024, p + 1)]))
+        np.testing.assert_array_equal(np.sort(idx[r]), exp)
+
+
+def test_topk_tiny_config_brute(L):
+    cfg = L.LsaConfig(index_topk=8, index_init_tokens=2, index_local_tokens=4)
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(11)
+    pos = np.array([0, 5, 7, 8, 9, 12, 30, 63], dtype=np.int64)
+    rows = [rng.integers(-3, 4, p + 1).astype(np.float32) for p in pos]
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, 64)
+    for r, p in enumerate(pos):
+        s64 = R.mask_and_force(rows[r].astype(np.float64), int(p), 64, ocfg)
+        exp, dense = R.select_topk(s64, int(p), ocfg)
+        n = min(int(p) + 1, 8)
+        assert cnt[r] == n
+        np.testing.assert_array_equal(np.sort(idx[r, :n]), exp)
+
+
+def test_topk_all_dense_status(L):
+    cfg = L.LsaConfig()
+    pos = np.array([0, 10, 2047], dtype=np.int64)
+    rows = [np.zeros(p + 1, dtype=np.float32) for p in pos]
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, 2048)
+    assert st == L.LSA_DENSE
+    assert list(cnt) == [1, 11, 2048]
+
+
+def test_topk_small_workspace_row_blocks(L):
+    # a workspace for 3 rows forces several row blocks
+    cfg = L.LsaConfig()
+    rng = np.random.default_rng(2)
+    pos = np.array([5000, 4000, 3000, 2500, 6000, 2049, 7000], dtype=np.int64)
+    max_len = 7001
+    s = np.full((len(pos), max_len), -np.inf, dtype=np.float32)
+    for r, p in enumerate(pos):
+        s[r, : p + 1] = rng.standard_normal(p + 1)
+    from sparse_attention_03_b200.lsa import LsaError  # noqa: F401
+    ws = torch.empty(3 * 40992 + 256, dtype=torch.uint8, device="cuda")
+    idx = torch.empty((len(pos), 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((len(pos),), dtype=torch.int32, device="cuda")
+    L.topk(cfg, i32_dev(pos), max_len, f32_dev(s), idx, cnt, ws)
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    ocfg = oracle_cfg(cfg)
+    for r, p in enumerate(pos):
+        exp, _ = R.select_topk(R.mask_and_force(s[r].astype(np.float64), int(p), max_len, ocfg), int(p), ocfg)
+        np.testing.assert_array_equal(np.sort(idx[r]), exp)
+
+
+# --------------------------------------------------------------------------
+# Sparse MLA on a given selection
+# --------------------------------------------------------------------------
+def _oracle_selection(wl, r, ocfg):
+    q, w, k, qa, lat = host_rows(wl, r)
+    p = int(wl.pos[r])
+    s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
+    sel, dense = R.select_topk(s, p, ocfg)
+    return sel, dense, qa, lat
+
+
+def test_mla_decode_on_selection(L):
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    lengths = [1, 64, 65, 2048, 2049, 5000, 9000, 4097]
+    wl = S.Workload(4, 0, lengths, cli=1)
+    d = _upload(wl)
+    B = wl.n_rows
+    idx = np.full((B, 2048), -1, dtype=np.int32)
+    cnt = np.zeros(B, dtype=np.int32)
+    exp = []
+    for r in range(B):
+        sel, dense, qa, lat = _oracle_selection(wl, r, ocfg)
+        idx[r, : len(sel)] = np.random.default_rng(r).permutation(sel)  # order must not matter
+        cnt[r] = len(sel)
+        exp.append(R.mla(qa[0], lat[0][sel], ocfg))
+    out = torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 32), device="cuda")
+    for use_ws in (True, False):   # split-K + merge, and single pass
+        ws = L.workspace(cfg, L.OP_MLA_DECODE, B, B, max(lengths)) if use_ws else None
+        L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], i32_dev(idx), i32_dev(cnt),
+                            max(lengths), out, lse, ws)
+        assert L.device_error() == 0
+        o, l = bf16_host_f64(out), lse.cpu().numpy()
+        for r in range(B):
+            assert_attention(o[r], l[r], exp[r][0], exp[r][1], where=f"row {r} ws={use_ws}")
+
+
+def test_mla_decode_dense(L):
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    lengths = [1, 33, 700, 2048, 3000]
+    wl = S.Workload(5, 0, lengths, cli=1)
+    d = _upload(wl)
+    out = torch.empty((len(lengths), 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((len(lengths), 32), device="cuda")
+    ws = L.workspace(cfg, L.OP_MLA_DECODE, len(lengths), len(lengths), max(lengths))
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], None, None, max(lengths), out, lse, ws)
+    o, l = bf16_host_f64(out), lse.cpu().numpy()
+    for r in range(len(lengths)):
+        _, _, _, qa, lat = host_rows(wl, r)
+        eo, el = R.dense_mla_row(qa[0], lat[0], lengths[r] - 1, ocfg)
+        assert_attention(o[r], l[r], eo, el, where=f"row {r}")
+
+
+def test_mla_prefill_on_selection(L):
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    n = 2600
+    wl = S.Workload(6, 0, [n], n_rows=n, q_start=0, cli=1)
+    d = _upload(wl)
+    rows = [0, 1, 100, 2046, 2047, 2048, 2049, 2599]
+    sub = np.array(rows)
+    idx = np.full((len(rows), 2048), -1, dtype=np.int32)
+    cnt = np.zeros(len(rows), dtype=np.int32)
+    exp = []
+    for i, r in enumerate(rows):
+        sel, dense, qa, lat = _oracle_selection(wl, r, ocfg)
+        idx[i, : len(sel)] = sel
+        cnt[i] = len(sel)
+        exp.append(R.mla(qa[0], lat[0][sel], ocfg))
+    out = torch.empty((len(rows), 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((len(rows), 32), device="cuda")
+    q_sub = d["q_abs"][0][torch.from_numpy(sub).cuda()].contiguous()
+    L.sparse_mla_prefill(cfg, i32_dev(sub), q_sub, d["latent"][0], i32_dev(idx), i32_dev(cnt), out, lse, None)
+    o, l = bf16_host_f64(out), lse.cpu().numpy()
+    for i in range(len(rows)):
+        assert_attention(o[i], l[i], exp[i][0], exp[i][1], where=f"row {rows[i]}")
+
+
+def test_mla_bad_index_is_flagged_not_faulting(L):
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    wl = S.Workload(7, 0, [3000], cli=1)
+    d = _upload(wl)
+    sel = np.arange(0, 3000, 2)[:1000].astype(np.int32)
+    bad = sel.copy()
+    bad[5] = 10 ** 9          # far outside the sequence
+    bad[6] = -3
+    idx = np.full((1, 2048), -1, dtype=np.int32)
+    idx[0, :1000] = bad
+    out = torch.empty((1, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, 32), device="cuda")
+    L.device_error()
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], i32_dev(idx), i32_dev(np.array([1000])),
+                        3000, out, lse, None)
+    assert L.device_error() & L.DEVERR_INDEX
+    _, _, _, qa, lat = host_rows(wl, 0)
+    keep = np.delete(sel, [5, 6])
+    eo, el = R.mla(qa[0], lat[0][keep], ocfg)
+    assert_attention(bf16_host_f64(out)[0], lse.cpu().numpy()[0], eo, el)
+
+
+# --------------------------------------------------------------------------
+# Whole layer through lsa_forward
+# --------------------------------------------------------------------------
+def _forward_check(L, wl, d, cfg, mode, rows_to_check, max_len):
+    ocfg = oracle_cfg(cfg)
+    n = wl.n_rows
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(cfg.cli_factor)]
+    lses = [torch.empty((n, 32), device="cuda") for _ in range(cfg.cli_factor)]
+    idx = torch.full((n, cfg.index_topk), -5, dtype=torch.int32, device="cuda")
+    cnt = torch.full((n,), -5, dtype=torch.int32, device="cuda")
+    op = L.OP_FORWARD_DECODE if mode == 0 else L.OP_FORWARD_PREFILL
+    ws = L.workspace(cfg, op, n, len(wl.lengths), max_len)
+    L.forward(cfg, mode, d["seq_of_row"] if mode == 0 else None, d["pos"], max_len, d["q_idx"], d["w"],
+              d["k_idx"], d["k_off"] if mode == 0 else None, d["q_abs"], d["latent"], outs, lses, ws,
+              idx_out=idx, count_out=cnt)
+    assert L.device_error() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    o = [bf16_host_f64(t) for t in outs]
+    l = [t.cpu().numpy() for t in lses]
+    dense_all = max_len <= cfg.index_topk
+    for r in rows_to_check:
+        q, w, k, qa, lat = host_rows(wl, r)
+        p = int(wl.pos[r])
+        sel, dense, res = R.lsa_row(q, w, k, p, qa, lat, ocfg)
+        exact = True
+        if not dense_all:
+            s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
+            exact = check_selection(idx[r], int(cnt[r]), s, p, ocfg, where=f"row {r}")
+        for z in range(cfg.cli_factor):
+            assert_attention(o[z][r], l[z][r], res[z][0], res[z][1], check_lse=exact, where=f"row {r} sub {z}")
+
+
+def test_forward_decode_varlen(L):
+    cfg = L.LsaConfig()
+    lengths = [2049, 3000, 4100, 5555, 7000, 8192, 2100, 6100]
+    wl = S.Workload(8, 3, lengths)
+    _forward_check(L, wl, _upload(wl), cfg, 0, range(len(lengths)), max(lengths))
+
+
+def test_forward_decode_dense_fallback(L):
+    cfg = L.LsaConfig()
+    lengths = [1, 100, 2048, 1500]
+    wl = S.Workload(9, 0, lengths)
+    _forward_check(L, wl, _upload(wl), cfg, 0, range(len(lengths)), max(lengths))
+
+
+def test_forward_prefill(L):
+    cfg = L.LsaConfig()
+    n = 2700
+    wl = S.Workload(10, 1, [n], n_rows=n, q_start=0)
+    rng = np.random.default_rng(1)
+    rows = sorted({0, 2047, 2048, 2049, n - 1} | set(rng.integers(2048, n, 6).tolist()) | {5, 700})
+    _forward_check(L, wl, _upload(wl), cfg, 1, rows, n)
+
+
+def test_forward_prefill_chunk_at_offset(L):
+    # a chunk of new rows appended to a longer cache (rows see q_start + t)
+    cfg = L.LsaConfig()
+    n_keys, n_rows = 4000, 300
+    wl = S.Workload(11, 0, [n_keys], n_rows=n_rows, q_start=n_keys - n_rows)
+    _forward_check(L, wl, _upload(wl), cfg, 1, [0, 1, 150, 299], n_keys)
+
+
+def test_forward_tiny_config(L):
+    cfg = L.LsaConfig(index_topk=8, index_init_tokens=2, index_local_tokens=4)
+    lengths = [1, 5, 8, 9, 10, 31, 64, 100]
+    wl = S.Workload(12, 0, lengths)
+    _forward_check(L, wl, _upload(wl), cfg, 0, range(len(lengths)), max(lengths))
+
+
+def test_empty_batch_is_noop(L):
+    cfg = L.LsaConfig()
+    e = torch.empty((0,), dtype=torch.int32, device="cuda")
+    assert L.index_scores(cfg, None, e, torch.empty((0, 32, 128), dtype=torch.bfloat16, device="cuda"),
+                          torch.empty((0, 32), device="cuda"),
+                          torch.empty((8, 128), dtype=torch.bfloat16, device="cuda"), None, 8,
+                          torch.empty((0, 8), device="cuda")) == 0
+
+
+def test_position_past_sequence_is_flagged(L):
+    cfg = L.LsaConfig()
+    wl = S.Workload(13, 0, [100, 200], cli=1)
+    d = _upload(wl)
+    pos = i32_dev(np.array([99, 250]))    # row 1 claims position 250 in a 200-key sequence
+    scores = torch.empty((2, 300), device="cuda")
+    L.device_error()
+    L.index_scores(cfg, d["seq_of_row"], pos, d["q_idx"], d["w"], d["k_idx"], d["k_off"], 300, scores)
+    assert L.device_error() & L.DEVERR_POS
+
+
+# --------------------------------------------------------------------------
+# Full-size workloads (device-drawn), sampled rows against the oracle
+# --------------------------------------------------------------------------
+def _oracle_row_from_stream(seed, layer, k_off, b, p, cfg, cli=2):
+    """The oracle on row b of a device-drawn decode workload, re-drawing inputs on the host."""
+    ocfg = oracle_cfg(cfg)
+    f = S.bf16_bits_to_f64
+    a, e = int(k_off[b]), int(k_off[b + 1])
+    q = f(S.normal_bf16(seed, S.tid(layer, S.Q_IDX), b * 4096, 4096)).reshape(32, 128)
+    w = S.normal_f32(seed, S.tid(layer, S.W), b * 32, 32, S.W_SIGMA).astype(np.float64)
+    k = f(S.rms_rows_bf16(seed, S.tid(layer, S.K_IDX), a, e - a, 128))
+    s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, e - a, ocfg)
+    sel, dense = R.select_topk(s, p, ocfg)
+    res = []
+    for z in range(cli):
+        qa = f(S.normal_bf16(seed, S.tid(layer, S.q_abs_kind(z)), b * 32 * 576, 32 * 576)).reshape(32, 576)
+        c = f(S.normal_bf16_rows(seed, S.tid(layer, S.lat_kind(z)), a + sel, 576))
+        res.append(R.mla(qa, c, ocfg))
+    return s, sel, res
+
+
+@pytest.mark.parametrize("name,batch,lo,hi,sample", [
+    ("decode_b64_16k_32k", 64, 16384, 32768, (0, 17, 63)),
+    ("decode_b16_128k", 16, 131072, 131072, (3, 15)),
+    ("decode_b4_983040", 4, 983040, 983040, (2,)),
+])
+def test_full_size_decode_sampled(L, name, batch, lo, hi, sample):
+    from sparse_attention_03_b200.device_inputs import DeviceWorkload
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    lengths = S.decode_lengths(0, batch, lo, hi)
+    wl = DeviceWorkload(0, 0, lengths)
+    n = wl.n_rows
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((n, 32), device="cuda") for _ in range(2)]
+    idx = torch.empty((n, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    ws = L.workspace(cfg, L.OP_FORWARD_DECODE, n, n, wl.max_len)
+    L.forward(cfg, 0, wl.seq_of_row, wl.pos, wl.max_len, wl.q_idx, wl.w, wl.k_idx, wl.k_off, wl.q_abs,
+              wl.latent, outs, lses, ws, idx_out=idx, count_out=cnt)
+    assert L.device_error() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    k_off = S.offsets(lengths)
+    for b in sample:
+        p = int(lengths[b]) - 1
+        s, sel, res = _oracle_row_from_stream(0, 0, k_off, b, p, cfg)
+        exact = check_selection(idx[b], int(cnt[b]), s, p, ocfg, where=f"{name} row {b}")
+        for z in range(2):
+            assert_attention(bf16_host_f64(outs[z][b]), lses[z][b].cpu().numpy(), res[z][0], res[z][1],
+                             check_lse=exact, where=f"{name} row {b} sub {z}")
+    del wl
+    torch.cuda.empty_cache()
+
+
+def test_full_size_prefill_16k_sampled(L):
+    from sparse_attention_03_b200.device_inputs import DeviceWorkload
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    n = 16384
+    wl = DeviceWorkload(0, 0, [n], n_rows=n, q_start=0)
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((n, 32), device="cuda") for _ in range(2)]
+    idx = torch.empty((n, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    ws = L.workspace(cfg, L.OP_FORWARD_PREFILL, n, 1, n)
+    L.forward(cfg, 1, None, wl.pos, n, wl.q_idx, wl.w, wl.k_idx, None, wl.q_abs, wl.latent, outs, lses, ws,
+              idx_out=idx, count_out=cnt)
+    assert L.device_error() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    f = S.bf16_bits_to_f64
+    k = f(S.rms_rows_bf16(0, S.tid(0, S.K_IDX), 0, n, 128))
+    for r in (0, 2047, 2048, 9000, n - 1):
+        q = f(S.normal_bf16(0, S.tid(0, S.Q_IDX), r * 4096, 4096)).reshape(32, 128)
+        w = S.normal_f32(0, S.tid(0, S.W), r * 32, 32, S.W_SIGMA).astype(np.float64)
+        s = R.mask_and_force(R.score_row(q, w, k[: r + 1]), r, n, ocfg)
+        exact = check_selection(idx[r], int(cnt[r]), s, r, ocfg, where=f"prefill row {r}")
+        sel, _ = R.select_topk(s, r, ocfg)
+        for z in range(2):
+            qa = f(S.normal_bf16(0, S.tid(0, S.q_abs_kind(z)), r * 32 * 576, 32 * 576)).reshape(32, 576)
+            c = f(S.normal_bf16_rows(0, S.tid(0, S.lat_kind(z)), sel, 576))
+            eo, el = R.mla(qa, c, ocfg)
+            assert_attention(bf16_host_f64(outs[z][r]), lses[z][r].cpu().numpy(), eo, el, check_lse=exact,
+                             where=f"prefill row {r} sub {z}")
