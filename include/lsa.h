@@ -67,6 +67,7 @@ typedef enum lsa_status {
 #define LSA_DEVERR_INDEX 2   /* a selected index outside the row's visible keys */
 #define LSA_DEVERR_COUNT 4   /* count[r] outside [0, index_topk] */
 #define LSA_DEVERR_SEQ 8     /* seq_of_row[r] outside [0, n_seq) */
+#define LSA_DEVERR_TIMEOUT 16 /* a bounded wait inside a kernel gave up (the CTA stopped early) */
 
 /*
  * Method constants, under the pages' config key names ([LSA-2.0] 模型架构配置;
@@ -117,9 +118,9 @@ LSA_API size_t lsa_workspace_size(const lsa_config* cfg, int32_t op, int32_t n_r
  *   scores[r, j] = sum_h w[r,h] * max(q_idx[r,h,:] . k_idx[k_off[b] + j, :], 0)
  *                  for j <= pos[r], b = seq_of_row[r];
  *                = +inf  if j <= pos[r] and (j < index_init_tokens or
- *                        j > pos[r] - index_local_tokens)   (forced columns);
- *                = -inf  for pos[r] < j < max_len            (causal mask).
- * Entries at j >= max_len are not written.
+ *                        j > pos[r] - index_local_tokens)   (forced columns).
+ * Entries at j > pos[r] are not written: the causal mask is applied by never
+ * reading them (lsa_topk reads columns 0..pos[r] only).
  *
  * q_idx   bf16 [n_rows, 32, 128]     w  fp32 [n_rows, 32]
  * k_idx   bf16 [sum L_b, 128]        k_off int64 [n_seq+1], or NULL: one

@@ -112,8 +112,7 @@ __global__ void __launch_bounds__(kThreads, 3)
   if (!ok) nvis = 0;
 
   float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
-  for (int64_t j = max(j0, nvis) + threadIdx.x; j < j1; j += kThreads) srow[j] = -INFINITY;
-  const int64_t jend = min(j1, nvis);
+  const int64_t jend = min(j1, nvis);  // columns after pos are never written
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   int64_t tile = j0 + warp * kKeysPerWarpTile;

@@ -34,6 +34,9 @@ struct IndexArgs {
 
 // Streaming indexer: each CTA scores a run of keys of one row (decode shape).
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st);
+// Tensor-core indexer for many rows of one sequence (prefill shape).
+bool index_prefill_supported(const IndexArgs& a);
+cudaError_t launch_index_prefill(const IndexArgs& a, cudaStream_t st);
 
 struct TopkArgs {
   const float* scores;

@@ -111,6 +111,7 @@ lsa_status run_index_scores(const lsa_config* c, int n_rows, int n_seq, const in
   a.scores = scores;
   a.ld = ld;
   a.err = device_error_word();
+  if (index_prefill_supported(a)) return cuda_status(launch_index_prefill(a, st), "lsa_index_scores");
   return cuda_status(launch_index_decode(a, st), "lsa_index_scores");
 }
 

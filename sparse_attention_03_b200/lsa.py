@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "liblsa.so")
 LSA_OK, LSA_DENSE = 0, 1
 LSA_ERR_INVALID, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_DEVICE = -1, -2, -3, -4, -5
 OP_TOPK, OP_MLA_DECODE, OP_MLA_PREFILL, OP_FORWARD_DECODE, OP_FORWARD_PREFILL = 1, 2, 3, 4, 5
-DEVERR_POS, DEVERR_INDEX, DEVERR_COUNT, DEVERR_SEQ = 1, 2, 4, 8
+DEVERR_POS, DEVERR_INDEX, DEVERR_COUNT, DEVERR_SEQ, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 
 EXPORTS = (
     "lsa_config_default", "lsa_workspace_size", "lsa_index_scores", "lsa_topk",
@@ -101,20 +101,59 @@ class LsaConfig:
     softmax_scale: float = 1.0 / (192.0 ** 0.5)
 
     def c(self) -> Config:
+        """A fresh C struct of this configuration (safe to modify)."""
         cfg = Config()
-        load().lsa_config_default(ctypes.byref(cfg))
-        cfg.index_topk = self.index_topk
-        cfg.index_init_tokens = self.index_init_tokens
-        cfg.index_local_tokens = self.index_local_tokens
-        cfg.cli_factor = self.cli_factor
-        cfg.softmax_scale = self.softmax_scale
+        ctypes.pointer(cfg)[0] = self._c()
         return cfg
+
+    def _c(self) -> Config:
+        """The cached C struct passed to the library (never modified)."""
+        key = (self.index_topk, self.index_init_tokens, self.index_local_tokens, self.cli_factor,
+               self.softmax_scale)
+        cfg = _CFG_CACHE.get(key)
+        if cfg is None:
+            cfg = Config()
+            load().lsa_config_default(ctypes.byref(cfg))
+            cfg.index_topk = self.index_topk
+            cfg.index_init_tokens = self.index_init_tokens
+            cfg.index_local_tokens = self.index_local_tokens
+            cfg.cli_factor = self.cli_factor
+            cfg.softmax_scale = self.softmax_scale
+            _CFG_CACHE[key] = cfg
+        return cfg
+
+
+_CFG_CACHE: dict = {}
 
 
 def _check(status: int, allow_dense: bool = False) -> int:
     if status < 0 or (status == LSA_DENSE and not allow_dense):
         raise LsaError(status, load().lsa_last_error().decode())
     return status
+
+
+class Bound:
+    """A C entry point with its arguments already marshalled: calling it only
+    crosses the ABI (for tight host loops that must stay ahead of the GPU).
+    The tensors it points at must outlive it; it launches on the stream that was
+    current when it was bound."""
+
+    __slots__ = ("fn", "args", "allow_dense", "keep")
+
+    def __init__(self, fn, args, allow_dense, keep=None):
+        self.fn, self.args, self.allow_dense, self.keep = fn, args, allow_dense, keep
+
+    def __call__(self) -> int:
+        st = self.fn(*self.args)
+        if st < 0 or (st == LSA_DENSE and not self.allow_dense):
+            raise LsaError(st, load().lsa_last_error().decode())
+        return st
+
+
+def _invoke(fn, args, allow_dense=False, bind=False, keep=None):
+    if bind:
+        return Bound(fn, args, allow_dense, keep)
+    return _check(fn(*args), allow_dense)
 
 
 def _ptr(t):
@@ -138,7 +177,7 @@ def _stream(stream):
 
 
 def workspace_size(cfg: LsaConfig, op: int, n_rows: int, n_seq: int, max_len: int) -> int:
-    return int(load().lsa_workspace_size(ctypes.byref(cfg.c()), op, n_rows, n_seq, max_len))
+    return int(load().lsa_workspace_size(ctypes.byref(cfg._c()), op, n_rows, n_seq, max_len))
 
 
 def workspace(cfg: LsaConfig, op: int, n_rows: int, n_seq: int, max_len: int, device=None) -> torch.Tensor:
@@ -146,46 +185,48 @@ def workspace(cfg: LsaConfig, op: int, n_rows: int, n_seq: int, max_len: int, de
     return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
 
 
-def index_scores(cfg, seq_of_row, pos, q_idx, w, k_idx, k_off, max_len, scores, n_seq=None, stream=None):
+def index_scores(cfg, seq_of_row, pos, q_idx, w, k_idx, k_off, max_len, scores, n_seq=None, stream=None,
+                 bind=False):
     _dt(q_idx, torch.bfloat16, "q_idx"); _dt(k_idx, torch.bfloat16, "k_idx"); _dt(w, torch.float32, "w")
     _dt(pos, torch.int32, "pos"); _dt(seq_of_row, torch.int32, "seq_of_row"); _dt(k_off, torch.int64, "k_off")
     _dt(scores, torch.float32, "scores")
     n_rows = pos.shape[0]
     if n_seq is None:
         n_seq = 1 if k_off is None else k_off.shape[0] - 1
-    return _check(load().lsa_index_scores(
-        ctypes.byref(cfg.c()), n_rows, n_seq, _ptr(seq_of_row), _ptr(pos), _ptr(q_idx), _ptr(w),
-        _ptr(k_idx), _ptr(k_off), int(max_len), _ptr(scores), scores.shape[1], _stream(stream)))
+    return _invoke(load().lsa_index_scores, (
+        ctypes.byref(cfg._c()), n_rows, n_seq, _ptr(seq_of_row), _ptr(pos), _ptr(q_idx), _ptr(w),
+        _ptr(k_idx), _ptr(k_off), int(max_len), _ptr(scores), scores.shape[1], _stream(stream)), bind=bind)
 
 
-def topk(cfg, pos, max_len, scores, idx, count, ws, stream=None):
+def topk(cfg, pos, max_len, scores, idx, count, ws, stream=None, bind=False):
     _dt(scores, torch.float32, "scores"); _dt(pos, torch.int32, "pos")
     _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
-    return _check(load().lsa_topk(
-        ctypes.byref(cfg.c()), pos.shape[0], _ptr(pos), int(max_len), _ptr(scores), scores.shape[1],
-        _ptr(idx), _ptr(count), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)), allow_dense=True)
+    return _invoke(load().lsa_topk, (
+        ctypes.byref(cfg._c()), pos.shape[0], _ptr(pos), int(max_len), _ptr(scores), scores.shape[1],
+        _ptr(idx), _ptr(count), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)), allow_dense=True,
+        bind=bind)
 
 
-def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None):
+def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None, bind=False):
     for t, n in ((q_abs, "q_abs"), (latent, "latent"), (out, "out")):
         _dt(t, torch.bfloat16, n)
     _dt(k_off, torch.int64, "k_off"); _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
     _dt(lse, torch.float32, "lse")
-    return _check(load().lsa_sparse_mla_decode(
-        ctypes.byref(cfg.c()), q_abs.shape[0], _ptr(q_abs), _ptr(latent), _ptr(k_off), _ptr(idx),
+    return _invoke(load().lsa_sparse_mla_decode, (
+        ctypes.byref(cfg._c()), q_abs.shape[0], _ptr(q_abs), _ptr(latent), _ptr(k_off), _ptr(idx),
         _ptr(count), int(max_len), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
-        _stream(stream)))
+        _stream(stream)), bind=bind)
 
 
-def sparse_mla_prefill(cfg, pos, q_abs, latent, idx, count, out, lse, ws, stream=None):
+def sparse_mla_prefill(cfg, pos, q_abs, latent, idx, count, out, lse, ws, stream=None, bind=False):
     for t, n in ((q_abs, "q_abs"), (latent, "latent"), (out, "out")):
         _dt(t, torch.bfloat16, n)
     _dt(pos, torch.int32, "pos"); _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
     _dt(lse, torch.float32, "lse")
-    return _check(load().lsa_sparse_mla_prefill(
-        ctypes.byref(cfg.c()), pos.shape[0], _ptr(pos), _ptr(q_abs), _ptr(latent), latent.shape[0],
+    return _invoke(load().lsa_sparse_mla_prefill, (
+        ctypes.byref(cfg._c()), pos.shape[0], _ptr(pos), _ptr(q_abs), _ptr(latent), latent.shape[0],
         _ptr(idx), _ptr(count), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
-        _stream(stream)))
+        _stream(stream)), bind=bind)
 
 
 def _ptr_array(ts):
@@ -196,7 +237,7 @@ def _ptr_array(ts):
 
 
 def forward(cfg, mode, seq_of_row, pos, max_len, q_idx, w, k_idx, k_off, q_abs, latent, out, lse,
-            ws, idx_out=None, count_out=None, n_seq=None, stream=None):
+            ws, idx_out=None, count_out=None, n_seq=None, stream=None, bind=False):
     """mode 0 decode / 1 prefill; q_abs, latent, out, lse: lists of cli_factor tensors."""
     for t in list(q_abs) + list(latent) + list(out):
         _dt(t, torch.bfloat16, "q_abs/latent/out")
@@ -208,10 +249,11 @@ def forward(cfg, mode, seq_of_row, pos, max_len, q_idx, w, k_idx, k_off, q_abs, 
     if n_seq is None:
         n_seq = 1 if k_off is None else k_off.shape[0] - 1
     keep = (_ptr_array(q_abs), _ptr_array(latent), _ptr_array(out), _ptr_array(lse) if lse else None)
-    return _check(load().lsa_forward(
-        ctypes.byref(cfg.c()), int(mode), pos.shape[0], n_seq, _ptr(seq_of_row), _ptr(pos), int(max_len),
+    return _invoke(load().lsa_forward, (
+        ctypes.byref(cfg._c()), int(mode), pos.shape[0], n_seq, _ptr(seq_of_row), _ptr(pos), int(max_len),
         _ptr(q_idx), _ptr(w), _ptr(k_idx), _ptr(k_off), keep[0], keep[1], keep[2], keep[3],
-        _ptr(idx_out), _ptr(count_out), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)))
+        _ptr(idx_out), _ptr(count_out), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+        bind=bind, keep=keep)
 
 
 def launch_count() -> int:

@@ -1,0 +1,111 @@
+"""Small single-kernel cases for profiling one kernel of the path under ncu.
+
+    python -m sparse_attention_03_b200.profile_cases CASE [--reps N]
+
+Each case draws its inputs on the device (a few GB at most, inputs larger than
+L2 where the kernel streams from HBM), runs one entry point --reps times on the
+current stream, checks the device error flags and exits. Cases:
+
+  index_decode   lsa_index_scores, 16 rows x 131072 keys (one 128K decode layer)
+  index_prefill  lsa_index_scores, 16384 causal rows over 16384 keys
+  topk_decode    lsa_topk on 16 rows x 131072 scores
+  mla_decode     lsa_sparse_mla_decode, 16 rows x 2048 selected keys of 131072
+  mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
+"""
+from __future__ import annotations
+
+import argparse
+import sys
+
+import numpy as np
+import torch
+
+
+from . import lsa
+from .device_inputs import DeviceWorkload
+
+
+def _decode_layer(draw_latent):
+    lengths = np.full(16, 131072, dtype=np.int64)
+    return DeviceWorkload(0, 0, lengths, cli=1, draw_latent=draw_latent)
+
+
+def case_index_decode(reps):
+    cfg = lsa.LsaConfig()
+    wl = _decode_layer(False)
+    scores = torch.empty((16, 131072), device="cuda")
+    for _ in range(reps):
+        lsa.index_scores(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, 131072, scores)
+
+
+def case_index_prefill(reps):
+    cfg = lsa.LsaConfig()
+    n = 16384
+    wl = DeviceWorkload(0, 0, [n], n_rows=n, q_start=0, cli=1, draw_latent=False)
+    scores = torch.empty((n, n), device="cuda")
+    for _ in range(reps):
+        lsa.index_scores(cfg, None, wl.pos, wl.q_idx, wl.w, wl.k_idx, None, n, scores)
+
+
+def case_topk_decode(reps):
+    cfg = lsa.LsaConfig()
+    wl = _decode_layer(False)
+    scores = torch.empty((16, 131072), device="cuda")
+    lsa.index_scores(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, 131072, scores)
+    idx = torch.empty((16, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((16,), dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(cfg, lsa.OP_TOPK, 16, 16, 131072)
+    for _ in range(reps):
+        lsa.topk(cfg, wl.pos, 131072, scores, idx, cnt, ws)
+
+
+def case_mla_decode(reps):
+    cfg = lsa.LsaConfig(cli_factor=1)
+    wl = _decode_layer(True)
+    rng = np.random.default_rng(0)
+    idx = torch.from_numpy(np.stack([np.sort(rng.choice(131072, 2048, replace=False)) for _ in range(16)])
+                           .astype(np.int32)).cuda()
+    cnt = torch.full((16,), 2048, dtype=torch.int32, device="cuda")
+    out = torch.empty((16, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((16, 32), device="cuda")
+    ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE, 16, 16, 131072)
+    for _ in range(reps):
+        lsa.sparse_mla_decode(cfg, wl.q_abs[0], wl.latent[0], wl.k_off, idx, cnt, 131072, out, lse, ws)
+
+
+def case_mla_prefill(reps):
+    cfg = lsa.LsaConfig(cli_factor=1)
+    n_keys, n_rows = 16384, 4096
+    wl = DeviceWorkload(0, 0, [n_keys], n_rows=n_rows, q_start=n_keys - n_rows, cli=1)
+    rng = np.random.default_rng(0)
+    idx = torch.from_numpy(np.stack([np.sort(rng.choice(int(p) + 1, 2048, replace=False))
+                                     for p in wl.pos.cpu().numpy()]).astype(np.int32)).cuda()
+    cnt = torch.full((n_rows,), 2048, dtype=torch.int32, device="cuda")
+    out = torch.empty((n_rows, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((n_rows, 32), device="cuda")
+    ws = lsa.workspace(cfg, lsa.OP_MLA_PREFILL, n_rows, 1, n_keys)
+    for _ in range(reps):
+        lsa.sparse_mla_prefill(cfg, wl.pos, wl.q_abs[0], wl.latent[0], idx, cnt, out, lse, ws)
+
+
+CASES = {name[5:]: fn for name, fn in globals().items() if name.startswith("case_")}
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=sorted(CASES))
+    ap.add_argument("--reps", type=int, default=3)
+    args = ap.parse_args(argv)
+    lsa.load()
+    CASES[args.case](args.reps)
+    torch.cuda.synchronize()
+    flags = lsa.device_error()
+    if flags:
+        print(f"device error flags 0x{flags:x}", file=sys.stderr)
+        return 1
+    print(f"{args.case}: ok")
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -74,7 +74,7 @@ def test_index_scores_decode_varlen(L):
     for r in range(wl.n_rows):
         q, w, k, _, _ = host_rows(wl, r)
         assert_scores(got[r, :max_len], q, w, k, int(wl.pos[r]), ocfg, where=f"row {r}")
-        assert np.isnan(got[r, max_len:]).all(), "columns past max_len must be untouched"
+        assert np.isnan(got[r, int(wl.pos[r]) + 1:]).all(), "columns after pos must stay unwritten"
 
 
 def test_index_scores_prefill_rows(L):
@@ -94,6 +94,46 @@ def test_index_scores_prefill_rows(L):
         assert_scores(got[r], q, w, k, r, ocfg, where=f"row {r}")
 
 
+def test_index_scores_prefill_streaming_path(L):
+    # the same prefill rows through the streaming kernel (a sequence offset given)
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    n = 1500
+    wl = S.Workload(1, 2, [n], n_rows=n, q_start=0, cli=1)
+    d = _upload(wl)
+    scores = torch.empty((n, n), device="cuda")
+    L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], n, scores)
+    got = scores.cpu().numpy().astype(np.float64)
+    for r in (0, 17, 1039, 1040, 1499):
+        q, w, k, _, _ = host_rows(wl, r)
+        assert_scores(got[r], q, w, k, r, ocfg, where=f"row {r}")
+
+
+@pytest.mark.parametrize("n_rows,n_keys,shuffle", [(1000, 1300, True), (16, 40000, False), (33, 777, True)])
+def test_index_scores_tensor_core_shapes(L, n_rows, n_keys, shuffle):
+    # ragged row blocks and key tiles, rows in any order, key-range splitting
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(n_rows)
+    wl = S.Workload(3, 4, [n_keys], n_rows=n_rows, q_start=n_keys - n_rows, cli=1)
+    pos = wl.pos.copy()
+    if shuffle:
+        pos = rng.permutation(np.arange(n_keys))[:n_rows].astype(np.int32)
+    d = _upload(wl)
+    ld = n_keys + 9
+    scores = torch.full((n_rows, ld), float("nan"), device="cuda")
+    L.device_error()
+    L.index_scores(cfg, None, i32_dev(pos), d["q_idx"], d["w"], d["k_idx"], None, n_keys, scores)
+    assert L.device_error() == 0
+    got = scores.cpu().numpy().astype(np.float64)
+    f = S.bf16_bits_to_f64
+    k = f(wl.k_idx)
+    rows = sorted(set(rng.integers(0, n_rows, 12).tolist()) | {0, n_rows - 1})
+    for r in rows:
+        assert_scores(got[r], f(wl.q_idx[r]), wl.w[r].astype(np.float64), k, int(pos[r]), ocfg, where=f"row {r}")
+        assert np.isnan(got[r, pos[r] + 1:]).all(), "columns after pos must stay unwritten"
+
+
 def test_index_scores_tiny_config_forcing(L):
     cfg = L.LsaConfig(index_topk=8, index_init_tokens=2, index_local_tokens=4)
     ocfg = oracle_cfg(cfg)
@@ -107,8 +147,10 @@ def test_index_scores_tiny_config_forcing(L):
         assert_scores(got[r], q, w, k, int(wl.pos[r]), ocfg, where=f"row {r}")
 
 
-def test_index_scores_many_rows_grid_chunks(L):
-    # more than 65535 rows: exercises the row-chunked launch
+@pytest.mark.parametrize("streaming", [True, False])
+def test_index_scores_many_rows_grid_chunks(L, streaming):
+    # more than 65535 rows: the row-chunked streaming launch, and 4375 row blocks
+    # of the tensor-core kernel
     cfg = L.LsaConfig()
     n_rows, n_keys = 70000, 40
     wl_q = S.normal_bf16(3, 0, 0, n_rows * 32 * 128).reshape(n_rows, 32, 128)
@@ -116,7 +158,8 @@ def test_index_scores_many_rows_grid_chunks(L):
     k = S.rms_rows_bf16(3, 2, 0, n_keys, 128)
     pos = (np.arange(n_rows) % n_keys).astype(np.int32)
     scores = torch.empty((n_rows, n_keys), device="cuda")
-    L.index_scores(cfg, None, i32_dev(pos), bf16_dev(wl_q), f32_dev(w), bf16_dev(k), None, n_keys, scores)
+    k_off = i64_dev(np.array([0, n_keys])) if streaming else None
+    L.index_scores(cfg, None, i32_dev(pos), bf16_dev(wl_q), f32_dev(w), bf16_dev(k), k_off, n_keys, scores)
     got = scores.cpu().numpy().astype(np.float64)
     f = S.bf16_bits_to_f64
     for r in (0, 39, 65535, 65536, 69999):
