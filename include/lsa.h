@@ -158,6 +158,32 @@ LSA_API lsa_status lsa_topk(const lsa_config* cfg, int32_t n_rows, const int32_t
                     size_t ws_bytes, void* stream);
 
 /*
+ * lsa_topk_static: the same selection as lsa_topk, for callers that cannot
+ * allocate device memory. The pages have no counterpart of this entry point.
+ *
+ * Who needs it: code being recorded into a CUDA graph (an allocation is not a
+ * stream operation, so a capture cannot contain one), serving loops that must
+ * not pay the device-wide synchronisation cudaMalloc/cudaFree may cause, and
+ * plugins whose host framework hands them only their input and output buffers.
+ * The caller passes exactly the buffers of lsa_topk except the workspace.
+ *
+ * Scratch: a file-scope device array of LSA_TOPK_STATIC_MAX_ROWS x 40992 bytes
+ * (2.5 MiB) inside the library; every GPU that loads the library keeps it
+ * until the process exits. The first call on a device looks up the array's
+ * device address (cudaGetSymbolAddress) with that device current: make that
+ * first call before any stream capture begins. The call allocates nothing.
+ * All calls share the one array and each call clears what must start at
+ * zero; calls whose kernels may overlap on the GPU (other streams, other host
+ * threads) race on it and must be serialised by the caller.
+ * n_rows > LSA_TOPK_STATIC_MAX_ROWS returns LSA_ERR_INVALID (split the rows or
+ * use lsa_topk). Statuses otherwise as lsa_topk.
+ */
+#define LSA_TOPK_STATIC_MAX_ROWS 64
+LSA_API lsa_status lsa_topk_static(const lsa_config* cfg, int32_t n_rows, const int32_t* pos,
+                                   int64_t max_len, const float* scores, int64_t ld, int32_t* idx,
+                                   int32_t* count, void* stream);
+
+/*
  * Sparse absorbed-latent MLA, decode ([Lite-Sparse] LSA section: at decode
  * the latent rows are gathered by the top-k indices; 架构总览: kv_lora_rank 512,
  * qk_rope_head_dim 64, 32 heads).
