@@ -268,15 +268,17 @@ def build_decode(device):
     cnt = torch.empty((B,), dtype=torch.int32, device=device)
     tk_ws = lsa.workspace(cfg, lsa.OP_TOPK, B, B, ctx, device=device)
     mla_ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE, B, B, ctx, device=device)
+    hist = lsa.topk_hist_buffer(B, device=device)
     D = dict(layers=layers, q_idx=q_idx, w=w, q_abs=q_abs, out=out, lse=lse, cfg=cfg, ws=ws, scores=scores,
-             idx=idx, cnt=cnt, tk_ws=tk_ws, mla_ws=mla_ws, ctx=ctx)
+             idx=idx, cnt=cnt, tk_ws=tk_ws, mla_ws=mla_ws, ctx=ctx, hist=hist)
     # Marshal every call once: the timed loops only cross the C-ABI.
     D["calls"] = []
     D["fwd"] = []
     for i, l in enumerate(layers):
         D["calls"].append((
-            lsa.index_scores(cfg, l.seq_of_row, l.pos, l.q_idx, l.w, l.k_idx, l.k_off, ctx, scores, bind=True),
-            lsa.topk(cfg, l.pos, ctx, scores, idx, cnt, tk_ws, bind=True),
+            lsa.index_scores(cfg, l.seq_of_row, l.pos, l.q_idx, l.w, l.k_idx, l.k_off, ctx, scores, bind=True,
+                             topk_hist=hist),
+            lsa.topk(cfg, l.pos, ctx, scores, idx, cnt, tk_ws, bind=True, topk_hist=hist),
             [lsa.sparse_mla_decode(cfg, l.q_abs[z], l.latent[z], l.k_off, idx, cnt, ctx, out[i, z], lse[i, z],
                                    mla_ws, bind=True) for z in range(2)]))
         D["fwd"].append(lsa.forward(cfg, 0, l.seq_of_row, l.pos, ctx, l.q_idx, l.w, l.k_idx, l.k_off, l.q_abs,
@@ -299,15 +301,29 @@ def decode_step(D, ev=None):
         mla_calls[1]()
 
 
-def decode_forward_e2e(D, h_in, h_out):
-    """One step through lsa_forward with the per-step inputs copied from pinned host
-    memory and the outputs copied back."""
-    D["q_idx"].copy_(h_in[0], non_blocking=True)
-    D["w"].copy_(h_in[1], non_blocking=True)
-    D["q_abs"].copy_(h_in[2], non_blocking=True)
-    for call in D["fwd"]:
+def decode_forward_e2e(D, h_in, h_out, pipe):
+    """One step through lsa_forward with every layer's inputs copied from pinned
+    host memory and its outputs copied back. The copies run on a second stream:
+    layer l+1's inputs travel while layer l computes, layer l's outputs while
+    layer l+1 computes."""
+    import torch
+    comp, copy, ev_in, ev_out = pipe
+    with torch.cuda.stream(copy):
+        copy.wait_stream(comp)  # the previous step's readers of these buffers are done
+        for i in range(len(D["fwd"])):
+            D["q_idx"][i].copy_(h_in[0][i], non_blocking=True)
+            D["w"][i].copy_(h_in[1][i], non_blocking=True)
+            D["q_abs"][i].copy_(h_in[2][i], non_blocking=True)
+            ev_in[i].record(copy)
+    for i, call in enumerate(D["fwd"]):
+        comp.wait_event(ev_in[i])
         call()
-    h_out.copy_(D["out"], non_blocking=True)
+        ev_out[i].record(comp)
+    with torch.cuda.stream(copy):
+        for i in range(len(D["fwd"])):
+            copy.wait_event(ev_out[i])
+            h_out[i].copy_(D["out"][i], non_blocking=True)
+    comp.wait_stream(copy)
 
 
 def time_region(fn, steps, world, device):
@@ -425,11 +441,13 @@ def gpu_arm(args):
     # end-to-end through lsa_forward with pinned host buffers
     h_in = [D["q_idx"].cpu().pin_memory(), D["w"].cpu().pin_memory(), D["q_abs"].cpu().pin_memory()]
     h_out = torch.empty(D["out"].shape, dtype=D["out"].dtype).pin_memory()
+    pipe = (torch.cuda.current_stream(), torch.cuda.Stream(),
+            [torch.cuda.Event() for _ in range(nl)], [torch.cuda.Event() for _ in range(nl)])
     for _ in range(max(3, args.warmup // 2)):
-        decode_forward_e2e(D, h_in, h_out)
+        decode_forward_e2e(D, h_in, h_out, pipe)
     torch.cuda.synchronize()
     e2e_steps = max(5, args.steps // 2)
-    te = time_region(lambda s: decode_forward_e2e(D, h_in, h_out), e2e_steps, world, device)
+    te = time_region(lambda s: decode_forward_e2e(D, h_in, h_out, pipe), e2e_steps, world, device)
     e2e_value, _ = aggregate(B * nl * e2e_steps, te, world, device)
     h2d = sum(x.numel() * x.element_size() for x in h_in)
     d2h = h_out.numel() * h_out.element_size()

@@ -128,12 +128,19 @@ LSA_API size_t lsa_workspace_size(const lsa_config* cfg, int32_t op, int32_t n_r
  * seq_of_row int32 [n_rows] or NULL (every row in sequence 0)
  * pos     int32 [n_rows]             scores fp32 [n_rows, ld], ld >= max_len
  * max_len host bound: every pos[r] < max_len.
+ * topk_hist: optional uint32 [n_rows, LSA_TOPK_HIST_WORDS] (device). When not
+ *   NULL it receives the first radix pass of the selection (a histogram of the
+ *   top 11 bits of the order-preserving key of every middle-column score of
+ *   rows with more than index_topk visible keys), built from the scores while
+ *   they are still in registers; pass it to lsa_topk with the same scores.
  * Products bf16 x bf16 exact in fp32, fp32 accumulation.
  */
+#define LSA_TOPK_HIST_WORDS 2056 /* uint32 words per row of a top-k histogram buffer */
 LSA_API lsa_status lsa_index_scores(const lsa_config* cfg, int32_t n_rows, int32_t n_seq,
                             const int32_t* seq_of_row, const int32_t* pos, const lsa_bf16* q_idx,
                             const float* w, const lsa_bf16* k_idx, const int64_t* k_off,
-                            int64_t max_len, float* scores, int64_t ld, void* stream);
+                            int64_t max_len, float* scores, int64_t ld, uint32_t* topk_hist,
+                            void* stream);
 
 /*
  * Top-k selection with the dense fallback ([Lite-Sparse] LSA section: the
@@ -150,12 +157,15 @@ LSA_API lsa_status lsa_index_scores(const lsa_config* cfg, int32_t n_rows, int32
  * 0..pos[r] are read). idx int32 [n_rows, index_topk], count int32 [n_rows].
  * max_len (host): every pos[r] < max_len. Returns LSA_DENSE when
  * max_len <= index_topk (every row dense; idx/count still written).
- * Workspace: lsa_workspace_size(LSA_OP_TOPK, ...); rows are processed in
- * blocks that fit (minimum one row, 40992 B).
+ * topk_hist: NULL, or the histogram lsa_index_scores wrote for these scores
+ *   (saves one pass over the scores).
+ * Workspace: lsa_workspace_size(LSA_OP_TOPK, ...). Only fewer than 256 rows
+ * longer than 16384 columns use it (then processed in blocks that fit,
+ * minimum one row of 40992 B); otherwise ws may be NULL.
  */
 LSA_API lsa_status lsa_topk(const lsa_config* cfg, int32_t n_rows, const int32_t* pos, int64_t max_len,
-                    const float* scores, int64_t ld, int32_t* idx, int32_t* count, void* ws,
-                    size_t ws_bytes, void* stream);
+                    const float* scores, int64_t ld, const uint32_t* topk_hist, int32_t* idx,
+                    int32_t* count, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * lsa_topk_static: the same selection as lsa_topk, for callers that cannot

@@ -19,6 +19,11 @@ constexpr int kMaxTopk = 2048;
 __host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 
+// Programmatic dependent launch: wait until the previous kernel on the stream
+// has completed (its writes visible); let the next kernel start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;\n" ::); }
+
 __device__ __forceinline__ void flag_error(int* err, int bits) {
   if (err) atomicOr(err, bits);
 }

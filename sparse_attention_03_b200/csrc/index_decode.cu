@@ -20,6 +20,7 @@
 // runs on the accumulators in registers, then two quad shuffles finish it.
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.h"
 
 namespace lsa {
 namespace {
@@ -85,8 +86,11 @@ __device__ __forceinline__ void score_tile(const KeyFrag& f, const uint4 (&qf)[4
   sb = y;
 }
 
+template <bool HIST>
 __global__ void __launch_bounds__(kThreads, 3)
-    index_decode_kernel(IndexArgs a, int keys_per_cta, int row0) {
+    index_decode_kernel(IndexArgs a, int keys_per_cta, int row0, uint32_t* hist, int topk) {
+  __shared__ uint32_t sh[HIST ? 2048 : 1];
+  pdl_wait();
   const int r = row0 + blockIdx.y;
   const int64_t j0 = (int64_t)blockIdx.x * keys_per_cta;
   if (j0 >= a.max_len) return;
@@ -116,7 +120,14 @@ __global__ void __launch_bounds__(kThreads, 3)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int g = lane >> 2, t = lane & 3;
   int64_t tile = j0 + warp * kKeysPerWarpTile;
-  if (tile >= jend) return;
+  // The top-k's histogram (top 11 bits of each middle-column score key) of rows
+  // that will be selected from, built here from the scores in registers.
+  const bool hist_row = HIST && ok && (p + 1 > topk);
+  if (HIST) {
+    for (int i = threadIdx.x; i < 2048; i += kThreads) sh[i] = 0;
+    __syncthreads();
+  }
+  if (tile < jend) {
 
   // Query B fragments (head 8nt+g, physical chunk 4c+t) and head weights.
   uint4 qf[4][4];
@@ -141,7 +152,9 @@ __global__ void __launch_bounds__(kThreads, 3)
       const int64_t j = tl + g + (t == 1 ? 8 : 0);
       if (j < jend) {
         const bool forced = (j < lo_force) || (j >= hi_force);
-        srow[j] = forced ? INFINITY : (t == 1 ? sb : sa);
+        const float v = t == 1 ? sb : sa;
+        srow[j] = forced ? INFINITY : v;
+        if (HIST && hist_row && !forced) atomicAdd(&sh[score_key(v) >> 21], 1u);
       }
     }
   };
@@ -164,11 +177,19 @@ __global__ void __launch_bounds__(kThreads, 3)
     if (nxt >= jend) break;
     tile = nxt;
   }
+  }
+  pdl_trigger();
+  if (HIST) {
+    __syncthreads();
+    uint32_t* hr = hist + (int64_t)r * kTopkHistStride;
+    for (int i = threadIdx.x; i < 2048; i += kThreads)
+      if (sh[i]) atomicAdd(&hr[i], sh[i]);
+  }
 }
 
 }  // namespace
 
-cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st) {
+cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st, uint32_t* hist, int topk) {
   if (a.n_rows <= 0) return cudaSuccess;
   // Keys per CTA: a multiple of one CTA pass (64 keys), large enough to amortise
   // the query-fragment load, small enough to give every SM several CTAs.
@@ -182,7 +203,12 @@ cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st) {
   const int64_t nx = (a.max_len + kpc - 1) / kpc;
   for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
     const int ny = min(65535, a.n_rows - row0);
-    index_decode_kernel<<<dim3((unsigned)nx, (unsigned)ny), kThreads, 0, st>>>(a, (int)kpc, row0);
+    const dim3 grid((unsigned)nx, (unsigned)ny);
+    const cudaError_t e =
+        hist ? launch_pdl(index_decode_kernel<true>, grid, dim3(kThreads), 0, st, a, (int)kpc, row0, hist, topk)
+             : launch_pdl(index_decode_kernel<false>, grid, dim3(kThreads), 0, st, a, (int)kpc, row0,
+                          (uint32_t*)nullptr, 0);
+    if (e != cudaSuccess) return e;
     count_launches(1);
   }
   return cudaGetLastError();

@@ -25,6 +25,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.h"
 
 namespace lsa {
 namespace {
@@ -159,6 +160,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   PrefillSmem& sm = *reinterpret_cast<PrefillSmem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
   // Heaviest (latest, longest-context) row blocks first.
   const int blk = gridDim.y - 1 - blockIdx.y;
   const int row0 = blk * kRowsPerBlock;
@@ -375,9 +377,11 @@ cudaError_t launch_index_prefill(const IndexArgs& a, cudaStream_t st) {
   p.tiles_per_cta = tiles_per_cta;
   p.err = a.err;
   if (n_blocks > 65535) return cudaErrorInvalidValue;
-  index_prefill_kernel<<<dim3((unsigned)chunks, (unsigned)n_blocks), kThreads, smem, st>>>(map_k, map_q, p);
+  const cudaError_t e =
+      launch_pdl(index_prefill_kernel, dim3((unsigned)chunks, (unsigned)n_blocks), dim3(kThreads), smem, st, map_k,
+                 map_q, p);
   count_launches(1);
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace lsa

@@ -33,7 +33,11 @@ struct IndexArgs {
 };
 
 // Streaming indexer: each CTA scores a run of keys of one row (decode shape).
-cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st);
+// With hist != null it also adds, for rows with more than `topk` visible keys,
+// the top 11 bits of every middle-column score key into hist (per row,
+// kTopkHistStride words apart, zeroed by the caller): the top-k's first pass.
+cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st, uint32_t* hist = nullptr,
+                                int topk = 0);
 // Tensor-core indexer for many rows of one sequence (prefill shape).
 bool index_prefill_supported(const IndexArgs& a);
 cudaError_t launch_index_prefill(const IndexArgs& a, cudaStream_t st);
@@ -49,10 +53,18 @@ struct TopkArgs {
   int32_t* count;
   void* ws;
   size_t ws_bytes;
+  // Per-row histograms built by the indexer (kTopkHistStride words apart), or
+  // null: the top-k then builds them itself.
+  const uint32_t* hist_ext = nullptr;
 };
 constexpr int kTopkCap = 4096;                              // candidates kept per row
 constexpr size_t kTopkRowBytes = 2048 * 4 + 32 + kTopkCap * 8;  // hist + ctl + candidates
+constexpr int kTopkHistStride = 2048 + 8;                   // words between rows' histograms
+
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
+bool topk_uses_workspace(int n_rows, int64_t max_len);
+// Fills hist (rows kTopkHistStride words apart, zeroed by the caller) from scores.
+cudaError_t launch_topk_hist_only(const TopkArgs& a, uint32_t* hist, cudaStream_t st);
 cudaError_t launch_topk_dense(const TopkArgs& a, cudaStream_t st);
 
 struct MlaArgs {

@@ -80,7 +80,7 @@ size_t mla_ws(int n_rows, int cli, int64_t max_list) {
 
 // Workspace of one forward block of R rows (sparse path).
 size_t forward_block_ws(const lsa_config* c, int R, int64_t max_len) {
-  return align_up((size_t)R * max_len * sizeof(float)) +
+  return align_up((size_t)R * max_len * sizeof(float)) + align_up((size_t)R * kTopkHistStride * sizeof(uint32_t)) +
          align_up((size_t)R * c->index_topk * sizeof(int32_t)) +
          align_up((size_t)R * sizeof(int32_t)) + topk_ws(R) + mla_ws(R, c->cli_factor, c->index_topk);
 }
@@ -94,7 +94,7 @@ int prefill_block_rows(int n_rows, int64_t max_len) {
 lsa_status run_index_scores(const lsa_config* c, int n_rows, int n_seq, const int32_t* seq_of_row,
                             int seq_identity, const int32_t* pos, const lsa_bf16* q_idx, const float* w,
                             const lsa_bf16* k_idx, const int64_t* k_off, int64_t max_len,
-                            float* scores, int64_t ld, cudaStream_t st) {
+                            float* scores, int64_t ld, cudaStream_t st, uint32_t* topk_hist = nullptr) {
   IndexArgs a;
   a.q_idx = q_idx;
   a.w = w;
@@ -111,13 +111,36 @@ lsa_status run_index_scores(const lsa_config* c, int n_rows, int n_seq, const in
   a.scores = scores;
   a.ld = ld;
   a.err = device_error_word();
-  if (index_prefill_supported(a)) return cuda_status(launch_index_prefill(a, st), "lsa_index_scores");
-  return cuda_status(launch_index_decode(a, st), "lsa_index_scores");
+  if (topk_hist) {
+    const lsa_status s0 = cuda_status(
+        cudaMemsetAsync(topk_hist, 0, (size_t)n_rows * kTopkHistStride * sizeof(uint32_t), st), "lsa_index_scores");
+    if (s0 != LSA_OK) return s0;
+  }
+  if (!index_prefill_supported(a))
+    return cuda_status(launch_index_decode(a, st, topk_hist, c->index_topk), "lsa_index_scores");
+  lsa_status s1 = cuda_status(launch_index_prefill(a, st), "lsa_index_scores");
+  if (s1 != LSA_OK || !topk_hist) return s1;
+  // The tensor-core epilogue has no room for per-row histograms: one pass over
+  // the fresh scores builds them instead.
+  TopkArgs t;
+  t.scores = scores;
+  t.ld = ld;
+  t.pos = pos;
+  t.n_rows = n_rows;
+  t.max_len = max_len;
+  t.topk = c->index_topk;
+  t.n_init = c->index_init_tokens;
+  t.n_loc = c->index_local_tokens;
+  t.idx = nullptr;
+  t.count = nullptr;
+  t.ws = nullptr;
+  t.ws_bytes = 0;
+  return cuda_status(launch_topk_hist_only(t, topk_hist, st), "lsa_index_scores");
 }
 
 lsa_status run_topk(const lsa_config* c, int n_rows, const int32_t* pos, int64_t max_len,
                     const float* scores, int64_t ld, int32_t* idx, int32_t* count, void* ws,
-                    size_t ws_bytes, cudaStream_t st) {
+                    size_t ws_bytes, cudaStream_t st, const uint32_t* hist_ext = nullptr) {
   TopkArgs a;
   a.scores = scores;
   a.ld = ld;
@@ -129,11 +152,12 @@ lsa_status run_topk(const lsa_config* c, int n_rows, const int32_t* pos, int64_t
   a.n_loc = c->index_local_tokens;
   a.idx = idx;
   a.count = count;
+  a.hist_ext = hist_ext;
   uintptr_t p = (reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~uintptr_t(kAlign - 1);
   a.ws = reinterpret_cast<void*>(p);
   const size_t slack = ws ? p - reinterpret_cast<uintptr_t>(ws) : 0;
   a.ws_bytes = ws_bytes > slack ? ws_bytes - slack : 0;
-  if (max_len > c->index_topk && a.ws_bytes < kTopkRowBytes)
+  if (max_len > c->index_topk && topk_uses_workspace(n_rows, max_len) && a.ws_bytes < kTopkRowBytes)
     return set_error(LSA_ERR_WORKSPACE, "lsa_topk: workspace below one row (%zu bytes)",
                      (size_t)kTopkRowBytes);
   const lsa_status st2 = cuda_status(launch_topk(a, st), "lsa_topk");
@@ -219,7 +243,8 @@ lsa_status lsa_device_error(int32_t* flags) {
 lsa_status lsa_index_scores(const lsa_config* c, int32_t n_rows, int32_t n_seq,
                             const int32_t* seq_of_row, const int32_t* pos, const lsa_bf16* q_idx,
                             const float* w, const lsa_bf16* k_idx, const int64_t* k_off,
-                            int64_t max_len, float* scores, int64_t ld, void* stream) {
+                            int64_t max_len, float* scores, int64_t ld, uint32_t* topk_hist,
+                            void* stream) {
   const char* fn = "lsa_index_scores";
   lsa_status s = check_cfg(c, fn);
   if (s != LSA_OK) return s;
@@ -232,12 +257,12 @@ lsa_status lsa_index_scores(const lsa_config* c, int32_t n_rows, int32_t n_seq,
   if (!aligned16(q_idx) || !aligned16(k_idx))
     return set_error(LSA_ERR_INVALID, "%s: q_idx and k_idx must be 16-byte aligned", fn);
   return run_index_scores(c, n_rows, n_seq, seq_of_row, 0, pos, q_idx, w, k_idx, k_off, max_len,
-                          scores, ld, (cudaStream_t)stream);
+                          scores, ld, (cudaStream_t)stream, topk_hist);
 }
 
 lsa_status lsa_topk(const lsa_config* c, int32_t n_rows, const int32_t* pos, int64_t max_len,
-                    const float* scores, int64_t ld, int32_t* idx, int32_t* count, void* ws,
-                    size_t ws_bytes, void* stream) {
+                    const float* scores, int64_t ld, const uint32_t* topk_hist, int32_t* idx,
+                    int32_t* count, void* ws, size_t ws_bytes, void* stream) {
   const char* fn = "lsa_topk";
   lsa_status s = check_cfg(c, fn);
   if (s != LSA_OK) return s;
@@ -245,8 +270,10 @@ lsa_status lsa_topk(const lsa_config* c, int32_t n_rows, const int32_t* pos, int
     return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0 and 1 <= max_len <= ld", fn);
   if (n_rows == 0) return max_len <= c->index_topk ? LSA_DENSE : LSA_OK;
   if (!pos || !scores || !idx || !count) return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
-  if (max_len > c->index_topk && !ws) return set_error(LSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
-  return run_topk(c, n_rows, pos, max_len, scores, ld, idx, count, ws, ws_bytes, (cudaStream_t)stream);
+  if (max_len > c->index_topk && !ws && topk_uses_workspace(n_rows, max_len))
+    return set_error(LSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
+  return run_topk(c, n_rows, pos, max_len, scores, ld, idx, count, ws, ws_bytes, (cudaStream_t)stream,
+                  topk_hist);
 }
 
 lsa_status lsa_sparse_mla_decode(const lsa_config* c, int32_t batch, const lsa_bf16* q_abs,
@@ -376,13 +403,18 @@ lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_
   char* p = reinterpret_cast<char*>(base);
   float* scores = reinterpret_cast<float*>(p);
   p += align_up((size_t)R * max_len * sizeof(float));
+  uint32_t* hist_ws = reinterpret_cast<uint32_t*>(p);
+  p += align_up((size_t)R * kTopkHistStride * sizeof(uint32_t));
   int32_t* idx_ws = reinterpret_cast<int32_t*>(p);
   p += align_up((size_t)R * c->index_topk * sizeof(int32_t));
   int32_t* cnt_ws = reinterpret_cast<int32_t*>(p);
   p += align_up((size_t)R * sizeof(int32_t));
-  void* topk_w = p;
+  void* topk_w = p;  // 256-byte aligned (every region above is a multiple of 256)
   const size_t topk_bytes = topk_ws(R);
   p += topk_bytes;
+  // Decode: the indexer builds the top-k's histogram while the scores are in
+  // registers, which saves the top-k one pass over the scores and one launch.
+  const bool fuse_hist = mode == 0;
   void* mla_w = p;
   const size_t mla_bytes = mla_ws(R, cli, c->index_topk);
 
@@ -390,11 +422,12 @@ lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_
     const int nr = std::min(R, n_rows - r0);
     int32_t* idx_b = idx_out ? idx_out + (int64_t)r0 * c->index_topk : idx_ws;
     int32_t* cnt_b = count_out ? count_out + r0 : cnt_ws;
+    uint32_t* hist = fuse_hist ? hist_ws : nullptr;
     s = run_index_scores(c, nr, n_seq, seq_of_row ? seq_of_row + r0 : nullptr, mode == 0, pos + r0,
                          q_idx + (int64_t)r0 * kHi * kDi, w + (int64_t)r0 * kHi, k_idx, k_off,
-                         max_len, scores, max_len, st);
+                         max_len, scores, max_len, st, hist);
     if (s != LSA_OK) return s;
-    s = run_topk(c, nr, pos + r0, max_len, scores, max_len, idx_b, cnt_b, topk_w, topk_bytes, st);
+    s = run_topk(c, nr, pos + r0, max_len, scores, max_len, idx_b, cnt_b, topk_w, topk_bytes, st, hist);
     if (s != LSA_OK && s != LSA_DENSE) return s;
     MlaArgs b = m;
     b.n_rows = nr;

@@ -9,18 +9,21 @@
 // same set. Both are computed here by gathering each row's selected keys, which
 // gives exactly the masked result without touching unselected keys.
 //
-// Design. One CTA handles one (query row, split of its key list, sub-block).
-// Latent rows are gathered by cp.async into a double-buffered shared-memory
-// tile of 64 keys (1152-byte rows padded to 1168 so ldmatrix is conflict-free).
-// S = Q K^T runs on mma.m16n8k16 with the 32 heads as M (2 tiles) and the keys
-// split across 4 warps; the online softmax (base-2, max-subtracted) reduces
-// across warps through shared memory; O += P V runs with the 512 value dims
-// split across the warps (128 each, fp32 accumulators in registers). With more
-// than one split per row the CTA writes an unnormalised partial (O, m, l) and a
-// merge kernel combines the splits; with one split it writes bf16 output and lse
-// directly. Gathered indices are bounds-checked against the row's visible keys.
+// Design. One CTA (8 warps) handles one (query row, split of its key list,
+// sub-block). Latent rows are gathered by cp.async into a double-buffered
+// shared-memory tile of 64 keys (1152-byte rows padded to 1168 so ldmatrix is
+// conflict-free). S = Q K^T runs on mma.m16n8k16 with the 576-dim contraction
+// split four ways across warps: each warp keeps its quarter of Q in registers
+// for the whole CTA and runs eight independent accumulator chains, and the
+// partial logits are summed through shared memory. The online softmax is
+// base-2 and max-subtracted. O += P V runs with the 512 value dims split across
+// the warps (64 each, fp32 accumulators in registers). With more than one split
+// per row the CTA writes an unnormalised partial (O, m, l) and a merge kernel
+// combines the splits; with one split it writes bf16 output and lse directly.
+// Gathered indices are bounds-checked against the row's visible keys.
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.h"
 
 namespace lsa {
 namespace {
@@ -29,24 +32,39 @@ constexpr int kTK = 64;             // keys per tile
 constexpr int kSRow = kDLat + 8;    // shared row stride (bf16): 1168 bytes
 constexpr int kPRow = kTK + 8;      // P row stride (bf16): 144 bytes
 constexpr int kMaxSplitKeys = 2048;
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;
 constexpr int kMaxSplits = 32;
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
 struct __align__(16) MlaSmem {
+  // Q staging at start; afterwards the per-warp partial logits
+  // [4 dim quarters][2 head halves][16 heads][kPartRow] fp32 (36864 B).
   uint16_t q[kH * kSRow];
   uint16_t k[2][kTK * kSRow];
   uint16_t p[kH * kPRow];
-  float red[2][4][kH];
+  float red_max[4][kH];
+  float red_sum[4][kH];
+  float alpha[kH];
+  float fin_m[kH];
+  float fin_l[kH];
   int32_t list[kMaxSplitKeys];
 };
+constexpr int kPartRow = 72;  // fp32 row stride of the partial logits (conflict-free float2 stores)
+static_assert(4 * 2 * 16 * kPartRow * 4 <= kH * kSRow * 2, "partial logits fit in the Q staging area");
 
 struct Split {
   int n_split;
   int split_keys;
 };
 
+// Warp roles. Logits S = Q K^T (32 heads x 64 keys per tile, contraction 576):
+// warp w takes head half mt = w & 1 and dim quarter kq = w >> 1 (9 k16 steps);
+// its Q fragments stay in registers for the whole CTA and it runs 8 independent
+// accumulator chains (one per 8-key n-tile) of 9 MMAs. The four dim-quarter
+// partials meet in shared memory. Softmax: warp w owns head half mt and key
+// quarter kg = w >> 1; each lane one head and 8 keys. O += P V: warp w owns
+// value dims 64w .. 64w+63 for all 32 heads (16 accumulator tiles).
 __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, float* part_o,
                                                           float2* part_ml) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -54,6 +72,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   const int s = blockIdx.x, r = blockIdx.y, z = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
+  const int mt = warp & 1, kq = warp >> 1;
+  pdl_wait();
 
   // ---- row geometry (clamped and flagged, never faulting) ----
   int64_t kbase = 0, nvis = 0;
@@ -69,7 +89,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
         int64_t p1 = (int64_t)a.pos[r] + 1;
         if (p1 < 1 || p1 > klen) {
           if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_POS);
-          p1 = max64(0, min(p1, klen));
+          p1 = max64(0, min64(p1, klen));
         }
         nvis = p1;
       }
@@ -78,7 +98,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     int64_t p1 = (int64_t)a.pos[r] + 1;
     if (p1 < 1 || p1 > a.n_keys) {
       if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_POS);
-      p1 = max64(0, min(p1, a.n_keys));
+      p1 = max64(0, min64(p1, a.n_keys));
     }
     nvis = p1;
   }
@@ -108,18 +128,18 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     cp_async16(smem_u32(&sm.q[h * kSRow + col * 8]), qg + h * kDLat + col * 8, 16);
   }
   cp_async_commit();
-  __syncthreads();
+  __syncthreads();  // list visible
 
   const uint16_t* __restrict__ latb = a.lat[z] + kbase * kDLat;
   const int n_tiles = (nk + kTK - 1) / kTK;
-  // Warp w gathers tile rows [16w, 16w+16): 16 x 72 16-byte chunks, 36 per lane,
+  // Warp w gathers tile rows [8w, 8w+8): 8 x 72 16-byte chunks, 18 per lane,
   // consecutive lanes on consecutive chunks of a row.
   auto issue_tile = [&](int tt) {
     uint16_t* dst = sm.k[tt & 1];
-#pragma unroll 4
-    for (int u = 0; u < 36; ++u) {
+#pragma unroll 6
+    for (int u = 0; u < 18; ++u) {
       const int qd = lane + 32 * u;
-      const int row = 16 * warp + qd / 72, col = qd % 72;
+      const int row = 8 * warp + qd / 72, col = qd % 72;
       const int slot = tt * kTK + row;
       const int key = slot < nk ? sm.list[slot] : -1;
       const uint16_t* src = key >= 0 ? latb + (int64_t)key * kDLat + col * 8 : a.lat[z];
@@ -129,143 +149,136 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   if (n_tiles > 0) issue_tile(0);
   cp_async_commit();
 
-  const float scale_log2 = a.scale * kLog2e;
-  float m_run[2][2], l_run[2][2];
-  float o[2][16][4];
+  // Q fragments of this warp: head half mt, k16 steps 9kq .. 9kq+8.
+  cp_async_wait<1>();
+  __syncthreads();
+  uint32_t qf[9][4];
+  {
+    const uint32_t qa = smem_u32(&sm.q[(16 * mt + (lane & 15)) * kSRow + 8 * (lane >> 4)]) + 9 * kq * 32;
 #pragma unroll
-  for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-      m_run[mt][hf] = -INFINITY;
-      l_run[mt][hf] = 0.f;
-    }
-#pragma unroll
-    for (int nt = 0; nt < 16; ++nt)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) o[mt][nt][i] = 0.f;
+    for (int ks = 0; ks < 9; ++ks) ldsm_x4(qa + ks * 32, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
   }
+  float* part = reinterpret_cast<float*>(sm.q);  // valid once every warp has its Q fragments
+
+  const float scale_log2 = a.scale * kLog2e;
+  // softmax state for this lane's head (head half mt, head 16mt + (lane >> 1))
+  const int sh = 16 * mt + (lane >> 1);
+  const int kg = warp >> 1, kb8 = 8 * (lane & 1);
+  float m_run = -INFINITY, l_run = 0.f;
+  // value accumulators: o[mtv][nt][4], heads 16mtv+g (+8), dims 64w + 8nt + 2t
+  float o[2][8][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) o[i][nt][j] = 0.f;
 
   for (int tt = 0; tt < n_tiles; ++tt) {
+    cp_async_wait<0>();
+    __syncthreads();  // (1) tile tt landed; every warp finished O += P V of tile tt-1
     if (tt + 1 < n_tiles) issue_tile(tt + 1);
     cp_async_commit();
-    cp_async_wait<1>();
-    __syncthreads();
     const uint16_t* kt = sm.k[tt & 1];
 
-    // ---- S = Q K^T for keys 16w .. 16w+15 of the tile ----
-    float sc[2][2][4];
+    // ---- partial logits over this warp's dim quarter ----
+    float sc[8][4];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+      for (int j = 0; j < 4; ++j) sc[nt][j] = 0.f;
+    const uint32_t kb0 = smem_u32(&kt[((lane & 7) + 8 * (lane >> 4)) * kSRow + 8 * ((lane >> 3) & 1)]) +
+                         9 * kq * 32;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) sc[mt][nt][i] = 0.f;
-    const uint32_t qa0 = smem_u32(&sm.q[(lane & 15) * kSRow + 8 * (lane >> 4)]);
-    const uint32_t qa1 = qa0 + 16 * kSRow * 2;
-    const uint32_t kb0 =
-        smem_u32(&kt[(16 * warp + (lane & 7) + 8 * (lane >> 4)) * kSRow + 8 * ((lane >> 3) & 1)]);
-#pragma unroll 4
-    for (int ks = 0; ks < kDLat / 16; ++ks) {
-      uint32_t a0[4], a1[4], b[4];
-      ldsm_x4(qa0 + ks * 32, a0[0], a0[1], a0[2], a0[3]);
-      ldsm_x4(qa1 + ks * 32, a1[0], a1[1], a1[2], a1[3]);
-      ldsm_x4(kb0 + ks * 32, b[0], b[1], b[2], b[3]);
-      mma_16816(sc[0][0], a0[0], a0[1], a0[2], a0[3], b[0], b[1]);
-      mma_16816(sc[0][1], a0[0], a0[1], a0[2], a0[3], b[2], b[3]);
-      mma_16816(sc[1][0], a1[0], a1[1], a1[2], a1[3], b[0], b[1]);
-      mma_16816(sc[1][1], a1[0], a1[1], a1[2], a1[3], b[2], b[3]);
+    for (int ks = 0; ks < 9; ++ks) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        uint32_t b[4];
+        ldsm_x4(kb0 + (16 * j * kSRow) * 2 + ks * 32, b[0], b[1], b[2], b[3]);
+        mma_16816(sc[2 * j], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b[0], b[1]);
+        mma_16816(sc[2 * j + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b[2], b[3]);
+      }
     }
+    {
+      float* pw = part + ((kq * 2 + mt) * 16) * kPartRow;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        *reinterpret_cast<float2*>(&pw[g * kPartRow + 8 * nt + 2 * t]) = make_float2(sc[nt][0], sc[nt][1]);
+        *reinterpret_cast<float2*>(&pw[(g + 8) * kPartRow + 8 * nt + 2 * t]) =
+            make_float2(sc[nt][2], sc[nt][3]);
+      }
+    }
+    __syncthreads();  // (2) partials complete
 
-    // ---- online softmax (base 2) ----
-    // sc[mt][nt][2*hf+e]: head 16mt+8hf+g, key 16w+8nt+2t+e.
+    // ---- sum the partials, mask, tile max (lane: head sh, keys 16kg+kb8 .. +7) ----
+    float x[8];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int i = 0; i < 8; ++i) x[i] = 0.f;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int slot = tt * kTK + 16 * warp + 8 * nt + 2 * t + e;
-        const bool valid = slot < nk && sm.list[slot] >= 0;
+    for (int q4 = 0; q4 < 4; ++q4) {
+      const float* pr = part + ((q4 * 2 + mt) * 16 + (lane >> 1)) * kPartRow + 16 * kg + kb8;
+      const float4 v0 = *reinterpret_cast<const float4*>(pr);
+      const float4 v1 = *reinterpret_cast<const float4*>(pr + 4);
+      x[0] += v0.x; x[1] += v0.y; x[2] += v0.z; x[3] += v0.w;
+      x[4] += v1.x; x[5] += v1.y; x[6] += v1.z; x[7] += v1.w;
+    }
+    float mx = -INFINITY;
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+    for (int i = 0; i < 8; ++i) {
+      const int slot = tt * kTK + 16 * kg + kb8 + i;
+      const bool valid = slot < nk && sm.list[slot] >= 0;
+      x[i] = valid ? x[i] * scale_log2 : -INFINITY;
+      mx = fmaxf(mx, x[i]);
+    }
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
+    if ((lane & 1) == 0) sm.red_max[kg][sh] = mx;
+    __syncthreads();  // (3) tile maxima
+    const float tmax = fmaxf(fmaxf(sm.red_max[0][sh], sm.red_max[1][sh]), fmaxf(sm.red_max[2][sh], sm.red_max[3][sh]));
+    const float m_new = fmaxf(m_run, tmax);
+    const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
+    const float alpha = exp2f(m_run - m_use);
+    m_run = m_new;
+    float ps = 0.f;
+    uint32_t pk[4];
 #pragma unroll
-          for (int hf = 0; hf < 2; ++hf)
-            sc[mt][nt][2 * hf + e] = valid ? sc[mt][nt][2 * hf + e] * scale_log2 : -INFINITY;
-      }
-    float mx[2][2];
+    for (int i = 0; i < 4; ++i) {
+      const float p0 = exp2f(x[2 * i] - m_use), p1 = exp2f(x[2 * i + 1] - m_use);
+      ps += p0 + p1;
+      pk[i] = pack_bf16x2(p0, p1);
+    }
+    *reinterpret_cast<uint4*>(&sm.p[sh * kPRow + 16 * kg + kb8]) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    ps += __shfl_xor_sync(0xffffffffu, ps, 1);
+    if ((lane & 1) == 0) {
+      sm.red_sum[kg][sh] = ps;
+      if (kg == 0) sm.alpha[sh] = alpha;
+    }
+    __syncthreads();  // (4) P, alpha and tile sums ready
+    l_run = l_run * alpha +
+            ((sm.red_sum[0][sh] + sm.red_sum[1][sh]) + (sm.red_sum[2][sh] + sm.red_sum[3][sh]));
+
+    // ---- O += P V, value dims 64w .. 64w+63 ----
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        float v = fmaxf(fmaxf(sc[mt][0][2 * hf], sc[mt][0][2 * hf + 1]),
-                        fmaxf(sc[mt][1][2 * hf], sc[mt][1][2 * hf + 1]));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 1));
-        v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, 2));
-        if (t == 0) sm.red[0][warp][16 * mt + 8 * hf + g] = v;
-      }
-    __syncthreads();
-    float alpha[2][2], m_use[2][2];
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int head = 16 * mt + 8 * hf + g;
-        const float tmax = fmaxf(fmaxf(sm.red[0][0][head], sm.red[0][1][head]),
-                                 fmaxf(sm.red[0][2][head], sm.red[0][3][head]));
-        const float m_new = fmaxf(m_run[mt][hf], tmax);
-        m_use[mt][hf] = (m_new == -INFINITY) ? 0.f : m_new;
-        alpha[mt][hf] = exp2f(m_run[mt][hf] - m_use[mt][hf]);
-        m_run[mt][hf] = m_new;
-        mx[mt][hf] = 0.f;
-      }
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
-          const float p0 = exp2f(sc[mt][nt][2 * hf] - m_use[mt][hf]);
-          const float p1 = exp2f(sc[mt][nt][2 * hf + 1] - m_use[mt][hf]);
-          mx[mt][hf] += p0 + p1;
-          const int head = 16 * mt + 8 * hf + g;
-          *reinterpret_cast<uint32_t*>(&sm.p[head * kPRow + 16 * warp + 8 * nt + 2 * t]) =
-              pack_bf16x2(p0, p1);
-        }
-#pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mv = 0; mv < 2; ++mv)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        float v = mx[mt][hf];
-        v += __shfl_xor_sync(0xffffffffu, v, 1);
-        v += __shfl_xor_sync(0xffffffffu, v, 2);
-        if (t == 0) sm.red[1][warp][16 * mt + 8 * hf + g] = v;
-      }
-    __syncthreads();
+        const float al = sm.alpha[16 * mv + 8 * hf + g];
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int head = 16 * mt + 8 * hf + g;
-        const float tsum = (sm.red[1][0][head] + sm.red[1][1][head]) +
-                           (sm.red[1][2][head] + sm.red[1][3][head]);
-        l_run[mt][hf] = l_run[mt][hf] * alpha[mt][hf] + tsum;
-#pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          o[mt][nt][2 * hf] *= alpha[mt][hf];
-          o[mt][nt][2 * hf + 1] *= alpha[mt][hf];
+        for (int nt = 0; nt < 8; ++nt) {
+          o[mv][nt][2 * hf] *= al;
+          o[mv][nt][2 * hf + 1] *= al;
         }
       }
-
-    // ---- O += P V for value dims 128w .. 128w+127 ----
     const uint32_t pa0 = smem_u32(&sm.p[(lane & 15) * kPRow + 8 * (lane >> 4)]);
     const uint32_t pa1 = pa0 + 16 * kPRow * 2;
-    const uint32_t vb0 = smem_u32(
-        &kt[((lane & 7) + 8 * ((lane >> 3) & 1)) * kSRow + 128 * warp + 8 * (lane >> 4)]);
+    const uint32_t vb0 =
+        smem_u32(&kt[((lane & 7) + 8 * ((lane >> 3) & 1)) * kSRow + 64 * warp + 8 * (lane >> 4)]);
 #pragma unroll
     for (int kk = 0; kk < kTK / 16; ++kk) {
       uint32_t p0[4], p1[4];
       ldsm_x4(pa0 + kk * 32, p0[0], p0[1], p0[2], p0[3]);
       ldsm_x4(pa1 + kk * 32, p1[0], p1[1], p1[2], p1[3]);
 #pragma unroll
-      for (int np = 0; np < 8; ++np) {
+      for (int np = 0; np < 4; ++np) {
         uint32_t v[4];
         ldsm_x4_t(vb0 + (kk * 16 * kSRow + 16 * np) * 2, v[0], v[1], v[2], v[3]);
         mma_16816(o[0][2 * np], p0[0], p0[1], p0[2], p0[3], v[0], v[1]);
@@ -274,87 +287,94 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
         mma_16816(o[1][2 * np + 1], p1[0], p1[1], p1[2], p1[3], v[2], v[3]);
       }
     }
-    __syncthreads();  // buffer tt&1, P and red are rewritten next iteration
   }
   cp_async_wait<0>();
+  pdl_trigger();
+  if (kg == 0 && (lane & 1) == 0) {
+    sm.fin_m[sh] = m_run;
+    sm.fin_l[sh] = l_run;
+  }
+  __syncthreads();
 
   // ---- epilogue ----
   if (sp.n_split == 1) {
     uint16_t* __restrict__ og = a.out[z] + (int64_t)r * kH * kDV;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mv = 0; mv < 2; ++mv)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        const int head = 16 * mt + 8 * hf + g;
-        const float l = l_run[mt][hf];
+        const int head = 16 * mv + 8 * hf + g;
+        const float l = sm.fin_l[head];
         const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          const int d = 128 * warp + 8 * nt + 2 * t;
+        for (int nt = 0; nt < 8; ++nt) {
+          const int d = 64 * warp + 8 * nt + 2 * t;
           *reinterpret_cast<uint32_t*>(&og[head * kDV + d]) =
-              pack_bf16x2(o[mt][nt][2 * hf] * inv, o[mt][nt][2 * hf + 1] * inv);
+              pack_bf16x2(o[mv][nt][2 * hf] * inv, o[mv][nt][2 * hf + 1] * inv);
         }
-        if (a.lse[z] && warp == 0 && t == 0)
-          a.lse[z][(int64_t)r * kH + head] =
-              l > 0.f ? (m_run[mt][hf] + log2f(l)) * kLn2 : -INFINITY;
       }
+    if (a.lse[z] && tid < kH) {
+      const float l = sm.fin_l[tid];
+      a.lse[z][(int64_t)r * kH + tid] = l > 0.f ? (sm.fin_m[tid] + log2f(l)) * kLn2 : -INFINITY;
+    }
   } else {
     const int64_t base = ((int64_t)z * a.n_rows + r) * sp.n_split + s;
     float* __restrict__ po = part_o + base * kH * kDV;
 #pragma unroll
-    for (int mt = 0; mt < 2; ++mt)
+    for (int mv = 0; mv < 2; ++mv)
 #pragma unroll
       for (int hf = 0; hf < 2; ++hf) {
-        const int head = 16 * mt + 8 * hf + g;
+        const int head = 16 * mv + 8 * hf + g;
 #pragma unroll
-        for (int nt = 0; nt < 16; ++nt) {
-          const int d = 128 * warp + 8 * nt + 2 * t;
-          *reinterpret_cast<float2*>(&po[head * kDV + d]) =
-              make_float2(o[mt][nt][2 * hf], o[mt][nt][2 * hf + 1]);
+        for (int nt = 0; nt < 8; ++nt) {
+          const int d = 64 * warp + 8 * nt + 2 * t;
+          *reinterpret_cast<float2*>(&po[head * kDV + d]) = make_float2(o[mv][nt][2 * hf], o[mv][nt][2 * hf + 1]);
         }
-        if (warp == 0 && t == 0) part_ml[base * kH + head] = make_float2(m_run[mt][hf], l_run[mt][hf]);
       }
+    if (tid < kH) part_ml[base * kH + tid] = make_float2(sm.fin_m[tid], sm.fin_l[tid]);
   }
 }
 
-__global__ void __launch_bounds__(256) mla_merge_kernel(MlaArgs a, Split sp, const float* part_o,
+// One CTA per (head, row, sub-block): 128 threads x 4 value dims, so that a
+// small decode batch still spreads the merge over many SMs.
+__global__ void __launch_bounds__(128) mla_merge_kernel(MlaArgs a, Split sp, const float* part_o,
                                                         const float2* part_ml) {
-  __shared__ float wgt[kMaxSplits][kH];
-  __shared__ float inv_l[kH];
-  const int r = blockIdx.x, z = blockIdx.y, tid = threadIdx.x;
+  __shared__ float wgt[kMaxSplits];
+  __shared__ float inv_l;
+  pdl_wait();
+  const int h = blockIdx.x, r = blockIdx.y, z = blockIdx.z, tid = threadIdx.x;
   const int64_t base = ((int64_t)z * a.n_rows + r) * sp.n_split;
-  if (tid < kH) {
-    float M = -INFINITY;
-    for (int s = 0; s < sp.n_split; ++s) M = fmaxf(M, part_ml[(base + s) * kH + tid].x);
-    float L = 0.f;
-    for (int s = 0; s < sp.n_split; ++s) {
-      const float2 ml = part_ml[(base + s) * kH + tid];
-      const float wv = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
-      wgt[s][tid] = wv;
-      L += wv * ml.y;
+  if (tid < 32) {
+    const float2 ml = tid < sp.n_split ? part_ml[(base + tid) * kH + h] : make_float2(-INFINITY, 0.f);
+    float M = ml.x;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float wv = (ml.x == -INFINITY) ? 0.f : exp2f(ml.x - M);
+    float L = wv * ml.y;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) L += __shfl_xor_sync(0xffffffffu, L, off);
+    if (tid < sp.n_split) wgt[tid] = wv;
+    if (tid == 0) {
+      inv_l = L > 0.f ? 1.f / L : 0.f;
+      if (a.lse[z]) a.lse[z][(int64_t)r * kH + h] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
     }
-    inv_l[tid] = L > 0.f ? 1.f / L : 0.f;
-    if (a.lse[z]) a.lse[z][(int64_t)r * kH + tid] = L > 0.f ? (M + log2f(L)) * kLn2 : -INFINITY;
   }
   __syncthreads();
-  uint16_t* __restrict__ og = a.out[z] + (int64_t)r * kH * kDV;
-  for (int e = tid * 4; e < kH * kDV; e += 256 * 4) {
-    const int head = e / kDV;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < sp.n_split; ++s) {
-      const float4 v = *reinterpret_cast<const float4*>(part_o + (base + s) * kH * kDV + e);
-      const float wv = wgt[s][head];
-      acc.x = fmaf(wv, v.x, acc.x);
-      acc.y = fmaf(wv, v.y, acc.y);
-      acc.z = fmaf(wv, v.z, acc.z);
-      acc.w = fmaf(wv, v.w, acc.w);
-    }
-    const float il = inv_l[head];
-    uint2 pk;
-    pk.x = pack_bf16x2(acc.x * il, acc.y * il);
-    pk.y = pack_bf16x2(acc.z * il, acc.w * il);
-    *reinterpret_cast<uint2*>(og + e) = pk;
+  const int e = tid * 4;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s = 0; s < sp.n_split; ++s) {
+    const float4 v = *reinterpret_cast<const float4*>(part_o + ((base + s) * kH + h) * kDV + e);
+    const float wv = wgt[s];
+    acc.x = fmaf(wv, v.x, acc.x);
+    acc.y = fmaf(wv, v.y, acc.y);
+    acc.z = fmaf(wv, v.z, acc.z);
+    acc.w = fmaf(wv, v.w, acc.w);
   }
+  const float il = inv_l;
+  uint2 pk;
+  pk.x = pack_bf16x2(acc.x * il, acc.y * il);
+  pk.y = pack_bf16x2(acc.z * il, acc.w * il);
+  *reinterpret_cast<uint2*>(a.out[z] + ((int64_t)r * kH + h) * kDV + e) = pk;
 }
 
 }  // namespace
@@ -433,11 +453,15 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
       b.k_off = a.k_off + row0;
       b.n_seq = a.n_seq - row0;
     }
-    mla_kernel<<<dim3(n_split, nr, a.cli), kThreads, sizeof(MlaSmem), st>>>(b, sp, part_o, part_ml);
-    if (n_split > 1) mla_merge_kernel<<<dim3(nr, a.cli), 256, 0, st>>>(b, sp, part_o, part_ml);
-    count_launches(n_split > 1 ? 2 : 1);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_pdl(mla_kernel, dim3(n_split, nr, a.cli), dim3(kThreads), sizeof(MlaSmem), st, b, sp,
+                               part_o, part_ml);
     if (e != cudaSuccess) return e;
+    if (n_split > 1) {
+      e = launch_pdl(mla_merge_kernel, dim3(kH, nr, a.cli), dim3(128), 0, st, b, sp, (const float*)part_o,
+                     (const float2*)part_ml);
+      if (e != cudaSuccess) return e;
+    }
+    count_launches(n_split > 1 ? 2 : 1);
   }
   return cudaSuccess;
 }

@@ -9,28 +9,28 @@
 // the budget (k_rem = topk - init - local) is chosen among the middle columns
 // [init, n - local) by a radix select on the order-preserving uint32 image of
 // the fp32 score, extended with the bit-inverted column index so that every
-// value is unique and ties go to the lower index. Three kernels per row block:
-//   1. histogram of the top 11 key bits (many CTAs per row, shared-memory
-//      counts flushed with global atomics);
-//   2. every CTA finds the threshold bin from the histogram, emits columns in
-//      higher bins straight to the output and appends columns in the threshold
-//      bin to a per-row candidate buffer;
-//   3. one CTA per row finishes the select on the candidates (the remaining 21
-//      key bits and 32 index bits, 11 bits per pass, stopping as soon as a bin
-//      holds exactly what is still needed), writes the forced columns, the
-//      count, and handles dense rows. If the candidate buffer overflowed (many
-//      equal scores), it rescans the row instead.
-// No kernel waits on another CTA; kernel boundaries order the passes.
+// value is unique and ties go to the lower index. The first pass is a histogram
+// of the top 11 key bits, built by the decode indexer while the scores are in
+// registers, or here. Two kernel shapes:
+//   * many or short rows: one CTA per row does everything, with the
+//     threshold-bin candidates in shared memory;
+//   * few long rows: many CTAs per row. Each finds the threshold bin, places
+//     its chunk's columns with one block-wide prefix sum and one global atomic,
+//     and the last CTA of the row (an atomic ticket) finishes the select on the
+//     candidates. If the candidate buffer overflowed (many equal scores), that
+//     CTA rescans the row instead.
+// No kernel waits on another CTA.
 #include "common.cuh"
 #include "kernels.h"
+#include "launch.h"
+#include "radix.cuh"
 
 namespace lsa {
 namespace {
 
-constexpr int kBins = 2048;
 constexpr int kHistThreads = 256;
-constexpr int kResolveThreads = 512;
-constexpr int64_t kChunk = 16384;
+constexpr int64_t kChunk = 4096;     // scores per CTA in the histogram and collect passes
+constexpr int kUnroll = 8;           // loads in flight per lane
 constexpr uint64_t kLow53 = (1ull << 53) - 1;
 
 // Per-row workspace: a zeroed histogram/control block, then the candidates.
@@ -56,55 +56,10 @@ __device__ __forceinline__ RowGeom row_geom(const TopkArgs& a, int r) {
   return g;
 }
 
-// For a histogram h[0..2048) and a budget `need`, finds the bin d such that
-// (count in bins above d) < need <= (count in bins >= d). Block-wide; every
-// thread returns the same answer.
-template <int THREADS>
-__device__ void find_threshold(const uint32_t* h, uint32_t need, int& bin_out,
-                               uint32_t& above_out, int* s_bin, uint32_t* s_above,
-                               uint32_t* s_warp) {
-  constexpr int PER = kBins / THREADS;
-  constexpr int WARPS = THREADS / 32;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) {
-    *s_bin = 0;
-    *s_above = 0;
-  }
-  uint32_t mine = 0;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) mine += h[tid * PER + i];
-  // inclusive suffix sum within the warp
-  uint32_t v = mine;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const uint32_t y = __shfl_down_sync(0xffffffffu, v, off);
-    if (lane + off < 32) v += y;
-  }
-  if (lane == 0) s_warp[warp] = v;  // warp total
-  __syncthreads();
-  uint32_t warp_above = 0;
-  for (int w2 = warp + 1; w2 < WARPS; ++w2) warp_above += s_warp[w2];
-  const uint32_t above = v - mine + warp_above;  // count in bins of higher threads
-  if (above < need && above + mine >= need) {
-    uint32_t cum = above;
-    for (int b = tid * PER + PER - 1; b >= tid * PER; --b) {
-      if (cum + h[b] >= need) {
-        *s_bin = b;
-        *s_above = cum;
-        break;
-      }
-      cum += h[b];
-    }
-  }
-  __syncthreads();
-  bin_out = *s_bin;
-  above_out = *s_above;
-  __syncthreads();
-}
-
 __global__ void __launch_bounds__(kHistThreads)
     topk_hist_kernel(TopkArgs a, int row0, HistCtl* hc) {
   __shared__ uint32_t h[kBins];
+  pdl_wait();
   const int r = row0 + blockIdx.y;
   const RowGeom g = row_geom(a, r);
   if (g.dense) return;
@@ -114,141 +69,293 @@ __global__ void __launch_bounds__(kHistThreads)
   for (int i = threadIdx.x; i < kBins; i += kHistThreads) h[i] = 0;
   __syncthreads();
   const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
-  for (int64_t j = s + threadIdx.x; j < e; j += kHistThreads)
-    atomicAdd(&h[score_key(srow[j]) >> 21], 1u);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  // each warp takes 32 * kUnroll consecutive scores per round, all loads first
+  for (int64_t base = s + warp * 32 * kUnroll; base < e; base += kHistThreads * kUnroll) {
+    float v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t j = base + lane + 32 * u;
+      v[u] = j < e ? srow[j] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u)
+      if (base + lane + 32 * u < e) atomicAdd(&h[score_key(v[u]) >> 21], 1u);
+  }
   __syncthreads();
   HistCtl& w = hc[blockIdx.y];
   for (int i = threadIdx.x; i < kBins; i += kHistThreads)
     if (h[i]) atomicAdd(&w.hist[i], h[i]);
 }
 
+// Every CTA finds the threshold bin from the row's histogram, then handles its
+// chunk with each thread's scores in registers: one block-wide prefix sum places
+// every emitted column, and one global atomic per CTA claims the row's slots
+// (no per-warp round trips to a shared counter). The last CTA of a row to finish
+// (an atomic ticket; nothing waits) selects the rest inside the threshold bin
+// from the candidates, staged in shared memory, and writes the forced columns.
+constexpr int kPerThread = kChunk / kHistThreads;  // 16 scores per thread
+static_assert(kPerThread == 2 * kUnroll, "two rounds of kUnroll loads per thread");
+
 __global__ void __launch_bounds__(kHistThreads)
-    topk_collect_kernel(TopkArgs a, int row0, HistCtl* hc, uint64_t* cand_all) {
+    topk_select_kernel(TopkArgs a, int row0, HistCtl* hc, uint64_t* cand_all) {
   __shared__ uint32_t h[kBins];
-  __shared__ int s_bin;
-  __shared__ uint32_t s_above, s_warp[kHistThreads / 32];
+  __shared__ uint64_t scand[kTopkCap];
+  __shared__ int s_bin, s_last;
+  __shared__ uint32_t s_above, s_warp[kHistThreads / 32], s_wu[kHistThreads / 32], s_we[kHistThreads / 32];
+  __shared__ uint32_t s_base_u, s_base_e, s_slot;
+  pdl_wait();
   const int r = row0 + blockIdx.y;
   const RowGeom g = row_geom(a, r);
-  if (g.dense) return;
+  int32_t* __restrict__ row_out = a.idx + (int64_t)r * a.topk;
+  const int tid = threadIdx.x;
+  if (g.dense) {
+    if (blockIdx.x == 0) {
+      for (int i = tid; i < a.topk; i += kHistThreads) row_out[i] = (i < g.n) ? i : -1;
+      if (tid == 0) a.count[r] = (int32_t)g.n;
+    }
+    return;
+  }
   const int64_t s = g.lo + (int64_t)blockIdx.x * kChunk;
   const int64_t e = min(s + kChunk, g.hi);
   if (s >= e) return;
+  const uint32_t n_chunks = (uint32_t)((g.hi - g.lo + kChunk - 1) / kChunk);
   HistCtl& w = hc[blockIdx.y];
   uint64_t* __restrict__ cand = cand_all + (int64_t)blockIdx.y * kTopkCap;
-  for (int i = threadIdx.x; i < kBins; i += kHistThreads) h[i] = w.hist[i];
+  const uint32_t* hsrc = a.hist_ext ? a.hist_ext + (int64_t)r * kTopkHistStride : w.hist;
+  for (int i = tid; i < kBins; i += kHistThreads) h[i] = hsrc[i];
   __syncthreads();
   const uint32_t k_rem = (uint32_t)(a.topk - a.n_init - a.n_loc);
   int bin;
   uint32_t above;
   find_threshold<kHistThreads>(h, k_rem, bin, above, &s_bin, &s_above, s_warp);
-  if (blockIdx.x == 0 && threadIdx.x == 0) {
-    w.ctl[2] = (uint32_t)bin;
-    w.ctl[3] = above;
-  }
   const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
-  int32_t* __restrict__ out = a.idx + (int64_t)r * a.topk + a.n_init + a.n_loc;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int64_t base = s + warp * 32; base < e; base += kHistThreads) {
-    const int64_t j = base + lane;
-    uint32_t key = 0;
-    int kb = -1;
-    if (j < e) {
-      key = score_key(srow[j]);
-      kb = (int)(key >> 21);
-    }
-    const uint32_t up = __ballot_sync(0xffffffffu, kb > bin);
-    const uint32_t eq = __ballot_sync(0xffffffffu, kb == bin);
-    if (up) {
-      uint32_t slot0 = 0;
-      if (lane == 0) slot0 = atomicAdd(&w.ctl[0], (uint32_t)__popc(up));
-      slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-      const uint32_t slot = slot0 + __popc(up & ((1u << lane) - 1u));
-      if (kb > bin && slot < k_rem) out[slot] = (int32_t)j;
-    }
-    if (eq) {
-      uint32_t slot0 = 0;
-      if (lane == 0) slot0 = atomicAdd(&w.ctl[1], (uint32_t)__popc(eq));
-      slot0 = __shfl_sync(0xffffffffu, slot0, 0);
-      const uint32_t slot = slot0 + __popc(eq & ((1u << lane) - 1u));
-      if (kb == bin && slot < (uint32_t)kTopkCap)
-        cand[slot] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+  const int lane = tid & 31, warp = tid >> 5;
+  const int64_t wbase = s + warp * 32 * kUnroll;  // the second round adds kHistThreads * kUnroll
+  uint32_t key[kPerThread];
+  int kb[kPerThread];
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t j = wbase + (i / kUnroll) * kHistThreads * kUnroll + lane + 32 * (i % kUnroll);
+    const float v = j < e ? srow[j] : 0.f;
+    key[i] = score_key(v);
+    kb[i] = j < e ? (int)(key[i] >> 21) : -1;
+  }
+  uint32_t nu = 0, ne = 0;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    nu += kb[i] > bin;
+    ne += kb[i] == bin;
+  }
+  // exclusive prefix sums over the CTA (warp scans, then the warp totals)
+  uint32_t iu = nu, ie = ne;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const uint32_t yu = __shfl_up_sync(0xffffffffu, iu, off);
+    const uint32_t ye = __shfl_up_sync(0xffffffffu, ie, off);
+    if (lane >= off) {
+      iu += yu;
+      ie += ye;
     }
   }
+  if (lane == 31) {
+    s_wu[warp] = iu;
+    s_we[warp] = ie;
+  }
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t tu = 0, te = 0;
+    for (int i = 0; i < kHistThreads / 32; ++i) {
+      const uint32_t a_u = s_wu[i], a_e = s_we[i];
+      s_wu[i] = tu;
+      s_we[i] = te;
+      tu += a_u;
+      te += a_e;
+    }
+    s_base_u = tu ? atomicAdd(&w.ctl[0], tu) : 0u;
+    s_base_e = te ? atomicAdd(&w.ctl[1], te) : 0u;
+  }
+  __syncthreads();
+  uint32_t ou = s_base_u + s_wu[warp] + iu - nu;
+  uint32_t oe = s_base_e + s_we[warp] + ie - ne;
+  int32_t* __restrict__ mid = row_out + a.n_init + a.n_loc;
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t j = wbase + (i / kUnroll) * kHistThreads * kUnroll + lane + 32 * (i % kUnroll);
+    if (kb[i] > bin) {
+      if (ou < k_rem) mid[ou] = (int32_t)j;
+      ++ou;
+    } else if (kb[i] == bin) {
+      if (oe < (uint32_t)kTopkCap) cand[oe] = ((uint64_t)key[i] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+      ++oe;
+    }
+  }
+
+  // ---- the last CTA of the row finishes it ----
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = atomicAdd(&w.ctl[4], 1u) == n_chunks - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int i = tid; i < a.n_init; i += kHistThreads) row_out[i] = i;
+  for (int i = tid; i < a.n_loc; i += kHistThreads) row_out[a.n_init + i] = (int32_t)(g.hi + i);
+  if (tid == 0) {
+    a.count[r] = a.topk;
+    s_slot = 0;
+  }
+  const uint32_t n_cand = __ldcg(&w.ctl[1]);
+  const bool in_smem = n_cand <= (uint32_t)kTopkCap;
+  if (in_smem)
+    for (uint32_t i = tid; i < n_cand; i += kHistThreads) scand[i] = __ldcg(&cand[i]);
+  __syncthreads();
+  auto for_each = [&](auto&& f) {
+    if (in_smem) {
+      for (uint32_t i = tid; i < n_cand; i += kHistThreads) {
+        const uint64_t c = scand[i];
+        f(c & kLow53, (int64_t)(0xFFFFFFFFu - (uint32_t)c));
+      }
+    } else {  // more equal-bin scores than the buffer holds: rescan the row
+      for (int64_t j = g.lo + tid; j < g.hi; j += kHistThreads) {
+        const uint32_t k2 = score_key(srow[j]);
+        if ((int)(k2 >> 21) == bin) f((((uint64_t)k2 << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j)) & kLow53, j);
+      }
+    }
+  };
+  const uint32_t need0 = k_rem - above;
+  uint64_t prefix;
+  int decided;
+  radix_levels<kHistThreads>(for_each, need0, h, &s_bin, &s_above, s_warp, prefix, decided);
+  int32_t* __restrict__ dst = mid + above;
+  const int shb = 53 - decided;
+  for_each([&](uint64_t v, int64_t j) {
+    if ((v >> shb) >= prefix) {
+      const uint32_t slot = atomicAdd(&s_slot, 1u);
+      if (slot < need0) dst[slot] = (int32_t)j;
+    }
+  });
 }
 
-__global__ void __launch_bounds__(kResolveThreads)
-    topk_resolve_kernel(TopkArgs a, int row0, const HistCtl* hc, const uint64_t* cand_all) {
+// One CTA per row: histogram (unless the indexer already built it), threshold,
+// one collect pass, and the rest of the select on candidates kept in shared
+// memory. For rows up to a few hundred thousand columns this is one launch
+// instead of three; the multi-CTA kernels above serve few, very long rows.
+constexpr int kRowThreads = 512;
+constexpr int kRowCap = 4608;  // 36 KB of candidates: static shared memory stays under 48 KB
+
+__global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int row0, const uint32_t* hist_in) {
   __shared__ uint32_t h[kBins];
+  __shared__ uint64_t cand[kRowCap];
   __shared__ int s_bin;
-  __shared__ uint32_t s_above, s_warp[kResolveThreads / 32], s_slot;
+  __shared__ uint32_t s_above, s_warp[kRowThreads / 32], s_up, s_nc, s_slot;
+  pdl_wait();
   const int r = row0 + blockIdx.x;
   const RowGeom g = row_geom(a, r);
   int32_t* __restrict__ out = a.idx + (int64_t)r * a.topk;
-  const int tid = threadIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (g.dense) {
-    for (int i = tid; i < a.topk; i += kResolveThreads) out[i] = (i < g.n) ? i : -1;
+    for (int i = tid; i < a.topk; i += kRowThreads) out[i] = (i < g.n) ? i : -1;
     if (tid == 0) a.count[r] = (int32_t)g.n;
     return;
   }
-  for (int i = tid; i < a.n_init; i += kResolveThreads) out[i] = i;
-  for (int i = tid; i < a.n_loc; i += kResolveThreads) out[a.n_init + i] = (int32_t)(g.hi + i);
-  if (tid == 0) a.count[r] = a.topk;
-
-  const HistCtl& w = hc[blockIdx.x];
-  const uint64_t* __restrict__ cand = cand_all + (int64_t)blockIdx.x * kTopkCap;
-  const uint32_t bin0 = w.ctl[2];
-  const uint32_t above0 = w.ctl[3];
-  const uint32_t n_cand = w.ctl[1];
-  const bool use_cand = n_cand <= (uint32_t)kTopkCap;
+  for (int i = tid; i < a.n_init; i += kRowThreads) out[i] = i;
+  for (int i = tid; i < a.n_loc; i += kRowThreads) out[a.n_init + i] = (int32_t)(g.hi + i);
+  if (tid == 0) {
+    a.count[r] = a.topk;
+    s_up = 0;
+    s_nc = 0;
+    s_slot = 0;
+  }
+  const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
   const uint32_t k_rem = (uint32_t)(a.topk - a.n_init - a.n_loc);
+  int bin0 = 0;
+  uint32_t above0 = 0;
+  const uint32_t* hr = hist_in ? hist_in + (int64_t)r * kTopkHistStride : nullptr;
+  if (hr) {
+    for (int i = tid; i < kBins; i += kRowThreads) h[i] = hr[i];
+    __syncthreads();
+  } else {
+    for (int i = tid; i < kBins; i += kRowThreads) h[i] = 0;
+    __syncthreads();
+    for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
+      float v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t j = base + lane + 32 * u;
+        v[u] = j < g.hi ? srow[j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u)
+        if (base + lane + 32 * u < g.hi) atomicAdd(&h[score_key(v[u]) >> 21], 1u);
+    }
+    __syncthreads();
+  }
+  find_threshold<kRowThreads>(h, k_rem, bin0, above0, &s_bin, &s_above, s_warp);
+  __syncthreads();  // s_up / s_nc initialised
+  int32_t* __restrict__ mid = out + a.n_init + a.n_loc;
+
+  // collect: higher bins straight out, the threshold bin into shared memory
+  for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
+    float v[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t j = base + lane + 32 * u;
+      v[u] = j < g.hi ? srow[j] : 0.f;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t j = base + lane + 32 * u;
+      uint32_t key = 0;
+      int kb = -1;
+      if (j < g.hi) {
+        key = score_key(v[u]);
+        kb = (int)(key >> 21);
+      }
+      const uint32_t up = __ballot_sync(0xffffffffu, kb > bin0);
+      const uint32_t eq = __ballot_sync(0xffffffffu, kb == bin0);
+      if (up) {
+        uint32_t s0 = 0;
+        if (lane == 0) s0 = atomicAdd(&s_up, (uint32_t)__popc(up));
+        s0 = __shfl_sync(0xffffffffu, s0, 0);
+        const uint32_t slot = s0 + __popc(up & ((1u << lane) - 1u));
+        if (kb > bin0 && slot < k_rem) mid[slot] = (int32_t)j;
+      }
+      if (eq) {
+        uint32_t s0 = 0;
+        if (lane == 0) s0 = atomicAdd(&s_nc, (uint32_t)__popc(eq));
+        s0 = __shfl_sync(0xffffffffu, s0, 0);
+        const uint32_t slot = s0 + __popc(eq & ((1u << lane) - 1u));
+        if (kb == bin0 && slot < (uint32_t)kRowCap)
+          cand[slot] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+      }
+    }
+  }
+  __syncthreads();
+  const uint32_t n_cand = s_nc;
+  const bool in_smem = n_cand <= (uint32_t)kRowCap;
   uint32_t need = k_rem - above0;
   const uint32_t need0 = need;
-  const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
 
-  // Calls f(v53, column) for every element of the threshold bin.
   auto for_each = [&](auto&& f) {
-    if (use_cand) {
-      for (uint32_t i = tid; i < n_cand; i += kResolveThreads) {
+    if (in_smem) {
+      for (uint32_t i = tid; i < n_cand; i += kRowThreads) {
         const uint64_t c = cand[i];
         f(c & kLow53, (int64_t)(0xFFFFFFFFu - (uint32_t)c));
       }
     } else {
-      for (int64_t j = g.lo + tid; j < g.hi; j += kResolveThreads) {
+      for (int64_t j = g.lo + tid; j < g.hi; j += kRowThreads) {
         const uint32_t key = score_key(srow[j]);
-        if ((key >> 21) == bin0) {
+        if ((int)(key >> 21) == bin0) {
           const uint64_t c = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
           f(c & kLow53, j);
         }
       }
     }
   };
-
-  uint64_t prefix = 0;
-  int decided = 0;  // bits of v53 fixed so far, from the top
-  const int widths[5] = {11, 11, 11, 11, 9};
-  for (int lvl = 0; lvl < 5; ++lvl) {
-    const int wdt = widths[lvl];
-    const int shift = 53 - decided - wdt;
-    for (int i = tid; i < kBins; i += kResolveThreads) h[i] = 0;
-    __syncthreads();
-    for_each([&](uint64_t v, int64_t) {
-      if ((v >> (53 - decided)) == prefix)
-        atomicAdd(&h[(uint32_t)(v >> shift) & ((1u << wdt) - 1u)], 1u);
-    });
-    __syncthreads();
-    int d;
-    uint32_t above;
-    find_threshold<kResolveThreads>(h, need, d, above, &s_bin, &s_above, s_warp);
-    const uint32_t cnt = h[d];
-    need -= above;
-    prefix = (prefix << wdt) | (uint64_t)d;
-    decided += wdt;
-    __syncthreads();
-    if (cnt == need) break;  // the whole bin is taken
-  }
-  if (tid == 0) s_slot = 0;
-  __syncthreads();
-  int32_t* __restrict__ dst = out + a.n_init + a.n_loc + above0;
+  uint64_t prefix;
+  int decided;
+  radix_levels<kRowThreads>(for_each, need, h, &s_bin, &s_above, s_warp, prefix, decided);
+  int32_t* __restrict__ dst = mid + above0;
   const int sh = 53 - decided;
   for_each([&](uint64_t v, int64_t j) {
     if ((v >> sh) >= prefix) {
@@ -261,34 +368,73 @@ __global__ void __launch_bounds__(kResolveThreads)
 }  // namespace
 
 cudaError_t launch_topk_dense(const TopkArgs& a, cudaStream_t st) {
+  // every row is dense: the per-row kernel writes 0..n-1 and the count
   for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
     const int nr = min(65535, a.n_rows - row0);
-    topk_resolve_kernel<<<nr, kResolveThreads, 0, st>>>(a, row0, nullptr, nullptr);
+    const cudaError_t e =
+        launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), 0, st, a, row0, (const uint32_t*)nullptr);
+    if (e != cudaSuccess) return e;
     count_launches(1);
   }
-  return cudaGetLastError();
+  return cudaSuccess;
 }
+
+// One CTA per row when there are enough rows to fill the GPU or the rows are
+// short; otherwise several CTAs per row. Only the multi-CTA kernels use the
+// workspace.
+bool topk_uses_workspace(int n_rows, int64_t max_len) { return n_rows < 256 && max_len > (int64_t)16384; }
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   if (a.n_rows <= 0) return cudaSuccess;
   if (a.max_len <= a.topk) return launch_topk_dense(a, st);
-  const int64_t rows_fit = (int64_t)(a.ws_bytes / kTopkRowBytes);
-  const int blk = (int)min64(min64(rows_fit, a.n_rows), 65535);
   const int64_t chunks = (a.max_len + kChunk - 1) / kChunk;
   HistCtl* hc = static_cast<HistCtl*>(a.ws);
+  const bool per_row = !topk_uses_workspace(a.n_rows, a.max_len);
+  if (per_row) {
+    const uint32_t* hist_in = a.hist_ext;
+    for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
+      const int nr = min(65535, a.n_rows - row0);
+      const cudaError_t e = launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), 0, st, a, row0, hist_in);
+      if (e != cudaSuccess) return e;
+      count_launches(1);
+    }
+    return cudaGetLastError();
+  }
+  const int64_t rows_fit = (int64_t)(a.ws_bytes / kTopkRowBytes);
+  const int blk = (int)min64(min64(rows_fit, a.n_rows), 65535);
   uint64_t* cand = reinterpret_cast<uint64_t*>(hc + blk);
   for (int row0 = 0; row0 < a.n_rows; row0 += blk) {
     const int nr = min(blk, a.n_rows - row0);
     cudaError_t e = cudaMemsetAsync(hc, 0, (size_t)nr * sizeof(HistCtl), st);
     if (e != cudaSuccess) return e;
-    topk_hist_kernel<<<dim3((unsigned)chunks, (unsigned)nr), kHistThreads, 0, st>>>(a, row0, hc);
-    topk_collect_kernel<<<dim3((unsigned)chunks, (unsigned)nr), kHistThreads, 0, st>>>(a, row0, hc, cand);
-    topk_resolve_kernel<<<nr, kResolveThreads, 0, st>>>(a, row0, hc, cand);
-    count_launches(3);
+    if (!a.hist_ext) {
+      e = launch_pdl(topk_hist_kernel, dim3((unsigned)chunks, (unsigned)nr), dim3(kHistThreads), 0, st, a, row0, hc);
+      if (e != cudaSuccess) return e;
+      count_launches(1);
+    }
+    e = launch_pdl(topk_select_kernel, dim3((unsigned)chunks, (unsigned)nr), dim3(kHistThreads), 0, st, a, row0, hc,
+                   cand);
+    if (e != cudaSuccess) return e;
+    count_launches(1);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   return cudaSuccess;
+}
+
+cudaError_t launch_topk_hist_only(const TopkArgs& a, uint32_t* hist, cudaStream_t st) {
+  if (a.n_rows <= 0 || a.max_len <= a.topk) return cudaSuccess;
+  static_assert(sizeof(HistCtl) == kTopkHistStride * sizeof(uint32_t), "histogram row stride");
+  const int64_t chunks = (a.max_len + kChunk - 1) / kChunk;
+  HistCtl* hc = reinterpret_cast<HistCtl*>(hist);
+  for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
+    const int nr = min(65535, a.n_rows - row0);
+    const cudaError_t e = launch_pdl(topk_hist_kernel, dim3((unsigned)chunks, (unsigned)nr), dim3(kHistThreads), 0,
+                                     st, a, row0, hc + row0);
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace lsa

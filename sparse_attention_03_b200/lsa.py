@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "liblsa.so")
 LSA_OK, LSA_DENSE = 0, 1
 LSA_ERR_INVALID, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_DEVICE = -1, -2, -3, -4, -5
 OP_TOPK, OP_MLA_DECODE, OP_MLA_PREFILL, OP_FORWARD_DECODE, OP_FORWARD_PREFILL = 1, 2, 3, 4, 5
+TOPK_HIST_WORDS = 2056
 DEVERR_POS, DEVERR_INDEX, DEVERR_COUNT, DEVERR_SEQ, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 
 EXPORTS = (
@@ -68,8 +69,9 @@ def load():
     lib.lsa_config_default.restype = None
     lib.lsa_workspace_size.argtypes = [ctypes.POINTER(Config), _I32, _I32, _I32, _I64]
     lib.lsa_workspace_size.restype = _SZ
-    lib.lsa_index_scores.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P]
-    lib.lsa_topk.argtypes = [ctypes.POINTER(Config), _I32, _P, _I64, _P, _I64, _P, _P, _P, _SZ, _P]
+    lib.lsa_index_scores.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P,
+                                     _P]
+    lib.lsa_topk.argtypes = [ctypes.POINTER(Config), _I32, _P, _I64, _P, _I64, _P, _P, _P, _P, _SZ, _P]
     lib.lsa_sparse_mla_decode.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]
     lib.lsa_sparse_mla_prefill.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
     lib.lsa_forward.argtypes = [ctypes.POINTER(Config), _I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P,
@@ -185,8 +187,13 @@ def workspace(cfg: LsaConfig, op: int, n_rows: int, n_seq: int, max_len: int, de
     return torch.empty(max(n, 1), dtype=torch.uint8, device=device or "cuda")
 
 
+def topk_hist_buffer(n_rows, device=None) -> torch.Tensor:
+    """A buffer for the optional top-k histogram lsa_index_scores can emit."""
+    return torch.empty((n_rows, TOPK_HIST_WORDS), dtype=torch.int32, device=device or "cuda")
+
+
 def index_scores(cfg, seq_of_row, pos, q_idx, w, k_idx, k_off, max_len, scores, n_seq=None, stream=None,
-                 bind=False):
+                 bind=False, topk_hist=None):
     _dt(q_idx, torch.bfloat16, "q_idx"); _dt(k_idx, torch.bfloat16, "k_idx"); _dt(w, torch.float32, "w")
     _dt(pos, torch.int32, "pos"); _dt(seq_of_row, torch.int32, "seq_of_row"); _dt(k_off, torch.int64, "k_off")
     _dt(scores, torch.float32, "scores")
@@ -195,16 +202,17 @@ def index_scores(cfg, seq_of_row, pos, q_idx, w, k_idx, k_off, max_len, scores, 
         n_seq = 1 if k_off is None else k_off.shape[0] - 1
     return _invoke(load().lsa_index_scores, (
         ctypes.byref(cfg._c()), n_rows, n_seq, _ptr(seq_of_row), _ptr(pos), _ptr(q_idx), _ptr(w),
-        _ptr(k_idx), _ptr(k_off), int(max_len), _ptr(scores), scores.shape[1], _stream(stream)), bind=bind)
+        _ptr(k_idx), _ptr(k_off), int(max_len), _ptr(scores), scores.shape[1], _ptr(topk_hist), _stream(stream)),
+        bind=bind)
 
 
-def topk(cfg, pos, max_len, scores, idx, count, ws, stream=None, bind=False):
+def topk(cfg, pos, max_len, scores, idx, count, ws, stream=None, bind=False, topk_hist=None):
     _dt(scores, torch.float32, "scores"); _dt(pos, torch.int32, "pos")
     _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
     return _invoke(load().lsa_topk, (
         ctypes.byref(cfg._c()), pos.shape[0], _ptr(pos), int(max_len), _ptr(scores), scores.shape[1],
-        _ptr(idx), _ptr(count), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)), allow_dense=True,
-        bind=bind)
+        _ptr(topk_hist), _ptr(idx), _ptr(count), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+        allow_dense=True, bind=bind)
 
 
 def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None, bind=False):

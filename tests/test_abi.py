@@ -64,10 +64,11 @@ def test_rejects_bad_config(lib):
     c = lsa.LsaConfig().c()
     c.index_n_heads = 16
     st = lib.lsa_index_scores(ctypes.byref(c), 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100,
-                              _fake(), 100, None)
+                              _fake(), 100, None, None)
     assert st == lsa.LSA_ERR_UNSUPPORTED
     assert b"32x128" in lib.lsa_last_error()
-    st = lib.lsa_index_scores(None, 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100, _fake(), 100, None)
+    st = lib.lsa_index_scores(None, 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100, _fake(), 100, None,
+                              None)
     assert st == lsa.LSA_ERR_INVALID
 
 
@@ -75,15 +76,15 @@ def test_rejects_bad_arguments(lib):
     c = lsa.LsaConfig().c()
     # ld < max_len
     assert lib.lsa_index_scores(ctypes.byref(c), 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100,
-                                _fake(), 50, None) == lsa.LSA_ERR_INVALID
+                                _fake(), 50, None, None) == lsa.LSA_ERR_INVALID
     # misaligned q_idx
     assert lib.lsa_index_scores(ctypes.byref(c), 4, 1, None, _fake(), ctypes.c_void_p(0x10002), _fake(),
-                                _fake(), None, 100, _fake(), 100, None) == lsa.LSA_ERR_INVALID
+                                _fake(), None, 100, _fake(), 100, None, None) == lsa.LSA_ERR_INVALID
     # several sequences without offsets
     assert lib.lsa_index_scores(ctypes.byref(c), 4, 3, None, _fake(), _fake(), _fake(), _fake(), None, 100,
-                                _fake(), 100, None) == lsa.LSA_ERR_INVALID
-    # top-k without a workspace on a sparse length
-    assert lib.lsa_topk(ctypes.byref(c), 4, _fake(), 5000, _fake(), 5000, _fake(), _fake(), None, 0,
+                                _fake(), 100, None, None) == lsa.LSA_ERR_INVALID
+    # top-k without a workspace on few long rows (the multi-CTA path)
+    assert lib.lsa_topk(ctypes.byref(c), 4, _fake(), 90000, _fake(), 90000, None, _fake(), _fake(), None, 0,
                         None) == lsa.LSA_ERR_WORKSPACE
     # decode MLA without offsets
     assert lib.lsa_sparse_mla_decode(ctypes.byref(c), 2, _fake(), _fake(), None, None, None, 10, _fake(),
@@ -102,7 +103,7 @@ def test_rejects_bad_arguments(lib):
 def test_empty_inputs_are_noops(lib):
     c = lsa.LsaConfig().c()
     assert lib.lsa_index_scores(ctypes.byref(c), 0, 1, None, None, None, None, None, None, 10, None, 10,
-                                None) == lsa.LSA_OK
-    assert lib.lsa_topk(ctypes.byref(c), 0, None, 10, None, 10, None, None, None, 0, None) == lsa.LSA_DENSE
+                                None, None) == lsa.LSA_OK
+    assert lib.lsa_topk(ctypes.byref(c), 0, None, 10, None, 10, None, None, None, None, 0, None) == lsa.LSA_DENSE
     assert lib.lsa_sparse_mla_prefill(ctypes.byref(c), 0, None, None, None, 5, None, None, None, None, None,
                                       0, None) == lsa.LSA_OK

@@ -224,6 +224,52 @@ def test_topk_all_equal_overflow_path(L):
         np.testing.assert_array_equal(np.sort(idx[r]), exp)
 
 
+def test_topk_multi_cta_long_rows(L):
+    # few long rows take the multi-CTA kernels, including their rescan path when
+    # the threshold bin overflows
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(21)
+    pos = np.array([300000, 270001, 2048, 400000, 5000], dtype=np.int64)
+    rows = [rng.standard_normal(pos[0] + 1).astype(np.float32) * 8,
+            np.round(rng.standard_normal(pos[1] + 1) * 3).astype(np.float32),
+            rng.standard_normal(pos[2] + 1).astype(np.float32),
+            np.full(pos[3] + 1, 0.25, dtype=np.float32),
+            rng.standard_normal(pos[4] + 1).astype(np.float32)]
+    max_len = int(pos.max()) + 1
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, max_len)
+    for r, p in enumerate(pos):
+        exp, dense = R.select_topk(R.mask_and_force(rows[r].astype(np.float64), int(p), max_len, ocfg), int(p), ocfg)
+        n = min(int(p) + 1, 2048)
+        assert cnt[r] == n
+        np.testing.assert_array_equal(np.sort(idx[r, :n]), exp, err_msg=f"row {r}")
+
+
+@pytest.mark.parametrize("streaming", [True, False])
+def test_topk_with_indexer_histogram(L, streaming):
+    # the histogram lsa_index_scores emits gives lsa_topk the same selection as
+    # its own first pass (both indexer kernels: streaming, and tensor-core + one pass)
+    cfg = L.LsaConfig()
+    n = 6000
+    wl = S.Workload(14, 0, [n], n_rows=300, q_start=n - 300, cli=1)
+    d = _upload(wl)
+    k_off = d["k_off"] if streaming else None
+    seq = torch.zeros(300, dtype=torch.int32, device="cuda") if streaming else None
+    scores = torch.empty((300, n), device="cuda")
+    hist = L.topk_hist_buffer(300)
+    L.index_scores(cfg, seq, d["pos"], d["q_idx"], d["w"], d["k_idx"], k_off, n, scores, topk_hist=hist)
+    ws = L.workspace(cfg, L.OP_TOPK, 300, 1, n)
+    outs = []
+    for h in (hist, None):
+        idx = torch.full((300, 2048), -3, dtype=torch.int32, device="cuda")
+        cnt = torch.full((300,), -3, dtype=torch.int32, device="cuda")
+        L.topk(cfg, d["pos"], n, scores, idx, cnt, ws, topk_hist=h)
+        outs.append((np.sort(idx.cpu().numpy(), axis=1), cnt.cpu().numpy()))
+    np.testing.assert_array_equal(outs[0][0], outs[1][0])
+    np.testing.assert_array_equal(outs[0][1], outs[1][1])
+    assert L.device_error() == 0
+
+
 def test_topk_tiny_config_brute(L):
     cfg = L.LsaConfig(index_topk=8, index_init_tokens=2, index_local_tokens=4)
     ocfg = oracle_cfg(cfg)
