@@ -6,9 +6,9 @@ Each case draws its inputs on the device (a few GB at most, inputs larger than
 L2 where the kernel streams from HBM), runs one entry point --reps times on the
 current stream, checks the device error flags and exits. Cases:
 
-  index_decode   lsa_index_scores, 16 rows x 131072 keys (one 128K decode layer)
+  index_decode   lsa_index_scores with the top-k histogram, 16 rows x 131072 keys (one 128K decode layer)
   index_prefill  lsa_index_scores, 16384 causal rows over 16384 keys
-  topk_decode    lsa_topk on 16 rows x 131072 scores
+  topk_decode    lsa_topk on 16 rows x 131072 scores, with the indexer's histogram
   mla_decode     lsa_sparse_mla_decode, 16 rows x 2048 selected keys of 131072
   mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
 """
@@ -31,11 +31,14 @@ def _decode_layer(draw_latent):
 
 
 def case_index_decode(reps):
+    # as the decode step runs it: the scores and the top-k's first radix pass
     cfg = lsa.LsaConfig()
     wl = _decode_layer(False)
     scores = torch.empty((16, 131072), device="cuda")
+    hist = lsa.topk_hist_buffer(16)
     for _ in range(reps):
-        lsa.index_scores(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, 131072, scores)
+        lsa.index_scores(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, 131072, scores,
+                         topk_hist=hist)
 
 
 def case_index_prefill(reps):
@@ -51,12 +54,14 @@ def case_topk_decode(reps):
     cfg = lsa.LsaConfig()
     wl = _decode_layer(False)
     scores = torch.empty((16, 131072), device="cuda")
-    lsa.index_scores(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, 131072, scores)
+    hist = lsa.topk_hist_buffer(16)
+    lsa.index_scores(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, 131072, scores,
+                     topk_hist=hist)
     idx = torch.empty((16, 2048), dtype=torch.int32, device="cuda")
     cnt = torch.empty((16,), dtype=torch.int32, device="cuda")
     ws = lsa.workspace(cfg, lsa.OP_TOPK, 16, 16, 131072)
     for _ in range(reps):
-        lsa.topk(cfg, wl.pos, 131072, scores, idx, cnt, ws)
+        lsa.topk(cfg, wl.pos, 131072, scores, idx, cnt, ws, topk_hist=hist)
 
 
 def case_mla_decode(reps):

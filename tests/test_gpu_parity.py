@@ -353,6 +353,31 @@ def test_mla_decode_on_selection(L):
             assert_attention(o[r], l[r], exp[r][0], exp[r][1], where=f"row {r} ws={use_ws}")
 
 
+def test_mla_rising_logits_rescale(L):
+    # logits that keep rising from tile to tile by far more than 2^8 force the
+    # attention kernel to rescale its running output; the oracle is exact fp64
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(17)
+    n = 2048
+    c = (rng.standard_normal((n, 576)) * 0.1).astype(np.float32)
+    c[:, 0] = np.linspace(-40.0, 60.0, n)                      # logit driver along dim 0
+    perm = rng.permutation(n)                                   # rising within the list order too
+    q = (rng.standard_normal((32, 576)) * 0.05).astype(np.float32)
+    q[:, 0] = 12.0
+    c_bits, q_bits = S.f32_to_bf16_bits(c), S.f32_to_bf16_bits(q)
+    idx = np.full((1, 2048), -1, dtype=np.int32)
+    idx[0] = np.sort(perm)                                      # ascending = rising logits
+    out = torch.empty((1, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((1, 32), device="cuda")
+    for ws in (None, L.workspace(cfg, L.OP_MLA_DECODE, 1, 1, n)):
+        L.sparse_mla_decode(cfg, bf16_dev(q_bits[None]), bf16_dev(c_bits), i64_dev(np.array([0, n])),
+                            i32_dev(idx), i32_dev(np.array([2048])), n, out, lse, ws)
+        assert L.device_error() == 0
+        eo, el = R.mla(S.bf16_bits_to_f64(q_bits), S.bf16_bits_to_f64(c_bits), ocfg)
+        assert_attention(bf16_host_f64(out)[0], lse.cpu().numpy()[0], eo, el)
+
+
 def test_mla_decode_dense(L):
     cfg = L.LsaConfig(cli_factor=1)
     ocfg = oracle_cfg(cfg)
