@@ -24,7 +24,6 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "launch.h"
-#include "tc.cuh"
 
 namespace lsa {
 namespace {
@@ -336,338 +335,6 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   }
 }
 
-// ---------------------------------------------------------------------------
-// Tensor-core (tcgen05) form. Per CTA: one (row, split, sub-block).
-//  * Gathered keys: 64 per tile, double-buffered; each tile is nine 64-dim
-//    blocks of [64 keys x 128 B] in the 128-byte-swizzled layout. The same
-//    bytes are the K-major B operand of S = Q K^T (N = keys, K = dims) and the
-//    MN-major B operand of O += P V (N = dims, K = keys).
-//  * S = Q K^T: M = 64 (the 32 heads; rows 32-63 are padding whose operand rows
-//    alias the next shared-memory block and whose results are never read),
-//    N = 64 keys, K = 576: 36 MMAs into tensor memory.
-//  * Softmax: one thread per head reads its 64 logits from tensor memory, so
-//    the max and the sum stay in-thread. The running reference max moves only
-//    when a tile's max exceeds it by more than 8 (base 2); then O is rescaled
-//    in tensor memory. P (bf16, 64 x 64) goes to shared memory (swizzled).
-//  * O += P V: M = 64, N = 256 (x2), K = 16 (x4) into 512 fp32 columns.
-//  Tensor memory: O in the lower half of every 32-lane subpartition (the M=64
-//  layout), S in the upper half. Warps: 0-1 softmax (lanes 16-31) and O owners
-//  (lanes 0-15); 2, 3, 5, 6 gather (cp.async, then a proxy fence and an
-//  mbarrier arrive); 4 allocates tensor memory and issues the MMAs.
-constexpr int kTcTK = 64;
-constexpr int kTcThreads = 7 * 32;
-constexpr uint32_t kTcKBlock = kTcTK * 128;          // 8 KB: 64 keys x 64 dims
-constexpr uint32_t kTcKTile = 9 * kTcKBlock;         // 72 KB
-constexpr uint32_t kTcQBlock = 32 * 128;             // 4 KB: 32 heads x 64 dims
-constexpr uint32_t kTcPBytes = 64 * 128;             // 8 KB: 64 rows x 64 keys
-constexpr uint32_t kIdescS = (1u << 4) | (1u << 7) | (1u << 10) | ((64u >> 3) << 17) | ((64u >> 4) << 24);
-constexpr uint32_t kIdescPV =
-    (1u << 4) | (1u << 7) | (1u << 10) | (1u << 16) | ((256u >> 3) << 17) | ((64u >> 4) << 24);
-
-struct __align__(1024) TcSmem {
-  uint8_t k[2][kTcKTile];
-  uint8_t q[9 * kTcQBlock];  // the last block's padding rows alias p[0]
-  uint8_t p[2][kTcPBytes];
-  int32_t list[kMaxSplitKeys];
-  uint64_t kfull[2], kempty[2], pfull[2], pvd[2], sfull;
-  uint32_t tmem_base;
-  int abort_flag;
-};
-
-__global__ void __launch_bounds__(kTcThreads, 1) mla_tc_kernel(MlaArgs a, Split sp, float* part_o,
-                                                                 float2* part_ml) {
-  extern __shared__ __align__(1024) unsigned char smem_raw[];
-  if ((smem_u32(smem_raw) & 1023u) != 0) {
-    if (threadIdx.x == 0) flag_error(a.err, LSA_DEVERR_TIMEOUT);
-    return;
-  }
-  TcSmem& sm = *reinterpret_cast<TcSmem*>(smem_raw);
-  const int s = blockIdx.x, r = blockIdx.y, z = blockIdx.z;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  pdl_wait();
-
-  // ---- row geometry (clamped and flagged, never faulting) ----
-  int64_t kbase = 0, nvis = 0;
-  if (a.decode) {
-    const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
-    if (seq < 0 || seq >= a.n_seq) {
-      if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_SEQ);
-    } else {
-      kbase = a.k_off[seq];
-      const int64_t klen = a.k_off[seq + 1] - kbase;
-      nvis = klen;
-      if (a.pos) {
-        int64_t p1 = (int64_t)a.pos[r] + 1;
-        if (p1 < 1 || p1 > klen) {
-          if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_POS);
-          p1 = max64(0, min64(p1, klen));
-        }
-        nvis = p1;
-      }
-    }
-  } else {
-    int64_t p1 = (int64_t)a.pos[r] + 1;
-    if (p1 < 1 || p1 > a.n_keys) {
-      if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_POS);
-      p1 = max64(0, min64(p1, a.n_keys));
-    }
-    nvis = p1;
-  }
-  int64_t n_list = nvis;
-  if (a.idx) {
-    int c = a.count[r];
-    if (c < 0 || c > a.topk) {
-      if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_COUNT);
-      c = max(0, min(c, a.topk));
-    }
-    n_list = c;
-  }
-  const int64_t b0 = (int64_t)s * sp.split_keys;
-  const int nk = (int)max64(0, min64(sp.split_keys, n_list - b0));
-  for (int i = tid; i < nk; i += kTcThreads) {
-    int64_t key = a.idx ? (int64_t)a.idx[(int64_t)r * a.topk + b0 + i] : b0 + i;
-    if (key < 0 || key >= nvis) {
-      flag_error(a.err, LSA_DEVERR_INDEX);
-      key = -1;
-    }
-    sm.list[i] = (int32_t)key;
-  }
-  // Q: 32 heads x 576 dims into nine swizzled 32-row blocks.
-  const uint16_t* __restrict__ qg = a.q[z] + (int64_t)r * kH * kDLat;
-  for (int c = tid; c < kH * 72; c += kTcThreads) {
-    const int h = c / 72, cg = c % 72, kb = cg >> 3, cc = cg & 7;
-    cp_async16(smem_u32(sm.q + kb * kTcQBlock + h * 128 + ((cc ^ (h & 7)) << 4)), qg + h * kDLat + cg * 8, 16);
-  }
-  cp_async_commit();
-  if (tid == 0) {
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sm.kfull[i], 128);
-      mbar_init(&sm.kempty[i], 1);
-      mbar_init(&sm.pfull[i], 2);
-      mbar_init(&sm.pvd[i], 1);
-    }
-    mbar_init(&sm.sfull, 1);
-    sm.abort_flag = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
-  }
-  cp_async_wait<0>();
-  fence_proxy_async();
-  if (warp == 4) tmem_alloc(&sm.tmem_base, 512);
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = sm.tmem_base;
-  volatile int* abort_flag = &sm.abort_flag;
-  const int n_tiles = (nk + kTcTK - 1) / kTcTK;
-  const uint16_t* __restrict__ latb = a.lat[z] + kbase * kDLat;
-  const float scale_log2 = a.scale * kLog2e;
-
-  if (warp == 2 || warp == 3 || warp == 5 || warp == 6) {
-    // ---------------- gather producers ----------------
-    const int ptid = (warp < 4 ? warp - 2 : warp - 3) * 32 + lane;  // 0..127
-    for (int t = 0; t < n_tiles; ++t) {
-      const int b = t & 1;
-      if (t >= 2 && !mbar_wait(&sm.kempty[b], ((t >> 1) - 1) & 1, abort_flag)) break;
-      uint8_t* dst = sm.k[b];
-#pragma unroll 4
-      for (int u = 0; u < 36; ++u) {
-        const int qd = ptid + 128 * u;  // 64 keys x 72 chunks
-        const int row = qd / 72, cg = qd % 72, kb = cg >> 3, cc = cg & 7;
-        const int slot = t * kTcTK + row;
-        const int key = slot < nk ? sm.list[slot] : -1;
-        const uint16_t* src = key >= 0 ? latb + (int64_t)key * kDLat + cg * 8 : a.lat[z];
-        cp_async16(smem_u32(dst + kb * kTcKBlock + row * 128 + ((cc ^ (row & 7)) << 4)), src, key >= 0 ? 16 : 0);
-      }
-      cp_async_commit();
-      cp_async_wait<0>();
-      fence_proxy_async();
-      mbar_arrive(&sm.kfull[b]);
-    }
-  } else if (warp == 4) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0 && n_tiles > 0) {
-      const uint32_t q_base = smem_u32(sm.q);
-      const uint32_t d_s = tmem + (16u << 16);
-      auto issue_s = [&](int t) -> bool {
-        const int b = t & 1;
-        if (!mbar_wait(&sm.kfull[b], (t >> 1) & 1, abort_flag)) return false;
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(sm.k[b]);
-#pragma unroll 4
-        for (int ks = 0; ks < 36; ++ks) {
-          const int kb = ks >> 2;
-          const uint32_t off = (ks & 3) * 32;
-          umma_f16(d_s, sw128_desc(q_base + kb * kTcQBlock + off), sw128_desc(k_base + kb * kTcKBlock + off),
-                   kIdescS, ks > 0 ? 1u : 0u);
-        }
-        umma_commit(&sm.sfull);
-        return true;
-      };
-      bool ok = issue_s(0);
-      for (int t = 0; ok && t < n_tiles; ++t) {
-        const int b = t & 1;
-        if (!mbar_wait(&sm.pfull[b], (t >> 1) & 1, abort_flag)) break;
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(sm.k[b]);
-        const uint32_t p_base = smem_u32(sm.p[b]);
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-#pragma unroll
-          for (int nh = 0; nh < 2; ++nh)
-            umma_f16(tmem + nh * 256, sw128_desc(p_base + ks * 32),
-                     sw128_mn_desc(k_base + nh * 4 * kTcKBlock + ks * 2048, kTcKBlock), kIdescPV,
-                     (t > 0 || ks > 0) ? 1u : 0u);
-        umma_commit(&sm.kempty[b]);
-        umma_commit(&sm.pvd[b]);
-        if (t + 1 < n_tiles) ok = issue_s(t + 1);
-      }
-    }
-  } else if (warp < 2) {
-    // ---------------- softmax (lanes 16-31) and O owners (lanes 0-15) ----------------
-    const bool smx = lane >= 16;
-    const int h = 16 * warp + (lane & 15);
-    const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-    float m_ref = -INFINITY, l = 0.f;
-    for (int t = 0; t < n_tiles; ++t) {
-      const int b = t & 1;
-      int ok = 1;
-      if (lane == 0) ok = mbar_wait(&sm.sfull, t & 1, abort_flag);
-      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-      tc_fence_after();
-      float x[64];
-      {
-        float v[32];
-        tmem_ld32(tmem + lane_base, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[i] = v[i];
-        tmem_ld32(tmem + lane_base + 32, v);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) x[32 + i] = v[i];
-      }
-      // (x holds O columns 0-63 in lanes 0-15; only lanes 16-31 use it)
-      float mt = -INFINITY;
-#pragma unroll
-      for (int i = 0; i < 64; ++i) {
-        const int slot = t * kTcTK + i;
-        const bool valid = slot < nk && sm.list[slot] >= 0;
-        x[i] = valid ? x[i] * scale_log2 : -INFINITY;
-        mt = fmaxf(mt, x[i]);
-      }
-      // The reference max moves only when a tile's max exceeds it by more than 8
-      // (base 2), so P stays below 2^8 and O is rescaled rarely.
-      bool need = false;
-      float alpha = 1.f;
-      if (smx) {
-        if (t == 0) {
-          m_ref = mt;
-        } else if (mt > m_ref + 8.f) {
-          alpha = (m_ref == -INFINITY) ? 0.f : exp2f(m_ref - mt);
-          m_ref = mt;
-          l *= alpha;
-          need = true;
-        }
-      }
-      if (t > 0 && __any_sync(0xffffffffu, need)) {
-        // O must hold tiles 0..t-1 completely before it is rescaled in place
-        int ok2 = 1;
-        if (lane == 0) ok2 = mbar_wait(&sm.pvd[(t - 1) & 1], ((t - 1) >> 1) & 1, abort_flag);
-        if (!__shfl_sync(0xffffffffu, ok2, 0)) break;
-        tc_fence_after();
-        const float al_o = __shfl_sync(0xffffffffu, alpha, (lane & 15) + 16);
-        const float al = smx ? 1.f : al_o;  // lanes 16-31 write back what they read (S, consumed)
-        for (int c = 0; c < 512; c += 32) {
-          float v[32];
-          tmem_ld32(tmem + lane_base + c, v);
-#pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] *= al;
-          tmem_st32(tmem + lane_base + c, v);
-        }
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-      float ps = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int i = 0; i < 32; ++i) {
-        const float p0 = exp2f(x[2 * i] - m_use), p1 = exp2f(x[2 * i + 1] - m_use);
-        ps += p0 + p1;
-        pk[i] = pack_bf16x2(p0, p1);
-      }
-      if (smx) l += ps;
-      // P buffer b is free once O += P V of tile t-2 completed
-      if (t >= 2) {
-        int ok3 = 1;
-        if (lane == 0) ok3 = mbar_wait(&sm.pvd[b], ((t >> 1) - 1) & 1, abort_flag);
-        if (!__shfl_sync(0xffffffffu, ok3, 0)) break;
-      }
-      if (smx) {
-        uint8_t* prow = sm.p[b] + (lane - 16 + 16 * warp) * 128;
-        const int hh = h & 7;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4*>(prow + ((c ^ hh) << 4)) = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      fence_proxy_async();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.pfull[b]);
-    }
-    // ---- epilogue: O complete after the last tile's O += P V ----
-    if (!*abort_flag) {
-      int ok4 = 1;
-      if (n_tiles > 0 && lane == 0) ok4 = mbar_wait(&sm.pvd[(n_tiles - 1) & 1], ((n_tiles - 1) >> 1) & 1, abort_flag);
-      ok4 = __shfl_sync(0xffffffffu, ok4, 0);
-      tc_fence_after();
-      const float l_o = __shfl_sync(0xffffffffu, l, (lane & 15) + 16);
-      const float m_o = __shfl_sync(0xffffffffu, m_ref, (lane & 15) + 16);
-      if (ok4) {
-        if (sp.n_split == 1) {
-          uint16_t* __restrict__ og = a.out[z] + ((int64_t)r * kH + h) * kDV;
-          const float inv = l_o > 0.f ? 1.f / l_o : 0.f;
-          for (int c = 0; c < 512; c += 32) {
-            float v[32];
-            if (n_tiles > 0) tmem_ld32(tmem + lane_base + c, v);
-            else
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = 0.f;
-            if (!smx) {
-#pragma unroll
-              for (int i = 0; i < 32; i += 8)
-                *reinterpret_cast<uint4*>(og + c + i) =
-                    make_uint4(pack_bf16x2(v[i] * inv, v[i + 1] * inv), pack_bf16x2(v[i + 2] * inv, v[i + 3] * inv),
-                               pack_bf16x2(v[i + 4] * inv, v[i + 5] * inv), pack_bf16x2(v[i + 6] * inv, v[i + 7] * inv));
-            }
-          }
-          if (!smx && a.lse[z])
-            a.lse[z][(int64_t)r * kH + h] = l_o > 0.f ? (m_o + log2f(l_o)) * kLn2 : -INFINITY;
-        } else {
-          const int64_t base = ((int64_t)z * a.n_rows + r) * sp.n_split + s;
-          float* __restrict__ po = part_o + (base * kH + h) * kDV;
-          for (int c = 0; c < 512; c += 32) {
-            float v[32];
-            if (n_tiles > 0) tmem_ld32(tmem + lane_base + c, v);
-            else
-#pragma unroll
-              for (int i = 0; i < 32; ++i) v[i] = 0.f;
-            if (!smx)
-#pragma unroll
-              for (int i = 0; i < 32; i += 4)
-                *reinterpret_cast<float4*>(po + c + i) = make_float4(v[i], v[i + 1], v[i + 2], v[i + 3]);
-          }
-          if (!smx) part_ml[base * kH + h] = make_float2(n_tiles > 0 ? m_o : -INFINITY, n_tiles > 0 ? l_o : 0.f);
-        }
-      }
-    }
-  }
-  if (*abort_flag && tid == 0) flag_error(a.err, LSA_DEVERR_TIMEOUT);
-  pdl_trigger();
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 4) {
-    tc_fence_after();
-    tmem_dealloc(tmem, 512);
-  }
-}
-
 // One CTA per (head, row, sub-block): 128 threads x 4 value dims, so that a
 // small decode batch still spreads the merge over many SMs.
 __global__ void __launch_bounds__(128) mla_merge_kernel(MlaArgs a, Split sp, const float* part_o,
@@ -757,8 +424,8 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(mla_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)sizeof(TcSmem));
+    cudaError_t e = cudaFuncSetAttribute(mla_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)sizeof(MlaSmem));
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
@@ -786,8 +453,8 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
       b.k_off = a.k_off + row0;
       b.n_seq = a.n_seq - row0;
     }
-    cudaError_t e = launch_pdl(mla_tc_kernel, dim3(n_split, nr, a.cli), dim3(kTcThreads), sizeof(TcSmem), st, b,
-                               sp, part_o, part_ml);
+    cudaError_t e = launch_pdl(mla_kernel, dim3(n_split, nr, a.cli), dim3(kThreads), sizeof(MlaSmem), st, b, sp,
+                               part_o, part_ml);
     if (e != cudaSuccess) return e;
     if (n_split > 1) {
       e = launch_pdl(mla_merge_kernel, dim3(kH, nr, a.cli), dim3(128), 0, st, b, sp, (const float*)part_o,
