@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(kHistThreads)
 constexpr int kPerThread = kChunk / kHistThreads;  // 16 scores per thread
 static_assert(kPerThread == 2 * kUnroll, "two rounds of kUnroll loads per thread");
 
-__global__ void __launch_bounds__(kHistThreads)
+__global__ void __launch_bounds__(kHistThreads, 4)
     topk_select_kernel(TopkArgs a, int row0, HistCtl* hc, uint64_t* cand_all) {
   __shared__ uint32_t h[kBins];
   __shared__ uint64_t scand[kTopkCap];
@@ -122,6 +122,17 @@ __global__ void __launch_bounds__(kHistThreads)
   const uint32_t n_chunks = (uint32_t)((g.hi - g.lo + kChunk - 1) / kChunk);
   HistCtl& w = hc[blockIdx.y];
   uint64_t* __restrict__ cand = cand_all + (int64_t)blockIdx.y * kTopkCap;
+  // This chunk's scores are requested first; the histogram and the threshold
+  // search overlap their latency.
+  const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
+  const int lane = tid & 31, warp = tid >> 5;
+  const int64_t wbase = s + warp * 32 * kUnroll;  // the second round adds kHistThreads * kUnroll
+  float sv[kPerThread];
+#pragma unroll
+  for (int i = 0; i < kPerThread; ++i) {
+    const int64_t j = wbase + (i / kUnroll) * kHistThreads * kUnroll + lane + 32 * (i % kUnroll);
+    sv[i] = j < e ? srow[j] : 0.f;
+  }
   const uint32_t* hsrc = a.hist_ext ? a.hist_ext + (int64_t)r * kTopkHistStride : w.hist;
   for (int i = tid; i < kBins; i += kHistThreads) h[i] = hsrc[i];
   __syncthreads();
@@ -129,23 +140,17 @@ __global__ void __launch_bounds__(kHistThreads)
   int bin;
   uint32_t above;
   find_threshold<kHistThreads>(h, k_rem, bin, above, &s_bin, &s_above, s_warp);
-  const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
-  const int lane = tid & 31, warp = tid >> 5;
-  const int64_t wbase = s + warp * 32 * kUnroll;  // the second round adds kHistThreads * kUnroll
-  uint32_t key[kPerThread];
-  int kb[kPerThread];
-#pragma unroll
-  for (int i = 0; i < kPerThread; ++i) {
+  // bin of each score; -1 marks positions past the chunk's end
+  auto kbin = [&](int i) -> int {
     const int64_t j = wbase + (i / kUnroll) * kHistThreads * kUnroll + lane + 32 * (i % kUnroll);
-    const float v = j < e ? srow[j] : 0.f;
-    key[i] = score_key(v);
-    kb[i] = j < e ? (int)(key[i] >> 21) : -1;
-  }
+    return j < e ? (int)(score_key(sv[i]) >> 21) : -1;
+  };
   uint32_t nu = 0, ne = 0;
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
-    nu += kb[i] > bin;
-    ne += kb[i] == bin;
+    const int kb = kbin(i);
+    nu += kb > bin;
+    ne += kb == bin;
   }
   // exclusive prefix sums over the CTA (warp scans, then the warp totals)
   uint32_t iu = nu, ie = ne;
@@ -182,11 +187,13 @@ __global__ void __launch_bounds__(kHistThreads)
 #pragma unroll
   for (int i = 0; i < kPerThread; ++i) {
     const int64_t j = wbase + (i / kUnroll) * kHistThreads * kUnroll + lane + 32 * (i % kUnroll);
-    if (kb[i] > bin) {
+    const int kb = kbin(i);
+    if (kb > bin) {
       if (ou < k_rem) mid[ou] = (int32_t)j;
       ++ou;
-    } else if (kb[i] == bin) {
-      if (oe < (uint32_t)kTopkCap) cand[oe] = ((uint64_t)key[i] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+    } else if (kb == bin) {
+      if (oe < (uint32_t)kTopkCap)
+        cand[oe] = ((uint64_t)score_key(sv[i]) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
       ++oe;
     }
   }

@@ -395,6 +395,26 @@ def test_mla_decode_dense(L):
         assert_attention(o[r], l[r], eo, el, where=f"row {r}")
 
 
+def test_mla_decode_dense_many_splits(L):
+    # a long dense list splits beyond one cluster (more than 8 CTAs per row), so
+    # the partials go through the workspace and the merge kernel
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    lengths = [20000, 9000]
+    wl = S.Workload(18, 0, lengths, cli=1)
+    d = _upload(wl)
+    out = torch.empty((2, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((2, 32), device="cuda")
+    ws = L.workspace(cfg, L.OP_MLA_DECODE, 2, 2, max(lengths))
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], None, None, max(lengths), out, lse, ws)
+    assert L.device_error() == 0
+    o, l = bf16_host_f64(out), lse.cpu().numpy()
+    for r in range(2):
+        _, _, _, qa, lat = host_rows(wl, r)
+        eo, el = R.dense_mla_row(qa[0], lat[0], lengths[r] - 1, ocfg)
+        assert_attention(o[r], l[r], eo, el, where=f"row {r}")
+
+
 def test_mla_prefill_on_selection(L):
     cfg = L.LsaConfig(cli_factor=1)
     ocfg = oracle_cfg(cfg)
