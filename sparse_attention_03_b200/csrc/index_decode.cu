@@ -191,14 +191,28 @@ __global__ void __launch_bounds__(kThreads, 3)
 
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st, uint32_t* hist, int topk) {
   if (a.n_rows <= 0) return cudaSuccess;
-  // Keys per CTA: a multiple of one CTA pass (64 keys), large enough to amortise
-  // the query-fragment load, small enough to give every SM several CTAs.
-  int sms = 148;
+  // One wave: as many CTAs as the SMs hold at once (a second, partial wave of
+  // these short-lived CTAs costs more than the larger per-CTA key range saves).
+  // Keys per CTA are a multiple of one CTA pass (64 keys), at least 256 so the
+  // query-fragment load is amortised, and at most 8192.
+  // Cached per device (a benign race: every thread writes the same values).
+  static int cache_sms[64], cache_occ[64];
   int dev = 0;
-  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t target_ctas = (int64_t)sms * 6;
-  int64_t kpc = (a.max_len * a.n_rows + target_ctas - 1) / target_ctas;
-  kpc = ((kpc + 255) / 256) * 256;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) dev = 0;
+  if (cache_sms[dev] == 0) {
+    int s = 148, o = 3;
+    cudaDeviceGetAttribute(&s, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&o, index_decode_kernel<true>, kThreads, 0) != cudaSuccess ||
+        o < 1)
+      o = 3;
+    cache_occ[dev] = o;
+    cache_sms[dev] = s;
+  }
+  const int sms = cache_sms[dev], occ = cache_occ[dev];
+  const int64_t wave = (int64_t)sms * occ;
+  const int64_t per_row = max64(1, wave / a.n_rows);
+  int64_t kpc = (a.max_len + per_row - 1) / per_row;
+  kpc = ((kpc + 63) / 64) * 64;
   kpc = max64(256, min64(kpc, 8192));
   const int64_t nx = (a.max_len + kpc - 1) / kpc;
   for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {

@@ -9,70 +9,111 @@
 // same set. Both are computed here by gathering each row's selected keys, which
 // gives exactly the masked result without touching unselected keys.
 //
-// Design. One CTA (8 warps) handles one (query row, split of its key list,
-// sub-block). Latent rows are gathered by cp.async into a double-buffered
-// shared-memory tile of 64 keys (1152-byte rows padded to 1168 so ldmatrix is
-// conflict-free). S = Q K^T runs on mma.m16n8k16 with the 576-dim contraction
-// split four ways across warps: each warp keeps its quarter of Q in registers
-// for the whole CTA and runs eight independent accumulator chains, and the
-// partial logits are summed through shared memory. The online softmax is
-// base-2 and max-subtracted. O += P V runs with the 512 value dims split across
-// the warps (64 each, fp32 accumulators in registers). With more than one split
-// per row the CTA writes an unnormalised partial (O, m, l) and a merge kernel
-// combines the splits; with one split it writes bf16 output and lse directly.
-// Gathered indices are bounds-checked against the row's visible keys.
+// Design. One CTA handles one (query row, split of its key list, sub-block):
+// eight math warps and one producer warp. The producer gathers each selected
+// 1152-byte latent row with one bulk asynchronous copy per lane (the TMA engine
+// moves the bytes; no register staging) into a four-stage ring of 32-key tiles
+// (rows padded to 1168 bytes so ldmatrix is conflict-free); full/empty
+// mbarriers hand stages between producer and math warps, so three tiles are in
+// flight while one is computed. S = Q K^T runs on mma.m16n8k16 with the
+// 576-dim contraction split four ways across warps: each warp keeps its quarter
+// of Q in registers for the whole CTA, and the partial logits are summed through
+// shared memory. The online softmax is base-2 and max-subtracted. O += P V runs
+// with the 512 value dims split across the warps (64 each, fp32 accumulators in
+// registers). A row's key list is cut into splits of whole tiles, balanced per
+// row; with more than one split the CTA writes an unnormalised partial
+// (O, m, l) and a merge kernel combines the splits; with one split it writes
+// bf16 output and lse directly. Gathered indices are bounds-checked against the
+// row's visible keys; every wait is bounded.
 #include "common.cuh"
 #include "kernels.h"
 #include "launch.h"
+#include "tc.cuh"
 
 namespace lsa {
 namespace {
 
-constexpr int kTK = 64;             // keys per tile
+constexpr int kTK = 32;             // keys per tile
+constexpr int kStages = 4;          // tiles in the ring
 constexpr int kSRow = kDLat + 8;    // shared row stride (bf16): 1168 bytes
-constexpr int kPRow = kTK + 8;      // P row stride (bf16): 144 bytes
-constexpr int kMaxSplitKeys = 2048;
-constexpr int kThreads = 256;
+constexpr int kPRow = kTK + 8;      // P row stride (bf16): 80 bytes
+constexpr int kMathWarps = 8;
+constexpr int kMathThreads = kMathWarps * 32;
+constexpr int kThreads = kMathThreads + 32;  // + the producer warp
 constexpr int kMaxSplits = 32;
+constexpr int kRowBytes = kDLat * 2;  // 1152
 constexpr float kLn2 = 0.69314718055994530942f;
 constexpr float kLog2e = 1.44269504088896340736f;
 
-struct __align__(16) MlaSmem {
-  // Q staging at start; afterwards the per-warp partial logits
-  // [4 dim quarters][2 head halves][16 heads][kPartRow] fp32 (36864 B).
+constexpr int kPartRow = kTK + 8;   // fp32 row stride of the partial logits (conflict-free float2 stores)
+
+struct __align__(128) MlaSmem {
+  uint16_t k[kStages][kTK * kSRow];
+  // Q rows at start; afterwards the per-warp partial logits
+  // [4 dim quarters][2 head halves][16 heads][kPartRow] fp32.
   uint16_t q[kH * kSRow];
-  uint16_t k[2][kTK * kSRow];
   uint16_t p[kH * kPRow];
   float red_max[4][kH];
   float red_sum[4][kH];
   float alpha[kH];
   float fin_m[kH];
   float fin_l[kH];
-  int32_t list[kMaxSplitKeys];
+  int32_t keys[kStages][kTK];  // gathered key of each tile slot, -1 when masked
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  uint64_t qbar;
+  int abort_flag;
 };
-constexpr int kPartRow = 72;  // fp32 row stride of the partial logits (conflict-free float2 stores)
-static_assert(4 * 2 * 16 * kPartRow * 4 <= kH * kSRow * 2, "partial logits fit in the Q staging area");
+static_assert(4 * 2 * 16 * kPartRow * 4 <= kH * kSRow * 2, "partial logits fit in the Q area");
+static_assert((kSRow * 2) % 16 == 0 && kRowBytes % 16 == 0, "bulk copies need 16-byte rows");
 
 struct Split {
   int n_split;
-  int split_keys;
 };
 
-// Warp roles. Logits S = Q K^T (32 heads x 64 keys per tile, contraction 576):
-// warp w takes head half mt = w & 1 and dim quarter kq = w >> 1 (9 k16 steps);
-// its Q fragments stay in registers for the whole CTA and it runs 8 independent
-// accumulator chains (one per 8-key n-tile) of 9 MMAs. The four dim-quarter
-// partials meet in shared memory. Softmax: warp w owns head half mt and key
-// quarter kg = w >> 1; each lane one head and 8 keys. O += P V: warp w owns
-// value dims 64w .. 64w+63 for all 32 heads (16 accumulator tiles).
+__device__ __forceinline__ void bulk_row(void* dst, const void* src, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(kRowBytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+// A wait that ignores the abort flag, used once at exit so that no copy is
+// still in flight into this CTA's shared memory when it retires.
+__device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
+  const long long t0 = global_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (global_ns() - t0 > kWaitLimitNs) return;
+}
+
+// Named barrier over the eight math warps (the producer never joins it).
+__device__ __forceinline__ void math_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(kMathThreads) : "memory"); }
+
+// Warp roles (math warps 0..7). Logits S = Q K^T (32 heads x 32 keys per tile,
+// contraction 576): warp w takes head half mt = w & 1 and dim quarter
+// kq = w >> 1 (9 k16 steps), with its Q fragments in registers and four
+// accumulator chains (one per 8-key n-tile). The four dim-quarter partials meet
+// in shared memory. Softmax: warp w owns head half mt and key group kg = w >> 1
+// (8 keys); each lane one head and 4 keys. O += P V: warp w owns value dims
+// 64w .. 64w+63 for all 32 heads (16 accumulator tiles).
 __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, float* part_o,
                                                           float2* part_ml) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   MlaSmem& sm = *reinterpret_cast<MlaSmem*>(smem_raw);
   const int s = blockIdx.x, r = blockIdx.y, z = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = lane >> 2, t = lane & 3;
-  const int mt = warp & 1, kq = warp >> 1;
+  if (tid == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sm.full[i], 32);
+      mbar_init(&sm.empty[i], kMathWarps);
+    }
+    mbar_init(&sm.qbar, 32);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::);
+  }
+  __syncthreads();
+  volatile int* abort_flag = &sm.abort_flag;
   pdl_wait();
 
   // ---- row geometry (clamped and flagged, never faulting) ----
@@ -111,59 +152,84 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     }
     n_list = c;
   }
-  const int64_t b0 = (int64_t)s * sp.split_keys;
-  const int nk = (int)max64(0, min64(sp.split_keys, n_list - b0));
+  // This split's whole tiles of the row's list.
+  const int64_t row_tiles = (n_list + kTK - 1) / kTK;
+  const int64_t t_lo = row_tiles * s / sp.n_split, t_hi = row_tiles * (s + 1) / sp.n_split;
+  const int64_t b0 = t_lo * kTK, b_end = min64(t_hi * kTK, n_list);
+  const int n_tiles = (int)(t_hi - t_lo);
 
-  for (int i = tid; i < nk; i += kThreads) {
-    int64_t key = a.idx ? (int64_t)a.idx[(int64_t)r * a.topk + b0 + i] : b0 + i;
-    if (key < 0 || key >= nvis) {
-      flag_error(a.err, LSA_DEVERR_INDEX);
-      key = -1;
+  if (warp == kMathWarps) {
+    // ================= producer warp =================
+    const uint16_t* __restrict__ qg = a.q[z] + ((int64_t)r * kH + lane) * kDLat;
+    mbar_expect_tx(&sm.qbar, kRowBytes);
+    bulk_row(&sm.q[lane * kSRow], qg, &sm.qbar);
+    const uint16_t* __restrict__ latb = a.lat[z] + kbase * kDLat;
+    const int32_t* __restrict__ irow = a.idx ? a.idx + (int64_t)r * a.topk : nullptr;
+    auto load_key = [&](int tt) -> int {
+      const int64_t slot = b0 + (int64_t)tt * kTK + lane;
+      if (tt >= n_tiles || slot >= b_end) return -1;
+      const int64_t key = irow ? (int64_t)__ldg(irow + slot) : slot;
+      if (key < 0 || key >= nvis) {
+        flag_error(a.err, LSA_DEVERR_INDEX);
+        return -1;
+      }
+      return (int)key;
+    };
+    int kr[kStages];
+#pragma unroll
+    for (int i = 0; i < kStages; ++i) kr[i] = load_key(i);
+    for (int base = 0; base < n_tiles; base += kStages) {
+#pragma unroll
+      for (int i = 0; i < kStages; ++i) {
+        const int tt = base + i;
+        if (tt < n_tiles) {
+          const int key = kr[i];
+          kr[i] = load_key(tt + kStages);
+          if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag);
+          sm.keys[i][lane] = key;
+          uint16_t* dst = &sm.k[i][lane * kSRow];
+          if (key >= 0) {
+            mbar_expect_tx(&sm.full[i], kRowBytes);
+            bulk_row(dst, latb + (int64_t)key * kDLat, &sm.full[i]);
+          } else {
+            // a masked slot: zero row (its weight is exactly 0, and 0 * 0 stays finite)
+#pragma unroll 8
+            for (int c = 0; c < kDLat / 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = make_uint4(0, 0, 0, 0);
+            fence_proxy_async();
+            mbar_arrive(&sm.full[i]);
+          }
+        }
+      }
     }
-    sm.list[i] = (int32_t)key;
-  }
-  const uint16_t* __restrict__ qg = a.q[z] + (int64_t)r * kH * kDLat;
-  for (int c = tid; c < kH * (kDLat / 8); c += kThreads) {
-    const int h = c / (kDLat / 8), col = c % (kDLat / 8);
-    cp_async16(smem_u32(&sm.q[h * kSRow + col * 8]), qg + h * kDLat + col * 8, 16);
-  }
-  cp_async_commit();
-  __syncthreads();  // list visible
-
-  const uint16_t* __restrict__ latb = a.lat[z] + kbase * kDLat;
-  const int n_tiles = (nk + kTK - 1) / kTK;
-  // Warp w gathers tile rows [8w, 8w+8): 8 x 72 16-byte chunks, 18 per lane,
-  // consecutive lanes on consecutive chunks of a row.
-  auto issue_tile = [&](int tt) {
-    uint16_t* dst = sm.k[tt & 1];
-#pragma unroll 6
-    for (int u = 0; u < 18; ++u) {
-      const int qd = lane + 32 * u;
-      const int row = 8 * warp + qd / 72, col = qd % 72;
-      const int slot = tt * kTK + row;
-      const int key = slot < nk ? sm.list[slot] : -1;
-      const uint16_t* src = key >= 0 ? latb + (int64_t)key * kDLat + col * 8 : a.lat[z];
-      cp_async16(smem_u32(dst + row * kSRow + col * 8), src, key >= 0 ? 16 : 0);
+    // Retire only after every copy into this CTA's shared memory has landed.
+    if (lane == 0) {
+      mbar_drain(&sm.qbar, 0);
+      for (int i = 0; i < kStages && i < n_tiles; ++i) {
+        const int last = i + ((n_tiles - 1 - i) / kStages) * kStages;
+        mbar_drain(&sm.full[i], (last / kStages) & 1);
+      }
     }
-  };
-  if (n_tiles > 0) issue_tile(0);
-  cp_async_commit();
+    return;
+  }
 
+  // ================= math warps =================
+  const int g = lane >> 2, t = lane & 3;
+  const int mt = warp & 1, kq = warp >> 1;
+  mbar_wait(&sm.qbar, 0, abort_flag);
   // Q fragments of this warp: head half mt, k16 steps 9kq .. 9kq+8.
-  cp_async_wait<1>();
-  __syncthreads();
   uint32_t qf[9][4];
   {
     const uint32_t qa = smem_u32(&sm.q[(16 * mt + (lane & 15)) * kSRow + 8 * (lane >> 4)]) + 9 * kq * 32;
 #pragma unroll
     for (int ks = 0; ks < 9; ++ks) ldsm_x4(qa + ks * 32, qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3]);
   }
-  float* part = reinterpret_cast<float*>(sm.q);  // valid once every warp has its Q fragments
+  math_sync();  // every warp holds its Q fragments: the Q area becomes the partial logits
+  float* part = reinterpret_cast<float*>(sm.q);
 
   const float scale_log2 = a.scale * kLog2e;
   // softmax state for this lane's head (head half mt, head 16mt + (lane >> 1))
   const int sh = 16 * mt + (lane >> 1);
-  const int kg = warp >> 1, kb8 = 8 * (lane & 1);
+  const int kg = warp >> 1, kb4 = 8 * kg + 4 * (lane & 1);
   float m_run = -INFINITY, l_run = 0.f;
   // value accumulators: o[mtv][nt][4], heads 16mtv+g (+8), dims 64w + 8nt + 2t
   float o[2][8][4];
@@ -175,16 +241,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
       for (int j = 0; j < 4; ++j) o[i][nt][j] = 0.f;
 
   for (int tt = 0; tt < n_tiles; ++tt) {
-    cp_async_wait<0>();
-    __syncthreads();  // (1) tile tt landed; every warp finished O += P V of tile tt-1
-    if (tt + 1 < n_tiles) issue_tile(tt + 1);
-    cp_async_commit();
-    const uint16_t* kt = sm.k[tt & 1];
+    const int st = tt % kStages;
+    mbar_wait(&sm.full[st], (tt / kStages) & 1, abort_flag);
+    const uint16_t* kt = sm.k[st];
 
     // ---- partial logits over this warp's dim quarter ----
-    float sc[8][4];
+    float sc[4][4];
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+    for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
       for (int j = 0; j < 4; ++j) sc[nt][j] = 0.f;
     const uint32_t kb0 = smem_u32(&kt[((lane & 7) + 8 * (lane >> 4)) * kSRow + 8 * ((lane >> 3) & 1)]) +
@@ -192,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
 #pragma unroll
     for (int ks = 0; ks < 9; ++ks) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
+      for (int j = 0; j < 2; ++j) {
         uint32_t b[4];
         ldsm_x4(kb0 + (16 * j * kSRow) * 2 + ks * 32, b[0], b[1], b[2], b[3]);
         mma_16816(sc[2 * j], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b[0], b[1]);
@@ -202,57 +266,45 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     {
       float* pw = part + ((kq * 2 + mt) * 16) * kPartRow;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
+      for (int nt = 0; nt < 4; ++nt) {
         *reinterpret_cast<float2*>(&pw[g * kPartRow + 8 * nt + 2 * t]) = make_float2(sc[nt][0], sc[nt][1]);
         *reinterpret_cast<float2*>(&pw[(g + 8) * kPartRow + 8 * nt + 2 * t]) =
             make_float2(sc[nt][2], sc[nt][3]);
       }
     }
-    __syncthreads();  // (2) partials complete
+    math_sync();  // (1) partials complete
 
-    // ---- sum the partials, mask, tile max (lane: head sh, keys 16kg+kb8 .. +7) ----
-    float x[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) x[i] = 0.f;
+    // ---- sum the partials, mask, tile max (lane: head sh, keys kb4 .. kb4+3) ----
+    float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
-      const float* pr = part + ((q4 * 2 + mt) * 16 + (lane >> 1)) * kPartRow + 16 * kg + kb8;
-      const float4 v0 = *reinterpret_cast<const float4*>(pr);
-      const float4 v1 = *reinterpret_cast<const float4*>(pr + 4);
-      x[0] += v0.x; x[1] += v0.y; x[2] += v0.z; x[3] += v0.w;
-      x[4] += v1.x; x[5] += v1.y; x[6] += v1.z; x[7] += v1.w;
+      const float4 v = *reinterpret_cast<const float4*>(part + ((q4 * 2 + mt) * 16 + (lane >> 1)) * kPartRow + kb4);
+      x[0] += v.x; x[1] += v.y; x[2] += v.z; x[3] += v.w;
     }
     float mx = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int slot = tt * kTK + 16 * kg + kb8 + i;
-      const bool valid = slot < nk && sm.list[slot] >= 0;
-      x[i] = valid ? x[i] * scale_log2 : -INFINITY;
+    for (int i = 0; i < 4; ++i) {
+      x[i] = sm.keys[st][kb4 + i] >= 0 ? x[i] * scale_log2 : -INFINITY;
       mx = fmaxf(mx, x[i]);
     }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
     if ((lane & 1) == 0) sm.red_max[kg][sh] = mx;
-    __syncthreads();  // (3) tile maxima
+    math_sync();  // (2) tile maxima
     const float tmax = fmaxf(fmaxf(sm.red_max[0][sh], sm.red_max[1][sh]), fmaxf(sm.red_max[2][sh], sm.red_max[3][sh]));
     const float m_new = fmaxf(m_run, tmax);
     const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
     const float alpha = exp2f(m_run - m_use);
     m_run = m_new;
-    float ps = 0.f;
-    uint32_t pk[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float p0 = exp2f(x[2 * i] - m_use), p1 = exp2f(x[2 * i + 1] - m_use);
-      ps += p0 + p1;
-      pk[i] = pack_bf16x2(p0, p1);
-    }
-    *reinterpret_cast<uint4*>(&sm.p[sh * kPRow + 16 * kg + kb8]) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+    const float p0 = exp2f(x[0] - m_use), p1 = exp2f(x[1] - m_use);
+    const float p2 = exp2f(x[2] - m_use), p3 = exp2f(x[3] - m_use);
+    float ps = (p0 + p1) + (p2 + p3);
+    *reinterpret_cast<uint2*>(&sm.p[sh * kPRow + kb4]) = make_uint2(pack_bf16x2(p0, p1), pack_bf16x2(p2, p3));
     ps += __shfl_xor_sync(0xffffffffu, ps, 1);
     if ((lane & 1) == 0) {
       sm.red_sum[kg][sh] = ps;
       if (kg == 0) sm.alpha[sh] = alpha;
     }
-    __syncthreads();  // (4) P, alpha and tile sums ready
+    math_sync();  // (3) P, alpha and tile sums ready
     l_run = l_run * alpha +
             ((sm.red_sum[0][sh] + sm.red_sum[1][sh]) + (sm.red_sum[2][sh] + sm.red_sum[3][sh]));
 
@@ -274,27 +326,29 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
         smem_u32(&kt[((lane & 7) + 8 * ((lane >> 3) & 1)) * kSRow + 64 * warp + 8 * (lane >> 4)]);
 #pragma unroll
     for (int kk = 0; kk < kTK / 16; ++kk) {
-      uint32_t p0[4], p1[4];
-      ldsm_x4(pa0 + kk * 32, p0[0], p0[1], p0[2], p0[3]);
-      ldsm_x4(pa1 + kk * 32, p1[0], p1[1], p1[2], p1[3]);
+      uint32_t pf0[4], pf1[4];
+      ldsm_x4(pa0 + kk * 32, pf0[0], pf0[1], pf0[2], pf0[3]);
+      ldsm_x4(pa1 + kk * 32, pf1[0], pf1[1], pf1[2], pf1[3]);
 #pragma unroll
       for (int np = 0; np < 4; ++np) {
         uint32_t v[4];
         ldsm_x4_t(vb0 + (kk * 16 * kSRow + 16 * np) * 2, v[0], v[1], v[2], v[3]);
-        mma_16816(o[0][2 * np], p0[0], p0[1], p0[2], p0[3], v[0], v[1]);
-        mma_16816(o[0][2 * np + 1], p0[0], p0[1], p0[2], p0[3], v[2], v[3]);
-        mma_16816(o[1][2 * np], p1[0], p1[1], p1[2], p1[3], v[0], v[1]);
-        mma_16816(o[1][2 * np + 1], p1[0], p1[1], p1[2], p1[3], v[2], v[3]);
+        mma_16816(o[0][2 * np], pf0[0], pf0[1], pf0[2], pf0[3], v[0], v[1]);
+        mma_16816(o[0][2 * np + 1], pf0[0], pf0[1], pf0[2], pf0[3], v[2], v[3]);
+        mma_16816(o[1][2 * np], pf1[0], pf1[1], pf1[2], pf1[3], v[0], v[1]);
+        mma_16816(o[1][2 * np + 1], pf1[0], pf1[1], pf1[2], pf1[3], v[2], v[3]);
       }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.empty[st]);  // this warp is done with the stage
   }
-  cp_async_wait<0>();
   pdl_trigger();
   if (kg == 0 && (lane & 1) == 0) {
     sm.fin_m[sh] = m_run;
     sm.fin_l[sh] = l_run;
   }
-  __syncthreads();
+  math_sync();
+  if (tid == 0 && *abort_flag) flag_error(a.err, LSA_DEVERR_TIMEOUT);
 
   // ---- epilogue ----
   if (sp.n_split == 1) {
@@ -386,17 +440,15 @@ size_t mla_ws_bytes(int n_rows, int cli, int n_split) {
 }
 
 int mla_choose_splits(int n_rows, int cli, int64_t max_list) {
-  // Enough CTAs to cover the SMs about twice, splits of at least 256 keys,
-  // each split at most 2048 keys (the shared-memory index list).
+  // One wave at one CTA per SM: split the rows' key lists until the CTAs cover
+  // the SMs, keeping at least four tiles per split (the ring's depth) and at
+  // most kMaxSplits splits.
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t work = (int64_t)n_rows * cli;
-  int64_t by_len = (max_list + 255) / 256;
-  int64_t want = (2 * sms + work - 1) / max64(work, 1);
-  int64_t n = min(by_len, want);
-  const int64_t min_for_list = (max_list + kMaxSplitKeys - 1) / kMaxSplitKeys;
-  n = max(n, min_for_list);
+  const int64_t work = max64((int64_t)n_rows * cli, 1);
+  const int64_t by_len = (max_list + kStages * kTK - 1) / (kStages * kTK);
+  int64_t n = min64(by_len, sms / work);
   n = max64(1, min64(n, kMaxSplits));
   return (int)n;
 }
@@ -404,15 +456,10 @@ int mla_choose_splits(int n_rows, int cli, int64_t max_list) {
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
   if (a.n_rows <= 0) return cudaSuccess;
   int n_split = mla_choose_splits(a.n_rows, a.cli, a.max_list);
-  const int64_t min_for_list = (a.max_list + kMaxSplitKeys - 1) / kMaxSplitKeys;
-  // Shrink split-K to what the workspace holds (never below what the list needs).
-  while (n_split > 1 && n_split > min_for_list && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes)
-    --n_split;
-  if (n_split > 1 && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes) return cudaErrorInvalidValue;
+  // Shrink split-K to what the workspace holds.
+  while (n_split > 1 && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes) --n_split;
   Split sp;
   sp.n_split = n_split;
-  sp.split_keys = (int)(((a.max_list + n_split - 1) / n_split + kTK - 1) / kTK * kTK);
-  if (sp.split_keys > kMaxSplitKeys) return cudaErrorInvalidValue;
   float* part_o = nullptr;
   float2* part_ml = nullptr;
   if (n_split > 1) {
