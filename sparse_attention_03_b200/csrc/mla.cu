@@ -59,6 +59,7 @@ struct __align__(128) MlaSmem {
   float fin_m[kH];
   float fin_l[kH];
   int32_t keys[kStages][kTK];  // gathered key of each tile slot, -1 when masked
+  int32_t list[kMaxTopk];      // this split's validated keys
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t qbar;
@@ -69,6 +70,7 @@ static_assert((kSRow * 2) % 16 == 0 && kRowBytes % 16 == 0, "bulk copies need 16
 
 struct Split {
   int n_split;
+  int list_tiles;  // tiles of the longest key list (the split boundaries)
 };
 
 __device__ __forceinline__ void bulk_row(void* dst, const void* src, uint64_t* bar) {
@@ -87,16 +89,62 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
     if (global_ns() - t0 > kWaitLimitNs) return;
 }
 
-// Named barrier over the eight math warps (the producer never joins it).
+// Named barriers: 1 = the eight math warps, 2 + h = the four warps of head half h.
 __device__ __forceinline__ void math_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(kMathThreads) : "memory"); }
+__device__ __forceinline__ void half_sync(int h) { asm volatile("bar.sync %0, 128;\n" ::"r"(2 + h) : "memory"); }
 
-// Warp roles (math warps 0..7). Logits S = Q K^T (32 heads x 32 keys per tile,
-// contraction 576): warp w takes head half mt = w & 1 and dim quarter
-// kq = w >> 1 (9 k16 steps), with its Q fragments in registers and four
-// accumulator chains (one per 8-key n-tile). The four dim-quarter partials meet
-// in shared memory. Softmax: warp w owns head half mt and key group kg = w >> 1
-// (8 keys); each lane one head and 4 keys. O += P V: warp w owns value dims
-// 64w .. 64w+63 for all 32 heads (16 accumulator tiles).
+struct RowGeom {
+  int64_t kbase, nvis, n_list;
+};
+
+// Row geometry, with every out-of-range input clamped (and flagged by one thread).
+__device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool report) {
+  RowGeom g{0, 0, 0};
+  if (a.decode) {
+    const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
+    if (seq < 0 || seq >= a.n_seq) {
+      if (report) flag_error(a.err, LSA_DEVERR_SEQ);
+    } else {
+      g.kbase = a.k_off[seq];
+      const int64_t klen = a.k_off[seq + 1] - g.kbase;
+      g.nvis = klen;
+      if (a.pos) {
+        int64_t p1 = (int64_t)a.pos[r] + 1;
+        if (p1 < 1 || p1 > klen) {
+          if (report) flag_error(a.err, LSA_DEVERR_POS);
+          p1 = max64(0, min64(p1, klen));
+        }
+        g.nvis = p1;
+      }
+    }
+  } else {
+    int64_t p1 = (int64_t)a.pos[r] + 1;
+    if (p1 < 1 || p1 > a.n_keys) {
+      if (report) flag_error(a.err, LSA_DEVERR_POS);
+      p1 = max64(0, min64(p1, a.n_keys));
+    }
+    g.nvis = p1;
+  }
+  g.n_list = g.nvis;
+  if (a.idx) {
+    int c = a.count[r];
+    if (c < 0 || c > a.topk) {
+      if (report) flag_error(a.err, LSA_DEVERR_COUNT);
+      c = max(0, min(c, a.topk));
+    }
+    g.n_list = c;
+  }
+  return g;
+}
+
+// Warp roles (math warps 0..7): head half mt = w >> 2 (heads 16mt .. 16mt+15)
+// and quarter kq = w & 3, so each SM sub-partition runs one warp of each half
+// and the two halves, which share nothing but the key tiles, drift apart and
+// overlap one half's softmax with the other's MMAs. Logits: warp w contracts
+// dim quarter kq (9 k16 steps) for its 16 heads x 32 keys, Q fragments in
+// registers, two accumulator chains per 8-key n-tile; the four quarters meet in
+// shared memory. Softmax: warp w owns key group kq (8 keys); each lane one head
+// and 4 keys. O += P V: warp w owns value dims 128kq .. 128kq+127 of its heads.
 __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, float* part_o,
                                                           float2* part_ml) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -116,75 +164,64 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   volatile int* abort_flag = &sm.abort_flag;
   pdl_wait();
 
-  // ---- row geometry (clamped and flagged, never faulting) ----
-  int64_t kbase = 0, nvis = 0;
-  if (a.decode) {
-    const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
-    if (seq < 0 || seq >= a.n_seq) {
-      if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_SEQ);
-    } else {
-      kbase = a.k_off[seq];
-      const int64_t klen = a.k_off[seq + 1] - kbase;
-      nvis = klen;
-      if (a.pos) {
-        int64_t p1 = (int64_t)a.pos[r] + 1;
-        if (p1 < 1 || p1 > klen) {
-          if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_POS);
-          p1 = max64(0, min64(p1, klen));
-        }
-        nvis = p1;
-      }
-    }
-  } else {
-    int64_t p1 = (int64_t)a.pos[r] + 1;
-    if (p1 < 1 || p1 > a.n_keys) {
-      if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_POS);
-      p1 = max64(0, min64(p1, a.n_keys));
-    }
-    nvis = p1;
-  }
-  int64_t n_list = nvis;
-  if (a.idx) {
-    int c = a.count[r];
-    if (c < 0 || c > a.topk) {
-      if (s == 0 && tid == 0) flag_error(a.err, LSA_DEVERR_COUNT);
-      c = max(0, min(c, a.topk));
-    }
-    n_list = c;
-  }
-  // This split's whole tiles of the row's list.
-  const int64_t row_tiles = (n_list + kTK - 1) / kTK;
-  const int64_t t_lo = row_tiles * s / sp.n_split, t_hi = row_tiles * (s + 1) / sp.n_split;
-  const int64_t b0 = t_lo * kTK, b_end = min64(t_hi * kTK, n_list);
-  const int n_tiles = (int)(t_hi - t_lo);
+  // This split's slots: whole tiles of the longest list, clipped to the row's own.
+  const int64_t t_lo = (int64_t)sp.list_tiles * s / sp.n_split;
+  const int64_t t_hi = (int64_t)sp.list_tiles * (s + 1) / sp.n_split;
+  const int64_t b0 = t_lo * kTK;
+  const int cap = (int)((t_hi - t_lo) * kTK);
 
   if (warp == kMathWarps) {
     // ================= producer warp =================
+    // Q and the first indices go out before the row geometry is known.
     const uint16_t* __restrict__ qg = a.q[z] + ((int64_t)r * kH + lane) * kDLat;
     mbar_expect_tx(&sm.qbar, kRowBytes);
     bulk_row(&sm.q[lane * kSRow], qg, &sm.qbar);
-    const uint16_t* __restrict__ latb = a.lat[z] + kbase * kDLat;
-    const int32_t* __restrict__ irow = a.idx ? a.idx + (int64_t)r * a.topk : nullptr;
-    auto load_key = [&](int tt) -> int {
-      const int64_t slot = b0 + (int64_t)tt * kTK + lane;
-      if (tt >= n_tiles || slot >= b_end) return -1;
-      const int64_t key = irow ? (int64_t)__ldg(irow + slot) : slot;
-      if (key < 0 || key >= nvis) {
-        flag_error(a.err, LSA_DEVERR_INDEX);
-        return -1;
-      }
-      return (int)key;
-    };
-    int kr[kStages];
+    const int32_t* __restrict__ irow = a.idx ? a.idx + (int64_t)r * a.topk + b0 : nullptr;
+    constexpr int kChunk = 16;
+    int v[kChunk];
+    // never past this row's topk entries (the tiles round topk up to 32)
+    const int first = irow ? (int)min64(min64((int64_t)cap, (int64_t)a.topk - b0), 32 * kChunk) : 0;
 #pragma unroll
-    for (int i = 0; i < kStages; ++i) kr[i] = load_key(i);
+    for (int u = 0; u < kChunk; ++u) {
+      const int i = u * 32 + lane;
+      v[u] = (irow && i < first) ? __ldg(irow + i) : 0;
+    }
+    const RowGeom geo = row_geometry(a, r, false);
+    const int nk = (int)max64(0, min64((int64_t)cap, geo.n_list - b0));
+    // With an index list the split holds at most topk <= kMaxTopk keys (the
+    // launcher sizes the splits from topk); a dense row's keys are b0 + slot and
+    // need no list.
+    for (int c0 = 0; irow && c0 < nk; c0 += 32 * kChunk) {
+      if (c0 > 0) {
+#pragma unroll
+        for (int u = 0; u < kChunk; ++u) {
+          const int i = c0 + u * 32 + lane;
+          v[u] = (irow && i < nk) ? __ldg(irow + i) : 0;
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < kChunk; ++u) {
+        const int i = c0 + u * 32 + lane;
+        if (i < nk) {
+          int64_t key = v[u];
+          if (key < 0 || key >= geo.nvis) {
+            flag_error(a.err, LSA_DEVERR_INDEX);
+            key = -1;
+          }
+          sm.list[i] = (int32_t)key;
+        }
+      }
+    }
+    __syncwarp();
+    const int n_tiles = (nk + kTK - 1) / kTK;
+    const uint16_t* __restrict__ latb = a.lat[z] + geo.kbase * kDLat;
     for (int base = 0; base < n_tiles; base += kStages) {
 #pragma unroll
       for (int i = 0; i < kStages; ++i) {
         const int tt = base + i;
         if (tt < n_tiles) {
-          const int key = kr[i];
-          kr[i] = load_key(tt + kStages);
+          const int sl = tt * kTK + lane;
+          const int key = sl < nk ? (irow ? sm.list[sl] : (int)(b0 + sl)) : -1;
           if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag);
           sm.keys[i][lane] = key;
           uint16_t* dst = &sm.k[i][lane * kSRow];
@@ -213,10 +250,13 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   }
 
   // ================= math warps =================
+  const RowGeom geo = row_geometry(a, r, s == 0 && tid == 0);
+  const int nk = (int)max64(0, min64((int64_t)cap, geo.n_list - b0));
+  const int n_tiles = (nk + kTK - 1) / kTK;
   const int g = lane >> 2, t = lane & 3;
-  const int mt = warp & 1, kq = warp >> 1;
+  const int mt = warp >> 2, kq = warp & 3;
   mbar_wait(&sm.qbar, 0, abort_flag);
-  // Q fragments of this warp: head half mt, k16 steps 9kq .. 9kq+8.
+  // Q fragments of this warp: heads 16mt .. 16mt+15, k16 steps 9kq .. 9kq+8.
   uint32_t qf[9][4];
   {
     const uint32_t qa = smem_u32(&sm.q[(16 * mt + (lane & 15)) * kSRow + 8 * (lane >> 4)]) + 9 * kq * 32;
@@ -227,18 +267,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   float* part = reinterpret_cast<float*>(sm.q);
 
   const float scale_log2 = a.scale * kLog2e;
-  // softmax state for this lane's head (head half mt, head 16mt + (lane >> 1))
+  // softmax state for this lane's head
   const int sh = 16 * mt + (lane >> 1);
-  const int kg = warp >> 1, kb4 = 8 * kg + 4 * (lane & 1);
+  const int kb4 = 8 * kq + 4 * (lane & 1);
   float m_run = -INFINITY, l_run = 0.f;
-  // value accumulators: o[mtv][nt][4], heads 16mtv+g (+8), dims 64w + 8nt + 2t
-  float o[2][8][4];
+  // value accumulators: o[nt][4], heads 16mt+g (+8), dims 128kq + 8nt + 2t
+  float o[16][4];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int nt = 0; nt < 16; ++nt)
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) o[i][nt][j] = 0.f;
+    for (int j = 0; j < 4; ++j) o[nt][j] = 0.f;
 
   for (int tt = 0; tt < n_tiles; ++tt) {
     const int st = tt % kStages;
@@ -246,40 +284,45 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     const uint16_t* kt = sm.k[st];
 
     // ---- partial logits over this warp's dim quarter ----
-    float sc[4][4];
+    float sc[2][4][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt)
+    for (int c = 0; c < 2; ++c)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) sc[nt][j] = 0.f;
+      for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) sc[c][nt][j] = 0.f;
     const uint32_t kb0 = smem_u32(&kt[((lane & 7) + 8 * (lane >> 4)) * kSRow + 8 * ((lane >> 3) & 1)]) +
                          9 * kq * 32;
 #pragma unroll
     for (int ks = 0; ks < 9; ++ks) {
+      const int c = ks & 1;
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         uint32_t b[4];
         ldsm_x4(kb0 + (16 * j * kSRow) * 2 + ks * 32, b[0], b[1], b[2], b[3]);
-        mma_16816(sc[2 * j], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b[0], b[1]);
-        mma_16816(sc[2 * j + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b[2], b[3]);
+        mma_16816(sc[c][2 * j], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b[0], b[1]);
+        mma_16816(sc[c][2 * j + 1], qf[ks][0], qf[ks][1], qf[ks][2], qf[ks][3], b[2], b[3]);
       }
     }
     {
       float* pw = part + ((kq * 2 + mt) * 16) * kPartRow;
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
-        *reinterpret_cast<float2*>(&pw[g * kPartRow + 8 * nt + 2 * t]) = make_float2(sc[nt][0], sc[nt][1]);
+        *reinterpret_cast<float2*>(&pw[g * kPartRow + 8 * nt + 2 * t]) =
+            make_float2(sc[0][nt][0] + sc[1][nt][0], sc[0][nt][1] + sc[1][nt][1]);
         *reinterpret_cast<float2*>(&pw[(g + 8) * kPartRow + 8 * nt + 2 * t]) =
-            make_float2(sc[nt][2], sc[nt][3]);
+            make_float2(sc[0][nt][2] + sc[1][nt][2], sc[0][nt][3] + sc[1][nt][3]);
       }
     }
-    math_sync();  // (1) partials complete
+    half_sync(mt);  // (1) this half's partials complete
 
     // ---- sum the partials, mask, tile max (lane: head sh, keys kb4 .. kb4+3) ----
     float x[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) {
-      const float4 v = *reinterpret_cast<const float4*>(part + ((q4 * 2 + mt) * 16 + (lane >> 1)) * kPartRow + kb4);
-      x[0] += v.x; x[1] += v.y; x[2] += v.z; x[3] += v.w;
+      const float4 vv =
+          *reinterpret_cast<const float4*>(part + ((q4 * 2 + mt) * 16 + (lane >> 1)) * kPartRow + kb4);
+      x[0] += vv.x; x[1] += vv.y; x[2] += vv.z; x[3] += vv.w;
     }
     float mx = -INFINITY;
 #pragma unroll
@@ -288,8 +331,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
       mx = fmaxf(mx, x[i]);
     }
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    if ((lane & 1) == 0) sm.red_max[kg][sh] = mx;
-    math_sync();  // (2) tile maxima
+    if ((lane & 1) == 0) sm.red_max[kq][sh] = mx;
+    half_sync(mt);  // (2) tile maxima
     const float tmax = fmaxf(fmaxf(sm.red_max[0][sh], sm.red_max[1][sh]), fmaxf(sm.red_max[2][sh], sm.red_max[3][sh]));
     const float m_new = fmaxf(m_run, tmax);
     const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
@@ -301,49 +344,44 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     *reinterpret_cast<uint2*>(&sm.p[sh * kPRow + kb4]) = make_uint2(pack_bf16x2(p0, p1), pack_bf16x2(p2, p3));
     ps += __shfl_xor_sync(0xffffffffu, ps, 1);
     if ((lane & 1) == 0) {
-      sm.red_sum[kg][sh] = ps;
-      if (kg == 0) sm.alpha[sh] = alpha;
+      sm.red_sum[kq][sh] = ps;
+      if (kq == 0) sm.alpha[sh] = alpha;
     }
-    math_sync();  // (3) P, alpha and tile sums ready
+    half_sync(mt);  // (3) P, alpha and tile sums of this half ready
     l_run = l_run * alpha +
             ((sm.red_sum[0][sh] + sm.red_sum[1][sh]) + (sm.red_sum[2][sh] + sm.red_sum[3][sh]));
 
-    // ---- O += P V, value dims 64w .. 64w+63 ----
+    // ---- O += P V, heads of this half, value dims 128kq .. 128kq+127 ----
+    {
+      const float al0 = sm.alpha[16 * mt + g], al1 = sm.alpha[16 * mt + 8 + g];
 #pragma unroll
-    for (int mv = 0; mv < 2; ++mv)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const float al = sm.alpha[16 * mv + 8 * hf + g];
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          o[mv][nt][2 * hf] *= al;
-          o[mv][nt][2 * hf + 1] *= al;
-        }
+      for (int nt = 0; nt < 16; ++nt) {
+        o[nt][0] *= al0;
+        o[nt][1] *= al0;
+        o[nt][2] *= al1;
+        o[nt][3] *= al1;
       }
-    const uint32_t pa0 = smem_u32(&sm.p[(lane & 15) * kPRow + 8 * (lane >> 4)]);
-    const uint32_t pa1 = pa0 + 16 * kPRow * 2;
+    }
+    const uint32_t pa = smem_u32(&sm.p[(16 * mt + (lane & 15)) * kPRow + 8 * (lane >> 4)]);
     const uint32_t vb0 =
-        smem_u32(&kt[((lane & 7) + 8 * ((lane >> 3) & 1)) * kSRow + 64 * warp + 8 * (lane >> 4)]);
+        smem_u32(&kt[((lane & 7) + 8 * ((lane >> 3) & 1)) * kSRow + 128 * kq + 8 * (lane >> 4)]);
 #pragma unroll
     for (int kk = 0; kk < kTK / 16; ++kk) {
-      uint32_t pf0[4], pf1[4];
-      ldsm_x4(pa0 + kk * 32, pf0[0], pf0[1], pf0[2], pf0[3]);
-      ldsm_x4(pa1 + kk * 32, pf1[0], pf1[1], pf1[2], pf1[3]);
+      uint32_t pf[4];
+      ldsm_x4(pa + kk * 32, pf[0], pf[1], pf[2], pf[3]);
 #pragma unroll
-      for (int np = 0; np < 4; ++np) {
-        uint32_t v[4];
-        ldsm_x4_t(vb0 + (kk * 16 * kSRow + 16 * np) * 2, v[0], v[1], v[2], v[3]);
-        mma_16816(o[0][2 * np], pf0[0], pf0[1], pf0[2], pf0[3], v[0], v[1]);
-        mma_16816(o[0][2 * np + 1], pf0[0], pf0[1], pf0[2], pf0[3], v[2], v[3]);
-        mma_16816(o[1][2 * np], pf1[0], pf1[1], pf1[2], pf1[3], v[0], v[1]);
-        mma_16816(o[1][2 * np + 1], pf1[0], pf1[1], pf1[2], pf1[3], v[2], v[3]);
+      for (int np = 0; np < 8; ++np) {
+        uint32_t vv[4];
+        ldsm_x4_t(vb0 + (kk * 16 * kSRow + 16 * np) * 2, vv[0], vv[1], vv[2], vv[3]);
+        mma_16816(o[2 * np], pf[0], pf[1], pf[2], pf[3], vv[0], vv[1]);
+        mma_16816(o[2 * np + 1], pf[0], pf[1], pf[2], pf[3], vv[2], vv[3]);
       }
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&sm.empty[st]);  // this warp is done with the stage
   }
   pdl_trigger();
-  if (kg == 0 && (lane & 1) == 0) {
+  if (kq == 0 && (lane & 1) == 0) {
     sm.fin_m[sh] = m_run;
     sm.fin_l[sh] = l_run;
   }
@@ -351,22 +389,17 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   if (tid == 0 && *abort_flag) flag_error(a.err, LSA_DEVERR_TIMEOUT);
 
   // ---- epilogue ----
+  const int h0 = 16 * mt + g, h1 = h0 + 8;
   if (sp.n_split == 1) {
     uint16_t* __restrict__ og = a.out[z] + (int64_t)r * kH * kDV;
+    const float l0 = sm.fin_l[h0], l1 = sm.fin_l[h1];
+    const float i0 = l0 > 0.f ? 1.f / l0 : 0.f, i1 = l1 > 0.f ? 1.f / l1 : 0.f;
 #pragma unroll
-    for (int mv = 0; mv < 2; ++mv)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int head = 16 * mv + 8 * hf + g;
-        const float l = sm.fin_l[head];
-        const float inv = l > 0.f ? 1.f / l : 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const int d = 64 * warp + 8 * nt + 2 * t;
-          *reinterpret_cast<uint32_t*>(&og[head * kDV + d]) =
-              pack_bf16x2(o[mv][nt][2 * hf] * inv, o[mv][nt][2 * hf + 1] * inv);
-        }
-      }
+    for (int nt = 0; nt < 16; ++nt) {
+      const int d = 128 * kq + 8 * nt + 2 * t;
+      *reinterpret_cast<uint32_t*>(&og[h0 * kDV + d]) = pack_bf16x2(o[nt][0] * i0, o[nt][1] * i0);
+      *reinterpret_cast<uint32_t*>(&og[h1 * kDV + d]) = pack_bf16x2(o[nt][2] * i1, o[nt][3] * i1);
+    }
     if (a.lse[z] && tid < kH) {
       const float l = sm.fin_l[tid];
       a.lse[z][(int64_t)r * kH + tid] = l > 0.f ? (sm.fin_m[tid] + log2f(l)) * kLn2 : -INFINITY;
@@ -375,16 +408,11 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     const int64_t base = ((int64_t)z * a.n_rows + r) * sp.n_split + s;
     float* __restrict__ po = part_o + base * kH * kDV;
 #pragma unroll
-    for (int mv = 0; mv < 2; ++mv)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        const int head = 16 * mv + 8 * hf + g;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-          const int d = 64 * warp + 8 * nt + 2 * t;
-          *reinterpret_cast<float2*>(&po[head * kDV + d]) = make_float2(o[mv][nt][2 * hf], o[mv][nt][2 * hf + 1]);
-        }
-      }
+    for (int nt = 0; nt < 16; ++nt) {
+      const int d = 128 * kq + 8 * nt + 2 * t;
+      *reinterpret_cast<float2*>(&po[h0 * kDV + d]) = make_float2(o[nt][0], o[nt][1]);
+      *reinterpret_cast<float2*>(&po[h1 * kDV + d]) = make_float2(o[nt][2], o[nt][3]);
+    }
     if (tid < kH) part_ml[base * kH + tid] = make_float2(sm.fin_m[tid], sm.fin_l[tid]);
   }
 }
@@ -460,6 +488,9 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
   while (n_split > 1 && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes) --n_split;
   Split sp;
   sp.n_split = n_split;
+  // With an index list no row has more than topk keys (the shared list's size).
+  const int64_t max_list = a.idx ? min64(a.max_list, (int64_t)min(a.topk, kMaxTopk)) : a.max_list;
+  sp.list_tiles = (int)((max_list + kTK - 1) / kTK);
   float* part_o = nullptr;
   float2* part_ml = nullptr;
   if (n_split > 1) {
