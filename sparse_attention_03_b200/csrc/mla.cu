@@ -92,6 +92,10 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
 // Named barriers: 1 = the eight math warps, 2 + h = the four warps of head half h.
 __device__ __forceinline__ void math_sync() { asm volatile("bar.sync 1, %0;\n" ::"n"(kMathThreads) : "memory"); }
 __device__ __forceinline__ void half_sync(int h) { asm volatile("bar.sync %0, 128;\n" ::"r"(2 + h) : "memory"); }
+// Barrier 4 staggers the halves once: half 0 arrives after its first logits,
+// half 1 waits for that before starting.
+__device__ __forceinline__ void stagger_arrive() { asm volatile("bar.arrive 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
+__device__ __forceinline__ void stagger_wait() { asm volatile("bar.sync 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 
 struct RowGeom {
   int64_t kbase, nvis, n_list;
@@ -278,6 +282,10 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
 #pragma unroll
     for (int j = 0; j < 4; ++j) o[nt][j] = 0.f;
 
+  // Half 1 starts one logits phase behind half 0, so that from then on one
+  // half's softmax runs while the other issues MMAs (both halves see the same
+  // n_tiles, so the barrier is taken by both or by neither).
+  if (mt == 1 && n_tiles > 0) stagger_wait();
   for (int tt = 0; tt < n_tiles; ++tt) {
     const int st = tt % kStages;
     mbar_wait(&sm.full[st], (tt / kStages) & 1, abort_flag);
@@ -314,6 +322,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
             make_float2(sc[0][nt][2] + sc[1][nt][2], sc[0][nt][3] + sc[1][nt][3]);
       }
     }
+    if (mt == 0 && tt == 0) stagger_arrive();
     half_sync(mt);  // (1) this half's partials complete
 
     // ---- sum the partials, mask, tile max (lane: head sh, keys kb4 .. kb4+3) ----
