@@ -11,8 +11,11 @@ caches read are ~8.6 GB (> L2), so no L2 flush is needed between steps.
 
 Also reported: prefill tok/s of one 16384-token causal sequence (same path in
 prefill form), the roofline fraction of the dominant kernel, the fp64 CPU
-oracle on a bounded sample, and an end-to-end number through lsa_forward with
-pinned host buffers and host<->device copies inside the timed region.
+oracle on a bounded sample, an end-to-end number through lsa_forward with
+pinned host buffers and host<->device copies inside the timed region, and an
+MTP draft round ("mtp": one index pass and top-k per layer shared by three
+draft steps of sparse MLA over one latent cache; tokens = 3 per sequence per
+layer per round).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
@@ -283,7 +286,30 @@ def build_decode(device):
                                    mla_ws, bind=True) for z in range(2)]))
         D["fwd"].append(lsa.forward(cfg, 0, l.seq_of_row, l.pos, ctx, l.q_idx, l.w, l.k_idx, l.k_off, l.q_abs,
                                     l.latent, [out[i, 0], out[i, 1]], [lse[i, 0], lse[i, 1]], ws, bind=True))
+    # MTP draft round: one index pass shared by three draft steps, each attending
+    # over the same latent cache with its own absorbed query
+    q3 = torch.empty((nl, B, 32, 576), dtype=torch.bfloat16, device=device)
+    for i in range(nl):
+        lsa.synth_normal_bf16(q3[i], 0, 16 * (100 + i) + 3)
+    out3 = torch.empty((B, 32, 512), dtype=torch.bfloat16, device=device)
+    lse3 = torch.empty((B, 32), dtype=torch.float32, device=device)
+    D["mtp"] = []
+    for i, l in enumerate(layers):
+        qs = [l.q_abs[0], l.q_abs[1], q3[i]]
+        D["mtp"].append([lsa.sparse_mla_decode(cfg, qs[st], l.latent[0], l.k_off, idx, cnt, ctx, out3, lse3,
+                                               mla_ws, bind=True) for st in range(3)])
+    D["q3"] = q3
     return D
+
+
+def mtp_round(D):
+    """One MTP draft round through every layer: the index pass and top-k once,
+    then three draft steps of sparse MLA over that one selection."""
+    for (idx_call, topk_call, _), steps in zip(D["calls"], D["mtp"]):
+        idx_call()
+        topk_call()
+        for call in steps:
+            call()
 
 
 def decode_step(D, ev=None):
@@ -451,6 +477,13 @@ def gpu_arm(args):
     e2e_value, _ = aggregate(B * nl * e2e_steps, te, world, device)
     h2d = sum(x.numel() * x.element_size() for x in h_in)
     d2h = h_out.numel() * h_out.element_size()
+
+    # MTP draft rounds (three draft tokens per sequence and layer per round)
+    for _ in range(3):
+        mtp_round(D)
+    mtp_steps = max(5, args.steps // 2)
+    tm = time_region(lambda s: mtp_round(D), mtp_steps, world, device)
+    mtp_value, _ = aggregate(3 * B * nl * mtp_steps, tm, world, device)
     assert lsa.device_error() == 0
 
     del D
@@ -477,6 +510,9 @@ def gpu_arm(args):
         "gpu_launches": launches,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
+    line["mtp"] = {"value": mtp_value, "unit": "tokens/s/layer", "ms_per_round": 1e3 * tm / mtp_steps,
+                   "config": {"workload": "mtp_draft_round_b16_ctx131072_14layers", "draft_steps": 3,
+                              "index_passes_per_round": 1}}
     if prefill:
         line["prefill"] = prefill
     if world == 1 and not args.no_cpu_baseline:

@@ -533,6 +533,50 @@ def test_forward_tiny_config(L):
     _forward_check(L, wl, _upload(wl), cfg, 0, range(len(lengths)), max(lengths))
 
 
+def test_mtp_draft_steps_share_one_index_pass(L):
+    # [LSA-2.0] "多token预测模块集成": all three MTP draft steps share one index
+    # pass. Reading: the indexer and the top-k run once, for the first draft
+    # step's query at position p; the three draft steps (positions p, p+1, p+2,
+    # their tokens already appended to the cache) attend over that one
+    # selection with their own absorbed queries.
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    lengths = [2052, 3000, 5002, 9001, 2049]
+    wl = S.Workload(21, 0, lengths, cli=1)
+    wl.pos = (wl.lengths - 3).astype(np.int32)   # the index owner is the first draft step
+    d = _upload(wl)
+    B, max_len = wl.n_rows, max(lengths)
+    q_steps = [S.normal_bf16(21, S.tid(50 + st, S.Q_ABS0), 0, B * 32 * 576).reshape(B, 32, 576)
+               for st in range(3)]
+    scores = torch.empty((B, max_len), device="cuda")
+    idx = torch.empty((B, cfg.index_topk), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((B,), dtype=torch.int32, device="cuda")
+    hist = L.topk_hist_buffer(B)
+    L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], max_len, scores,
+                   topk_hist=hist)
+    L.topk(cfg, d["pos"], max_len, scores, idx, cnt, L.workspace(cfg, L.OP_TOPK, B, B, max_len), topk_hist=hist)
+    mws = L.workspace(cfg, L.OP_MLA_DECODE, B, B, max_len)
+    got = []
+    for st in range(3):
+        out = torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((B, 32), device="cuda")
+        L.sparse_mla_decode(cfg, bf16_dev(q_steps[st]), d["latent"][0], d["k_off"], idx, cnt, max_len, out, lse,
+                            mws)
+        got.append((bf16_host_f64(out), lse.cpu().numpy()))
+    assert L.device_error() == 0
+    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    for r in range(B):
+        q, w, k, _, lat = host_rows(wl, r)
+        p = int(wl.pos[r])
+        s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
+        exact = check_selection(gi[r], int(gc[r]), s, p, ocfg, where=f"row {r}")
+        sel, _ = R.select_topk(s, p, ocfg)
+        assert gi[r, : gc[r]].max() <= p, "the shared set holds no key after the index owner's position"
+        for st in range(3):
+            eo, el = R.mla(S.bf16_bits_to_f64(q_steps[st][r]), lat[0][sel], ocfg)
+            assert_attention(got[st][0][r], got[st][1][r], eo, el, check_lse=exact, where=f"row {r} step {st}")
+
+
 def test_empty_batch_is_noop(L):
     cfg = L.LsaConfig()
     e = torch.empty((0,), dtype=torch.int32, device="cuda")
