@@ -28,6 +28,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "launch.h"
+#include "mla_common.cuh"
 #include "tc.cuh"
 
 namespace lsa {
@@ -96,50 +97,6 @@ __device__ __forceinline__ void half_sync(int h) { asm volatile("bar.sync %0, 12
 // half 1 waits for that before starting.
 __device__ __forceinline__ void stagger_arrive() { asm volatile("bar.arrive 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 __device__ __forceinline__ void stagger_wait() { asm volatile("bar.sync 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
-
-struct RowGeom {
-  int64_t kbase, nvis, n_list;
-};
-
-// Row geometry, with every out-of-range input clamped (and flagged by one thread).
-__device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool report) {
-  RowGeom g{0, 0, 0};
-  if (a.decode) {
-    const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
-    if (seq < 0 || seq >= a.n_seq) {
-      if (report) flag_error(a.err, LSA_DEVERR_SEQ);
-    } else {
-      g.kbase = a.k_off[seq];
-      const int64_t klen = a.k_off[seq + 1] - g.kbase;
-      g.nvis = klen;
-      if (a.pos) {
-        int64_t p1 = (int64_t)a.pos[r] + 1;
-        if (p1 < 1 || p1 > klen) {
-          if (report) flag_error(a.err, LSA_DEVERR_POS);
-          p1 = max64(0, min64(p1, klen));
-        }
-        g.nvis = p1;
-      }
-    }
-  } else {
-    int64_t p1 = (int64_t)a.pos[r] + 1;
-    if (p1 < 1 || p1 > a.n_keys) {
-      if (report) flag_error(a.err, LSA_DEVERR_POS);
-      p1 = max64(0, min64(p1, a.n_keys));
-    }
-    g.nvis = p1;
-  }
-  g.n_list = g.nvis;
-  if (a.idx) {
-    int c = a.count[r];
-    if (c < 0 || c > a.topk) {
-      if (report) flag_error(a.err, LSA_DEVERR_COUNT);
-      c = max(0, min(c, a.topk));
-    }
-    g.n_list = c;
-  }
-  return g;
-}
 
 // Warp roles (math warps 0..7): head half mt = w >> 2 (heads 16mt .. 16mt+15)
 // and quarter kq = w & 3, so each SM sub-partition runs one warp of each half
@@ -492,6 +449,9 @@ int mla_choose_splits(int n_rows, int cli, int64_t max_list) {
 
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
   if (a.n_rows <= 0) return cudaSuccess;
+  // The tcgen05 form passes every parity test but is bound by the TMA gather4
+  // rate (about 14 GB/s per SM); it stays off until its gather is faster.
+  const bool tc = false && a.lat_rows > 0 && mla_tc_supported();
   int n_split = mla_choose_splits(a.n_rows, a.cli, a.max_list);
   // Shrink split-K to what the workspace holds.
   while (n_split > 1 && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes) --n_split;
@@ -540,8 +500,9 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
       b.k_off = a.k_off + row0;
       b.n_seq = a.n_seq - row0;
     }
-    cudaError_t e = launch_pdl(mla_kernel, dim3(n_split, nr, a.cli), dim3(kThreads), sizeof(MlaSmem), st, b, sp,
-                               part_o, part_ml);
+    cudaError_t e = tc ? launch_mla_tc_chunk(b, n_split, a.max_list, a.lat_rows, part_o, part_ml, st)
+                       : launch_pdl(mla_kernel, dim3(n_split, nr, a.cli), dim3(kThreads), sizeof(MlaSmem), st, b,
+                                    sp, part_o, part_ml);
     if (e != cudaSuccess) return e;
     if (n_split > 1) {
       e = launch_pdl(mla_merge_kernel, dim3(kH, nr, a.cli), dim3(128), 0, st, b, sp, (const float*)part_o,

@@ -1,0 +1,54 @@
+// Row geometry shared by the sparse-MLA kernels: where a query row's keys live
+// in the latent cache, how many it may see, and how long its key list is.
+#pragma once
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace lsa {
+
+struct RowGeom {
+  int64_t kbase, nvis, n_list;
+};
+
+// Row geometry, with every out-of-range input clamped (and flagged by one thread).
+__device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool report) {
+  RowGeom g{0, 0, 0};
+  if (a.decode) {
+    const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
+    if (seq < 0 || seq >= a.n_seq) {
+      if (report) flag_error(a.err, LSA_DEVERR_SEQ);
+    } else {
+      g.kbase = a.k_off[seq];
+      const int64_t klen = a.k_off[seq + 1] - g.kbase;
+      g.nvis = klen;
+      if (a.pos) {
+        int64_t p1 = (int64_t)a.pos[r] + 1;
+        if (p1 < 1 || p1 > klen) {
+          if (report) flag_error(a.err, LSA_DEVERR_POS);
+          p1 = max64(0, min64(p1, klen));
+        }
+        g.nvis = p1;
+      }
+    }
+  } else {
+    int64_t p1 = (int64_t)a.pos[r] + 1;
+    if (p1 < 1 || p1 > a.n_keys) {
+      if (report) flag_error(a.err, LSA_DEVERR_POS);
+      p1 = max64(0, min64(p1, a.n_keys));
+    }
+    g.nvis = p1;
+  }
+  g.n_list = g.nvis;
+  if (a.idx) {
+    int c = a.count[r];
+    if (c < 0 || c > a.topk) {
+      if (report) flag_error(a.err, LSA_DEVERR_COUNT);
+      c = max(0, min(c, a.topk));
+    }
+    g.n_list = c;
+  }
+  return g;
+}
+
+}  // namespace lsa
