@@ -80,7 +80,6 @@ struct MlaArgs {
   int n_rows, n_seq, topk, decode, cli;
   int64_t n_keys;            // prefill: rows in latent
   int64_t max_list;          // host bound on keys per row (sizes split-K)
-  int64_t lat_rows = 0;      // bound on the latent rows a key may address (0: unknown)
   float scale;
   void* ws;
   size_t ws_bytes;
@@ -90,9 +89,5 @@ struct MlaArgs {
 size_t mla_ws_bytes(int n_rows, int cli, int n_split);
 int mla_choose_splits(int n_rows, int cli, int64_t max_list);
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st);
-// The tensor-core (tcgen05) form of the same kernel, one chunk of <= 65535 rows.
-bool mla_tc_supported();
-cudaError_t launch_mla_tc_chunk(const MlaArgs& b, int n_split, int64_t max_list, int64_t lat_rows, float* part_o,
-                                float2* part_ml, cudaStream_t st);
 
 }  // namespace lsa

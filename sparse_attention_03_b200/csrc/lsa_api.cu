@@ -299,7 +299,6 @@ lsa_status lsa_sparse_mla_decode(const lsa_config* c, int32_t batch, const lsa_b
   a.idx = idx;
   a.count = count;
   a.max_list = idx ? c->index_topk : max_len;
-  a.lat_rows = (int64_t)batch * max_len;
   a.ws = ws;
   a.ws_bytes = ws ? ws_bytes : 0;
   return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
@@ -328,7 +327,6 @@ lsa_status lsa_sparse_mla_prefill(const lsa_config* c, int32_t n_rows, const int
   a.idx = idx;
   a.count = count;
   a.max_list = idx ? c->index_topk : n_keys;
-  a.lat_rows = n_keys;
   a.ws = ws;
   a.ws_bytes = ws ? ws_bytes : 0;
   return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
@@ -382,7 +380,6 @@ lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_
   m.n_seq = n_seq;
   m.pos = pos;
   m.n_keys = max_len;
-  m.lat_rows = mode == 0 ? (int64_t)n_seq * max_len : max_len;
 
   if (dense) {
     // The pages' fallback: no index pass, dense MLA in every sub-block.

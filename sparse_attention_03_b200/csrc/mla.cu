@@ -449,9 +449,6 @@ int mla_choose_splits(int n_rows, int cli, int64_t max_list) {
 
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
   if (a.n_rows <= 0) return cudaSuccess;
-  // The tcgen05 form passes every parity test but is bound by the TMA gather4
-  // rate (about 14 GB/s per SM); it stays off until its gather is faster.
-  const bool tc = false && a.lat_rows > 0 && mla_tc_supported();
   int n_split = mla_choose_splits(a.n_rows, a.cli, a.max_list);
   // Shrink split-K to what the workspace holds.
   while (n_split > 1 && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes) --n_split;
@@ -500,9 +497,8 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
       b.k_off = a.k_off + row0;
       b.n_seq = a.n_seq - row0;
     }
-    cudaError_t e = tc ? launch_mla_tc_chunk(b, n_split, a.max_list, a.lat_rows, part_o, part_ml, st)
-                       : launch_pdl(mla_kernel, dim3(n_split, nr, a.cli), dim3(kThreads), sizeof(MlaSmem), st, b,
-                                    sp, part_o, part_ml);
+    cudaError_t e = launch_pdl(mla_kernel, dim3(n_split, nr, a.cli), dim3(kThreads), sizeof(MlaSmem), st, b, sp,
+                               part_o, part_ml);
     if (e != cudaSuccess) return e;
     if (n_split > 1) {
       e = launch_pdl(mla_merge_kernel, dim3(kH, nr, a.cli), dim3(128), 0, st, b, sp, (const float*)part_o,
