@@ -183,3 +183,49 @@ def absorb_query(q_nope, q_rope, w_uk):
 def unembed_out(o_lat, w_uv):
     """unembed_out: map each head's 512-d latent output back, out[h] = W_UV[h] o_lat[h]."""
     return np.stack([w_uv[h] @ o_lat[h] for h in range(o_lat.shape[0])])
+
+
+# ---------------------------------------------------------------------------
+# Upstream of the path: the indexer's own projections and the cache append.
+# [Lite-Sparse] LSA section (the indexer's structure): wq_b maps the q-LoRA
+# representation (q_lora_rank dims) to index_n_heads x index_head_dim; wk maps
+# the hidden state to the index key, which is RMS-normalised; weights_proj
+# gives one scalar per index head; the index query and key share MLA's RoPE
+# configuration (qk_rope_head_dim, rope_theta).
+# Readings (the pages leave these open): the RoPE part is the last
+# qk_rope_head_dim dims of each 128-dim vector (MLA keeps its rope dims last),
+# rotated in rotate-half form, pairs (i, i + rope/2) at angle
+# pos * theta^(-2i/rope); no rope scaling; RMSNorm = x / sqrt(mean(x^2) + eps)
+# times a per-dim weight, eps = 1e-6; no scale on the head weights.
+# ---------------------------------------------------------------------------
+Q_LORA, HIDDEN, ROPE_DIM, ROPE_THETA, NORM_EPS = 1536, 3072, 64, 1.0e6, 1e-6
+
+
+def rope(x: np.ndarray, pos: float, theta: float = ROPE_THETA, rope_dim: int = ROPE_DIM) -> np.ndarray:
+    """Rotary embedding of the last rope_dim dims of x[..., d] at position pos (fp64)."""
+    x = np.array(x, dtype=np.float64)
+    d = x.shape[-1]
+    r0, half = d - rope_dim, rope_dim // 2
+    ang = float(pos) * theta ** (-2.0 * np.arange(half) / rope_dim)
+    c, s = np.cos(ang), np.sin(ang)
+    a = x[..., r0:r0 + half].copy()
+    b = x[..., r0 + half:].copy()
+    x[..., r0:r0 + half] = a * c - b * s
+    x[..., r0 + half:] = a * s + b * c
+    return x
+
+
+def rms_norm(x: np.ndarray, weight: np.ndarray, eps: float = NORM_EPS) -> np.ndarray:
+    x = np.asarray(x, dtype=np.float64)
+    return x / np.sqrt(np.mean(x * x, axis=-1, keepdims=True) + eps) * weight
+
+
+def index_project_row(c_q, h, wq_b, wk, wproj, k_norm_w, pos, theta=ROPE_THETA, eps=NORM_EPS):
+    """One token's indexer inputs from its q-LoRA vector c_q [1536] and hidden
+    state h [3072]: q_idx [32, 128] = RoPE(wq_b c_q), k [128] = RoPE(RMSNorm(wk h)),
+    w [32] = weights_proj h. Weights are [out, in]."""
+    q = (np.asarray(wq_b, np.float64) @ np.asarray(c_q, np.float64)).reshape(-1, 128)
+    q = rope(q, pos, theta)
+    k = rope(rms_norm(np.asarray(wk, np.float64) @ np.asarray(h, np.float64), k_norm_w, eps), pos, theta)
+    w = np.asarray(wproj, np.float64) @ np.asarray(h, np.float64)
+    return q, k, w

@@ -324,3 +324,62 @@ def test_tiny_config_whole_row():
         if not dense:
             assert {0, 1, p - 3, p - 2, p - 1, p} <= set(sel.tolist())
         assert np.isfinite(outs[0][0]).all()
+
+
+# --------------------------------------------------------------------------
+# Indexer projection (upstream of the path): RoPE, RMSNorm, the projections.
+# --------------------------------------------------------------------------
+def test_rope_closed_form_frequencies():
+    # pair i of the rope part turns by pos * theta^(-2i/64): a unit vector on the
+    # pair's first dim lands on (cos, sin) of exactly that angle
+    pos = 777
+    for i in (0, 1, 17, 31):
+        x = np.zeros(128)
+        x[64 + i] = 1.0
+        y = R.rope(x, pos)
+        ang = pos * R.ROPE_THETA ** (-2.0 * i / 64)
+        assert abs(y[64 + i] - np.cos(ang)) < 1e-12 and abs(y[96 + i] - np.sin(ang)) < 1e-12
+        assert np.count_nonzero(np.abs(y) > 1e-15) <= 2
+
+
+def test_rope_relative_position_and_norms():
+    # dot products of rotated vectors depend only on the position difference;
+    # a sign slip in one half of the rotation breaks this; norms of pairs are kept
+    rng = np.random.default_rng(5)
+    q, k = rng.standard_normal((2, 128))
+    for p1, p2 in ((10, 3), (983039, 5), (1, 1)):
+        lhs = R.rope(q, p1)[64:] @ R.rope(k, p2)[64:]
+        rhs = R.rope(q, p1 - p2)[64:] @ k[64:]
+        assert abs(lhs - rhs) < 1e-9 * (1 + abs(rhs))
+    y = R.rope(q, 12345)
+    np.testing.assert_array_equal(y[:64], q[:64])          # the non-rope half is untouched
+    np.testing.assert_allclose(y[64:96] ** 2 + y[96:] ** 2, q[64:96] ** 2 + q[96:] ** 2, rtol=1e-12)
+
+
+def test_rms_norm_closed_form():
+    w = np.linspace(0.5, 1.5, 128)
+    for c in (3.0, -0.25):
+        y = R.rms_norm(np.full(128, c), w)
+        np.testing.assert_allclose(y, np.sign(c) * abs(c) / np.sqrt(c * c + R.NORM_EPS) * w, rtol=1e-13)
+    x = np.zeros(128)
+    x[0], x[1] = 3.0, 4.0            # mean square 25/128
+    np.testing.assert_allclose(R.rms_norm(x, np.ones(128))[:2], np.array([3.0, 4.0]) / np.sqrt(25 / 128 + 1e-6),
+                               rtol=1e-13)
+
+
+def test_index_project_layout_and_pieces():
+    # head-major query rows, the key normalised before it is rotated, raw weights
+    rng = np.random.default_rng(6)
+    K = 16
+    c_q, h = rng.standard_normal(K), rng.standard_normal(K)
+    wq_b, wk, wp = rng.standard_normal((4096, K)), rng.standard_normal((128, K)), rng.standard_normal((32, K))
+    g = rng.uniform(0.5, 1.5, 128)
+    q, k, w = R.index_project_row(c_q, h, wq_b, wk, wp, g, pos=0)
+    for head in (0, 13, 31):
+        np.testing.assert_allclose(q[head], wq_b[128 * head:128 * (head + 1)] @ c_q, rtol=1e-12)
+    raw = wk @ h
+    np.testing.assert_allclose(k, raw / np.sqrt(np.mean(raw * raw) + 1e-6) * g, rtol=1e-12)
+    np.testing.assert_allclose(w, wp @ h, rtol=1e-12)
+    q5, k5, _ = R.index_project_row(c_q, h, wq_b, wk, wp, g, pos=5)
+    np.testing.assert_allclose(q5, R.rope(q, 5), rtol=1e-12)
+    np.testing.assert_allclose(k5, R.rope(k, 5), rtol=1e-12)
