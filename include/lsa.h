@@ -98,6 +98,7 @@ LSA_API void lsa_config_default(lsa_config* cfg);
 #define LSA_OP_MLA_PREFILL 3
 #define LSA_OP_FORWARD_DECODE 4
 #define LSA_OP_FORWARD_PREFILL 5
+#define LSA_OP_INDEX_PROJECT 6
 
 /*
  * Bytes of workspace the operation uses at full speed for these sizes (host
@@ -192,6 +193,42 @@ LSA_API lsa_status lsa_topk(const lsa_config* cfg, int32_t n_rows, const int32_t
 LSA_API lsa_status lsa_topk_static(const lsa_config* cfg, int32_t n_rows, const int32_t* pos,
                                    int64_t max_len, const float* scores, int64_t ld, int32_t* idx,
                                    int32_t* count, void* stream);
+
+/*
+ * The indexer's own inputs from the model's activations, and the key-cache
+ * append ([Lite-Sparse] LSA section, the indexer's structure: wq_b maps the
+ * q-LoRA representation to index_n_heads x index_head_dim, wk maps the hidden
+ * state to the index key, which is RMS-normalised (index_k_norm_type rms),
+ * weights_proj gives one scalar per index head, and the index query and key
+ * share MLA's RoPE configuration (qk_rope_head_dim, rope_theta)). This is
+ * upstream of lsa_index_scores; it feeds its q_idx, w and k_idx.
+ *
+ * For each row r (sequence seq_of_row[r], position pos[r]):
+ *   q_idx[r,h,:] = RoPE(wq_b c_q[r])[h*128 .. h*128+127]          (bf16 out)
+ *   w[r,:]       = weights_proj hidden[r]                           (fp32 out)
+ *   k_cache[k_off[seq] + pos[r], :] = RoPE(RMSNorm(wk hidden[r]))   (bf16 out)
+ * RoPE rotates the last qk_rope_head_dim (64) dims of each 128-dim vector in
+ * rotate-half form: pairs (i, i+32) by pos * rope_theta^(-2i/64). RMSNorm:
+ * x / sqrt(mean(x^2) + 1e-6) * k_norm_w. These readings fill what the pages
+ * leave open (which dims carry RoPE, its form, the epsilon); no rope scaling.
+ * c_q bf16 [n_rows, q_lora_rank]; hidden bf16 [n_rows, hidden_size]; wq_b bf16
+ * [32*128, q_lora_rank]; wk bf16 [128, hidden_size]; wproj bf16 [32,
+ * hidden_size]; k_norm_w bf16 [128]; q_idx bf16 [n_rows, 32, 128]; w fp32
+ * [n_rows, 32]; k_cache bf16 packed [sum L, 128] (only the rows' own slots are
+ * written). q_lora_rank and hidden_size must be positive multiples of 32; every
+ * pointer 16-byte aligned. seq_of_row NULL: row r is sequence r when k_off is
+ * given, else every row is sequence 0 with k_cache rows = positions. max_len
+ * (host) bounds every position. A row whose sequence or position is out of
+ * range writes no cache row and raises a device error flag.
+ * Workspace (fp32 products): lsa_workspace_size(LSA_OP_INDEX_PROJECT).
+ */
+LSA_API lsa_status lsa_index_project(const lsa_config* cfg, int32_t n_rows, int32_t n_seq,
+                                     const int32_t* seq_of_row, const int32_t* pos, const int64_t* k_off,
+                                     int64_t max_len, const lsa_bf16* c_q, const lsa_bf16* hidden,
+                                     const lsa_bf16* wq_b, const lsa_bf16* wk, const lsa_bf16* wproj,
+                                     const lsa_bf16* k_norm_w, int32_t q_lora_rank, int32_t hidden_size,
+                                     float rope_theta, lsa_bf16* q_idx, float* w, lsa_bf16* k_cache, void* ws,
+                                     size_t ws_bytes, void* stream);
 
 /*
  * Sparse absorbed-latent MLA, decode ([Lite-Sparse] LSA section: at decode

@@ -138,6 +138,9 @@ def uniform_int(seed: int, tid: int, first: int, n: int, lo: int, hi: int) -> np
 # Tensor ids. One stream per tensor; per layer and attention sub-block.
 # ---------------------------------------------------------------------------
 Q_IDX, W, K_IDX, Q_ABS0, Q_ABS1, LAT0, LAT1, LENS = range(8)
+# inputs of the indexer's own projections: q-LoRA vectors, hidden states, the
+# weights wq_b / wk / weights_proj (N(0, 1/fan_in)) and the key-norm weight
+C_Q, HIDDEN, WQ_B, WK, WPROJ, KNORM = range(8, 14)
 
 
 def tid(layer: int, kind: int) -> int:

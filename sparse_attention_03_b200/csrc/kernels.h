@@ -67,6 +67,29 @@ bool topk_uses_workspace(int n_rows, int64_t max_len);
 cudaError_t launch_topk_hist_only(const TopkArgs& a, uint32_t* hist, cudaStream_t st);
 cudaError_t launch_topk_dense(const TopkArgs& a, cudaStream_t st);
 
+// The indexer's own projections and the key-cache append (upstream of the path).
+struct ProjectLaunch {
+  const uint16_t* c_q;      // [n_rows, q_lora] bf16
+  const uint16_t* hidden;   // [n_rows, hidden_dim] bf16
+  const uint16_t* wq_b;     // [32 * 128, q_lora] bf16
+  const uint16_t* wk;       // [128, hidden_dim] bf16
+  const uint16_t* wproj;    // [32, hidden_dim] bf16
+  const uint16_t* k_norm_w; // [128] bf16
+  const int32_t* seq_of_row;
+  const int32_t* pos;
+  const int64_t* k_off;
+  int n_rows, n_seq, q_lora, hidden_dim;
+  int64_t max_len;
+  double theta;
+  uint16_t* q_out;
+  float* w_out;
+  uint16_t* k_cache;
+  void* ws;
+  int* err;
+};
+size_t project_ws_bytes(int n_rows);
+cudaError_t launch_index_project(const ProjectLaunch& L, cudaStream_t st);
+
 struct MlaArgs {
   const uint16_t* q[2];
   const uint16_t* lat[2];

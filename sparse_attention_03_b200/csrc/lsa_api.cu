@@ -221,6 +221,8 @@ size_t lsa_workspace_size(const lsa_config* c, int32_t op, int32_t n_rows, int32
     case LSA_OP_FORWARD_PREFILL:
       if (max_len <= c->index_topk) return mla_ws(n_rows, c->cli_factor, max_len) + kAlign;
       return forward_block_ws(c, prefill_block_rows(n_rows, max_len), max_len) + kAlign;
+    case LSA_OP_INDEX_PROJECT:
+      return project_ws_bytes(n_rows) + kAlign;
     default:
       return 0;
   }
@@ -274,6 +276,54 @@ lsa_status lsa_topk(const lsa_config* c, int32_t n_rows, const int32_t* pos, int
     return set_error(LSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
   return run_topk(c, n_rows, pos, max_len, scores, ld, idx, count, ws, ws_bytes, (cudaStream_t)stream,
                   topk_hist);
+}
+
+lsa_status lsa_index_project(const lsa_config* c, int32_t n_rows, int32_t n_seq, const int32_t* seq_of_row,
+                             const int32_t* pos, const int64_t* k_off, int64_t max_len, const lsa_bf16* c_q,
+                             const lsa_bf16* hidden, const lsa_bf16* wq_b, const lsa_bf16* wk,
+                             const lsa_bf16* wproj, const lsa_bf16* k_norm_w, int32_t q_lora_rank,
+                             int32_t hidden_size, float rope_theta, lsa_bf16* q_idx, float* w, lsa_bf16* k_cache,
+                             void* ws, size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_index_project";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (n_rows < 0 || n_seq < 1 || max_len < 1)
+    return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0, n_seq >= 1, max_len >= 1", fn);
+  if (q_lora_rank <= 0 || q_lora_rank % 32 || hidden_size <= 0 || hidden_size % 32)
+    return set_error(LSA_ERR_INVALID, "%s: q_lora_rank and hidden_size must be positive multiples of 32", fn);
+  if (!(rope_theta > 1.f)) return set_error(LSA_ERR_INVALID, "%s: rope_theta must exceed 1", fn);
+  if (n_rows == 0) return LSA_OK;
+  if (!pos || !c_q || !hidden || !wq_b || !wk || !wproj || !k_norm_w || !q_idx || !w || !k_cache)
+    return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (n_seq > 1 && !k_off) return set_error(LSA_ERR_INVALID, "%s: several sequences need k_off", fn);
+  const void* al[] = {c_q, hidden, wq_b, wk, wproj, k_norm_w, q_idx, w, k_cache};
+  for (const void* p : al)
+    if (!aligned16(p)) return set_error(LSA_ERR_INVALID, "%s: arrays must be 16-byte aligned", fn);
+  if (!ws || ws_bytes < project_ws_bytes(n_rows))
+    return set_error(LSA_ERR_WORKSPACE, "%s: workspace of %zu bytes needed", fn, project_ws_bytes(n_rows));
+  if ((n_rows + 63) / 64 > 65535) return set_error(LSA_ERR_UNSUPPORTED, "%s: at most 4194240 rows", fn);
+  ProjectLaunch L;
+  L.c_q = reinterpret_cast<const uint16_t*>(c_q);
+  L.hidden = reinterpret_cast<const uint16_t*>(hidden);
+  L.wq_b = reinterpret_cast<const uint16_t*>(wq_b);
+  L.wk = reinterpret_cast<const uint16_t*>(wk);
+  L.wproj = reinterpret_cast<const uint16_t*>(wproj);
+  L.k_norm_w = reinterpret_cast<const uint16_t*>(k_norm_w);
+  L.seq_of_row = seq_of_row;
+  L.pos = pos;
+  L.k_off = k_off;
+  L.n_rows = n_rows;
+  L.n_seq = n_seq;
+  L.q_lora = q_lora_rank;
+  L.hidden_dim = hidden_size;
+  L.max_len = max_len;
+  L.theta = rope_theta;
+  L.q_out = reinterpret_cast<uint16_t*>(q_idx);
+  L.w_out = w;
+  L.k_cache = reinterpret_cast<uint16_t*>(k_cache);
+  L.ws = ws;
+  L.err = device_error_word();
+  return cuda_status(launch_index_project(L, (cudaStream_t)stream), fn);
 }
 
 lsa_status lsa_sparse_mla_decode(const lsa_config* c, int32_t batch, const lsa_bf16* q_abs,

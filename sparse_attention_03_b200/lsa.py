@@ -20,6 +20,7 @@ LIB_PATH = os.path.join(_HERE, "liblsa.so")
 LSA_OK, LSA_DENSE = 0, 1
 LSA_ERR_INVALID, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_DEVICE = -1, -2, -3, -4, -5
 OP_TOPK, OP_MLA_DECODE, OP_MLA_PREFILL, OP_FORWARD_DECODE, OP_FORWARD_PREFILL = 1, 2, 3, 4, 5
+OP_INDEX_PROJECT = 6
 TOPK_HIST_WORDS = 2056
 DEVERR_POS, DEVERR_INDEX, DEVERR_COUNT, DEVERR_SEQ, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 
@@ -27,7 +28,7 @@ EXPORTS = (
     "lsa_config_default", "lsa_workspace_size", "lsa_index_scores", "lsa_topk",
     "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill", "lsa_forward", "lsa_last_error",
     "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16", "lsa_synth_normal_f32",
-    "lsa_synth_rms_rows_bf16", "lsa_launch_count",
+    "lsa_synth_rms_rows_bf16", "lsa_launch_count", "lsa_index_project",
 )
 
 
@@ -77,6 +78,8 @@ def load():
     lib.lsa_forward.argtypes = [ctypes.POINTER(Config), _I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P,
                                 ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
                                 _P, _P, _P, _SZ, _P]
+    lib.lsa_index_project.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P,
+                                      _I32, _I32, ctypes.c_float, _P, _P, _P, _P, _SZ, _P]
     lib.lsa_last_error.argtypes = []
     lib.lsa_last_error.restype = ctypes.c_char_p
     lib.lsa_device_error.argtypes = [ctypes.POINTER(_I32)]
@@ -87,7 +90,7 @@ def load():
     lib.lsa_synth_normal_f32.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
     lib.lsa_synth_rms_rows_bf16.argtypes = [_P, _I64, _I32, _U64, _U64, _I64, _P]
     for name in ("lsa_index_scores", "lsa_topk", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
-                 "lsa_forward", "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16",
+                 "lsa_forward", "lsa_index_project", "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16",
                  "lsa_synth_normal_f32", "lsa_synth_rms_rows_bf16"):
         getattr(lib, name).restype = _I32
     _lib = lib
@@ -234,6 +237,26 @@ def sparse_mla_prefill(cfg, pos, q_abs, latent, idx, count, out, lse, ws, stream
     return _invoke(load().lsa_sparse_mla_prefill, (
         ctypes.byref(cfg._c()), pos.shape[0], _ptr(pos), _ptr(q_abs), _ptr(latent), latent.shape[0],
         _ptr(idx), _ptr(count), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
+        _stream(stream)), bind=bind)
+
+
+def index_project(cfg, seq_of_row, pos, k_off, max_len, c_q, hidden, wq_b, wk, wproj, k_norm_w, q_idx, w, k_cache,
+                  ws, rope_theta=1.0e6, stream=None, bind=False):
+    """The indexer's q_idx [rows, 32, 128] and w [rows, 32] from c_q / hidden, and the
+    rows' keys appended to k_cache (see lsa_index_project in include/lsa.h)."""
+    for t, n in ((c_q, "c_q"), (hidden, "hidden"), (wq_b, "wq_b"), (wk, "wk"), (wproj, "wproj"),
+                 (k_norm_w, "k_norm_w"), (q_idx, "q_idx"), (k_cache, "k_cache")):
+        _dt(t, torch.bfloat16, n)
+    _dt(w, torch.float32, "w"); _dt(pos, torch.int32, "pos")
+    if seq_of_row is not None:
+        _dt(seq_of_row, torch.int32, "seq_of_row")
+    if k_off is not None:
+        _dt(k_off, torch.int64, "k_off")
+    n_seq = 1 if k_off is None else k_off.shape[0] - 1
+    return _invoke(load().lsa_index_project, (
+        ctypes.byref(cfg._c()), pos.shape[0], n_seq, _ptr(seq_of_row), _ptr(pos), _ptr(k_off), int(max_len),
+        _ptr(c_q), _ptr(hidden), _ptr(wq_b), _ptr(wk), _ptr(wproj), _ptr(k_norm_w), c_q.shape[1], hidden.shape[1],
+        float(rope_theta), _ptr(q_idx), _ptr(w), _ptr(k_cache), _ptr(ws), 0 if ws is None else ws.numel(),
         _stream(stream)), bind=bind)
 
 

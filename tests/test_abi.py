@@ -107,3 +107,15 @@ def test_empty_inputs_are_noops(lib):
     assert lib.lsa_topk(ctypes.byref(c), 0, None, 10, None, 10, None, None, None, None, 0, None) == lsa.LSA_DENSE
     assert lib.lsa_sparse_mla_prefill(ctypes.byref(c), 0, None, None, None, 5, None, None, None, None, None,
                                       0, None) == lsa.LSA_OK
+
+
+def test_index_project_validation(lib):
+    c = lsa.LsaConfig().c()
+    args = lambda q_lora, hidden, ws, theta=1.0e6: (ctypes.byref(c), 4, 1, None, _fake(), None, 100, _fake(), _fake(),
+                                                    _fake(), _fake(), _fake(), _fake(), q_lora, hidden, theta,
+                                                    _fake(), _fake(), _fake(), ws, 10 ** 9 if ws else 0, None)
+    assert lib.lsa_index_project(*args(1536, 3000, _fake())) == lsa.LSA_ERR_INVALID     # hidden % 32
+    assert b"multiples of 32" in lib.lsa_last_error()
+    assert lib.lsa_index_project(*args(1536, 3072, None)) == lsa.LSA_ERR_WORKSPACE      # no workspace
+    assert lib.lsa_index_project(*args(1536, 3072, _fake(), 0.5)) == lsa.LSA_ERR_INVALID
+    assert lsa.workspace_size(lsa.LsaConfig(), lsa.OP_INDEX_PROJECT, 16, 16, 100) >= 16 * (4096 + 160) * 4

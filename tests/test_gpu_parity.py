@@ -680,3 +680,83 @@ def test_full_size_prefill_16k_sampled(L):
             eo, el = R.mla(qa, c, ocfg)
             assert_attention(bf16_host_f64(outs[z][r]), lses[z][r].cpu().numpy(), eo, el, check_lse=exact,
                              where=f"prefill row {r} sub {z}")
+
+
+# --------------------------------------------------------------------------
+# The indexer's own projections and the key-cache append (upstream of the path)
+# --------------------------------------------------------------------------
+def _project_inputs(seed, n_rows, q_lora=1536, hidden=3072):
+    f = S.bf16_bits_to_f64
+    c_q = S.normal_bf16(seed, S.tid(0, S.C_Q), 0, n_rows * q_lora).reshape(n_rows, q_lora)
+    h = S.normal_bf16(seed, S.tid(0, S.HIDDEN), 0, n_rows * hidden).reshape(n_rows, hidden)
+    wq_b = S.normal_bf16(seed, S.tid(0, S.WQ_B), 0, 4096 * q_lora, 1 / np.sqrt(q_lora)).reshape(4096, q_lora)
+    wk = S.normal_bf16(seed, S.tid(0, S.WK), 0, 128 * hidden, 1 / np.sqrt(hidden)).reshape(128, hidden)
+    wp = S.normal_bf16(seed, S.tid(0, S.WPROJ), 0, 32 * hidden, 1 / np.sqrt(hidden)).reshape(32, hidden)
+    g = S.f32_to_bf16_bits((1.0 + 0.1 * f(S.normal_bf16(seed, S.tid(0, S.KNORM), 0, 128))).astype(np.float32))
+    return c_q, h, wq_b, wk, wp, g
+
+
+def _pair_bound(m):
+    # |error| after RoPE of a pair (a, b) is at most the sum of both inputs' errors
+    m = m.copy()
+    a, b = m[..., 64:96].copy(), m[..., 96:].copy()
+    m[..., 64:96] = a + b
+    m[..., 96:] = a + b
+    return m
+
+
+def _check_bf16(got, exp, mag, where):
+    # bf16 output: one bf16 ulp (2^-8 relative) of rounding plus the fp32
+    # accumulation error, bounded by 2e-4 x sum |W x| (K <= 3072 terms, 2^-24 each)
+    tol = 2.0 ** -8 * np.abs(exp) + 2e-4 * mag + 1e-30
+    bad = np.abs(got - exp) > tol
+    assert not bad.any(), f"{where}: {bad.sum()} elements off, worst {np.abs(got - exp)[bad].max():.3g}"
+
+
+def _project_check(L, seed, lengths, rows_pos, k_off_given=True):
+    f = S.bf16_bits_to_f64
+    c_q, h, wq_b, wk, wp, g = _project_inputs(seed, len(rows_pos))
+    lengths = np.asarray(lengths, dtype=np.int64)
+    off = S.offsets(lengths)
+    total = int(off[-1])
+    cache0 = S.normal_bf16(seed, S.tid(1, S.K_IDX), 0, total * 128).reshape(total, 128)
+    k_cache = bf16_dev(cache0)
+    n = len(rows_pos)
+    seq = np.array([s for s, _ in rows_pos], dtype=np.int32)
+    pos = np.array([p for _, p in rows_pos], dtype=np.int32)
+    q_out = torch.empty((n, 32, 128), dtype=torch.bfloat16, device="cuda")
+    w_out = torch.empty((n, 32), device="cuda")
+    cfg = L.LsaConfig()
+    ws = L.workspace(cfg, L.OP_INDEX_PROJECT, n, 1, int(lengths.max()))
+    L.index_project(cfg, i32_dev(seq) if k_off_given else None, i32_dev(pos), i64_dev(off) if k_off_given else None,
+                    int(lengths.max()), bf16_dev(c_q), bf16_dev(h), bf16_dev(wq_b), bf16_dev(wk), bf16_dev(wp),
+                    bf16_dev(g), q_out, w_out, k_cache, ws)
+    assert L.device_error() == 0
+    gq, gw = bf16_host_f64(q_out), w_out.cpu().numpy().astype(np.float64)
+    gk = k_cache.view(torch.int16).cpu().numpy().view(np.uint16)
+    slots = (off[seq] + pos) if k_off_given else pos.astype(np.int64)
+    untouched = np.ones(total, dtype=bool)
+    untouched[slots] = False
+    np.testing.assert_array_equal(gk[untouched], cache0[untouched])   # only the rows' own slots change
+    Wq, Wk, Wp, G = f(wq_b), f(wk), f(wp), f(g)
+    for r in range(n):
+        cq, hr = f(c_q[r]), f(h[r])
+        q, k, w = R.index_project_row(cq, hr, Wq, Wk, Wp, G, int(pos[r]))
+        mq = _pair_bound((np.abs(Wq) @ np.abs(cq)).reshape(32, 128))
+        raw = Wk @ hr
+        scale = np.abs(G) / np.sqrt(np.mean(raw * raw) + 1e-6)
+        mk = _pair_bound(scale * (np.abs(Wk) @ np.abs(hr)))
+        _check_bf16(gq[r], q, mq, f"q row {r}")
+        _check_bf16(f(gk[slots[r]]), k, mk, f"k row {r}")
+        assert np.all(np.abs(gw[r] - w) <= 2e-4 * (np.abs(Wp) @ np.abs(hr))), f"w row {r}"
+
+
+def test_index_project_decode_varlen(L):
+    # one new token per sequence, at the last slot of its (already extended) cache
+    lengths = [3, 100, 2050, 5000, 777, 100000]
+    _project_check(L, 31, lengths, [(b, lengths[b] - 1) for b in range(len(lengths))])
+
+
+def test_index_project_prefill_rows(L):
+    # rows of one sequence at positions 2000 .. 2299 (tiles of 64 rows, a ragged last one)
+    _project_check(L, 32, [2300], [(0, 2000 + t) for t in range(300)], k_off_given=False)
