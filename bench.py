@@ -15,7 +15,8 @@ oracle on a bounded sample, an end-to-end number through lsa_forward with
 pinned host buffers and host<->device copies inside the timed region, and an
 MTP draft round ("mtp": one index pass and top-k per layer shared by three
 draft steps of sparse MLA over one latent cache; tokens = 3 per sequence per
-layer per round).
+layer per round), and the indexer's own projections with the key-cache append
+("project": one decode token per sequence per layer, with its HBM roofline).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
@@ -302,6 +303,40 @@ def build_decode(device):
     return D
 
 
+def build_project(D, device):
+    """Per layer: the indexer's projection weights (wq_b, wk, weights_proj, key-norm
+    weight) and one decode token's q-LoRA vector and hidden state per sequence."""
+    import torch
+    from sparse_attention_03_b200 import lsa
+    import lsa_synth as S
+    B, nl = DECODE["batch"], DECODE["layers"]
+    ql, hd = 1536, 3072
+    P = []
+    for i, l in enumerate(D["layers"]):
+        def draw(shape, kind, sigma=1.0):
+            t = torch.empty(shape, dtype=torch.bfloat16, device=device)
+            lsa.synth_normal_bf16(t, 0, S.tid(200 + i, kind), sigma=sigma)
+            return t
+        wq_b, wk, wp = draw((4096, ql), S.WQ_B, ql ** -0.5), draw((128, hd), S.WK, hd ** -0.5), draw((32, hd), S.WPROJ, hd ** -0.5)
+        g = (1.0 + 0.1 * draw((128,), S.KNORM).float()).to(torch.bfloat16)
+        c_q, h = draw((B, ql), S.C_Q), draw((B, hd), S.HIDDEN)
+        q_out = torch.empty((B, 32, 128), dtype=torch.bfloat16, device=device)
+        w_out = torch.empty((B, 32), dtype=torch.float32, device=device)
+        ws = lsa.workspace(D["cfg"], lsa.OP_INDEX_PROJECT, B, B, D["ctx"], device=device)
+        P.append(dict(keep=(wq_b, wk, wp, g, c_q, h, q_out, w_out, ws),
+                      call=lsa.index_project(D["cfg"], l.seq_of_row, l.pos, l.k_off, D["ctx"], c_q, h, wq_b, wk, wp,
+                                             g, q_out, w_out, l.k_idx, ws, bind=True)))
+    D["project"] = P
+    wbytes = (4096 * ql + 128 * hd + 32 * hd + 128) * 2
+    io = B * ((ql + hd) * 2 + 32 * 128 * 2 + 32 * 4 + 128 * 2)
+    D["project_bytes"] = wbytes + io
+
+
+def project_step(D):
+    for p in D["project"]:
+        p["call"]()
+
+
 def mtp_round(D):
     """One MTP draft round through every layer: the index pass and top-k once,
     then three draft steps of sparse MLA over that one selection."""
@@ -478,6 +513,17 @@ def gpu_arm(args):
     h2d = sum(x.numel() * x.element_size() for x in h_in)
     d2h = h_out.numel() * h_out.element_size()
 
+    # the indexer's own projections and key append for one decode token per sequence
+    # (runs after the timed decode step: it rewrites the newest key row of each cache)
+    build_project(D, device)
+    D_bytes = D["project_bytes"]
+    for _ in range(3):
+        project_step(D)
+    pj_steps = max(5, args.steps // 2)
+    tp = time_region(lambda s: project_step(D), pj_steps, world, device)
+    pj_value, _ = aggregate(B * nl * pj_steps, tp, world, device)
+    pj_layer_s = tp / (pj_steps * nl)
+
     # MTP draft rounds (three draft tokens per sequence and layer per round)
     for _ in range(3):
         mtp_round(D)
@@ -510,6 +556,11 @@ def gpu_arm(args):
         "gpu_launches": launches,
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
+    line["project"] = {"value": pj_value, "unit": "tokens/s/layer", "us_per_layer": 1e6 * pj_layer_s,
+                       "config": {"workload": "index_project_b16_qlora1536_hidden3072_14layers"},
+                       "roofline": {"bound": "hbm", "achieved": D_bytes / pj_layer_s / 1e9, "peak": peak,
+                                    "unit": "GB/s", "frac": D_bytes / pj_layer_s / 1e9 / peak,
+                                    "peak_source": f"{psrc} hbm_gbs"}}
     line["mtp"] = {"value": mtp_value, "unit": "tokens/s/layer", "ms_per_round": 1e3 * tm / mtp_steps,
                    "config": {"workload": "mtp_draft_round_b16_ctx131072_14layers", "draft_steps": 3,
                               "index_passes_per_round": 1}}

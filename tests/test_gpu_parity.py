@@ -713,9 +713,9 @@ def _check_bf16(got, exp, mag, where):
     assert not bad.any(), f"{where}: {bad.sum()} elements off, worst {np.abs(got - exp)[bad].max():.3g}"
 
 
-def _project_check(L, seed, lengths, rows_pos, k_off_given=True):
+def _project_check(L, seed, lengths, rows_pos, k_off_given=True, q_lora=1536, hidden=3072):
     f = S.bf16_bits_to_f64
-    c_q, h, wq_b, wk, wp, g = _project_inputs(seed, len(rows_pos))
+    c_q, h, wq_b, wk, wp, g = _project_inputs(seed, len(rows_pos), q_lora, hidden)
     lengths = np.asarray(lengths, dtype=np.int64)
     off = S.offsets(lengths)
     total = int(off[-1])
@@ -755,6 +755,21 @@ def test_index_project_decode_varlen(L):
     # one new token per sequence, at the last slot of its (already extended) cache
     lengths = [3, 100, 2050, 5000, 777, 100000]
     _project_check(L, 31, lengths, [(b, lengths[b] - 1) for b in range(len(lengths))])
+
+
+def test_index_project_row_blocks(L):
+    # 37 rows over 4 sequences: three 16-row blocks of the fused decode launch, the last ragged
+    lengths = [40, 9000, 1, 300]
+    rows = [(b, lengths[b] - 1 - i) for b in range(4) for i in range(min(lengths[b], 12))][:37]
+    assert len(rows) == 37
+    _project_check(L, 33, lengths, rows)
+
+
+@pytest.mark.parametrize("q_lora,hidden,n", [(512, 1024, 64), (160, 224, 5), (1536, 3072, 65)])
+def test_index_project_dims(L, q_lora, hidden, n):
+    # fused launch at its row limit; K not a multiple of 512 (tiled GEMMs with split K on
+    # few rows); one row past the fused limit
+    _project_check(L, 34, [n + 10], [(0, 10 + t) for t in range(n)], q_lora=q_lora, hidden=hidden)
 
 
 def test_index_project_prefill_rows(L):
