@@ -229,3 +229,72 @@ def index_project_row(c_q, h, wq_b, wk, wproj, k_norm_w, pos, theta=ROPE_THETA, 
     k = rope(rms_norm(np.asarray(wk, np.float64) @ np.asarray(h, np.float64), k_norm_w, eps), pos, theta)
     w = np.asarray(wproj, np.float64) @ np.asarray(h, np.float64)
     return q, k, w
+
+
+# ---------------------------------------------------------------------------
+# Hierarchical indexing ([LSA-2.0] 分层索引): coarse-to-fine, two-stage scoring;
+# approximate block-level scores first, then token-level selection inside the
+# surviving blocks, so the indexer's candidate space shrinks.
+# The page gives only that structure. Readings:
+# * a block is `block` consecutive cached keys of one sequence (block b holds
+#   positions b*block .. b*block + block - 1; the last one may be short);
+# * a block's approximate score is the indexer's own score of the block's
+#   summary key, the mean of its keys, rounded once to bf16 like every stored
+#   key;
+# * the coarse stage is the flat selection one level up: a row at position p
+#   sees blocks 0 .. p // block; the ceil(n_init / block) sink blocks and the
+#   ceil(n_loc / block) + 1 most recent blocks are forced in (together they
+#   hold every forced token), and the n_blocks best of the others are kept,
+#   ties to the lower block, with the same dense fallback (every block kept
+#   when the row sees no more than that many);
+# * the fine stage is the flat selection (mask, forcing, top-k, dense
+#   fallback) over the tokens of the kept blocks only.
+# ---------------------------------------------------------------------------
+HIER_BLOCK, HIER_BLOCKS = 64, 128
+
+
+def bf16_round(x) -> np.ndarray:
+    """fp64 -> the nearest bf16 value (8 significant bits, ties to even), as fp64.
+    Finite, normal-range inputs; computed on the fp64 bit pattern directly."""
+    b = np.ascontiguousarray(np.asarray(x, dtype=np.float64)).view(np.uint64)
+    drop = np.uint64(52 - 7)                       # fp64 keeps 52 fraction bits, bf16 7
+    half = np.uint64(1) << (drop - np.uint64(1))
+    lsb = (b >> drop) & np.uint64(1)
+    r = (b + half - np.uint64(1) + lsb) >> drop << drop
+    return r.view(np.float64)
+
+
+def block_summaries(k_seq: np.ndarray, block: int = HIER_BLOCK) -> np.ndarray:
+    """Summary keys of every block of one sequence's cache k_seq [L, d]: the mean
+    of the block's keys, rounded to bf16 -> [ceil(L / block), d]."""
+    k = np.asarray(k_seq, dtype=np.float64)
+    n = -(-k.shape[0] // block)
+    return np.stack([bf16_round(k[b * block:(b + 1) * block].mean(axis=0)) for b in range(n)])
+
+
+def hier_config(cfg: LsaConfig, block: int, n_blocks: int) -> LsaConfig:
+    """The flat selection's constants one level up (blocks instead of tokens)."""
+    n_init = -(-cfg.index_init_tokens // block)
+    n_loc = -(-cfg.index_local_tokens // block) + 1
+    return LsaConfig(index_topk=n_init + n_loc + n_blocks, index_init_tokens=n_init, index_local_tokens=n_loc,
+                     cli_factor=cfg.cli_factor)
+
+
+def hier_select(q, w, k_seq, k_blk, p, cfg: LsaConfig = PAGES, block: int = HIER_BLOCK,
+                n_blocks: int = HIER_BLOCKS):
+    """Hierarchical selection of one query row at position p over its sequence's
+    keys k_seq [L, d] and block summaries k_blk [ceil(L / block), d].
+
+    Returns (selected columns (sorted), dense flag, kept blocks (sorted)).
+    """
+    pb = p // block
+    bcfg = hier_config(cfg, block, n_blocks)
+    coarse = score_row(q, w, k_blk[: pb + 1])
+    kept, _ = select_topk(mask_and_force(coarse, pb, pb + 1, bcfg), pb, bcfg)
+    n = p + 1
+    if n <= cfg.index_topk:
+        return np.arange(n, dtype=np.int64), True, kept
+    cand = np.concatenate([np.arange(b * block, min((b + 1) * block, n)) for b in kept])
+    s = mask_and_force(score_row(q, w, k_seq[: p + 1]), p, p + 1, cfg)[cand]
+    order = np.lexsort((cand, -s))                 # score descending, then lower column
+    return np.sort(cand[order[: cfg.index_topk]]).astype(np.int64), False, kept

@@ -383,3 +383,147 @@ def test_index_project_layout_and_pieces():
     q5, k5, _ = R.index_project_row(c_q, h, wq_b, wk, wp, g, pos=5)
     np.testing.assert_allclose(q5, R.rope(q, 5), rtol=1e-12)
     np.testing.assert_allclose(k5, R.rope(k, 5), rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------
+# Hierarchical indexing ([LSA-2.0] 分层索引)
+# ---------------------------------------------------------------------------
+def test_bf16_round_ties_and_halfway():
+    one = 1.0
+    ulp = 2.0 ** -7
+    cases = {
+        one + ulp / 2: one,                        # tie -> even (1.0)
+        one + 3 * ulp / 2: one + 2 * ulp,          # tie -> even (1 + 2 ulp)
+        one + ulp / 2 + 2.0 ** -40: one + ulp,     # just above the tie rounds up
+        one + ulp / 2 - 2.0 ** -40: one,           # just below rounds down
+        -(one + 3 * ulp / 2): -(one + 2 * ulp),
+        255.5: 256.0,                              # 8 significant bits: 255.5 is a tie, 256 is even
+        3.0 * 2.0 ** -100: 3.0 * 2.0 ** -100,      # already representable
+    }
+    got = R.bf16_round(np.array(list(cases)))
+    np.testing.assert_array_equal(got, np.array(list(cases.values())))
+
+
+def test_bf16_round_matches_torch_on_fp32_values():
+    # inputs exactly representable in fp32, where torch's conversion rounds once
+    x = np.random.default_rng(3).standard_normal(20000).astype(np.float32).astype(np.float64)
+    ref = torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(R.bf16_round(x), ref)
+
+
+def test_block_summaries_closed_forms():
+    k = np.zeros((10, 3))
+    k[0:4] = [1.0, 2.0, -3.0]                      # a block of identical keys -> that key
+    k[4:8] = [[0, 0, 1], [0, 0, 3], [1, 1, 5], [3, 1, 7]]   # mean (1, 0.5, 4)
+    k[8:10] = [[2, 4, 8], [4, 8, 16]]              # short last block: mean of its 2 keys
+    s = R.block_summaries(k, 4)
+    np.testing.assert_array_equal(s, [[1, 2, -3], [1, 0.5, 4], [3, 6, 12]])
+
+
+def test_hier_config_forced_blocks_cover_forced_tokens():
+    # every forced token lies in a forced block, for every alignment of p
+    for cfg, block in ((TINY, 4), (TINY, 2), (PAGES, 64), (PAGES, 16), (PAGES, 128)):
+        bcfg = R.hier_config(cfg, block, 4)
+        for p in range(0, 4 * cfg.index_local_tokens + 3 * block, max(1, block // 3)):
+            pb = p // block
+            j = np.arange(p + 1)
+            forced = j[(j < cfg.index_init_tokens) | (j >= p + 1 - cfg.index_local_tokens)]
+            b = np.arange(pb + 1)
+            fb = set(b[(b < bcfg.index_init_tokens) | (b >= pb + 1 - bcfg.index_local_tokens)].tolist())
+            assert set((forced // block).tolist()) <= fb, (cfg, block, p)
+
+
+def _rand_case(rng, L, d=8, heads=4):
+    q = rng.standard_normal((heads, d))
+    w = rng.standard_normal(heads)
+    k = R.bf16_round(rng.standard_normal((L, d)))
+    return q, w, k
+
+
+@pytest.mark.parametrize("trial", range(6))
+def test_hier_with_every_block_kept_is_flat_lsa(trial):
+    # n_blocks at least the number of blocks: the coarse stage keeps everything and
+    # the result is the flat selection
+    rng = np.random.default_rng(100 + trial)
+    L, block = 300, 8
+    q, w, k = _rand_case(rng, L)
+    kb = R.block_summaries(k, block)
+    for p in (3, 7, 8, 9, 100, 299):
+        sel, dense, kept = R.hier_select(q, w, k, kb, p, TINY, block, n_blocks=L)
+        np.testing.assert_array_equal(kept, np.arange(p // block + 1))
+        flat, fdense = R.select_topk(R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, L, TINY), p, TINY)
+        assert dense == fdense
+        np.testing.assert_array_equal(sel, flat)
+
+
+def _brute_hier(q, w, k, p, cfg, block, n_blocks):
+    # independent restatement with explicit loops and tuple sorts
+    nb = p // block + 1
+    n_init = math.ceil(cfg.index_init_tokens / block)
+    n_loc = math.ceil(cfg.index_local_tokens / block) + 1
+    def score(key):
+        return sum(w[h] * max(float(np.dot(q[h], key)), 0.0) for h in range(len(w)))
+    means = []
+    for b in range(nb):
+        rows = k[b * block: min((b + 1) * block, len(k))]
+        means.append(R.bf16_round(sum(rows) / len(rows)))
+    if nb <= n_init + n_loc + n_blocks:
+        kept = list(range(nb))
+    else:
+        forced = [b for b in range(nb) if b < n_init or b >= nb - n_loc]
+        rest = sorted((b for b in range(nb) if b not in forced), key=lambda b: (-score(means[b]), b))
+        kept = sorted(forced + rest[:n_blocks])
+    if p + 1 <= cfg.index_topk:
+        return list(range(p + 1)), kept
+    cand = [j for b in kept for j in range(b * block, min((b + 1) * block, p + 1))]
+    def key(j):
+        forced = j < cfg.index_init_tokens or j >= p + 1 - cfg.index_local_tokens
+        return (0 if forced else 1, -score(k[j]) if not forced else 0.0, j)
+    return sorted(sorted(cand, key=key)[: cfg.index_topk]), kept
+
+
+@pytest.mark.parametrize("trial", range(10))
+def test_hier_brute_force_tiny(trial):
+    rng = np.random.default_rng(200 + trial)
+    L, block, nbk = 90, 4, 3
+    q, w, k = _rand_case(rng, L)
+    kb = R.block_summaries(k, block)
+    for p in (5, 9, 20, 47, 60, 89):
+        sel, dense, kept = R.hier_select(q, w, k, kb, p, TINY, block, nbk)
+        bsel, bkept = _brute_hier(q, w, k, p, TINY, block, nbk)
+        np.testing.assert_array_equal(kept, bkept)
+        np.testing.assert_array_equal(sel, bsel)
+
+
+def test_hier_planted_blocks_survive():
+    # keys of blocks 10 and 20 point along the query; everything else is orthogonal
+    rng = np.random.default_rng(7)
+    L, block, d = 2000, 16, 8
+    q = np.zeros((2, d)); q[:, 0] = 1.0
+    w = np.array([1.0, 0.5])
+    k = np.zeros((L, d)); k[:, 1:] = R.bf16_round(rng.standard_normal((L, d - 1)))
+    k[10 * block:11 * block, 0] = 2.0
+    k[20 * block:21 * block, 0] = 1.0
+    kb = R.block_summaries(k, block)
+    cfg = LsaConfig(index_topk=24, index_init_tokens=2, index_local_tokens=4)
+    sel, dense, kept = R.hier_select(q, w, k, kb, L - 1, cfg, block, n_blocks=2)
+    # sink block 0, the ceil(4/16)+1 = 2 most recent blocks, and the planted two
+    np.testing.assert_array_equal(kept, [0, 10, 20, 123, 124])
+    # forced tokens (0, 1, and the last 4) plus the 16 keys of block 10 and the
+    # lowest-index 2 of block 20 (all its keys tie)
+    expect = sorted([0, 1, *range(L - 4, L), *range(160, 176), 320, 321])
+    np.testing.assert_array_equal(sel, expect)
+    assert not dense
+
+
+def test_hier_kept_sets_nest_with_n_blocks():
+    rng = np.random.default_rng(11)
+    L, block = 3000, 16
+    q, w, k = _rand_case(rng, L)
+    kb = R.block_summaries(k, block)
+    prev = None
+    for nbk in (1, 2, 5, 10, 40, 200):
+        _, _, kept = R.hier_select(q, w, k, kb, L - 1, PAGES, block, nbk)
+        if prev is not None:
+            assert set(prev) <= set(kept)
+        prev = kept
