@@ -231,6 +231,56 @@ LSA_API lsa_status lsa_index_project(const lsa_config* cfg, int32_t n_rows, int3
                                      size_t ws_bytes, void* stream);
 
 /*
+ * Hierarchical indexing ([LSA-2.0] "分层索引": coarse-to-fine two-stage
+ * scoring, approximate block-level scores first, then token selection inside
+ * the surviving blocks, so the indexer handles a smaller candidate space).
+ * The page gives only that structure; the readings taken are: a block is
+ * `block` consecutive cached keys of one sequence; its summary key is the mean
+ * of its keys rounded once to bf16; the coarse stage is the flat selection one
+ * level up (the ceil(init/block) sink blocks and the ceil(local/block) + 1 most
+ * recent blocks forced in, the n_blocks best other blocks kept, ties to the
+ * lower block, every block kept when the row sees no more than that many); the
+ * fine stage is the flat selection (mask, forcing, top-k, dense fallback) over
+ * the tokens of the kept blocks.
+ *
+ * lsa_block_summaries: for each item i, the summary of block item_blk[i] of
+ * sequence item_seq[i] (the mean of its keys at positions < the sequence's
+ * length, in fp64, rounded to nearest-even bf16). Call it for every block at
+ * build time and, after each append, for the block holding the new key.
+ *   k_idx: packed [sum L, 128] bf16 with k_off int64 [n_seq+1] (as lsa_index_scores).
+ *   blk_off: int64 [n_seq+1], blk_off[s+1] - blk_off[s] >= ceil(L_s / block).
+ *   k_blk: packed [blk_off[n_seq], 128] bf16 (16-byte aligned), caller-owned.
+ *   block: 16 .. 1024, a multiple of 16.
+ * An item naming a sequence or block out of range is skipped and sets
+ * LSA_DEVERR_SEQ / LSA_DEVERR_POS.
+ */
+LSA_API lsa_status lsa_block_summaries(const lsa_config* cfg, int32_t n_items, int32_t n_seq,
+                                       const int32_t* item_seq, const int32_t* item_blk, const lsa_bf16* k_idx,
+                                       const int64_t* k_off, const int64_t* blk_off, int32_t block,
+                                       lsa_bf16* k_blk, void* stream);
+
+/*
+ * lsa_hier_select: the two-stage selection of every row, output as lsa_topk's
+ * (idx int32 [n_rows, index_topk] unordered, count int32 [n_rows]; rows with
+ * pos + 1 <= index_topk are dense: 0..pos).
+ *   Rows, queries and keys as lsa_index_scores (seq_of_row NULL: sequence 0);
+ *   k_blk / blk_off as written by lsa_block_summaries for the same caches.
+ *   n_blocks: blocks kept by score per row; n_blocks * block >= index_topk, and
+ *   the coarse selection's size ceil(init/block) + ceil(local/block) + 1 +
+ *   n_blocks <= 2048.
+ *   Workspace: lsa_hier_workspace_size(cfg, n_rows, max_len, block, n_blocks).
+ * Returns LSA_DENSE when max_len <= index_topk (every row dense).
+ */
+LSA_API size_t lsa_hier_workspace_size(const lsa_config* cfg, int32_t n_rows, int64_t max_len, int32_t block,
+                                       int32_t n_blocks);
+LSA_API lsa_status lsa_hier_select(const lsa_config* cfg, int32_t n_rows, int32_t n_seq,
+                                   const int32_t* seq_of_row, const int32_t* pos, const lsa_bf16* q_idx,
+                                   const float* w, const lsa_bf16* k_idx, const int64_t* k_off,
+                                   const lsa_bf16* k_blk, const int64_t* blk_off, int64_t max_len, int32_t block,
+                                   int32_t n_blocks, int32_t* idx, int32_t* count, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/*
  * Sparse absorbed-latent MLA, decode ([Lite-Sparse] LSA section: at decode
  * the latent rows are gathered by the top-k indices; 架构总览: kv_lora_rank 512,
  * qk_rope_head_dim 64, 32 heads).

@@ -28,6 +28,7 @@ namespace {
 constexpr int kWarps = 4;
 constexpr int kThreads = kWarps * 32;
 constexpr int kKeysPerWarpTile = 16;
+constexpr int kMaxHierBlocks = 2048;  // kept blocks per row (the top-k's own limit)
 
 struct KeyFrag {
   uint4 lo[4];  // key g:   physical dims 8*(4c+t) .. +7, c = 0..3
@@ -187,6 +188,111 @@ __global__ void __launch_bounds__(kThreads, 3)
   }
 }
 
+
+// ---------------------------------------------------------------------------
+// Hierarchical indexing, fine stage ([LSA-2.0] "分层索引"): the same scoring
+// over only the tokens of each row's kept blocks, written to a compact row
+// (slot i = token sorted[i / block] * block + i % block, blocks in ascending
+// order so that the top-k's lower-slot tie rule is the lower-column rule).
+// Forced tokens are +inf, tokens after the row's position -inf.
+__global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, int blocks_per_cta) {
+  __shared__ int32_t ids[kMaxHierBlocks];
+  __shared__ int32_t srt[kMaxHierBlocks];
+  pdl_wait();
+  const IndexArgs& a = h.ix;
+  const int r = blockIdx.y;
+  const int n = min(h.kept_n[r], h.kb);
+  const int32_t* __restrict__ kr = h.kept + (int64_t)r * h.kb;
+  // (a kept id is a visible block, >= 0; clamping and pre-filling keep every
+  // token index below non-negative even for a malformed list)
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    ids[i] = max(kr[i], 0);
+    srt[i] = 0;
+  }
+  __syncthreads();
+  // ascending order by counting (the ids of a row are distinct)
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    const int v = ids[i];
+    int rank = 0;
+    for (int j = 0; j < n; ++j) rank += ids[j] < v;
+    srt[rank] = v;
+  }
+  __syncthreads();
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < n; i += kThreads) h.sorted[(int64_t)r * h.kb + i] = srt[i];
+    if (threadIdx.x == 0) h.pos_c[r] = n * h.block - 1;
+  }
+
+  // row geometry, clamped and flagged as in the flat indexer
+  const int seq = a.seq_of_row ? a.seq_of_row[r] : (a.seq_identity ? r : 0);
+  int64_t kbase = 0, klen = a.max_len;
+  bool ok = true;
+  if (seq < 0 || seq >= a.n_seq) {
+    ok = false;
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(a.err, LSA_DEVERR_SEQ);
+  } else if (a.k_off) {
+    kbase = a.k_off[seq];
+    klen = a.k_off[seq + 1] - kbase;
+  }
+  const int64_t p = a.pos[r];
+  int64_t nvis = p + 1;
+  if (ok && (p < 0 || nvis > klen || nvis > a.max_len)) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(a.err, LSA_DEVERR_POS);
+    nvis = max64(0, min(nvis, min(klen, a.max_len)));
+  }
+  if (!ok) nvis = 0;
+
+  const int64_t s_lo = (int64_t)blockIdx.x * blocks_per_cta * h.block;
+  const int64_t s_hi = min((int64_t)(blockIdx.x + 1) * blocks_per_cta, (int64_t)n) * h.block;
+  if (s_lo >= s_hi) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  uint4 qf[4][4];
+  const uint16_t* __restrict__ qr = a.q_idx + (int64_t)r * kHi * kDi;
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      qf[nt][c] = __ldg(reinterpret_cast<const uint4*>(qr + (8 * nt + g) * kDi + 8 * (4 * c + t)));
+  float wf[4][2];
+#pragma unroll
+  for (int nt = 0; nt < 4; ++nt)
+#pragma unroll
+    for (int e = 0; e < 2; ++e) wf[nt][e] = __ldg(a.w + (int64_t)r * kHi + 8 * nt + 2 * t + e);
+  const uint16_t* __restrict__ kb = a.k_idx + kbase * kDi;
+  const int64_t lo_force = a.n_init, hi_force = p + 1 - a.n_loc;
+  float* __restrict__ crow = h.cand + (int64_t)r * h.ld_c;
+  // slot tiles of 16 (a block is a multiple of 16 keys, so a tile never straddles two)
+  auto tok = [&](int64_t s) { return (int64_t)srt[s / h.block] * h.block + s % h.block; };
+  auto put = [&](int64_t s, float sa, float sb) {
+    if (t < 2) {
+      const int64_t j = tok(s) + g + (t == 1 ? 8 : 0);
+      const bool forced = (j < lo_force) || (j >= hi_force);
+      crow[s + g + (t == 1 ? 8 : 0)] = j >= nvis ? -INFINITY : forced ? INFINITY : (t == 1 ? sb : sa);
+    }
+  };
+  const int64_t step = kWarps * kKeysPerWarpTile;
+  int64_t s = s_lo + warp * kKeysPerWarpTile;
+  if (s >= s_hi) return;
+  KeyFrag f0, f1;
+  load_keys(f0, kb, tok(s) + g, nvis, t);
+  while (true) {
+    int64_t nxt = s + step;
+    if (nxt < s_hi) load_keys(f1, kb, tok(nxt) + g, nvis, t);
+    float sa, sb;
+    score_tile(f0, qf, wf, sa, sb);
+    put(s, sa, sb);
+    if (nxt >= s_hi) break;
+    s = nxt;
+    nxt = s + step;
+    if (nxt < s_hi) load_keys(f0, kb, tok(nxt) + g, nvis, t);
+    score_tile(f1, qf, wf, sa, sb);
+    put(s, sa, sb);
+    if (nxt >= s_hi) break;
+    s = nxt;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st, uint32_t* hist, int topk) {
@@ -226,6 +332,40 @@ cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st, uint32_t* h
     count_launches(1);
   }
   return cudaGetLastError();
+}
+
+}  // namespace lsa
+
+namespace lsa {
+
+cudaError_t launch_hier_fine(const HierFineArgs& h, cudaStream_t st) {
+  if (h.ix.n_rows <= 0) return cudaSuccess;
+  if (h.kb > kMaxHierBlocks || h.block % kKeysPerWarpTile != 0) return cudaErrorInvalidValue;
+  // one wave of CTAs (three per SM), each a whole number of kept blocks
+  int sms = 148, dev = 0;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t wave = 3LL * sms;
+  const int64_t per_row = max64(1, wave / h.ix.n_rows);
+  const int bpc = (int)max64(1, (h.kb + per_row - 1) / per_row);
+  const int nx = (h.kb + bpc - 1) / bpc;
+  for (int row0 = 0; row0 < h.ix.n_rows; row0 += 65535) {
+    HierFineArgs b = h;
+    const int ny = min(65535, h.ix.n_rows - row0);
+    b.ix.n_rows = ny;
+    b.ix.pos += row0;
+    if (b.ix.seq_of_row) b.ix.seq_of_row += row0;
+    b.ix.q_idx += (int64_t)row0 * kHi * kDi;
+    b.ix.w += (int64_t)row0 * kHi;
+    b.kept += (int64_t)row0 * h.kb;
+    b.kept_n += row0;
+    b.sorted += (int64_t)row0 * h.kb;
+    b.pos_c += row0;
+    b.cand += (int64_t)row0 * h.ld_c;
+    const cudaError_t e = launch_pdl(hier_fine_kernel, dim3(nx, ny), dim3(kThreads), 0, st, b, bpc);
+    if (e != cudaSuccess) return e;
+    count_launches(1);
+  }
+  return cudaSuccess;
 }
 
 }  // namespace lsa

@@ -114,3 +114,42 @@ int mla_choose_splits(int n_rows, int cli, int64_t max_list);
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st);
 
 }  // namespace lsa
+
+namespace lsa {
+
+// Hierarchical indexing: block summaries, and the pieces of the two-stage
+// selection that are not the flat indexer and top-k themselves.
+struct BlockSumArgs {
+  const uint16_t* k_idx;   // packed [sum L, 128] bf16
+  const int64_t* k_off;    // [n_seq+1]
+  const int64_t* blk_off;  // [n_seq+1]
+  const int32_t* item_seq;
+  const int32_t* item_blk;
+  int n_items, n_seq, block;
+  uint16_t* k_blk;         // packed [sum ceil(L/block), 128] bf16
+  int* err;
+};
+cudaError_t launch_block_summaries(const BlockSumArgs& a, cudaStream_t st);
+
+// pos_b[r] = pos[r] / block (-1 for a negative position).
+cudaError_t launch_hier_prep(const int32_t* pos, int n_rows, int block, int32_t* pos_b, cudaStream_t st);
+
+struct HierFineArgs {
+  IndexArgs ix;             // token-level rows, keys and forcing (scores unused)
+  const int32_t* kept;      // [n_rows, kb] kept blocks, unordered
+  const int32_t* kept_n;    // [n_rows]
+  int kb, block;
+  int32_t* sorted;          // out [n_rows, kb]: the kept blocks in ascending order
+  int32_t* pos_c;           // out [n_rows]: kept_n * block - 1
+  float* cand;              // out [n_rows, ld_c]: slot i = token sorted[i / block] * block + i % block
+  int64_t ld_c;
+};
+// Scores the tokens of each row's kept blocks into the compact rows.
+cudaError_t launch_hier_fine(const HierFineArgs& a, cudaStream_t st);
+
+// Maps compact selections to token columns in place; dense rows (pos + 1 <=
+// topk) get 0..pos.
+cudaError_t launch_hier_map(const int32_t* pos, const int32_t* sorted, int kb, int block, int n_rows, int topk,
+                            int32_t* idx, int32_t* count, cudaStream_t st);
+
+}  // namespace lsa

@@ -176,6 +176,47 @@ MlaArgs mla_args(const lsa_config* c, int cli, int n_rows, int decode) {
   return a;
 }
 
+
+// Hierarchical selection: the block-level constants and the workspace layout.
+struct HierPlan {
+  int n_init_b, n_loc_b, kb;  // forced sink / recent blocks, blocks kept per row
+  int64_t nb_max, ld_b, ld_c; // blocks per row at most, coarse and compact row strides
+  size_t off_pos_b, off_pos_c, off_coarse, off_kept, off_kept_n, off_sorted, off_cand, off_topk, total;
+};
+
+HierPlan hier_plan(const lsa_config* c, int n_rows, int64_t max_len, int block, int n_blocks) {
+  HierPlan h;
+  h.n_init_b = (c->index_init_tokens + block - 1) / block;
+  h.n_loc_b = (c->index_local_tokens + block - 1) / block + 1;
+  h.kb = h.n_init_b + h.n_loc_b + n_blocks;
+  h.nb_max = (max_len + block - 1) / block;
+  h.ld_b = (h.nb_max + 3) / 4 * 4;
+  h.ld_c = (int64_t)h.kb * block;
+  const size_t R = (size_t)n_rows;
+  size_t o = 0;
+  h.off_pos_b = o;  o += align_up(R * 4);
+  h.off_pos_c = o;  o += align_up(R * 4);
+  h.off_coarse = o; o += align_up(R * h.ld_b * 4);
+  h.off_kept = o;   o += align_up(R * h.kb * 4);
+  h.off_kept_n = o; o += align_up(R * 4);
+  h.off_sorted = o; o += align_up(R * h.kb * 4);
+  h.off_cand = o;   o += align_up(R * h.ld_c * 4);
+  h.off_topk = o;   o += topk_ws(n_rows);
+  h.total = o + kAlign;
+  return h;
+}
+
+lsa_status check_hier(const lsa_config* c, int block, int n_blocks, const char* fn) {
+  if (block < 16 || block > 1024 || block % 16 != 0)
+    return set_error(LSA_ERR_UNSUPPORTED, "%s: block must be a multiple of 16 in [16, 1024]", fn);
+  if (n_blocks < 1 || (int64_t)n_blocks * block < c->index_topk)
+    return set_error(LSA_ERR_UNSUPPORTED, "%s: need n_blocks >= 1 and n_blocks * block >= index_topk", fn);
+  const int64_t kb = (int64_t)(c->index_init_tokens + block - 1) / block +
+                     (c->index_local_tokens + block - 1) / block + 1 + n_blocks;
+  if (kb > 2048) return set_error(LSA_ERR_UNSUPPORTED, "%s: the coarse selection exceeds 2048 blocks", fn);
+  return LSA_OK;
+}
+
 }  // namespace
 }  // namespace lsa
 
@@ -498,6 +539,138 @@ lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_
     if (s != LSA_OK) return s;
   }
   return LSA_OK;
+}
+
+
+lsa_status lsa_block_summaries(const lsa_config* c, int32_t n_items, int32_t n_seq, const int32_t* item_seq,
+                               const int32_t* item_blk, const lsa_bf16* k_idx, const int64_t* k_off,
+                               const int64_t* blk_off, int32_t block, lsa_bf16* k_blk, void* stream) {
+  const char* fn = "lsa_block_summaries";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (block < 16 || block > 1024 || block % 16 != 0)
+    return set_error(LSA_ERR_UNSUPPORTED, "%s: block must be a multiple of 16 in [16, 1024]", fn);
+  if (n_items < 0 || n_seq < 1) return set_error(LSA_ERR_INVALID, "%s: need n_items >= 0 and n_seq >= 1", fn);
+  if (n_items == 0) return LSA_OK;
+  if (!item_seq || !item_blk || !k_idx || !k_off || !blk_off || !k_blk)
+    return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (!aligned16(k_idx) || !aligned16(k_blk))
+    return set_error(LSA_ERR_INVALID, "%s: k_idx and k_blk must be 16-byte aligned", fn);
+  BlockSumArgs a;
+  a.k_idx = k_idx;
+  a.k_off = k_off;
+  a.blk_off = blk_off;
+  a.item_seq = item_seq;
+  a.item_blk = item_blk;
+  a.n_items = n_items;
+  a.n_seq = n_seq;
+  a.block = block;
+  a.k_blk = k_blk;
+  a.err = device_error_word();
+  return cuda_status(launch_block_summaries(a, (cudaStream_t)stream), fn);
+}
+
+size_t lsa_hier_workspace_size(const lsa_config* c, int32_t n_rows, int64_t max_len, int32_t block,
+                               int32_t n_blocks) {
+  if (check_cfg(c, "lsa_hier_workspace_size") != LSA_OK || n_rows < 0 || max_len < 1 ||
+      check_hier(c, block, n_blocks, "lsa_hier_workspace_size") != LSA_OK)
+    return 0;
+  if (n_rows == 0) return kAlign;
+  return hier_plan(c, n_rows, max_len, block, n_blocks).total;
+}
+
+lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, const int32_t* seq_of_row,
+                           const int32_t* pos, const lsa_bf16* q_idx, const float* w, const lsa_bf16* k_idx,
+                           const int64_t* k_off, const lsa_bf16* k_blk, const int64_t* blk_off, int64_t max_len,
+                           int32_t block, int32_t n_blocks, int32_t* idx, int32_t* count, void* ws,
+                           size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_hier_select";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  s = check_hier(c, block, n_blocks, fn);
+  if (s != LSA_OK) return s;
+  if (n_rows < 0 || n_seq < 1 || max_len < 1)
+    return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0, n_seq >= 1, max_len >= 1", fn);
+  if ((!k_off || !blk_off) && n_seq != 1)
+    return set_error(LSA_ERR_INVALID, "%s: k_off / blk_off NULL with n_seq > 1", fn);
+  if (!k_off || !blk_off) return set_error(LSA_ERR_INVALID, "%s: k_off and blk_off are required", fn);
+  if (n_rows == 0) return max_len <= c->index_topk ? LSA_DENSE : LSA_OK;
+  if (!pos || !q_idx || !w || !k_idx || !k_blk || !idx || !count)
+    return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (!aligned16(q_idx) || !aligned16(k_idx) || !aligned16(k_blk))
+    return set_error(LSA_ERR_INVALID, "%s: q_idx, k_idx and k_blk must be 16-byte aligned", fn);
+  cudaStream_t st = (cudaStream_t)stream;
+  const HierPlan h = hier_plan(c, n_rows, max_len, block, n_blocks);
+  if (!ws || ws_bytes < h.total)
+    return set_error(LSA_ERR_WORKSPACE, "%s: workspace %zu below %zu", fn, ws_bytes, h.total);
+  char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~uintptr_t(kAlign - 1));
+  int32_t* pos_b = reinterpret_cast<int32_t*>(base + h.off_pos_b);
+  int32_t* pos_c = reinterpret_cast<int32_t*>(base + h.off_pos_c);
+  float* coarse = reinterpret_cast<float*>(base + h.off_coarse);
+  int32_t* kept = reinterpret_cast<int32_t*>(base + h.off_kept);
+  int32_t* kept_n = reinterpret_cast<int32_t*>(base + h.off_kept_n);
+  int32_t* sorted = reinterpret_cast<int32_t*>(base + h.off_sorted);
+  float* cand = reinterpret_cast<float*>(base + h.off_cand);
+  void* topk_w = base + h.off_topk;
+  const size_t topk_bytes = topk_ws(n_rows);
+
+  if (max_len <= c->index_topk) {  // every row dense: nothing to score
+    s = cuda_status(launch_hier_map(pos, sorted, h.kb, block, n_rows, c->index_topk, idx, count, st), fn);
+    return s == LSA_OK ? LSA_DENSE : s;
+  }
+  // coarse stage: the indexer over the summaries, then the flat top-k one level up
+  s = cuda_status(launch_hier_prep(pos, n_rows, block, pos_b, st), fn);
+  if (s != LSA_OK) return s;
+  IndexArgs a;
+  a.q_idx = q_idx;
+  a.w = w;
+  a.k_idx = k_blk;
+  a.k_off = blk_off;
+  a.seq_of_row = seq_of_row;
+  a.seq_identity = 0;
+  a.pos = pos_b;
+  a.n_rows = n_rows;
+  a.n_seq = n_seq;
+  a.max_len = h.nb_max;
+  a.n_init = h.n_init_b;
+  a.n_loc = h.n_loc_b;
+  a.scores = coarse;
+  a.ld = h.ld_b;
+  a.err = device_error_word();
+  s = cuda_status(index_prefill_supported(a) ? launch_index_prefill(a, st) : launch_index_decode(a, st), fn);
+  if (s != LSA_OK) return s;
+  lsa_config cb = *c;
+  cb.index_topk = h.kb;
+  cb.index_init_tokens = h.n_init_b;
+  cb.index_local_tokens = h.n_loc_b;
+  s = run_topk(&cb, n_rows, pos_b, h.nb_max, coarse, h.ld_b, kept, kept_n, topk_w, topk_bytes, st);
+  if (s != LSA_OK && s != LSA_DENSE) return s;
+  // fine stage: the kept blocks' tokens into compact rows, the flat top-k over them
+  HierFineArgs f;
+  f.ix = a;
+  f.ix.k_idx = k_idx;
+  f.ix.k_off = k_off;
+  f.ix.pos = pos;
+  f.ix.max_len = max_len;
+  f.ix.n_init = c->index_init_tokens;
+  f.ix.n_loc = c->index_local_tokens;
+  f.ix.scores = nullptr;
+  f.kept = kept;
+  f.kept_n = kept_n;
+  f.kb = h.kb;
+  f.block = block;
+  f.sorted = sorted;
+  f.pos_c = pos_c;
+  f.cand = cand;
+  f.ld_c = h.ld_c;
+  s = cuda_status(launch_hier_fine(f, st), fn);
+  if (s != LSA_OK) return s;
+  lsa_config cc = *c;
+  cc.index_init_tokens = 0;
+  cc.index_local_tokens = 0;
+  s = run_topk(&cc, n_rows, pos_c, h.ld_c, cand, h.ld_c, idx, count, topk_w, topk_bytes, st);
+  if (s != LSA_OK && s != LSA_DENSE) return s;
+  return cuda_status(launch_hier_map(pos, sorted, h.kb, block, n_rows, c->index_topk, idx, count, st), fn);
 }
 
 }  // extern "C"

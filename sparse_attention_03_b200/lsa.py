@@ -28,8 +28,10 @@ EXPORTS = (
     "lsa_config_default", "lsa_workspace_size", "lsa_index_scores", "lsa_topk",
     "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill", "lsa_forward", "lsa_last_error",
     "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16", "lsa_synth_normal_f32",
-    "lsa_synth_rms_rows_bf16", "lsa_launch_count", "lsa_index_project",
+    "lsa_synth_rms_rows_bf16", "lsa_launch_count", "lsa_index_project", "lsa_block_summaries",
+    "lsa_hier_workspace_size", "lsa_hier_select",
 )
+HIER_BLOCK, HIER_BLOCKS = 64, 128
 
 
 class LsaError(RuntimeError):
@@ -80,6 +82,11 @@ def load():
                                 _P, _P, _P, _SZ, _P]
     lib.lsa_index_project.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _P,
                                       _I32, _I32, ctypes.c_float, _P, _P, _P, _P, _SZ, _P]
+    lib.lsa_block_summaries.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _P, _P, _I32, _P, _P]
+    lib.lsa_hier_workspace_size.argtypes = [ctypes.POINTER(Config), _I32, _I64, _I32, _I32]
+    lib.lsa_hier_workspace_size.restype = _SZ
+    lib.lsa_hier_select.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _P, _I64, _I32,
+                                    _I32, _P, _P, _P, _SZ, _P]
     lib.lsa_last_error.argtypes = []
     lib.lsa_last_error.restype = ctypes.c_char_p
     lib.lsa_device_error.argtypes = [ctypes.POINTER(_I32)]
@@ -90,7 +97,7 @@ def load():
     lib.lsa_synth_normal_f32.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
     lib.lsa_synth_rms_rows_bf16.argtypes = [_P, _I64, _I32, _U64, _U64, _I64, _P]
     for name in ("lsa_index_scores", "lsa_topk", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
-                 "lsa_forward", "lsa_index_project", "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16",
+                 "lsa_forward", "lsa_index_project", "lsa_block_summaries", "lsa_hier_select", "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16",
                  "lsa_synth_normal_f32", "lsa_synth_rms_rows_bf16"):
         getattr(lib, name).restype = _I32
     _lib = lib
@@ -313,3 +320,45 @@ def synth_rms_rows_bf16(dst, seed, tid, first_row=0, stream=None):
     _dt(dst, torch.bfloat16, "dst")
     n_rows, d = dst.shape
     return _check(load().lsa_synth_rms_rows_bf16(_ptr(dst), n_rows, d, seed, tid, first_row, _stream(stream)))
+
+
+def block_offsets(lengths, block=HIER_BLOCK):
+    """blk_off for packed caches of the given lengths: ceil(L / block) blocks each."""
+    n = [(int(L) + block - 1) // block for L in lengths]
+    off = [0]
+    for x in n:
+        off.append(off[-1] + x)
+    return off
+
+
+def block_summaries(cfg, item_seq, item_blk, k_idx, k_off, blk_off, k_blk, block=HIER_BLOCK, stream=None,
+                    bind=False):
+    """Summary keys (bf16 mean of the block's keys) of blocks item_blk[i] of
+    sequences item_seq[i] into k_blk (hierarchical indexing)."""
+    _dt(k_idx, torch.bfloat16, "k_idx"); _dt(k_blk, torch.bfloat16, "k_blk")
+    _dt(item_seq, torch.int32, "item_seq"); _dt(item_blk, torch.int32, "item_blk")
+    _dt(k_off, torch.int64, "k_off"); _dt(blk_off, torch.int64, "blk_off")
+    return _invoke(load().lsa_block_summaries, (
+        ctypes.byref(cfg._c()), item_seq.numel(), k_off.numel() - 1, _ptr(item_seq), _ptr(item_blk), _ptr(k_idx),
+        _ptr(k_off), _ptr(blk_off), block, _ptr(k_blk), _stream(stream)), bind=bind)
+
+
+def hier_workspace(cfg, n_rows, max_len, block=HIER_BLOCK, n_blocks=HIER_BLOCKS, device=None) -> torch.Tensor:
+    n = int(load().lsa_hier_workspace_size(ctypes.byref(cfg._c()), n_rows, max_len, block, n_blocks))
+    if n == 0:
+        raise LsaError(LSA_ERR_UNSUPPORTED, load().lsa_last_error().decode())
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def hier_select(cfg, seq_of_row, pos, q_idx, w, k_idx, k_off, k_blk, blk_off, max_len, idx, count, ws,
+                block=HIER_BLOCK, n_blocks=HIER_BLOCKS, stream=None, bind=False):
+    """Two-stage (block, then token) selection of every row into idx / count,
+    shaped like topk's output."""
+    _dt(q_idx, torch.bfloat16, "q_idx"); _dt(k_idx, torch.bfloat16, "k_idx"); _dt(k_blk, torch.bfloat16, "k_blk")
+    _dt(w, torch.float32, "w"); _dt(pos, torch.int32, "pos"); _dt(idx, torch.int32, "idx")
+    _dt(count, torch.int32, "count"); _dt(k_off, torch.int64, "k_off"); _dt(blk_off, torch.int64, "blk_off")
+    _dt(seq_of_row, torch.int32, "seq_of_row")
+    return _invoke(load().lsa_hier_select, (
+        ctypes.byref(cfg._c()), pos.numel(), k_off.numel() - 1, _ptr(seq_of_row), _ptr(pos), _ptr(q_idx), _ptr(w),
+        _ptr(k_idx), _ptr(k_off), _ptr(k_blk), _ptr(blk_off), int(max_len), block, n_blocks, _ptr(idx),
+        _ptr(count), _ptr(ws), ws.numel(), _stream(stream)), allow_dense=True, bind=bind)

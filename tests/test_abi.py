@@ -119,3 +119,26 @@ def test_index_project_validation(lib):
     assert lib.lsa_index_project(*args(1536, 3072, None)) == lsa.LSA_ERR_WORKSPACE      # no workspace
     assert lib.lsa_index_project(*args(1536, 3072, _fake(), 0.5)) == lsa.LSA_ERR_INVALID
     assert lsa.workspace_size(lsa.LsaConfig(), lsa.OP_INDEX_PROJECT, 16, 16, 100) >= 16 * (4096 + 160) * 4
+
+
+def test_hier_validation(lib):
+    c = lsa.LsaConfig().c()
+    f = _fake
+    sel = lambda block, n_blocks, ws=None, wsb=0, k_blk=f(): (
+        ctypes.byref(c), 4, 1, None, f(), f(), f(), f(), f(), k_blk, f(), 100000, block, n_blocks, f(), f(), ws,
+        wsb, None)
+    assert lib.lsa_hier_select(*sel(8, 500)) == lsa.LSA_ERR_UNSUPPORTED          # block below 16
+    assert lib.lsa_hier_select(*sel(48 + 1, 100)) == lsa.LSA_ERR_UNSUPPORTED     # not a multiple of 16
+    assert lib.lsa_hier_select(*sel(64, 31)) == lsa.LSA_ERR_UNSUPPORTED          # 31 x 64 < index_topk
+    assert b"n_blocks * block" in lib.lsa_last_error()
+    assert lib.lsa_hier_select(*sel(16, 2000)) == lsa.LSA_ERR_UNSUPPORTED        # coarse selection > 2048
+    assert lib.lsa_hier_select(*sel(64, 32)) == lsa.LSA_ERR_WORKSPACE            # no workspace
+    assert lib.lsa_hier_select(*sel(64, 32, f(), 10 ** 9, k_blk=None)) == lsa.LSA_ERR_INVALID
+    n = lib.lsa_hier_workspace_size(ctypes.byref(c), 16, 131072, 64, 128)
+    # coarse scores (2048 blocks) + compact rows ((1 + 17 + 128) x 64 slots) per row, fp32
+    assert n >= 16 * (2048 + 146 * 64) * 4
+    assert lib.lsa_hier_workspace_size(ctypes.byref(c), 16, 131072, 64, 10) == 0
+    summ = lambda block, k_blk=f(): (ctypes.byref(c), 3, 2, f(), f(), f(), f(), f(), block, k_blk, None)
+    assert lib.lsa_block_summaries(*summ(20)) == lsa.LSA_ERR_UNSUPPORTED
+    assert lib.lsa_block_summaries(*summ(64, None)) == lsa.LSA_ERR_INVALID
+    assert lsa.block_offsets([1, 64, 65, 0], 64) == [0, 1, 2, 4, 4]

@@ -9,7 +9,7 @@ import pytest
 import torch
 
 import lsa_synth as S
-from lsa_testutil import (assert_attention, assert_scores, bf16_dev, bf16_host_f64, check_selection,
+from lsa_testutil import (GAP_RTOL, assert_attention, assert_scores, bf16_dev, bf16_host_f64, check_selection,
                           f32_dev, host_rows, i32_dev, i64_dev, oracle_cfg)
 from oracle import lsa_ref as R
 
@@ -775,3 +775,187 @@ def test_index_project_dims(L, q_lora, hidden, n):
 def test_index_project_prefill_rows(L):
     # rows of one sequence at positions 2000 .. 2299 (tiles of 64 rows, a ragged last one)
     _project_check(L, 32, [2300], [(0, 2000 + t) for t in range(300)], k_off_given=False)
+
+
+# --------------------------------------------------------------------------
+# Hierarchical indexing ([LSA-2.0] 分层索引)
+# --------------------------------------------------------------------------
+def _hier_inputs(seed, lengths, n_rows):
+    off = S.offsets(np.asarray(lengths, dtype=np.int64))
+    k = S.rms_rows_bf16(seed, S.tid(0, S.K_IDX), 0, int(off[-1]), 128)
+    q = S.normal_bf16(seed, S.tid(0, S.Q_IDX), 0, n_rows * 4096).reshape(n_rows, 32, 128)
+    w = S.normal_f32(seed, S.tid(0, S.W), 0, n_rows * 32, S.W_SIGMA).reshape(n_rows, 32)
+    return off, k, q, w
+
+
+def _summaries_dev(L, cfg, lengths, k_d, off_d, block):
+    blk_off = np.array(L.block_offsets(lengths, block), dtype=np.int64)
+    items = [(s, b) for s in range(len(lengths)) for b in range(int(blk_off[s + 1] - blk_off[s]))]
+    items = [items[i] for i in np.random.default_rng(1).permutation(len(items))]   # any order
+    k_blk = torch.empty((max(int(blk_off[-1]), 1), 128), dtype=torch.bfloat16, device="cuda")
+    L.block_summaries(cfg, i32_dev([s for s, _ in items]), i32_dev([b for _, b in items]), k_d, off_d,
+                      i64_dev(blk_off), k_blk, block)
+    return blk_off, k_blk
+
+
+def test_block_summaries_bit_exact(L):
+    cfg = L.LsaConfig()
+    lengths = [1, 63, 64, 65, 1000, 4097]
+    off, k, _, _ = _hier_inputs(41, lengths, 1)
+    f = S.bf16_bits_to_f64
+    for block in (16, 64, 1024):
+        blk_off, k_blk = _summaries_dev(L, cfg, lengths, bf16_dev(k), i64_dev(off), block)
+        assert L.device_error() == 0
+        got = k_blk.view(torch.int16).cpu().numpy().view(np.uint16)
+        for s in range(len(lengths)):
+            exp = R.block_summaries(f(k[off[s]:off[s + 1]]), block)
+            np.testing.assert_array_equal(f(got[blk_off[s]:blk_off[s + 1]]), exp, err_msg=f"block {block} seq {s}")
+
+
+def test_block_summary_update_after_append(L):
+    # decode: after appending a key, re-summarise only the block that holds it
+    cfg = L.LsaConfig()
+    f = S.bf16_bits_to_f64
+    lengths = [130, 64, 1]
+    off, k, _, _ = _hier_inputs(42, lengths, 1)
+    k_d = bf16_dev(k)
+    blk_off = np.array(L.block_offsets([200, 200, 200], 64), dtype=np.int64)   # room to grow
+    k_blk = torch.zeros((int(blk_off[-1]), 128), dtype=torch.bfloat16, device="cuda")
+    last = [(L_ - 1) // 64 for L_ in lengths]
+    L.block_summaries(cfg, i32_dev([0, 1, 2]), i32_dev(last), k_d, i64_dev(off), i64_dev(blk_off), k_blk, 64)
+    assert L.device_error() == 0
+    got = k_blk.view(torch.int16).cpu().numpy().view(np.uint16)
+    for s in range(3):
+        exp = R.block_summaries(f(k[off[s]:off[s + 1]]), 64)[last[s]]
+        np.testing.assert_array_equal(f(got[blk_off[s] + last[s]]), exp)
+
+
+def test_block_summary_bad_item_is_flagged(L):
+    cfg = L.LsaConfig()
+    off, k, _, _ = _hier_inputs(43, [100], 1)
+    blk_off = i64_dev([0, 2])
+    k_blk = torch.zeros((2, 128), dtype=torch.bfloat16, device="cuda")
+    L.block_summaries(cfg, i32_dev([0]), i32_dev([5]), bf16_dev(k), i64_dev(off), blk_off, k_blk, 64)
+    assert L.device_error() == L.DEVERR_POS
+    assert not k_blk.view(torch.int16).any()
+
+
+def _hier_check_row(got_idx, got_cnt, q, w, k_seq, p, ocfg, block, n_blocks, where):
+    """Checks one row of a GPU hierarchical selection against the oracle.
+    Returns True when the row was compared bit for bit."""
+    kb = R.block_summaries(k_seq, block)
+    sel, dense, kept = R.hier_select(q, w, k_seq, kb, p, ocfg, block, n_blocks)
+    n = p + 1
+    if dense:
+        assert got_cnt == n, where
+        np.testing.assert_array_equal(np.sort(got_idx[:n]), np.arange(n))
+        assert np.all(got_idx[n:] == -1)
+        return True
+    assert got_cnt == ocfg.index_topk, where
+    g = got_idx[: ocfg.index_topk]
+    assert len(np.unique(g)) == len(g) and g.min() >= 0 and g.max() <= p, where
+    forced = set(range(min(ocfg.index_init_tokens, n))) | set(range(max(0, n - ocfg.index_local_tokens), n))
+    assert forced <= set(g.tolist()), f"forced token missing {where}"
+    # coarse boundary: relative gap between the n_blocks-th and next best unforced block
+    bc = R.hier_config(ocfg, block, n_blocks)
+    nb = p // block + 1
+    b = np.arange(nb)
+    mid = (b >= bc.index_init_tokens) & (b < nb - bc.index_local_tokens)
+    cs = np.sort(R.score_row(q, w, kb[:nb])[mid])[::-1]
+    if len(cs) > n_blocks and abs(cs[n_blocks - 1] - cs[n_blocks]) <= GAP_RTOL * abs(cs[n_blocks - 1]):
+        return False            # kept blocks may legitimately differ: validity checked above
+    kept_tok = set(np.concatenate([np.arange(x * block, min((x + 1) * block, n)) for x in kept]).tolist())
+    assert set(g.tolist()) <= kept_tok, f"token outside the kept blocks {where}"
+    s = R.score_row(q, w, k_seq[:n])
+    cand = np.array(sorted(kept_tok - forced))
+    v = np.sort(s[cand])[::-1]
+    k_rem = ocfg.index_topk - len(forced)
+    if len(v) <= k_rem or abs(v[k_rem - 1] - v[k_rem]) > GAP_RTOL * abs(v[k_rem - 1]):
+        np.testing.assert_array_equal(np.sort(g), sel, err_msg=where)
+        return True
+    a, e = s[sorted(set(g.tolist()) - forced)].sum(), s[sorted(set(sel.tolist()) - forced)].sum()
+    assert abs(a - e) <= GAP_RTOL * abs(e), f"near-tie sum {where}"
+    return False
+
+
+def _hier_run(L, cfg, seed, lengths, rows, block, n_blocks):
+    """rows: (sequence, position) pairs. Returns (idx, count, status) and the host inputs."""
+    off, k, q, w = _hier_inputs(seed, lengths, len(rows))
+    k_d, off_d = bf16_dev(k), i64_dev(off)
+    blk_off, k_blk = _summaries_dev(L, cfg, lengths, k_d, off_d, block)
+    n = len(rows)
+    max_len = int(max(lengths))
+    idx = torch.full((n, cfg.index_topk), -7, dtype=torch.int32, device="cuda")
+    cnt = torch.full((n,), -7, dtype=torch.int32, device="cuda")
+    ws = L.hier_workspace(cfg, n, max_len, block, n_blocks)
+    st = L.hier_select(cfg, i32_dev([s for s, _ in rows]), i32_dev([p for _, p in rows]), bf16_dev(q), f32_dev(w),
+                       k_d, off_d, k_blk, i64_dev(blk_off), max_len, idx, cnt, ws, block, n_blocks)
+    assert L.device_error() == 0
+    return idx.cpu().numpy(), cnt.cpu().numpy(), st, (off, k, q, w)
+
+
+def _hier_check(L, cfg, seed, lengths, rows, block, n_blocks, min_exact):
+    idx, cnt, _, (off, k, q, w) = _hier_run(L, cfg, seed, lengths, rows, block, n_blocks)
+    f = S.bf16_bits_to_f64
+    ocfg = oracle_cfg(cfg)
+    exact = 0
+    for r, (s, p) in enumerate(rows):
+        exact += _hier_check_row(idx[r], int(cnt[r]), f(q[r]), w[r].astype(np.float64), f(k[off[s]:off[s + 1]]),
+                                 p, ocfg, block, n_blocks, f"row {r} (seq {s}, pos {p})")
+    assert exact >= min_exact, f"only {exact} of {len(rows)} rows compared exactly"
+
+
+def test_hier_select_decode_varlen(L):
+    lengths = [3000, 5000, 777, 20000, 2049, 2048, 40000]
+    rows = [(s, n - 1) for s, n in enumerate(lengths)]
+    _hier_check(L, L.LsaConfig(), 5, lengths, rows, 64, 32, min_exact=6)   # one fine-stage near-tie
+
+
+def test_hier_select_prefill_rows(L):
+    # 200 rows of one sequence at consecutive positions (prefill shape)
+    rows = [(0, 11800 + t) for t in range(200)]
+    # (of the 200 rows, 111 have no near-tie at either stage's boundary in the oracle)
+    _hier_check(L, L.LsaConfig(), 6, [12000], rows, 32, 80, min_exact=111)
+
+
+@pytest.mark.parametrize("block,n_blocks,n_exact", [(16, 256, 1), (128, 16, 3), (1024, 2, 3)])
+def test_hier_select_block_sizes(L, block, n_blocks, n_exact):
+    # n_exact: rows without a near-tie at either boundary in the oracle
+    lengths = [6000, 15000, 2500]
+    rows = [(s, n - 1) for s, n in enumerate(lengths)] + [(1, 9000), (1, 100)]
+    _hier_check(L, L.LsaConfig(), 7, lengths, rows, block, n_blocks, min_exact=n_exact)
+
+
+def test_hier_select_tiny_config(L):
+    cfg = L.LsaConfig(index_topk=8, index_init_tokens=2, index_local_tokens=4)
+    lengths = [40, 100, 300, 5]
+    rows = [(s, n - 1) for s, n in enumerate(lengths)] + [(2, 150), (2, 16)]
+    _hier_check(L, cfg, 8, lengths, rows, 16, 1, min_exact=6)
+
+
+def test_hier_every_block_kept_is_the_flat_selection(L):
+    # n_blocks covering every block: the GPU's two-stage result equals its flat
+    # indexer + top-k on the same inputs, set for set
+    cfg = L.LsaConfig()
+    lengths = [9000, 30000, 1500]
+    rows = [(s, n - 1) for s, n in enumerate(lengths)]
+    idx, cnt, _, (off, k, q, w) = _hier_run(L, cfg, 9, lengths, rows, 64, 2048 - 18)
+    max_len = int(max(lengths))
+    scores = torch.empty((len(rows), max_len), device="cuda")
+    L.index_scores(cfg, i32_dev([s for s, _ in rows]), i32_dev([p for _, p in rows]), bf16_dev(q), f32_dev(w),
+                   bf16_dev(k), i64_dev(off), max_len, scores)
+    fidx = torch.empty((len(rows), cfg.index_topk), dtype=torch.int32, device="cuda")
+    fcnt = torch.empty((len(rows),), dtype=torch.int32, device="cuda")
+    L.topk(cfg, i32_dev([p for _, p in rows]), max_len, scores, fidx, fcnt,
+           L.workspace(cfg, L.OP_TOPK, len(rows), len(rows), max_len))
+    fidx, fcnt = fidx.cpu().numpy(), fcnt.cpu().numpy()
+    np.testing.assert_array_equal(cnt, fcnt)
+    for r in range(len(rows)):
+        np.testing.assert_array_equal(np.sort(idx[r, :cnt[r]]), np.sort(fidx[r, :fcnt[r]]))
+
+
+def test_hier_all_dense_status(L):
+    cfg = L.LsaConfig()
+    _, cnt, st, _ = _hier_run(L, cfg, 10, [2048, 500], [(0, 2047), (1, 499)], 64, 32)
+    assert st == L.LSA_DENSE
+    np.testing.assert_array_equal(cnt, [2048, 500])
