@@ -16,7 +16,12 @@ pinned host buffers and host<->device copies inside the timed region, and an
 MTP draft round ("mtp": one index pass and top-k per layer shared by three
 draft steps of sparse MLA over one latent cache; tokens = 3 per sequence per
 layer per round), and the indexer's own projections with the key-cache append
-("project": one decode token per sequence per layer, with its HBM roofline).
+("project": one decode token per sequence per layer, with its HBM roofline),
+and the decode step with hierarchical indexing ("hier": per layer the newest
+block's summary, a coarse pass over 64-key block summaries keeping the sink /
+recent blocks and the 128 best others, the fine selection over their tokens,
+then both MLA sub-blocks; also the selection alone against the flat index pass
+and top-k).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
@@ -332,6 +337,52 @@ def build_project(D, device):
     D["project_bytes"] = wbytes + io
 
 
+def build_hier(D, device, block=64, n_blocks=128):
+    """Per layer: block summaries of the index-key cache (built once, untimed), the
+    per-step update of each sequence's newest block, and the two-stage selection
+    bound into the decode step's idx / count buffers."""
+    import torch
+    from sparse_attention_03_b200 import lsa
+    B, ctx, cfg = DECODE["batch"], D["ctx"], D["cfg"]
+    blk_off_h = lsa.block_offsets([ctx] * B, block)
+    blk_off = torch.tensor(blk_off_h, dtype=torch.int64, device=device)
+    nb = ctx // block if ctx % block == 0 else ctx // block + 1
+    all_seq = torch.arange(B, dtype=torch.int32, device=device).repeat_interleave(nb)
+    all_blk = torch.arange(nb, dtype=torch.int32, device=device).repeat(B)
+    new_seq = torch.arange(B, dtype=torch.int32, device=device)
+    new_blk = torch.full((B,), (ctx - 1) // block, dtype=torch.int32, device=device)
+    ws = lsa.hier_workspace(cfg, B, ctx, block, n_blocks, device=device)
+    H = []
+    for l in D["layers"]:
+        k_blk = torch.empty((blk_off_h[-1], 128), dtype=torch.bfloat16, device=device)
+        lsa.block_summaries(cfg, all_seq, all_blk, l.k_idx, l.k_off, blk_off, k_blk, block)
+        H.append(dict(k_blk=k_blk,
+                      update=lsa.block_summaries(cfg, new_seq, new_blk, l.k_idx, l.k_off, blk_off, k_blk, block,
+                                                 bind=True),
+                      select=lsa.hier_select(cfg, l.seq_of_row, l.pos, l.q_idx, l.w, l.k_idx, l.k_off, k_blk,
+                                             blk_off, ctx, D["idx"], D["cnt"], ws, block, n_blocks, bind=True)))
+    D["hier"] = H
+    D["hier_keep"] = (blk_off, all_seq, all_blk, new_seq, new_blk, ws)
+    D["hier_cfg"] = {"block": block, "n_blocks": n_blocks}
+
+
+def hier_step(D, select_only=False):
+    """One decode step with hierarchical selection: per layer the newest block's
+    summary, the two-stage selection, then both MLA sub-blocks on it."""
+    for h, (_, _, mla_calls) in zip(D["hier"], D["calls"]):
+        h["update"]()
+        h["select"]()
+        if not select_only:
+            for call in mla_calls:
+                call()
+
+
+def flat_select_step(D):
+    for idx_call, topk_call, _ in D["calls"]:
+        idx_call()
+        topk_call()
+
+
 def project_step(D):
     for p in D["project"]:
         p["call"]()
@@ -532,6 +583,19 @@ def gpu_arm(args):
     mtp_value, _ = aggregate(3 * B * nl * mtp_steps, tm, world, device)
     assert lsa.device_error() == 0
 
+    # hierarchical indexing: the same decode step with the two-stage selection,
+    # and the selection alone against the flat index pass + top-k
+    build_hier(D, device)
+    for _ in range(3):
+        hier_step(D)
+    h_steps = max(5, args.steps // 2)
+    th = time_region(lambda s: hier_step(D), h_steps, world, device)
+    hier_value, _ = aggregate(B * nl * h_steps, th, world, device)
+    ths = time_region(lambda s: hier_step(D, select_only=True), h_steps, world, device)
+    tfs = time_region(lambda s: flat_select_step(D), h_steps, world, device)
+    assert lsa.device_error() == 0
+
+    D_hier_cfg = D["hier_cfg"]
     del D
     torch.cuda.empty_cache()
     prefill = None
@@ -564,6 +628,12 @@ def gpu_arm(args):
     line["mtp"] = {"value": mtp_value, "unit": "tokens/s/layer", "ms_per_round": 1e3 * tm / mtp_steps,
                    "config": {"workload": "mtp_draft_round_b16_ctx131072_14layers", "draft_steps": 3,
                               "index_passes_per_round": 1}}
+    hc = D_hier_cfg
+    line["hier"] = {"value": hier_value, "unit": "tokens/s/layer", "ms_per_step": 1e3 * th / h_steps,
+                    "select_us_per_layer": 1e6 * ths / (h_steps * nl),
+                    "flat_select_us_per_layer": 1e6 * tfs / (h_steps * nl),
+                    "config": {"workload": f"hier_decode_b16_ctx131072_14layers_block{hc['block']}"
+                                           f"_keep{hc['n_blocks']}", **hc}}
     if prefill:
         line["prefill"] = prefill
     if world == 1 and not args.no_cpu_baseline:

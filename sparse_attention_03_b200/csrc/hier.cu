@@ -9,10 +9,10 @@
 // (sink and most recent blocks forced, the n_blocks best others kept); the
 // fine stage is the flat selection over the kept blocks' tokens.
 //
-// The coarse scores come from the streaming indexer run over the summaries,
-// the coarse and fine selections from the flat top-k; this file holds the
-// summaries, the per-row block positions and the map from compact selections
-// back to token columns.
+// The coarse scores come from the streaming indexer run over the summaries
+// (row positions divided by the block size as it reads them), the coarse and
+// fine selections from the flat top-k (the fine one mapping compact slots back
+// to token columns as it writes them); this file holds the summaries.
 #include "common.cuh"
 #include "kernels.h"
 #include "launch.h"
@@ -60,43 +60,20 @@ __global__ void __launch_bounds__(kDi) block_summary_kernel(BlockSumArgs a) {
   const uint16_t* __restrict__ k = a.k_idx + (base + t0) * kDi + d;
   // fp64 sum: exact for up to 1024 bf16 terms spanning fewer than 35 binades, so
   // the mean is the correctly rounded fp64 quotient before the bf16 rounding
-  double sum = 0.0;
-  for (int64_t t = 0; t < t1 - t0; ++t) sum += (double)__uint_as_float((uint32_t)__ldg(k + t * kDi) << 16);
-  a.k_blk[(bbase + b) * kDi + d] = f64_to_bf16_rne(sum / (double)(t1 - t0));
-  pdl_trigger();
-}
-
-__global__ void hier_prep_kernel(const int32_t* __restrict__ pos, int n_rows, int block, int32_t* __restrict__ pos_b) {
-  pdl_wait();
-  const int r = blockIdx.x * blockDim.x + threadIdx.x;
-  if (r < n_rows) {
-    const int p = pos[r];
-    pos_b[r] = p >= 0 ? p / block : -1;
+  // (the order of the exact additions is free: eight chains keep eight loads in flight)
+  const int n = (int)(t1 - t0);
+  double part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  int t = 0;
+  for (; t + 8 <= n; t += 8) {
+    uint16_t v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = __ldg(k + (int64_t)(t + u) * kDi);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) part[u] += (double)__uint_as_float((uint32_t)v[u] << 16);
   }
-  pdl_trigger();
-}
-
-// One CTA per row.
-__global__ void __launch_bounds__(256) hier_map_kernel(const int32_t* __restrict__ pos,
-                                                       const int32_t* __restrict__ sorted, int kb, int block,
-                                                       int topk, int32_t* __restrict__ idx,
-                                                       int32_t* __restrict__ count) {
-  pdl_wait();
-  const int r = blockIdx.x;
-  const int p = pos[r];
-  int32_t* __restrict__ ir = idx + (int64_t)r * topk;
-  if (p < 0 || p + 1 <= topk) {  // dense row (or an invalid one, flagged upstream: empty)
-    const int n = p < 0 ? 0 : p + 1;
-    for (int i = threadIdx.x; i < topk; i += blockDim.x) ir[i] = i < n ? i : -1;
-    if (threadIdx.x == 0) count[r] = n;
-  } else {
-    const int n = count[r];
-    const int32_t* __restrict__ sr = sorted + (int64_t)r * kb;
-    for (int i = threadIdx.x; i < topk; i += blockDim.x) {
-      const int c = ir[i];
-      if (i < n && c >= 0) ir[i] = sr[c / block] * block + c % block;
-    }
-  }
+  for (; t < n; ++t) part[0] += (double)__uint_as_float((uint32_t)__ldg(k + (int64_t)t * kDi) << 16);
+  const double sum = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
+  a.k_blk[(bbase + b) * kDi + d] = f64_to_bf16_rne(sum / (double)n);
   pdl_trigger();
 }
 
@@ -106,19 +83,6 @@ cudaError_t launch_block_summaries(const BlockSumArgs& a, cudaStream_t st) {
   if (a.n_items <= 0) return cudaSuccess;
   count_launches(1);
   return launch_pdl(block_summary_kernel, dim3(a.n_items), dim3(kDi), 0, st, a);
-}
-
-cudaError_t launch_hier_prep(const int32_t* pos, int n_rows, int block, int32_t* pos_b, cudaStream_t st) {
-  if (n_rows <= 0) return cudaSuccess;
-  count_launches(1);
-  return launch_pdl(hier_prep_kernel, dim3((n_rows + 255) / 256), dim3(256), 0, st, pos, n_rows, block, pos_b);
-}
-
-cudaError_t launch_hier_map(const int32_t* pos, const int32_t* sorted, int kb, int block, int n_rows, int topk,
-                            int32_t* idx, int32_t* count, cudaStream_t st) {
-  if (n_rows <= 0) return cudaSuccess;
-  count_launches(1);
-  return launch_pdl(hier_map_kernel, dim3(n_rows), dim3(256), 0, st, pos, sorted, kb, block, topk, idx, count);
 }
 
 }  // namespace lsa

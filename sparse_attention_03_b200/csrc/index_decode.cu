@@ -108,7 +108,8 @@ __global__ void __launch_bounds__(kThreads, 3)
     kbase = a.k_off[seq];
     klen = a.k_off[seq + 1] - kbase;
   }
-  const int64_t p = a.pos[r];
+  const int pr = a.pos[r];
+  const int64_t p = a.pos_div == 1 ? pr : (pr >= 0 ? pr / a.pos_div : -1);
   int64_t nvis = p + 1;
   if (ok && (p < 0 || nvis > klen || nvis > a.max_len)) {
     if (blockIdx.x == 0 && threadIdx.x == 0) flag_error(a.err, LSA_DEVERR_POS);
@@ -220,7 +221,12 @@ __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, 
   __syncthreads();
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i < n; i += kThreads) h.sorted[(int64_t)r * h.kb + i] = srt[i];
-    if (threadIdx.x == 0) h.pos_c[r] = n * h.block - 1;
+    // a dense row keeps every block 0 .. pos / block, so its compact slots 0 .. pos
+    // are its tokens 0 .. pos in order
+    if (threadIdx.x == 0) {
+      const int pr = a.pos[r];
+      h.pos_c[r] = (pr >= 0 && pr + 1 <= h.topk) ? pr : n * h.block - 1;
+    }
   }
 
   // row geometry, clamped and flagged as in the flat indexer

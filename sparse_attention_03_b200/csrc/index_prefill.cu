@@ -260,7 +260,7 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t rows, uint32_t box_rows
 }  // namespace
 
 bool index_prefill_supported(const IndexArgs& a) {
-  return a.k_off == nullptr && a.n_seq == 1 && a.seq_of_row == nullptr && a.n_rows >= kRowsPerBlock &&
+  return a.k_off == nullptr && a.n_seq == 1 && a.seq_of_row == nullptr && a.pos_div == 1 && a.n_rows >= kRowsPerBlock &&
          encode_fn() != nullptr;
 }
 

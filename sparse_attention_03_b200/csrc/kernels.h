@@ -24,6 +24,7 @@ struct IndexArgs {
   const int32_t* seq_of_row;  // null: sequence r (seq_identity) or sequence 0
   int seq_identity;
   const int32_t* pos;
+  int pos_div = 1;          // the row's position is pos[r] / pos_div (-1 when pos[r] < 0)
   int n_rows, n_seq;
   int64_t max_len;
   int n_init, n_loc;
@@ -46,6 +47,7 @@ struct TopkArgs {
   const float* scores;
   int64_t ld;
   const int32_t* pos;
+  int pos_div = 1;          // as IndexArgs::pos_div
   int n_rows;
   int64_t max_len;
   int topk, n_init, n_loc;
@@ -56,6 +58,12 @@ struct TopkArgs {
   // Per-row histograms built by the indexer (kTopkHistStride words apart), or
   // null: the top-k then builds them itself.
   const uint32_t* hist_ext = nullptr;
+  // Optional map from column j to the emitted index: col_map[r * col_ld + j /
+  // col_block] * col_block + j % col_block (compact rows of whole blocks). With a
+  // map every row goes through the one-CTA-per-row kernel.
+  const int32_t* col_map = nullptr;
+  int col_block = 1;
+  int64_t col_ld = 0;
 };
 constexpr int kTopkCap = 4096;                              // candidates kept per row
 constexpr size_t kTopkRowBytes = 2048 * 4 + 32 + kTopkCap * 8;  // hist + ctl + candidates
@@ -131,8 +139,6 @@ struct BlockSumArgs {
 };
 cudaError_t launch_block_summaries(const BlockSumArgs& a, cudaStream_t st);
 
-// pos_b[r] = pos[r] / block (-1 for a negative position).
-cudaError_t launch_hier_prep(const int32_t* pos, int n_rows, int block, int32_t* pos_b, cudaStream_t st);
 
 struct HierFineArgs {
   IndexArgs ix;             // token-level rows, keys and forcing (scores unused)
@@ -140,16 +146,13 @@ struct HierFineArgs {
   const int32_t* kept_n;    // [n_rows]
   int kb, block;
   int32_t* sorted;          // out [n_rows, kb]: the kept blocks in ascending order
-  int32_t* pos_c;           // out [n_rows]: kept_n * block - 1
+  int32_t* pos_c;           // out [n_rows]: kept_n * block - 1, or pos for a dense row (pos + 1 <= topk)
+  int topk;
   float* cand;              // out [n_rows, ld_c]: slot i = token sorted[i / block] * block + i % block
   int64_t ld_c;
 };
 // Scores the tokens of each row's kept blocks into the compact rows.
 cudaError_t launch_hier_fine(const HierFineArgs& a, cudaStream_t st);
 
-// Maps compact selections to token columns in place; dense rows (pos + 1 <=
-// topk) get 0..pos.
-cudaError_t launch_hier_map(const int32_t* pos, const int32_t* sorted, int kb, int block, int n_rows, int topk,
-                            int32_t* idx, int32_t* count, cudaStream_t st);
 
 }  // namespace lsa

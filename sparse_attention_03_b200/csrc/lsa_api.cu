@@ -181,7 +181,7 @@ MlaArgs mla_args(const lsa_config* c, int cli, int n_rows, int decode) {
 struct HierPlan {
   int n_init_b, n_loc_b, kb;  // forced sink / recent blocks, blocks kept per row
   int64_t nb_max, ld_b, ld_c; // blocks per row at most, coarse and compact row strides
-  size_t off_pos_b, off_pos_c, off_coarse, off_kept, off_kept_n, off_sorted, off_cand, off_topk, total;
+  size_t off_pos_c, off_coarse, off_kept, off_kept_n, off_sorted, off_cand, off_topk, total;
 };
 
 HierPlan hier_plan(const lsa_config* c, int n_rows, int64_t max_len, int block, int n_blocks) {
@@ -194,7 +194,6 @@ HierPlan hier_plan(const lsa_config* c, int n_rows, int64_t max_len, int block, 
   h.ld_c = (int64_t)h.kb * block;
   const size_t R = (size_t)n_rows;
   size_t o = 0;
-  h.off_pos_b = o;  o += align_up(R * 4);
   h.off_pos_c = o;  o += align_up(R * 4);
   h.off_coarse = o; o += align_up(R * h.ld_b * 4);
   h.off_kept = o;   o += align_up(R * h.kb * 4);
@@ -604,7 +603,6 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   if (!ws || ws_bytes < h.total)
     return set_error(LSA_ERR_WORKSPACE, "%s: workspace %zu below %zu", fn, ws_bytes, h.total);
   char* base = reinterpret_cast<char*>((reinterpret_cast<uintptr_t>(ws) + kAlign - 1) & ~uintptr_t(kAlign - 1));
-  int32_t* pos_b = reinterpret_cast<int32_t*>(base + h.off_pos_b);
   int32_t* pos_c = reinterpret_cast<int32_t*>(base + h.off_pos_c);
   float* coarse = reinterpret_cast<float*>(base + h.off_coarse);
   int32_t* kept = reinterpret_cast<int32_t*>(base + h.off_kept);
@@ -614,13 +612,32 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   void* topk_w = base + h.off_topk;
   const size_t topk_bytes = topk_ws(n_rows);
 
-  if (max_len <= c->index_topk) {  // every row dense: nothing to score
-    s = cuda_status(launch_hier_map(pos, sorted, h.kb, block, n_rows, c->index_topk, idx, count, st), fn);
+  // the flat top-k's arguments over this call's rows (a per-call view of the workspace)
+  auto topk_args = [&](const float* scores, int64_t ld, int64_t len, int topk, int n_init, int n_loc, int32_t* out,
+                       int32_t* cnt) {
+    TopkArgs t;
+    t.scores = scores;
+    t.ld = ld;
+    t.pos = pos;
+    t.n_rows = n_rows;
+    t.max_len = len;
+    t.topk = topk;
+    t.n_init = n_init;
+    t.n_loc = n_loc;
+    t.idx = out;
+    t.count = cnt;
+    t.ws = topk_w;
+    t.ws_bytes = topk_bytes;
+    return t;
+  };
+  if (max_len <= c->index_topk) {  // every row dense: 0 .. pos, nothing to score
+    const TopkArgs t = topk_args(coarse, h.ld_b, max_len, c->index_topk, c->index_init_tokens,
+                                 c->index_local_tokens, idx, count);
+    s = cuda_status(launch_topk(t, st), fn);
     return s == LSA_OK ? LSA_DENSE : s;
   }
-  // coarse stage: the indexer over the summaries, then the flat top-k one level up
-  s = cuda_status(launch_hier_prep(pos, n_rows, block, pos_b, st), fn);
-  if (s != LSA_OK) return s;
+  // coarse stage: the indexer over the summaries and the flat top-k one level up,
+  // both reading each row's position divided by the block size
   IndexArgs a;
   a.q_idx = q_idx;
   a.w = w;
@@ -628,7 +645,8 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   a.k_off = blk_off;
   a.seq_of_row = seq_of_row;
   a.seq_identity = 0;
-  a.pos = pos_b;
+  a.pos = pos;
+  a.pos_div = block;
   a.n_rows = n_rows;
   a.n_seq = n_seq;
   a.max_len = h.nb_max;
@@ -637,20 +655,19 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   a.scores = coarse;
   a.ld = h.ld_b;
   a.err = device_error_word();
-  s = cuda_status(index_prefill_supported(a) ? launch_index_prefill(a, st) : launch_index_decode(a, st), fn);
+  s = cuda_status(launch_index_decode(a, st), fn);
   if (s != LSA_OK) return s;
-  lsa_config cb = *c;
-  cb.index_topk = h.kb;
-  cb.index_init_tokens = h.n_init_b;
-  cb.index_local_tokens = h.n_loc_b;
-  s = run_topk(&cb, n_rows, pos_b, h.nb_max, coarse, h.ld_b, kept, kept_n, topk_w, topk_bytes, st);
-  if (s != LSA_OK && s != LSA_DENSE) return s;
-  // fine stage: the kept blocks' tokens into compact rows, the flat top-k over them
+  TopkArgs tb = topk_args(coarse, h.ld_b, h.nb_max, h.kb, h.n_init_b, h.n_loc_b, kept, kept_n);
+  tb.pos_div = block;
+  s = cuda_status(launch_topk(tb, st), fn);
+  if (s != LSA_OK) return s;
+  // fine stage: the kept blocks' tokens into compact rows, then the flat top-k
+  // over them, writing token columns
   HierFineArgs f;
   f.ix = a;
   f.ix.k_idx = k_idx;
   f.ix.k_off = k_off;
-  f.ix.pos = pos;
+  f.ix.pos_div = 1;
   f.ix.max_len = max_len;
   f.ix.n_init = c->index_init_tokens;
   f.ix.n_loc = c->index_local_tokens;
@@ -661,16 +678,17 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   f.block = block;
   f.sorted = sorted;
   f.pos_c = pos_c;
+  f.topk = c->index_topk;
   f.cand = cand;
   f.ld_c = h.ld_c;
   s = cuda_status(launch_hier_fine(f, st), fn);
   if (s != LSA_OK) return s;
-  lsa_config cc = *c;
-  cc.index_init_tokens = 0;
-  cc.index_local_tokens = 0;
-  s = run_topk(&cc, n_rows, pos_c, h.ld_c, cand, h.ld_c, idx, count, topk_w, topk_bytes, st);
-  if (s != LSA_OK && s != LSA_DENSE) return s;
-  return cuda_status(launch_hier_map(pos, sorted, h.kb, block, n_rows, c->index_topk, idx, count, st), fn);
+  TopkArgs tc = topk_args(cand, h.ld_c, h.ld_c, c->index_topk, 0, 0, idx, count);
+  tc.pos = pos_c;
+  tc.col_map = sorted;
+  tc.col_block = block;
+  tc.col_ld = h.kb;
+  return cuda_status(launch_topk(tc, st), fn);
 }
 
 }  // extern "C"

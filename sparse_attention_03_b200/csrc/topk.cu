@@ -47,7 +47,8 @@ struct RowGeom {
 
 __device__ __forceinline__ RowGeom row_geom(const TopkArgs& a, int r) {
   RowGeom g;
-  g.n = (int64_t)a.pos[r] + 1;
+  const int pr = a.pos[r];
+  g.n = (int64_t)(a.pos_div == 1 ? pr : (pr >= 0 ? pr / a.pos_div : -1)) + 1;
   if (g.n < 0) g.n = 0;
   if (g.n > a.max_len) g.n = a.max_len;
   g.dense = g.n <= a.topk;
@@ -260,13 +261,17 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
   const RowGeom g = row_geom(a, r);
   int32_t* __restrict__ out = a.idx + (int64_t)r * a.topk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int32_t* __restrict__ cmap = a.col_map ? a.col_map + (int64_t)r * a.col_ld : nullptr;
+  auto col = [&](int64_t j) -> int32_t {
+    return cmap ? cmap[j / a.col_block] * a.col_block + (int32_t)(j % a.col_block) : (int32_t)j;
+  };
   if (g.dense) {
-    for (int i = tid; i < a.topk; i += kRowThreads) out[i] = (i < g.n) ? i : -1;
+    for (int i = tid; i < a.topk; i += kRowThreads) out[i] = (i < g.n) ? col(i) : -1;
     if (tid == 0) a.count[r] = (int32_t)g.n;
     return;
   }
-  for (int i = tid; i < a.n_init; i += kRowThreads) out[i] = i;
-  for (int i = tid; i < a.n_loc; i += kRowThreads) out[a.n_init + i] = (int32_t)(g.hi + i);
+  for (int i = tid; i < a.n_init; i += kRowThreads) out[i] = col(i);
+  for (int i = tid; i < a.n_loc; i += kRowThreads) out[a.n_init + i] = col(g.hi + i);
   if (tid == 0) {
     a.count[r] = a.topk;
     s_up = 0;
@@ -325,7 +330,7 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
         if (lane == 0) s0 = atomicAdd(&s_up, (uint32_t)__popc(up));
         s0 = __shfl_sync(0xffffffffu, s0, 0);
         const uint32_t slot = s0 + __popc(up & ((1u << lane) - 1u));
-        if (kb > bin0 && slot < k_rem) mid[slot] = (int32_t)j;
+        if (kb > bin0 && slot < k_rem) mid[slot] = col(j);
       }
       if (eq) {
         uint32_t s0 = 0;
@@ -367,7 +372,7 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
   for_each([&](uint64_t v, int64_t j) {
     if ((v >> sh) >= prefix) {
       const uint32_t slot = atomicAdd(&s_slot, 1u);
-      if (slot < need0) dst[slot] = (int32_t)j;
+      if (slot < need0) dst[slot] = col(j);
     }
   });
 }
@@ -396,7 +401,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   if (a.max_len <= a.topk) return launch_topk_dense(a, st);
   const int64_t chunks = (a.max_len + kChunk - 1) / kChunk;
   HistCtl* hc = static_cast<HistCtl*>(a.ws);
-  const bool per_row = !topk_uses_workspace(a.n_rows, a.max_len);
+  const bool per_row = !topk_uses_workspace(a.n_rows, a.max_len) || a.col_map != nullptr;
   if (per_row) {
     const uint32_t* hist_in = a.hist_ext;
     for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {

@@ -11,6 +11,8 @@ current stream, checks the device error flags and exits. Cases:
   topk_decode    lsa_topk on 16 rows x 131072 scores, with the indexer's histogram
   mla_decode     lsa_sparse_mla_decode, 16 rows x 2048 selected keys of 131072
   mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
+  hier_decode    lsa_block_summaries of each row's newest block + lsa_hier_select (64-key blocks,
+                 128 kept), 16 rows x 131072 keys
 """
 from __future__ import annotations
 
@@ -91,6 +93,27 @@ def case_mla_prefill(reps):
     ws = lsa.workspace(cfg, lsa.OP_MLA_PREFILL, n_rows, 1, n_keys)
     for _ in range(reps):
         lsa.sparse_mla_prefill(cfg, wl.pos, wl.q_abs[0], wl.latent[0], idx, cnt, out, lse, ws)
+
+
+def case_hier_decode(reps):
+    cfg = lsa.LsaConfig()
+    wl = _decode_layer(False)
+    block, n_blocks, B, ctx = 64, 128, 16, 131072
+    blk_off = torch.tensor(lsa.block_offsets([ctx] * B, block), dtype=torch.int64, device="cuda")
+    nb = ctx // block
+    k_blk = torch.empty((B * nb, 128), dtype=torch.bfloat16, device="cuda")
+    lsa.block_summaries(cfg, torch.arange(B, dtype=torch.int32, device="cuda").repeat_interleave(nb),
+                        torch.arange(nb, dtype=torch.int32, device="cuda").repeat(B), wl.k_idx, wl.k_off, blk_off,
+                        k_blk, block)
+    new_seq = torch.arange(B, dtype=torch.int32, device="cuda")
+    new_blk = torch.full((B,), nb - 1, dtype=torch.int32, device="cuda")
+    idx = torch.empty((B, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((B,), dtype=torch.int32, device="cuda")
+    ws = lsa.hier_workspace(cfg, B, ctx, block, n_blocks)
+    for _ in range(reps):
+        lsa.block_summaries(cfg, new_seq, new_blk, wl.k_idx, wl.k_off, blk_off, k_blk, block)
+        lsa.hier_select(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, k_blk, blk_off, ctx, idx,
+                        cnt, ws, block, n_blocks)
 
 
 CASES = {name[5:]: fn for name, fn in globals().items() if name.startswith("case_")}
