@@ -195,41 +195,22 @@ __global__ void __launch_bounds__(kThreads, 3)
 // over only the tokens of each row's kept blocks, written to a compact row
 // (slot i = token sorted[i / block] * block + i % block, blocks in ascending
 // order so that the top-k's lower-slot tie rule is the lower-column rule).
-// Forced tokens are +inf, tokens after the row's position -inf.
+// Forced tokens are +inf, tokens after the row's position -inf. Each CTA also
+// adds its slots to the compact row's top-k histogram (the top 11 bits of every
+// slot's score key, as the top-k's own first pass would count them).
 __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, int blocks_per_cta) {
   __shared__ int32_t ids[kMaxHierBlocks];
   __shared__ int32_t srt[kMaxHierBlocks];
+  __shared__ uint32_t sh[2048];   // the kept blocks as a bitmap, then the histogram
+  __shared__ uint32_t pre[2048];  // set bits in the bitmap's earlier words
   pdl_wait();
   const IndexArgs& a = h.ix;
   const int r = blockIdx.y;
-  const int n = min(h.kept_n[r], h.kb);
-  const int32_t* __restrict__ kr = h.kept + (int64_t)r * h.kb;
-  // (a kept id is a visible block, >= 0; clamping and pre-filling keep every
-  // token index below non-negative even for a malformed list)
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    ids[i] = max(kr[i], 0);
-    srt[i] = 0;
-  }
-  __syncthreads();
-  // ascending order by counting (the ids of a row are distinct)
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    const int v = ids[i];
-    int rank = 0;
-    for (int j = 0; j < n; ++j) rank += ids[j] < v;
-    srt[rank] = v;
-  }
-  __syncthreads();
-  if (blockIdx.x == 0) {
-    for (int i = threadIdx.x; i < n; i += kThreads) h.sorted[(int64_t)r * h.kb + i] = srt[i];
-    // a dense row keeps every block 0 .. pos / block, so its compact slots 0 .. pos
-    // are its tokens 0 .. pos in order
-    if (threadIdx.x == 0) {
-      const int pr = a.pos[r];
-      h.pos_c[r] = (pr >= 0 && pr + 1 <= h.topk) ? pr : n * h.block - 1;
-    }
-  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int g = lane >> 2, t = lane & 3;
 
-  // row geometry, clamped and flagged as in the flat indexer
+  // row geometry, clamped and flagged as in the flat indexer; the query
+  // fragments and head weights are requested before the kept list is sorted
   const int seq = a.seq_of_row ? a.seq_of_row[r] : (a.seq_identity ? r : 0);
   int64_t kbase = 0, klen = a.max_len;
   bool ok = true;
@@ -247,12 +228,6 @@ __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, 
     nvis = max64(0, min(nvis, min(klen, a.max_len)));
   }
   if (!ok) nvis = 0;
-
-  const int64_t s_lo = (int64_t)blockIdx.x * blocks_per_cta * h.block;
-  const int64_t s_hi = min((int64_t)(blockIdx.x + 1) * blocks_per_cta, (int64_t)n) * h.block;
-  if (s_lo >= s_hi) return;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int g = lane >> 2, t = lane & 3;
   uint4 qf[4][4];
   const uint16_t* __restrict__ qr = a.q_idx + (int64_t)r * kHi * kDi;
 #pragma unroll
@@ -265,37 +240,111 @@ __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, 
   for (int nt = 0; nt < 4; ++nt)
 #pragma unroll
     for (int e = 0; e < 2; ++e) wf[nt][e] = __ldg(a.w + (int64_t)r * kHi + 8 * nt + 2 * t + e);
+
+  // the kept blocks in ascending order (the ids of a row are distinct; clamping
+  // and pre-filling keep every token index in range even for a malformed list):
+  // ranks from a bitmap of the ids and its prefix counts when the ids fit in
+  // 65536 bits, else by counting
+  const int n = min(h.kept_n[r], h.kb);
+  const int32_t* __restrict__ kr = h.kept + (int64_t)r * h.kb;
+  const bool bitmap = h.nb_max <= 2048 * 32;
+  const int n_words = bitmap ? (int)((h.nb_max + 31) / 32) : 0;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    ids[i] = min(max(kr[i], 0), (int)max64(h.nb_max - 1, 0));
+    srt[i] = 0;
+  }
+  for (int i = threadIdx.x; i < n_words; i += kThreads) sh[i] = 0;
+  __syncthreads();
+  if (bitmap) {
+    for (int i = threadIdx.x; i < n; i += kThreads) atomicOr(&sh[ids[i] >> 5], 1u << (ids[i] & 31));
+    __syncthreads();
+    if (warp == 0) {  // exclusive prefix of the words' popcounts, 32 words per step
+      uint32_t carry = 0;
+      for (int w0 = 0; w0 < n_words; w0 += 32) {
+        const uint32_t c = w0 + lane < n_words ? (uint32_t)__popc(sh[w0 + lane]) : 0u;
+        uint32_t x = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+          if (lane >= o) x += y;
+        }
+        if (w0 + lane < n_words) pre[w0 + lane] = carry + x - c;
+        carry += __shfl_sync(0xffffffffu, x, 31);
+      }
+    }
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const int v = ids[i];
+      srt[pre[v >> 5] + __popc(sh[v >> 5] & ((1u << (v & 31)) - 1u))] = v;
+    }
+  } else {
+    for (int i = threadIdx.x; i < n; i += kThreads) {
+      const int v = ids[i];
+      int rank = 0;
+      for (int j = 0; j < n; ++j) rank += ids[j] < v;
+      srt[rank] = v;
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < 2048; i += kThreads) sh[i] = 0;  // now the histogram
+  __syncthreads();
+  const bool dense_row = p >= 0 && p + 1 <= h.topk;
+  if (blockIdx.x == 0) {
+    for (int i = threadIdx.x; i < n; i += kThreads) h.sorted[(int64_t)r * h.kb + i] = srt[i];
+    // a dense row keeps every block 0 .. pos / block, so its compact slots 0 .. pos
+    // are its tokens 0 .. pos in order
+    if (threadIdx.x == 0) h.pos_c[r] = dense_row ? (int32_t)p : n * h.block - 1;
+  }
+
+  const int64_t s_lo = (int64_t)blockIdx.x * blocks_per_cta * h.block;
+  const int64_t s_hi = min((int64_t)(blockIdx.x + 1) * blocks_per_cta, (int64_t)n) * h.block;
   const uint16_t* __restrict__ kb = a.k_idx + kbase * kDi;
   const int64_t lo_force = a.n_init, hi_force = p + 1 - a.n_loc;
   float* __restrict__ crow = h.cand + (int64_t)r * h.ld_c;
   // slot tiles of 16 (a block is a multiple of 16 keys, so a tile never straddles two)
   auto tok = [&](int64_t s) { return (int64_t)srt[s / h.block] * h.block + s % h.block; };
+  // a tile whose tokens are all forced or all past the row's position needs no keys
+  auto needs_keys = [&](int64_t s) {
+    const int64_t j0 = tok(s);
+    return !(j0 + kKeysPerWarpTile <= lo_force || (j0 >= hi_force) || j0 >= nvis);
+  };
   auto put = [&](int64_t s, float sa, float sb) {
     if (t < 2) {
       const int64_t j = tok(s) + g + (t == 1 ? 8 : 0);
       const bool forced = (j < lo_force) || (j >= hi_force);
-      crow[s + g + (t == 1 ? 8 : 0)] = j >= nvis ? -INFINITY : forced ? INFINITY : (t == 1 ? sb : sa);
+      const float v = j >= nvis ? -INFINITY : forced ? INFINITY : (t == 1 ? sb : sa);
+      crow[s + g + (t == 1 ? 8 : 0)] = v;
+      atomicAdd(&sh[score_key(v) >> 21], 1u);
     }
   };
   const int64_t step = kWarps * kKeysPerWarpTile;
   int64_t s = s_lo + warp * kKeysPerWarpTile;
-  if (s >= s_hi) return;
-  KeyFrag f0, f1;
-  load_keys(f0, kb, tok(s) + g, nvis, t);
-  while (true) {
-    int64_t nxt = s + step;
-    if (nxt < s_hi) load_keys(f1, kb, tok(nxt) + g, nvis, t);
-    float sa, sb;
-    score_tile(f0, qf, wf, sa, sb);
-    put(s, sa, sb);
-    if (nxt >= s_hi) break;
-    s = nxt;
-    nxt = s + step;
-    if (nxt < s_hi) load_keys(f0, kb, tok(nxt) + g, nvis, t);
-    score_tile(f1, qf, wf, sa, sb);
-    put(s, sa, sb);
-    if (nxt >= s_hi) break;
-    s = nxt;
+  if (s < s_hi) {
+    KeyFrag f0, f1;
+    const int64_t tend = 0;  // (no key is read for a tile that needs none)
+    load_keys(f0, kb, tok(s) + g, needs_keys(s) ? nvis : tend, t);
+    while (true) {
+      int64_t nxt = s + step;
+      if (nxt < s_hi) load_keys(f1, kb, tok(nxt) + g, needs_keys(nxt) ? nvis : tend, t);
+      float sa, sb;
+      score_tile(f0, qf, wf, sa, sb);
+      put(s, sa, sb);
+      if (nxt >= s_hi) break;
+      s = nxt;
+      nxt = s + step;
+      if (nxt < s_hi) load_keys(f0, kb, tok(nxt) + g, needs_keys(nxt) ? nvis : tend, t);
+      score_tile(f1, qf, wf, sa, sb);
+      put(s, sa, sb);
+      if (nxt >= s_hi) break;
+      s = nxt;
+    }
+  }
+  pdl_trigger();
+  __syncthreads();
+  if (!dense_row && s_lo < s_hi) {
+    uint32_t* __restrict__ hr = h.hist + (int64_t)r * kTopkHistStride;
+    for (int i = threadIdx.x; i < 2048; i += kThreads)
+      if (sh[i]) atomicAdd(&hr[i], sh[i]);
   }
 }
 
@@ -367,6 +416,7 @@ cudaError_t launch_hier_fine(const HierFineArgs& h, cudaStream_t st) {
     b.sorted += (int64_t)row0 * h.kb;
     b.pos_c += row0;
     b.cand += (int64_t)row0 * h.ld_c;
+    b.hist += (int64_t)row0 * kTopkHistStride;
     const cudaError_t e = launch_pdl(hier_fine_kernel, dim3(nx, ny), dim3(kThreads), 0, st, b, bpc);
     if (e != cudaSuccess) return e;
     count_launches(1);

@@ -63,7 +63,11 @@ struct TopkArgs {
   // map every row goes through the one-CTA-per-row kernel.
   const int32_t* col_map = nullptr;
   int col_block = 1;
-  int64_t col_ld = 0;
+  int64_t col_ld = 0;      // <= 2048
+  // Optional: rows of another histogram buffer (kTopkHistStride words apart) that
+  // this call clears, row r by row r's CTA, for a later producer. Also forces
+  // the one-CTA-per-row kernel.
+  uint32_t* zero_hist = nullptr;
 };
 constexpr int kTopkCap = 4096;                              // candidates kept per row
 constexpr size_t kTopkRowBytes = 2048 * 4 + 32 + kTopkCap * 8;  // hist + ctl + candidates
@@ -145,11 +149,13 @@ struct HierFineArgs {
   const int32_t* kept;      // [n_rows, kb] kept blocks, unordered
   const int32_t* kept_n;    // [n_rows]
   int kb, block;
+  int64_t nb_max;           // blocks a row can have (bounds the kept ids)
   int32_t* sorted;          // out [n_rows, kb]: the kept blocks in ascending order
   int32_t* pos_c;           // out [n_rows]: kept_n * block - 1, or pos for a dense row (pos + 1 <= topk)
   int topk;
   float* cand;              // out [n_rows, ld_c]: slot i = token sorted[i / block] * block + i % block
   int64_t ld_c;
+  uint32_t* hist;           // out: the compact rows' top-k histograms (kTopkHistStride apart, zeroed)
 };
 // Scores the tokens of each row's kept blocks into the compact rows.
 cudaError_t launch_hier_fine(const HierFineArgs& a, cudaStream_t st);

@@ -181,7 +181,7 @@ MlaArgs mla_args(const lsa_config* c, int cli, int n_rows, int decode) {
 struct HierPlan {
   int n_init_b, n_loc_b, kb;  // forced sink / recent blocks, blocks kept per row
   int64_t nb_max, ld_b, ld_c; // blocks per row at most, coarse and compact row strides
-  size_t off_pos_c, off_coarse, off_kept, off_kept_n, off_sorted, off_cand, off_topk, total;
+  size_t off_pos_c, off_hist, off_coarse, off_kept, off_kept_n, off_sorted, off_cand, off_topk, total;
 };
 
 HierPlan hier_plan(const lsa_config* c, int n_rows, int64_t max_len, int block, int n_blocks) {
@@ -195,6 +195,7 @@ HierPlan hier_plan(const lsa_config* c, int n_rows, int64_t max_len, int block, 
   const size_t R = (size_t)n_rows;
   size_t o = 0;
   h.off_pos_c = o;  o += align_up(R * 4);
+  h.off_hist = o;   o += align_up(R * kTopkHistStride * 4);
   h.off_coarse = o; o += align_up(R * h.ld_b * 4);
   h.off_kept = o;   o += align_up(R * h.kb * 4);
   h.off_kept_n = o; o += align_up(R * 4);
@@ -609,6 +610,7 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   int32_t* kept_n = reinterpret_cast<int32_t*>(base + h.off_kept_n);
   int32_t* sorted = reinterpret_cast<int32_t*>(base + h.off_sorted);
   float* cand = reinterpret_cast<float*>(base + h.off_cand);
+  uint32_t* hist_c = reinterpret_cast<uint32_t*>(base + h.off_hist);
   void* topk_w = base + h.off_topk;
   const size_t topk_bytes = topk_ws(n_rows);
 
@@ -659,6 +661,7 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   if (s != LSA_OK) return s;
   TopkArgs tb = topk_args(coarse, h.ld_b, h.nb_max, h.kb, h.n_init_b, h.n_loc_b, kept, kept_n);
   tb.pos_div = block;
+  tb.zero_hist = hist_c;  // for the fine stage, which builds the compact rows' histograms
   s = cuda_status(launch_topk(tb, st), fn);
   if (s != LSA_OK) return s;
   // fine stage: the kept blocks' tokens into compact rows, then the flat top-k
@@ -676,15 +679,18 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   f.kept_n = kept_n;
   f.kb = h.kb;
   f.block = block;
+  f.nb_max = h.nb_max;
   f.sorted = sorted;
   f.pos_c = pos_c;
   f.topk = c->index_topk;
   f.cand = cand;
   f.ld_c = h.ld_c;
+  f.hist = hist_c;
   s = cuda_status(launch_hier_fine(f, st), fn);
   if (s != LSA_OK) return s;
   TopkArgs tc = topk_args(cand, h.ld_c, h.ld_c, c->index_topk, 0, 0, idx, count);
   tc.pos = pos_c;
+  tc.hist_ext = hist_c;
   tc.col_map = sorted;
   tc.col_block = block;
   tc.col_ld = h.kb;

@@ -256,14 +256,20 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
   __shared__ uint64_t cand[kRowCap];
   __shared__ int s_bin;
   __shared__ uint32_t s_above, s_warp[kRowThreads / 32], s_up, s_nc, s_slot;
+  extern __shared__ int32_t s_map[];  // the row's column map (col_ld entries) when there is one
   pdl_wait();
   const int r = row0 + blockIdx.x;
   const RowGeom g = row_geom(a, r);
   int32_t* __restrict__ out = a.idx + (int64_t)r * a.topk;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int32_t* __restrict__ cmap = a.col_map ? a.col_map + (int64_t)r * a.col_ld : nullptr;
+  if (a.zero_hist)
+    for (int i = tid; i < kBins; i += kRowThreads) a.zero_hist[(int64_t)r * kTopkHistStride + i] = 0;
+  if (a.col_map) {
+    for (int i = tid; i < a.col_ld; i += kRowThreads) s_map[i] = a.col_map[(int64_t)r * a.col_ld + i];
+    __syncthreads();
+  }
   auto col = [&](int64_t j) -> int32_t {
-    return cmap ? cmap[j / a.col_block] * a.col_block + (int32_t)(j % a.col_block) : (int32_t)j;
+    return a.col_map ? s_map[j / a.col_block] * a.col_block + (int32_t)(j % a.col_block) : (int32_t)j;
   };
   if (g.dense) {
     for (int i = tid; i < a.topk; i += kRowThreads) out[i] = (i < g.n) ? col(i) : -1;
@@ -314,32 +320,44 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
       const int64_t j = base + lane + 32 * u;
       v[u] = j < g.hi ? srow[j] : 0.f;
     }
+    // one pair of shared atomics per warp and round: the round's counts first
+    uint32_t key[kUnroll], upm[kUnroll], eqm[kUnroll];
+    int kb[kUnroll];
+    uint32_t n_up = 0, n_eq = 0;
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       const int64_t j = base + lane + 32 * u;
-      uint32_t key = 0;
-      int kb = -1;
+      key[u] = 0;
+      kb[u] = -1;
       if (j < g.hi) {
-        key = score_key(v[u]);
-        kb = (int)(key >> 21);
+        key[u] = score_key(v[u]);
+        kb[u] = (int)(key[u] >> 21);
       }
-      const uint32_t up = __ballot_sync(0xffffffffu, kb > bin0);
-      const uint32_t eq = __ballot_sync(0xffffffffu, kb == bin0);
-      if (up) {
-        uint32_t s0 = 0;
-        if (lane == 0) s0 = atomicAdd(&s_up, (uint32_t)__popc(up));
-        s0 = __shfl_sync(0xffffffffu, s0, 0);
-        const uint32_t slot = s0 + __popc(up & ((1u << lane) - 1u));
-        if (kb > bin0 && slot < k_rem) mid[slot] = col(j);
+      upm[u] = __ballot_sync(0xffffffffu, kb[u] > bin0);
+      eqm[u] = __ballot_sync(0xffffffffu, kb[u] == bin0);
+      n_up += __popc(upm[u]);
+      n_eq += __popc(eqm[u]);
+    }
+    uint32_t b_up = 0, b_eq = 0;
+    if (lane == 0) {
+      if (n_up) b_up = atomicAdd(&s_up, n_up);
+      if (n_eq) b_eq = atomicAdd(&s_nc, n_eq);
+    }
+    b_up = __shfl_sync(0xffffffffu, b_up, 0);
+    b_eq = __shfl_sync(0xffffffffu, b_eq, 0);
+    const uint32_t below = (1u << lane) - 1u;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t j = base + lane + 32 * u;
+      if (kb[u] > bin0) {
+        const uint32_t slot = b_up + __popc(upm[u] & below);
+        if (slot < k_rem) mid[slot] = col(j);
+      } else if (kb[u] == bin0) {
+        const uint32_t slot = b_eq + __popc(eqm[u] & below);
+        if (slot < (uint32_t)kRowCap) cand[slot] = ((uint64_t)key[u] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
       }
-      if (eq) {
-        uint32_t s0 = 0;
-        if (lane == 0) s0 = atomicAdd(&s_nc, (uint32_t)__popc(eq));
-        s0 = __shfl_sync(0xffffffffu, s0, 0);
-        const uint32_t slot = s0 + __popc(eq & ((1u << lane) - 1u));
-        if (kb == bin0 && slot < (uint32_t)kRowCap)
-          cand[slot] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
-      }
+      b_up += __popc(upm[u]);
+      b_eq += __popc(eqm[u]);
     }
   }
   __syncthreads();
@@ -379,12 +397,24 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
 
 }  // namespace
 
+// Dynamic shared memory of the per-row kernel: the column map, if any (at most
+// 2048 entries; the attribute allowing it above the 48 KB default is set once).
+static size_t row_map_smem(const TopkArgs& a) {
+  if (!a.col_map) return 0;
+  static bool attr_set = false;  // benign race: every caller sets the same value
+  if (!attr_set) {
+    cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2048 * 4);
+    attr_set = true;
+  }
+  return (size_t)a.col_ld * sizeof(int32_t);
+}
+
 cudaError_t launch_topk_dense(const TopkArgs& a, cudaStream_t st) {
   // every row is dense: the per-row kernel writes 0..n-1 and the count
   for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
     const int nr = min(65535, a.n_rows - row0);
     const cudaError_t e =
-        launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), 0, st, a, row0, (const uint32_t*)nullptr);
+        launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), row_map_smem(a), st, a, row0, (const uint32_t*)nullptr);
     if (e != cudaSuccess) return e;
     count_launches(1);
   }
@@ -401,12 +431,13 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   if (a.max_len <= a.topk) return launch_topk_dense(a, st);
   const int64_t chunks = (a.max_len + kChunk - 1) / kChunk;
   HistCtl* hc = static_cast<HistCtl*>(a.ws);
-  const bool per_row = !topk_uses_workspace(a.n_rows, a.max_len) || a.col_map != nullptr;
+  const bool per_row = !topk_uses_workspace(a.n_rows, a.max_len) || a.col_map != nullptr || a.zero_hist != nullptr;
   if (per_row) {
     const uint32_t* hist_in = a.hist_ext;
     for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
       const int nr = min(65535, a.n_rows - row0);
-      const cudaError_t e = launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), 0, st, a, row0, hist_in);
+      const cudaError_t e =
+          launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), row_map_smem(a), st, a, row0, hist_in);
       if (e != cudaSuccess) return e;
       count_launches(1);
     }
