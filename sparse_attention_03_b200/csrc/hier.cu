@@ -40,13 +40,21 @@ __device__ __forceinline__ uint16_t f64_to_bf16_rne(double x) {
   return (uint16_t)((sign << 15) | out);
 }
 
-// One CTA (128 threads, thread = dim d) per item: the mean of the block's keys.
-__global__ void __launch_bounds__(kDi) block_summary_kernel(BlockSumArgs a) {
+// One CTA per item: the mean of the block's keys. Thread (grp, c) sums keys
+// grp, grp + 16, ... over dims 8c .. 8c + 7 with 16-byte loads (every load of the
+// block in flight at once), then the 16 partial sums of each dim are added in a
+// fixed order (the fp64 sums are exact, so the order does not change them).
+constexpr int kSumThreads = 256;
+constexpr int kSumGroups = kSumThreads / (kDi / 8);  // 16 key groups
+
+__global__ void __launch_bounds__(kSumThreads) block_summary_kernel(BlockSumArgs a) {
+  __shared__ double part[kSumGroups][kDi];
   pdl_wait();
-  const int i = blockIdx.x, d = threadIdx.x;
+  const int i = blockIdx.x, tid = threadIdx.x;
+  const int grp = tid / (kDi / 8), c = tid % (kDi / 8);
   const int s = a.item_seq[i];
   if (s < 0 || s >= a.n_seq) {
-    if (d == 0) flag_error(a.err, LSA_DEVERR_SEQ);
+    if (tid == 0) flag_error(a.err, LSA_DEVERR_SEQ);
     return;
   }
   const int64_t base = a.k_off[s], len = a.k_off[s + 1] - base;
@@ -54,26 +62,36 @@ __global__ void __launch_bounds__(kDi) block_summary_kernel(BlockSumArgs a) {
   const int64_t b = a.item_blk[i];
   const int64_t t0 = b * a.block, t1 = min64(t0 + a.block, len);
   if (b < 0 || b >= nb || t0 >= len) {
-    if (d == 0) flag_error(a.err, LSA_DEVERR_POS);
+    if (tid == 0) flag_error(a.err, LSA_DEVERR_POS);
     return;
   }
-  const uint16_t* __restrict__ k = a.k_idx + (base + t0) * kDi + d;
-  // fp64 sum: exact for up to 1024 bf16 terms spanning fewer than 35 binades, so
-  // the mean is the correctly rounded fp64 quotient before the bf16 rounding
-  // (the order of the exact additions is free: eight chains keep eight loads in flight)
   const int n = (int)(t1 - t0);
-  double part[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-  int t = 0;
-  for (; t + 8 <= n; t += 8) {
-    uint16_t v[8];
+  const uint4* __restrict__ k = reinterpret_cast<const uint4*>(a.k_idx + (base + t0) * kDi) + c;
+  double acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+  for (int t = grp; t < n; t += kSumGroups * 4) {
+    uint4 v[4];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) v[u] = __ldg(k + (int64_t)(t + u) * kDi);
+    for (int u = 0; u < 4; ++u) v[u] = t + u * kSumGroups < n ? __ldg(k + (int64_t)(t + u * kSumGroups) * (kDi / 8))
+                                                              : make_uint4(0, 0, 0, 0);
 #pragma unroll
-    for (int u = 0; u < 8; ++u) part[u] += (double)__uint_as_float((uint32_t)v[u] << 16);
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        acc[2 * e] += (double)__uint_as_float(w[e] << 16);
+        acc[2 * e + 1] += (double)__uint_as_float(w[e] & 0xffff0000u);
+      }
+    }
   }
-  for (; t < n; ++t) part[0] += (double)__uint_as_float((uint32_t)__ldg(k + (int64_t)t * kDi) << 16);
-  const double sum = ((part[0] + part[1]) + (part[2] + part[3])) + ((part[4] + part[5]) + (part[6] + part[7]));
-  a.k_blk[(bbase + b) * kDi + d] = f64_to_bf16_rne(sum / (double)n);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) part[grp][8 * c + e] = acc[e];
+  __syncthreads();
+  if (tid < kDi) {
+    double sum = 0.0;
+#pragma unroll
+    for (int g2 = 0; g2 < kSumGroups; ++g2) sum += part[g2][tid];
+    a.k_blk[(bbase + b) * kDi + tid] = f64_to_bf16_rne(sum / (double)n);
+  }
   pdl_trigger();
 }
 
@@ -82,7 +100,7 @@ __global__ void __launch_bounds__(kDi) block_summary_kernel(BlockSumArgs a) {
 cudaError_t launch_block_summaries(const BlockSumArgs& a, cudaStream_t st) {
   if (a.n_items <= 0) return cudaSuccess;
   count_launches(1);
-  return launch_pdl(block_summary_kernel, dim3(a.n_items), dim3(kDi), 0, st, a);
+  return launch_pdl(block_summary_kernel, dim3(a.n_items), dim3(kSumThreads), 0, st, a);
 }
 
 }  // namespace lsa
