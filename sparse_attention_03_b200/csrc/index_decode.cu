@@ -195,9 +195,14 @@ __global__ void __launch_bounds__(kThreads, 3)
 // over only the tokens of each row's kept blocks, written to a compact row
 // (slot i = token sorted[i / block] * block + i % block, blocks in ascending
 // order so that the top-k's lower-slot tie rule is the lower-column rule).
-// Forced tokens are +inf, tokens after the row's position -inf. Each CTA also
-// adds its slots to the compact row's top-k histogram (the top 11 bits of every
-// slot's score key, as the top-k's own first pass would count them).
+// The kept blocks always include the sink blocks (first in order) and the most
+// recent blocks (last, consecutive), so in compact slots the sink tokens are
+// 0 .. init-1 and the local window is the `local` slots ending at the slot of
+// the row's own token, pos_c: the flat top-k then applies its own forcing to
+// the compact row with position pos_c, and only the tokens in between are
+// scored here. Each CTA also adds those slots to the compact row's top-k
+// histogram (the top 11 bits of each score key, as the top-k's first pass
+// would count its middle columns).
 __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, int blocks_per_cta) {
   __shared__ int32_t ids[kMaxHierBlocks];
   __shared__ int32_t srt[kMaxHierBlocks];
@@ -291,9 +296,9 @@ __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, 
   const bool dense_row = p >= 0 && p + 1 <= h.topk;
   if (blockIdx.x == 0) {
     for (int i = threadIdx.x; i < n; i += kThreads) h.sorted[(int64_t)r * h.kb + i] = srt[i];
-    // a dense row keeps every block 0 .. pos / block, so its compact slots 0 .. pos
-    // are its tokens 0 .. pos in order
-    if (threadIdx.x == 0) h.pos_c[r] = dense_row ? (int32_t)p : n * h.block - 1;
+    // the row's own token is in the last kept block (a dense row keeps every
+    // block, so there pos_c = pos); -1 for a row with no visible key
+    if (threadIdx.x == 0) h.pos_c[r] = (n > 0 && nvis > 0) ? (n - 1) * h.block + (int32_t)((nvis - 1) % h.block) : -1;
   }
 
   const int64_t s_lo = (int64_t)blockIdx.x * blocks_per_cta * h.block;
@@ -301,8 +306,13 @@ __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, 
   const uint16_t* __restrict__ kb = a.k_idx + kbase * kDi;
   const int64_t lo_force = a.n_init, hi_force = p + 1 - a.n_loc;
   float* __restrict__ crow = h.cand + (int64_t)r * h.ld_c;
-  // slot tiles of 16 (a block is a multiple of 16 keys, so a tile never straddles two)
-  auto tok = [&](int64_t s) { return (int64_t)srt[s / h.block] * h.block + s % h.block; };
+  // slot tiles of 16 (a block is a multiple of 16 keys, so a tile never straddles
+  // two); a compact row is shorter than 2^31 slots: 32-bit division
+  const uint32_t ub = (uint32_t)h.block;
+  auto tok = [&](int64_t s) {
+    const uint32_t su = (uint32_t)s, q = su / ub;
+    return (int64_t)srt[q] * h.block + (int64_t)(su - q * ub);
+  };
   // a tile whose tokens are all forced or all past the row's position needs no keys
   auto needs_keys = [&](int64_t s) {
     const int64_t j0 = tok(s);
@@ -312,9 +322,12 @@ __global__ void __launch_bounds__(kThreads, 3) hier_fine_kernel(HierFineArgs h, 
     if (t < 2) {
       const int64_t j = tok(s) + g + (t == 1 ? 8 : 0);
       const bool forced = (j < lo_force) || (j >= hi_force);
-      const float v = j >= nvis ? -INFINITY : forced ? INFINITY : (t == 1 ? sb : sa);
-      crow[s + g + (t == 1 ? 8 : 0)] = v;
-      atomicAdd(&sh[score_key(v) >> 21], 1u);
+      // forced slots and slots past the row's token are never read by the top-k
+      if (j < nvis && !forced) {
+        const float v = t == 1 ? sb : sa;
+        crow[s + g + (t == 1 ? 8 : 0)] = v;
+        atomicAdd(&sh[score_key(v) >> 21], 1u);
+      }
     }
   };
   const int64_t step = kWarps * kKeysPerWarpTile;

@@ -151,7 +151,7 @@ struct HierFineArgs {
   int kb, block;
   int64_t nb_max;           // blocks a row can have (bounds the kept ids)
   int32_t* sorted;          // out [n_rows, kb]: the kept blocks in ascending order
-  int32_t* pos_c;           // out [n_rows]: kept_n * block - 1, or pos for a dense row (pos + 1 <= topk)
+  int32_t* pos_c;           // out [n_rows]: the compact slot of the row's own token (see hier_fine_kernel)
   int topk;
   float* cand;              // out [n_rows, ld_c]: slot i = token sorted[i / block] * block + i % block
   int64_t ld_c;

@@ -688,7 +688,8 @@ lsa_status lsa_hier_select(const lsa_config* c, int32_t n_rows, int32_t n_seq, c
   f.hist = hist_c;
   s = cuda_status(launch_hier_fine(f, st), fn);
   if (s != LSA_OK) return s;
-  TopkArgs tc = topk_args(cand, h.ld_c, h.ld_c, c->index_topk, 0, 0, idx, count);
+  TopkArgs tc = topk_args(cand, h.ld_c, h.ld_c, c->index_topk, c->index_init_tokens, c->index_local_tokens, idx,
+                          count);
   tc.pos = pos_c;
   tc.hist_ext = hist_c;
   tc.col_map = sorted;

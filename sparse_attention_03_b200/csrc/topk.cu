@@ -268,8 +268,10 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
     for (int i = tid; i < a.col_ld; i += kRowThreads) s_map[i] = a.col_map[(int64_t)r * a.col_ld + i];
     __syncthreads();
   }
-  auto col = [&](int64_t j) -> int32_t {
-    return a.col_map ? s_map[j / a.col_block] * a.col_block + (int32_t)(j % a.col_block) : (int32_t)j;
+  auto col = [&](int64_t j) -> int32_t {  // (a mapped row is shorter than 2^31: 32-bit division)
+    if (!a.col_map) return (int32_t)j;
+    const uint32_t ju = (uint32_t)j, cb = (uint32_t)a.col_block, q = ju / cb;
+    return s_map[q] * a.col_block + (int32_t)(ju - q * cb);
   };
   if (g.dense) {
     for (int i = tid; i < a.topk; i += kRowThreads) out[i] = (i < g.n) ? col(i) : -1;
