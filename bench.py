@@ -149,16 +149,27 @@ def peaks():
     return PEAKS_FALLBACK, "fallback"
 
 
-def kernel_traffic(kernel: str, src: str):
-    """dram bytes per launch from the committed ncu summary, if it was taken on this source."""
+# the decode indexer's code: its kernel and its key-tile helpers
+INDEX_DECODE_SOURCES = ("index_decode.cu", "index_tile.cuh")
+
+
+def source_sha(srcs) -> str:
+    """sha256 over the kernel's source files (in order) under csrc/."""
+    h = hashlib.sha256()
+    for src in srcs:
+        h.update(open(os.path.join(ROOT, "sparse_attention_03_b200", "csrc", src), "rb").read())
+    return h.hexdigest()
+
+
+def kernel_traffic(kernel: str, srcs):
+    """dram bytes per launch from the committed ncu summary, if it was taken on these sources."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(kernel)
     if not d:
         return None
-    h = hashlib.sha256(open(os.path.join(ROOT, "sparse_attention_03_b200", "csrc", src), "rb").read()).hexdigest()
-    return d["bytes_per_launch"] if d.get("source_sha256") == h else None
+    return d["bytes_per_launch"] if d.get("source_sha256") == source_sha(srcs) else None
 
 
 # ---------------------------------------------------------------------------
@@ -614,7 +625,7 @@ def gpu_arm(args):
                    "l2": "inputs larger than L2 (8.6 GB of caches read per step), no flush"},
         "roofline": {"kernel": "index_decode_kernel", "bound": "hbm", "achieved": achieved, "peak": peak,
                      "unit": "GB/s", "frac": achieved / peak, "peak_source": f"{psrc} hbm_gbs",
-                     "traffic": kernel_traffic("index_decode_kernel", "index_decode.cu"),
+                     "traffic": kernel_traffic("index_decode_kernel", INDEX_DECODE_SOURCES),
                      "alg_bytes_per_launch": alg_bytes, "avg_launch_ms": statistics.mean(idx_ms)},
         "e2e": {"value": e2e_value, "unit": "tokens/s/layer", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": launches,
