@@ -300,7 +300,7 @@ def build_decode(device):
                              topk_hist=hist),
             lsa.topk(cfg, l.pos, ctx, scores, idx, cnt, tk_ws, bind=True, topk_hist=hist),
             [lsa.sparse_mla_decode(cfg, l.q_abs[z], l.latent[z], l.k_off, idx, cnt, ctx, out[i, z], lse[i, z],
-                                   mla_ws, bind=True) for z in range(2)]))
+                                   mla_ws, bind=True, lists_from_topk=True) for z in range(2)]))
         D["fwd"].append(lsa.forward(cfg, 0, l.seq_of_row, l.pos, ctx, l.q_idx, l.w, l.k_idx, l.k_off, l.q_abs,
                                     l.latent, [out[i, 0], out[i, 1]], [lse[i, 0], lse[i, 1]], ws, bind=True))
     # MTP draft round: one index pass shared by three draft steps, each attending
@@ -314,7 +314,7 @@ def build_decode(device):
     for i, l in enumerate(layers):
         qs = [l.q_abs[0], l.q_abs[1], q3[i]]
         D["mtp"].append([lsa.sparse_mla_decode(cfg, qs[st], l.latent[0], l.k_off, idx, cnt, ctx, out3, lse3,
-                                               mla_ws, bind=True) for st in range(3)])
+                                               mla_ws, bind=True, lists_from_topk=True) for st in range(3)])
     D["q3"] = q3
     return D
 

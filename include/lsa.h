@@ -295,6 +295,27 @@ LSA_API lsa_status lsa_hier_select(const lsa_config* cfg, int32_t n_rows, int32_
  * lse fp32 [batch, 32] or NULL. max_len (host) >= every L_b (sizes split-K).
  * Workspace optional (split-K partials): lsa_workspace_size(LSA_OP_MLA_DECODE).
  */
+/*
+ * lsa_sparse_mla_decode_topk: the same attention, for idx / count written by
+ * lsa_topk, lsa_forward or lsa_hier_select for these rows with this
+ * configuration. Every
+ * list then starts with the row's index_init_tokens sink columns and
+ * index_local_tokens local columns, which the position alone determines
+ * ([Lite-Sparse] LSA section: those columns are always selected), and the
+ * kernel gathers and attends over them before it waits for the previous kernel
+ * in the stream (the top-k); it reads idx and count only after that wait, and
+ * writes nothing before it. So q_abs, latent and k_off are read early: they
+ * must not be written by the immediately preceding kernel if that kernel lets
+ * its dependents start before it has finished (programmatic dependent launch);
+ * kernels of this library never write them. A count other than
+ * min(L_b, index_topk) sets LSA_DEVERR_COUNT. Arguments otherwise as
+ * lsa_sparse_mla_decode; idx must not be NULL.
+ */
+LSA_API lsa_status lsa_sparse_mla_decode_topk(const lsa_config* cfg, int32_t batch, const lsa_bf16* q_abs,
+                                              const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
+                                              const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,
+                                              void* ws, size_t ws_bytes, void* stream);
+
 LSA_API lsa_status lsa_sparse_mla_decode(const lsa_config* cfg, int32_t batch, const lsa_bf16* q_abs,
                                  const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
                                  const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,

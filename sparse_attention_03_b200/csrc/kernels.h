@@ -113,6 +113,10 @@ struct MlaArgs {
   const int32_t* idx;        // [n_rows, topk] or null (dense)
   const int32_t* count;
   int n_rows, n_seq, topk, decode, cli;
+  // The index lists were written by the top-k for these rows (every non-dense
+  // row's list starts with its n_init sink and n_loc local columns): the kernel
+  // attends over those before it waits for the previous kernel in the stream.
+  int forced_first = 0, n_init = 0, n_loc = 0;
   int64_t n_keys;            // prefill: rows in latent
   int64_t max_list;          // host bound on keys per row (sizes split-K)
   float scale;
@@ -122,7 +126,7 @@ struct MlaArgs {
 };
 // Split-K partial bytes for a given split count.
 size_t mla_ws_bytes(int n_rows, int cli, int n_split);
-int mla_choose_splits(int n_rows, int cli, int64_t max_list);
+int mla_choose_splits(int n_rows, int cli, int64_t max_list, bool forced_first = false);
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st);
 
 }  // namespace lsa

@@ -367,11 +367,13 @@ lsa_status lsa_index_project(const lsa_config* c, int32_t n_rows, int32_t n_seq,
   return cuda_status(launch_index_project(L, (cudaStream_t)stream), fn);
 }
 
-lsa_status lsa_sparse_mla_decode(const lsa_config* c, int32_t batch, const lsa_bf16* q_abs,
-                                 const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
-                                 const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,
-                                 void* ws, size_t ws_bytes, void* stream) {
-  const char* fn = "lsa_sparse_mla_decode";
+}  // extern "C"
+
+namespace {
+lsa_status mla_decode(const char* fn, bool lists_from_topk, const lsa_config* c, int32_t batch,
+                      const lsa_bf16* q_abs, const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
+                      const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse, void* ws, size_t ws_bytes,
+                      void* stream) {
   lsa_status s = check_cfg(c, fn);
   if (s != LSA_OK) return s;
   if (batch < 0 || max_len < 1) return set_error(LSA_ERR_INVALID, "%s: need batch >= 0, max_len >= 1", fn);
@@ -392,7 +394,32 @@ lsa_status lsa_sparse_mla_decode(const lsa_config* c, int32_t batch, const lsa_b
   a.max_list = idx ? c->index_topk : max_len;
   a.ws = ws;
   a.ws_bytes = ws ? ws_bytes : 0;
+  if (lists_from_topk) {
+    if (!idx) return set_error(LSA_ERR_INVALID, "%s: idx is NULL", fn);
+    a.forced_first = 1;
+    a.n_init = c->index_init_tokens;
+    a.n_loc = c->index_local_tokens;
+  }
   return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
+}
+}  // namespace
+
+extern "C" {
+
+lsa_status lsa_sparse_mla_decode(const lsa_config* c, int32_t batch, const lsa_bf16* q_abs,
+                                 const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
+                                 const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,
+                                 void* ws, size_t ws_bytes, void* stream) {
+  return mla_decode("lsa_sparse_mla_decode", false, c, batch, q_abs, latent, k_off, idx, count, max_len, out, lse,
+                    ws, ws_bytes, stream);
+}
+
+lsa_status lsa_sparse_mla_decode_topk(const lsa_config* c, int32_t batch, const lsa_bf16* q_abs,
+                                      const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
+                                      const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,
+                                      void* ws, size_t ws_bytes, void* stream) {
+  return mla_decode("lsa_sparse_mla_decode_topk", true, c, batch, q_abs, latent, k_off, idx, count, max_len, out,
+                    lse, ws, ws_bytes, stream);
 }
 
 lsa_status lsa_sparse_mla_prefill(const lsa_config* c, int32_t n_rows, const int32_t* pos,
@@ -532,6 +559,10 @@ lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_
     b.pos = pos + r0;
     b.idx = idx_b;
     b.count = cnt_b;
+    // the lists come from the top-k just above: the forced columns lead them
+    b.forced_first = 1;
+    b.n_init = c->index_init_tokens;
+    b.n_loc = c->index_local_tokens;
     b.max_list = c->index_topk;
     b.ws = mla_w;
     b.ws_bytes = mla_bytes;

@@ -98,6 +98,22 @@ __device__ __forceinline__ void half_sync(int h) { asm volatile("bar.sync %0, 12
 __device__ __forceinline__ void stagger_arrive() { asm volatile("bar.arrive 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 __device__ __forceinline__ void stagger_wait() { asm volatile("bar.sync 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 
+// A split's tiles of a forced-first list: whole tiles of the known prefix
+// [0, K), then whole tiles of the selected part [K, L), each part shared evenly
+// by the splits (only each part's last tile of a row can be partly empty).
+struct FfTiles {
+  int kt0, kt, ut0, ut;
+};
+__device__ __forceinline__ FfTiles ff_tiles(const ListPlan& p, int s, int n) {
+  const int Kt = (int)((p.K + kTK - 1) / kTK), Ut = (int)((p.L - p.K + kTK - 1) / kTK);
+  FfTiles f;
+  f.kt0 = Kt * s / n;
+  f.kt = Kt * (s + 1) / n - f.kt0;
+  f.ut0 = Ut * s / n;
+  f.ut = Ut * (s + 1) / n - f.ut0;
+  return f;
+}
+
 // Warp roles (math warps 0..7): head half mt = w >> 2 (heads 16mt .. 16mt+15)
 // and quarter kq = w & 3, so each SM sub-partition runs one warp of each half
 // and the two halves, which share nothing but the key tiles, drift apart and
@@ -123,13 +139,76 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   }
   __syncthreads();
   volatile int* abort_flag = &sm.abort_flag;
-  pdl_wait();
+  // Forced-first lists: the forced columns are gathered and attended over before
+  // the wait for the previous kernel (the top-k that writes idx / count); only
+  // the producer's index loads and the epilogue's stores come after it.
+  const bool ff = a.forced_first && a.idx;
+  if (!ff) pdl_wait();
 
   // This split's slots: whole tiles of the longest list, clipped to the row's own.
   const int64_t t_lo = (int64_t)sp.list_tiles * s / sp.n_split;
   const int64_t t_hi = (int64_t)sp.list_tiles * (s + 1) / sp.n_split;
   const int64_t b0 = t_lo * kTK;
   const int cap = (int)((t_hi - t_lo) * kTK);
+
+  if (warp == kMathWarps && ff) {
+    // ================= producer warp, forced-first list =================
+    const uint16_t* __restrict__ qg = a.q[z] + ((int64_t)r * kH + lane) * kDLat;
+    mbar_expect_tx(&sm.qbar, kRowBytes);
+    bulk_row(&sm.q[lane * kSRow], qg, &sm.qbar);
+    const RowGeom geo = row_base(a, r, false);
+    const ListPlan lp = list_plan(a, geo.nvis);
+    const FfTiles ft = ff_tiles(lp, s, sp.n_split);
+    const int n_tiles = ft.kt + ft.ut;
+    const uint16_t* __restrict__ latb = a.lat[z] + geo.kbase * kDLat;
+    auto issue = [&](int tt, int key) {
+      const int i = tt % kStages;
+      if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag);
+      sm.keys[i][lane] = key;
+      uint16_t* dst = &sm.k[i][lane * kSRow];
+      if (key >= 0) {
+        mbar_expect_tx(&sm.full[i], kRowBytes);
+        bulk_row(dst, latb + (int64_t)key * kDLat, &sm.full[i]);
+      } else {
+#pragma unroll 8
+        for (int c = 0; c < kDLat / 8; ++c) *reinterpret_cast<uint4*>(dst + 8 * c) = make_uint4(0, 0, 0, 0);
+        fence_proxy_async();
+        mbar_arrive(&sm.full[i]);
+      }
+    };
+    // the known slots (forced columns, or a dense row's whole list): keys by formula
+    for (int tt = 0; tt < ft.kt; ++tt) {
+      const int64_t sl = (int64_t)(ft.kt0 + tt) * kTK + lane;
+      issue(tt, sl < lp.K ? (int)known_key(lp, a, sl) : -1);
+    }
+    // the selected slots: the top-k's list, after it has finished
+    pdl_wait();
+    int c = a.count[r];
+    if (c != (int)lp.L && geo.nvis > 0) flag_error(a.err, LSA_DEVERR_COUNT);
+    const int64_t uend = max64(lp.K, min64((int64_t)c, lp.L));
+    const int32_t* __restrict__ irow = a.idx + (int64_t)r * a.topk;
+    for (int u = 0; u < ft.ut; ++u) {
+      const int64_t sl = lp.K + (int64_t)(ft.ut0 + u) * kTK + lane;
+      int64_t key = -1;
+      if (sl < uend) {
+        key = __ldg(irow + sl);
+        if (key < 0 || key >= geo.nvis) {
+          flag_error(a.err, LSA_DEVERR_INDEX);
+          key = -1;
+        }
+      }
+      sm.list[u * kTK + lane] = (int32_t)key;
+    }
+    for (int u = 0; u < ft.ut; ++u) issue(ft.kt + u, sm.list[u * kTK + lane]);
+    if (lane == 0) {
+      mbar_drain(&sm.qbar, 0);
+      for (int i = 0; i < kStages && i < n_tiles; ++i) {
+        const int last = i + ((n_tiles - 1 - i) / kStages) * kStages;
+        mbar_drain(&sm.full[i], (last / kStages) & 1);
+      }
+    }
+    return;
+  }
 
   if (warp == kMathWarps) {
     // ================= producer warp =================
@@ -211,9 +290,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   }
 
   // ================= math warps =================
-  const RowGeom geo = row_geometry(a, r, s == 0 && tid == 0);
-  const int nk = (int)max64(0, min64((int64_t)cap, geo.n_list - b0));
-  const int n_tiles = (nk + kTK - 1) / kTK;
+  int n_tiles;
+  if (ff) {
+    const RowGeom geo = row_base(a, r, s == 0 && tid == 0);
+    const FfTiles ft = ff_tiles(list_plan(a, geo.nvis), s, sp.n_split);
+    n_tiles = ft.kt + ft.ut;
+  } else {
+    const RowGeom geo = row_geometry(a, r, s == 0 && tid == 0);
+    const int nk = (int)max64(0, min64((int64_t)cap, geo.n_list - b0));
+    n_tiles = (nk + kTK - 1) / kTK;
+  }
   const int g = lane >> 2, t = lane & 3;
   const int mt = warp >> 2, kq = warp & 3;
   mbar_wait(&sm.qbar, 0, abort_flag);
@@ -355,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   if (tid == 0 && *abort_flag) flag_error(a.err, LSA_DEVERR_TIMEOUT);
 
   // ---- epilogue ----
+  if (ff) pdl_wait();  // the outputs and the split-K workspace may still be read by earlier kernels
   const int h0 = 16 * mt + g, h1 = h0 + 8;
   if (sp.n_split == 1) {
     uint16_t* __restrict__ og = a.out[z] + (int64_t)r * kH * kDV;
@@ -390,6 +477,7 @@ __global__ void __launch_bounds__(128) mla_merge_kernel(MlaArgs a, Split sp, con
   __shared__ float wgt[kMaxSplits];
   __shared__ float inv_l;
   pdl_wait();
+  pdl_trigger();  // the next MLA may start its forced columns; it waits for this grid before writing
   const int h = blockIdx.x, r = blockIdx.y, z = blockIdx.z, tid = threadIdx.x;
   const int64_t base = ((int64_t)z * a.n_rows + r) * sp.n_split;
   if (tid < 32) {
@@ -433,13 +521,16 @@ size_t mla_ws_bytes(int n_rows, int cli, int n_split) {
   return (size_t)n_rows * cli * n_split * per + 256;
 }
 
-int mla_choose_splits(int n_rows, int cli, int64_t max_list) {
+int mla_choose_splits(int n_rows, int cli, int64_t max_list, bool forced_first) {
   // One wave at one CTA per SM: split the rows' key lists until the CTAs cover
   // the SMs, keeping at least four tiles per split (the ring's depth) and at
-  // most kMaxSplits splits.
+  // most kMaxSplits splits. With forced-first lists the CTAs start while the
+  // top-k is still finishing, which holds one SM per row (its last CTA): leave
+  // those SMs out, so that no CTA starts only after the top-k.
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (forced_first) sms = max(sms - n_rows, sms / 2);
   const int64_t work = max64((int64_t)n_rows * cli, 1);
   const int64_t by_len = (max_list + kStages * kTK - 1) / (kStages * kTK);
   int64_t n = min64(by_len, sms / work);
@@ -449,7 +540,7 @@ int mla_choose_splits(int n_rows, int cli, int64_t max_list) {
 
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
   if (a.n_rows <= 0) return cudaSuccess;
-  int n_split = mla_choose_splits(a.n_rows, a.cli, a.max_list);
+  int n_split = mla_choose_splits(a.n_rows, a.cli, a.max_list, a.forced_first && a.idx);
   // Shrink split-K to what the workspace holds.
   while (n_split > 1 && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes) --n_split;
   Split sp;

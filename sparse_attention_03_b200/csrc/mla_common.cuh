@@ -11,6 +11,30 @@ struct RowGeom {
   int64_t kbase, nvis, n_list;
 };
 
+// Where the row's keys live and how many it sees, from the caller's inputs alone
+// (not the index list): clamped, and flagged by one thread. n_list = nvis.
+__device__ __forceinline__ RowGeom row_base(const MlaArgs& a, int r, bool report);
+
+// The list of a row whose index list came from the top-k (forced columns first):
+// the expected length L, its known prefix K (the forced columns, or the whole
+// list of a dense row) and the key of a known slot, all from the position.
+struct ListPlan {
+  int64_t L, K;
+  int64_t hi;  // first local-window column (non-dense rows)
+  bool dense;
+};
+__device__ __forceinline__ ListPlan list_plan(const MlaArgs& a, int64_t nvis) {
+  ListPlan p;
+  p.dense = nvis <= a.topk;
+  p.L = min64(nvis, (int64_t)a.topk);
+  p.K = p.dense ? p.L : min64(p.L, (int64_t)a.n_init + a.n_loc);
+  p.hi = nvis - a.n_loc;
+  return p;
+}
+__device__ __forceinline__ int64_t known_key(const ListPlan& p, const MlaArgs& a, int64_t i) {
+  return (p.dense || i < a.n_init) ? i : p.hi + (i - a.n_init);
+}
+
 // Row geometry, with every out-of-range input clamped (and flagged by one thread).
 __device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool report) {
   RowGeom g{0, 0, 0};
@@ -49,6 +73,12 @@ __device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool re
     g.n_list = c;
   }
   return g;
+}
+
+__device__ __forceinline__ RowGeom row_base(const MlaArgs& a, int r, bool report) {
+  MlaArgs b = a;
+  b.idx = nullptr;  // (row_geometry then reads no count)
+  return row_geometry(b, r, report);
 }
 
 }  // namespace lsa

@@ -61,6 +61,7 @@ __global__ void __launch_bounds__(kHistThreads)
     topk_hist_kernel(TopkArgs a, int row0, HistCtl* hc) {
   __shared__ uint32_t h[kBins];
   pdl_wait();
+  pdl_trigger();  // dependents may launch now; they wait for this grid before reading its outputs
   const int r = row0 + blockIdx.y;
   const RowGeom g = row_geom(a, r);
   if (g.dense) return;
@@ -106,6 +107,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
   __shared__ uint32_t s_above, s_warp[kHistThreads / 32], s_wu[kHistThreads / 32], s_we[kHistThreads / 32];
   __shared__ uint32_t s_base_u, s_base_e, s_slot;
   pdl_wait();
+  pdl_trigger();  // dependents may launch now; they wait for this grid before reading its outputs
   const int r = row0 + blockIdx.y;
   const RowGeom g = row_geom(a, r);
   int32_t* __restrict__ row_out = a.idx + (int64_t)r * a.topk;
@@ -258,6 +260,7 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
   __shared__ uint32_t s_above, s_warp[kRowThreads / 32], s_up, s_nc, s_slot;
   extern __shared__ int32_t s_map[];  // the row's column map (col_ld entries) when there is one
   pdl_wait();
+  pdl_trigger();  // dependents may launch now; they wait for this grid before reading its outputs
   const int r = row0 + blockIdx.x;
   const RowGeom g = row_geom(a, r);
   int32_t* __restrict__ out = a.idx + (int64_t)r * a.topk;

@@ -29,7 +29,7 @@ EXPORTS = (
     "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill", "lsa_forward", "lsa_last_error",
     "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16", "lsa_synth_normal_f32",
     "lsa_synth_rms_rows_bf16", "lsa_launch_count", "lsa_index_project", "lsa_block_summaries",
-    "lsa_hier_workspace_size", "lsa_hier_select",
+    "lsa_hier_workspace_size", "lsa_hier_select", "lsa_sparse_mla_decode_topk",
 )
 HIER_BLOCK, HIER_BLOCKS = 64, 128
 
@@ -76,6 +76,7 @@ def load():
                                      _P]
     lib.lsa_topk.argtypes = [ctypes.POINTER(Config), _I32, _P, _I64, _P, _I64, _P, _P, _P, _P, _SZ, _P]
     lib.lsa_sparse_mla_decode.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]
+    lib.lsa_sparse_mla_decode_topk.argtypes = lib.lsa_sparse_mla_decode.argtypes
     lib.lsa_sparse_mla_prefill.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
     lib.lsa_forward.argtypes = [ctypes.POINTER(Config), _I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P,
                                 ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
@@ -97,7 +98,8 @@ def load():
     lib.lsa_synth_normal_f32.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
     lib.lsa_synth_rms_rows_bf16.argtypes = [_P, _I64, _I32, _U64, _U64, _I64, _P]
     for name in ("lsa_index_scores", "lsa_topk", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
-                 "lsa_forward", "lsa_index_project", "lsa_block_summaries", "lsa_hier_select", "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16",
+                 "lsa_forward", "lsa_index_project", "lsa_block_summaries", "lsa_hier_select", "lsa_device_error",
+                 "lsa_sparse_mla_decode_topk", "lsa_abi_version", "lsa_synth_normal_bf16",
                  "lsa_synth_normal_f32", "lsa_synth_rms_rows_bf16"):
         getattr(lib, name).restype = _I32
     _lib = lib
@@ -225,12 +227,17 @@ def topk(cfg, pos, max_len, scores, idx, count, ws, stream=None, bind=False, top
         allow_dense=True, bind=bind)
 
 
-def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None, bind=False):
+def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None, bind=False,
+                      lists_from_topk=False):
+    """Sparse absorbed MLA over each row's selected keys. lists_from_topk: idx /
+    count were written by topk (or forward) for these rows and this config; the
+    kernel then attends over the forced columns before the top-k has finished."""
     for t, n in ((q_abs, "q_abs"), (latent, "latent"), (out, "out")):
         _dt(t, torch.bfloat16, n)
     _dt(k_off, torch.int64, "k_off"); _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
     _dt(lse, torch.float32, "lse")
-    return _invoke(load().lsa_sparse_mla_decode, (
+    fn = load().lsa_sparse_mla_decode_topk if lists_from_topk else load().lsa_sparse_mla_decode
+    return _invoke(fn, (
         ctypes.byref(cfg._c()), q_abs.shape[0], _ptr(q_abs), _ptr(latent), _ptr(k_off), _ptr(idx),
         _ptr(count), int(max_len), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
         _stream(stream)), bind=bind)

@@ -1005,3 +1005,61 @@ def test_full_size_hier_sampled(L, name, batch, lo, hi, sample, n_exact):
     assert exact >= n_exact
     del wl
     torch.cuda.empty_cache()
+
+
+# --------------------------------------------------------------------------
+# MLA over top-k lists with the forced columns attended first
+# --------------------------------------------------------------------------
+def _topk_lists(L, cfg, wl, d, max_len):
+    n = wl.n_rows
+    scores = torch.empty((n, max_len), device="cuda")
+    L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], max_len, scores)
+    idx = torch.full((n, cfg.index_topk), -3, dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    L.topk(cfg, d["pos"], max_len, scores, idx, cnt, L.workspace(cfg, L.OP_TOPK, n, n, max_len))
+    return idx, cnt
+
+
+def test_mla_decode_lists_from_topk(L):
+    # dense rows (<= 2048 keys) and selected rows, the lists from the library's top-k
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    lengths = [700, 2048, 2049, 3001, 5000, 9000, 12345, 1]
+    wl = S.Workload(11, 2, lengths)
+    d = _upload(wl)
+    n, max_len = wl.n_rows, max(lengths)
+    idx, cnt = _topk_lists(L, cfg, wl, d, max_len)
+    ws = L.workspace(cfg, L.OP_MLA_DECODE, n, n, max_len)
+    res = {}
+    for mode in (False, True):
+        out = torch.empty((n, 32, 512), dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((n, 32), device="cuda")
+        L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], idx, cnt, max_len, out, lse, ws,
+                            lists_from_topk=mode)
+        assert L.device_error() == 0
+        res[mode] = (bf16_host_f64(out), lse.cpu().numpy())
+    # the two entry points attend over the same sets in different orders
+    assert np.abs(res[True][0] - res[False][0]).max() <= 1e-2
+    assert np.abs(res[True][1] - res[False][1]).max() <= 1e-4
+    idx_h, cnt_h = idx.cpu().numpy(), cnt.cpu().numpy()
+    for r in range(n):
+        q, w, k, qa, lat = host_rows(wl, r)
+        p = int(wl.pos[r])
+        s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
+        exact = check_selection(idx_h[r], int(cnt_h[r]), s, p, ocfg, where=f"row {r}")
+        sel, _ = R.select_topk(s, p, ocfg)
+        o, l = R.mla(qa[0], lat[0][sel], ocfg)
+        assert_attention(res[True][0][r], res[True][1][r], o, l, check_lse=exact, where=f"row {r}")
+
+
+def test_mla_decode_topk_bad_count_is_flagged(L):
+    cfg = L.LsaConfig()
+    lengths = [5000, 3000]
+    wl = S.Workload(12, 2, lengths, cli=1)
+    d = _upload(wl)
+    idx, cnt = _topk_lists(L, cfg, wl, d, max(lengths))
+    cnt[1] = 100  # not what the top-k wrote for a row of 3000 keys
+    out = torch.empty((2, 32, 512), dtype=torch.bfloat16, device="cuda")
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], idx, cnt, max(lengths), out, None,
+                        L.workspace(cfg, L.OP_MLA_DECODE, 2, 2, max(lengths)), lists_from_topk=True)
+    assert L.device_error() == L.DEVERR_COUNT
