@@ -187,19 +187,25 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     if (c != (int)lp.L && geo.nvis > 0) flag_error(a.err, LSA_DEVERR_COUNT);
     const int64_t uend = max64(lp.K, min64((int64_t)c, lp.L));
     const int32_t* __restrict__ irow = a.idx + (int64_t)r * a.topk;
-    for (int u = 0; u < ft.ut; ++u) {
-      const int64_t sl = lp.K + (int64_t)(ft.ut0 + u) * kTK + lane;
-      int64_t key = -1;
-      if (sl < uend) {
-        key = __ldg(irow + sl);
-        if (key < 0 || key >= geo.nvis) {
-          flag_error(a.err, LSA_DEVERR_INDEX);
-          key = -1;
-        }
+    constexpr int kBatch = 8;  // tiles whose indices are requested together
+    for (int u0 = 0; u0 < ft.ut; u0 += kBatch) {
+      int key[kBatch];
+      bool listed[kBatch];
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        const int64_t sl = lp.K + (int64_t)(ft.ut0 + u0 + j) * kTK + lane;
+        listed[j] = u0 + j < ft.ut && sl < uend;
+        key[j] = listed[j] ? __ldg(irow + sl) : -1;
       }
-      sm.list[u * kTK + lane] = (int32_t)key;
+#pragma unroll
+      for (int j = 0; j < kBatch; ++j) {
+        if (listed[j] && (key[j] < 0 || key[j] >= geo.nvis)) {
+          flag_error(a.err, LSA_DEVERR_INDEX);
+          key[j] = -1;
+        }
+        if (u0 + j < ft.ut) issue(ft.kt + u0 + j, key[j]);
+      }
     }
-    for (int u = 0; u < ft.ut; ++u) issue(ft.kt + u, sm.list[u * kTK + lane]);
     if (lane == 0) {
       mbar_drain(&sm.qbar, 0);
       for (int i = 0; i < kStages && i < n_tiles; ++i) {
