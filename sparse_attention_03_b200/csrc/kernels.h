@@ -74,6 +74,8 @@ constexpr size_t kTopkRowBytes = 2048 * 4 + 32 + kTopkCap * 8;  // hist + ctl + 
 constexpr int kTopkHistStride = 2048 + 8;                   // words between rows' histograms
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
+// Clears n_words 32-bit words on the stream with a kernel (keeps the launch chain).
+cudaError_t launch_zero_words(void* p, size_t n_words, cudaStream_t st);
 bool topk_uses_workspace(int n_rows, int64_t max_len);
 // Fills hist (rows kTopkHistStride words apart, zeroed by the caller) from scores.
 cudaError_t launch_topk_hist_only(const TopkArgs& a, uint32_t* hist, cudaStream_t st);

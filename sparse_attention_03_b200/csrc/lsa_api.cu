@@ -113,7 +113,7 @@ lsa_status run_index_scores(const lsa_config* c, int n_rows, int n_seq, const in
   a.err = device_error_word();
   if (topk_hist) {
     const lsa_status s0 = cuda_status(
-        cudaMemsetAsync(topk_hist, 0, (size_t)n_rows * kTopkHistStride * sizeof(uint32_t), st), "lsa_index_scores");
+        launch_zero_words(topk_hist, (size_t)n_rows * kTopkHistStride, st), "lsa_index_scores");
     if (s0 != LSA_OK) return s0;
   }
   if (!index_prefill_supported(a))

@@ -400,7 +400,22 @@ __global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int r
   });
 }
 
+// Clears n words on the stream as a kernel (a memset between two kernels would
+// keep the second from launching while the first finishes).
+__global__ void zero_words_kernel(uint32_t* __restrict__ p, size_t n) {
+  pdl_wait();  // the previous kernel may still read these words
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) p[i] = 0;
+  pdl_trigger();
+}
+
 }  // namespace
+
+cudaError_t launch_zero_words(void* p, size_t n_words, cudaStream_t st) {
+  if (n_words == 0) return cudaSuccess;
+  const unsigned blocks = (unsigned)min64(148 * 4, (int64_t)((n_words + 255) / 256));
+  count_launches(1);
+  return launch_pdl(zero_words_kernel, dim3(blocks), dim3(256), 0, st, static_cast<uint32_t*>(p), n_words);
+}
 
 // Dynamic shared memory of the per-row kernel: the column map, if any (at most
 // 2048 entries; the attribute allowing it above the 48 KB default is set once).
@@ -453,7 +468,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   uint64_t* cand = reinterpret_cast<uint64_t*>(hc + blk);
   for (int row0 = 0; row0 < a.n_rows; row0 += blk) {
     const int nr = min(blk, a.n_rows - row0);
-    cudaError_t e = cudaMemsetAsync(hc, 0, (size_t)nr * sizeof(HistCtl), st);
+    cudaError_t e = launch_zero_words(hc, (size_t)nr * sizeof(HistCtl) / sizeof(uint32_t), st);
     if (e != cudaSuccess) return e;
     if (!a.hist_ext) {
       e = launch_pdl(topk_hist_kernel, dim3((unsigned)chunks, (unsigned)nr), dim3(kHistThreads), 0, st, a, row0, hc);
