@@ -159,13 +159,16 @@ LSA_API lsa_status lsa_index_scores(const lsa_config* cfg, int32_t n_rows, int32
  * max_len (host): every pos[r] < max_len. Returns LSA_DENSE when
  * max_len <= index_topk (every row dense; idx/count still written).
  * topk_hist: NULL, or the histogram lsa_index_scores wrote for these scores
- *   (saves one pass over the scores).
+ *   (saves one pass over the scores). Rows longer than 16384 columns (fewer
+ *   than 256 rows) also keep their counters in its 8 words after each row's
+ *   bins: they must be zero on entry, as lsa_index_scores leaves them, and are
+ *   zero again on return.
  * Workspace: lsa_workspace_size(LSA_OP_TOPK, ...). Only fewer than 256 rows
  * longer than 16384 columns use it (then processed in blocks that fit,
  * minimum one row of 40992 B); otherwise ws may be NULL.
  */
 LSA_API lsa_status lsa_topk(const lsa_config* cfg, int32_t n_rows, const int32_t* pos, int64_t max_len,
-                    const float* scores, int64_t ld, const uint32_t* topk_hist, int32_t* idx,
+                    const float* scores, int64_t ld, uint32_t* topk_hist, int32_t* idx,
                     int32_t* count, void* ws, size_t ws_bytes, void* stream);
 
 /*

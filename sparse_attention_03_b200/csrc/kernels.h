@@ -56,8 +56,10 @@ struct TopkArgs {
   void* ws;
   size_t ws_bytes;
   // Per-row histograms built by the indexer (kTopkHistStride words apart), or
-  // null: the top-k then builds them itself.
-  const uint32_t* hist_ext = nullptr;
+  // null: the top-k then builds them itself. The multi-CTA select keeps its
+  // per-row counters in the 8 words after each row's bins (zero on entry, as the
+  // indexer leaves them; the row's last CTA zeroes them again).
+  uint32_t* hist_ext = nullptr;
   // Optional map from column j to the emitted index: col_map[r * col_ld + j /
   // col_block] * col_block + j % col_block (compact rows of whole blocks). With a
   // map every row goes through the one-CTA-per-row kernel.

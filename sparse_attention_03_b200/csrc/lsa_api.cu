@@ -140,7 +140,7 @@ lsa_status run_index_scores(const lsa_config* c, int n_rows, int n_seq, const in
 
 lsa_status run_topk(const lsa_config* c, int n_rows, const int32_t* pos, int64_t max_len,
                     const float* scores, int64_t ld, int32_t* idx, int32_t* count, void* ws,
-                    size_t ws_bytes, cudaStream_t st, const uint32_t* hist_ext = nullptr) {
+                    size_t ws_bytes, cudaStream_t st, uint32_t* hist_ext = nullptr) {
   TopkArgs a;
   a.scores = scores;
   a.ld = ld;
@@ -304,7 +304,7 @@ lsa_status lsa_index_scores(const lsa_config* c, int32_t n_rows, int32_t n_seq,
 }
 
 lsa_status lsa_topk(const lsa_config* c, int32_t n_rows, const int32_t* pos, int64_t max_len,
-                    const float* scores, int64_t ld, const uint32_t* topk_hist, int32_t* idx,
+                    const float* scores, int64_t ld, uint32_t* topk_hist, int32_t* idx,
                     int32_t* count, void* ws, size_t ws_bytes, void* stream) {
   const char* fn = "lsa_topk";
   lsa_status s = check_cfg(c, fn);

@@ -137,6 +137,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
     sv[i] = j < e ? srow[j] : 0.f;
   }
   const uint32_t* hsrc = a.hist_ext ? a.hist_ext + (int64_t)r * kTopkHistStride : w.hist;
+  uint32_t* ctl = a.hist_ext ? a.hist_ext + (int64_t)r * kTopkHistStride + kBins : w.ctl;
   for (int i = tid; i < kBins; i += kHistThreads) h[i] = hsrc[i];
   __syncthreads();
   const uint32_t k_rem = (uint32_t)(a.topk - a.n_init - a.n_loc);
@@ -180,8 +181,8 @@ __global__ void __launch_bounds__(kHistThreads, 4)
       tu += a_u;
       te += a_e;
     }
-    s_base_u = tu ? atomicAdd(&w.ctl[0], tu) : 0u;
-    s_base_e = te ? atomicAdd(&w.ctl[1], te) : 0u;
+    s_base_u = tu ? atomicAdd(&ctl[0], tu) : 0u;
+    s_base_e = te ? atomicAdd(&ctl[1], te) : 0u;
   }
   __syncthreads();
   uint32_t ou = s_base_u + s_wu[warp] + iu - nu;
@@ -204,7 +205,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
   // ---- the last CTA of the row finishes it ----
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&w.ctl[4], 1u) == n_chunks - 1;
+  if (tid == 0) s_last = atomicAdd(&ctl[4], 1u) == n_chunks - 1;
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -214,7 +215,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
     a.count[r] = a.topk;
     s_slot = 0;
   }
-  const uint32_t n_cand = __ldcg(&w.ctl[1]);
+  const uint32_t n_cand = __ldcg(&ctl[1]);
   const bool in_smem = n_cand <= (uint32_t)kTopkCap;
   if (in_smem)
     for (uint32_t i = tid; i < n_cand; i += kHistThreads) scand[i] = __ldcg(&cand[i]);
@@ -244,6 +245,12 @@ __global__ void __launch_bounds__(kHistThreads, 4)
       if (slot < need0) dst[slot] = (int32_t)j;
     }
   });
+  // every CTA of the row has taken its ticket: the counters are free again
+  if (tid == 0) {
+    ctl[0] = 0;
+    ctl[1] = 0;
+    ctl[4] = 0;
+  }
 }
 
 // One CTA per row: histogram (unless the indexer already built it), threshold,
@@ -468,9 +475,10 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   uint64_t* cand = reinterpret_cast<uint64_t*>(hc + blk);
   for (int row0 = 0; row0 < a.n_rows; row0 += blk) {
     const int nr = min(blk, a.n_rows - row0);
-    cudaError_t e = launch_zero_words(hc, (size_t)nr * sizeof(HistCtl) / sizeof(uint32_t), st);
-    if (e != cudaSuccess) return e;
-    if (!a.hist_ext) {
+    cudaError_t e = cudaSuccess;
+    if (!a.hist_ext) {  // (with the indexer's histograms the counters live beside them)
+      e = launch_zero_words(hc, (size_t)nr * sizeof(HistCtl) / sizeof(uint32_t), st);
+      if (e != cudaSuccess) return e;
       e = launch_pdl(topk_hist_kernel, dim3((unsigned)chunks, (unsigned)nr), dim3(kHistThreads), 0, st, a, row0, hc);
       if (e != cudaSuccess) return e;
       count_launches(1);

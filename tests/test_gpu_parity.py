@@ -1063,3 +1063,30 @@ def test_mla_decode_topk_bad_count_is_flagged(L):
     L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], idx, cnt, max(lengths), out, None,
                         L.workspace(cfg, L.OP_MLA_DECODE, 2, 2, max(lengths)), lists_from_topk=True)
     assert L.device_error() == L.DEVERR_COUNT
+
+
+def test_topk_multi_cta_with_indexer_histogram_twice(L):
+    # few long rows (the multi-CTA select): its counters live beside the indexer's
+    # histogram and are cleared by the call itself, so a second call on the same
+    # histogram gives the same selection, as does the top-k's own first pass
+    cfg = L.LsaConfig()
+    lengths = [40000, 33000, 17000, 65536]
+    wl = S.Workload(15, 0, lengths, cli=1)
+    d = _upload(wl)
+    n, max_len = wl.n_rows, max(lengths)
+    scores = torch.empty((n, max_len), device="cuda")
+    hist = L.topk_hist_buffer(n)
+    L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], max_len, scores,
+                   topk_hist=hist)
+    ws = L.workspace(cfg, L.OP_TOPK, n, n, max_len)
+    outs = []
+    for h in (hist, hist, None):
+        idx = torch.full((n, 2048), -3, dtype=torch.int32, device="cuda")
+        cnt = torch.full((n,), -3, dtype=torch.int32, device="cuda")
+        L.topk(cfg, d["pos"], max_len, scores, idx, cnt, ws, topk_hist=h)
+        outs.append((np.sort(idx.cpu().numpy(), axis=1), cnt.cpu().numpy()))
+    for o in outs[1:]:
+        np.testing.assert_array_equal(outs[0][0], o[0])
+        np.testing.assert_array_equal(outs[0][1], o[1])
+    assert np.all(hist.cpu().numpy()[:, 2048:] == 0)
+    assert L.device_error() == 0
