@@ -260,7 +260,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
 constexpr int kRowThreads = 512;
 constexpr int kRowCap = 4608;  // 36 KB of candidates: static shared memory stays under 48 KB
 
-__global__ void __launch_bounds__(kRowThreads) topk_row_kernel(TopkArgs a, int row0, const uint32_t* hist_in) {
+__global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, int row0, const uint32_t* hist_in) {
   __shared__ uint32_t h[kBins];
   __shared__ uint64_t cand[kRowCap];
   __shared__ int s_bin;
