@@ -21,7 +21,10 @@ and the decode step with hierarchical indexing ("hier": per layer the newest
 block's summary, a coarse pass over 64-key block summaries keeping the sink /
 recent blocks and the 128 best others, the fine selection over their tokens,
 then both MLA sub-blocks; also the selection alone against the flat index pass
-and top-k).
+and top-k), and the other workloads of the pages' configuration list as one
+lsa_forward layer each ("configs": single-token decode latency at 8192 cached
+keys with L2 flushed before every step, 64 sequences of 16K-32K cached keys,
+4 sequences at 983040, and a 4096-token prefill chunk against 983040).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lsa|reference]
 Multi-GPU (torchrun): every rank runs its own batch (weak scaling, no
@@ -514,6 +517,91 @@ def run_prefill(device, steps, warmup):
                          "peak_source": f"{src} bf16_tflops_sustained", "traffic": None}}
 
 
+def _forward_case(device, lengths, n_rows=None, q_start=None):
+    """One layer's lsa_forward call (cli 2) on device-drawn inputs, bound once."""
+    import torch
+    from sparse_attention_03_b200 import lsa
+    from sparse_attention_03_b200.device_inputs import DeviceWorkload
+    cfg = lsa.LsaConfig()
+    wl = DeviceWorkload(0, 300, lengths, n_rows=n_rows, q_start=q_start, device=device)
+    n, max_len = wl.n_rows, wl.max_len
+    mode = 0 if n_rows is None else 1
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device=device) for _ in range(2)]
+    lses = [torch.empty((n, 32), device=device) for _ in range(2)]
+    n_seq = len(lengths) if mode == 0 else 1
+    ws = lsa.workspace(cfg, lsa.OP_FORWARD_DECODE if mode == 0 else lsa.OP_FORWARD_PREFILL, n, n_seq, max_len,
+                       device=device)
+    call = lsa.forward(cfg, mode, wl.seq_of_row, wl.pos, max_len, wl.q_idx, wl.w, wl.k_idx, wl.k_off, wl.q_abs,
+                       wl.latent, outs, lses, ws, bind=True)
+    return call, (wl, outs, lses, ws)
+
+
+def run_configs(device, steps):
+    """The other workloads of the pages' configuration list, one lsa_forward layer
+    (one index pass, top-k, two sub-blocks) per step: single-token latency at
+    8192 cached keys (caches fit in L2, so L2 is flushed before every step and
+    each step is event-timed alone), the 64-sequence varlen decode, and the
+    long-context pair (4 sequences at 983040 cached keys; a 4096-token prefill
+    chunk against the 983040-token cache)."""
+    import torch
+    from sparse_attention_03_b200 import lsa
+    res = {}
+
+    # decode, batch 1, 8192 cached keys: latency with a cold L2
+    call, keep = _forward_case(device, [8192])
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    lat = []
+    for i in range(steps + 3):
+        flush.fill_(i & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        call()
+        b.record()
+        torch.cuda.synchronize()
+        if i >= 3:
+            lat.append(a.elapsed_time(b))
+    res["decode_b1_ctx8192"] = {"value": 1e3 / statistics.median(lat), "unit": "tokens/s/layer",
+                                "us_per_layer": 1e3 * statistics.median(lat),
+                                "l2": "flushed (256 MB write) before every step; median of per-step events"}
+    del call, keep, flush
+
+    def timed(call, units, n_steps):
+        for _ in range(3):
+            call()
+        t = time_region(lambda s: call(), n_steps, 1, device)
+        return units * n_steps / t, 1e3 * t / n_steps
+
+    # decode, batch 64, cached lengths uniform in [16384, 32768]
+    lengths = S.decode_lengths(0, 64, 16384, 32768)
+    call, keep = _forward_case(device, lengths)
+    v, ms = timed(call, 64, steps)
+    res["decode_b64_ctx16k_32k"] = {"value": v, "unit": "tokens/s/layer", "ms_per_layer": ms,
+                                    "cached_keys": int(lengths.sum()),
+                                    "l2": f"{int(lengths.sum()) * 2560 / 1e9:.1f} GB of caches per step, no flush"}
+    del call, keep
+    torch.cuda.empty_cache()
+
+    # decode, batch 4, 983040 cached keys
+    call, keep = _forward_case(device, [983040] * 4)
+    v, ms = timed(call, 4, steps)
+    res["decode_b4_ctx983040"] = {"value": v, "unit": "tokens/s/layer", "ms_per_layer": ms,
+                                  "l2": "10.1 GB of caches per step, no flush"}
+    del call, keep
+    torch.cuda.empty_cache()
+
+    # prefill chunk of 4096 tokens at positions 983040 .. 987135
+    n, q0 = 4096, 983040
+    call, keep = _forward_case(device, [q0 + n], n_rows=n, q_start=q0)
+    v, ms = timed(call, n, max(3, steps // 4))
+    flops = 2.0 * 32 * 128 * (n * q0 + n * (n + 1) / 2)  # visible (row, key) pairs of the indexer
+    res["prefill_chunk4096_ctx983040"] = {"value": v, "unit": "tok/s", "ms_per_chunk": ms,
+                                          "indexer_tflop": flops / 1e12,
+                                          "l2": "16 GB score matrix and 2.5 GB of caches per step, no flush"}
+    del call, keep
+    torch.cuda.empty_cache()
+    return res
+
+
 def gpu_arm(args):
     import torch
     from sparse_attention_03_b200 import lsa
@@ -614,6 +702,9 @@ def gpu_arm(args):
     prefill = None
     if not args.no_prefill:
         prefill = run_prefill(device, max(3, args.steps // 20), 3)
+    configs = None
+    if not args.no_configs:
+        configs = run_configs(device, max(5, args.steps // 10))
 
     clocks = clk.summary()
     if rank != 0:
@@ -649,6 +740,8 @@ def gpu_arm(args):
                                            f"_keep{hc['n_blocks']}", **hc}}
     if prefill:
         line["prefill"] = prefill
+    if configs:
+        line["configs"] = configs
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline()
     print(json.dumps(line), flush=True)
@@ -662,6 +755,7 @@ def main():
     ap.add_argument("--impl", choices=["lsa", "reference"], default="lsa")
     ap.add_argument("--no-prefill", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true", help="skip the other workloads' lines")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

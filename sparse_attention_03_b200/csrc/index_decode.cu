@@ -140,7 +140,7 @@ cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st, uint32_t* h
   // these short-lived CTAs costs more than the larger per-CTA key range saves).
   // Keys per CTA are a multiple of one CTA pass (64 keys), at least 256 so the
   // query-fragment load is amortised (64 for rows of at most 16384 keys), and at
-  // most 8192.
+  // most 65536 (a few long rows then still fill exactly one wave).
   // Cached per device (a benign race: every thread writes the same values).
   static int cache_sms[64], cache_occ[64];
   int dev = 0;
@@ -161,7 +161,7 @@ cudaError_t launch_index_decode(const IndexArgs& a, cudaStream_t st, uint32_t* h
   kpc = ((kpc + 63) / 64) * 64;
   // short rows (block summaries) spread over more CTAs; long ones amortise the
   // query-fragment load over at least 256 keys
-  kpc = max64(a.max_len <= 16384 ? 64 : 256, min64(kpc, 8192));
+  kpc = max64(a.max_len <= 16384 ? 64 : 256, min64(kpc, 65536));
   const int64_t nx = (a.max_len + kpc - 1) / kpc;
   for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
     const int ny = min(65535, a.n_rows - row0);

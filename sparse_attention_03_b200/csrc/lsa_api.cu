@@ -70,8 +70,16 @@ lsa_status cuda_status(cudaError_t e, const char* fn) {
   return set_error(LSA_ERR_CUDA, "%s: %s", fn, cudaGetErrorString(e));
 }
 
-size_t topk_ws(int n_rows) {
-  return (size_t)std::min(n_rows, kTopkPreferredRows) * kTopkRowBytes + kAlign;
+// The top-k's workspace. Rows taken by several CTAs each also get room for the
+// threshold bin's candidates beyond the kTopkCap of the base layout: a sixteenth
+// of the row (at most 2^18), so that the bin rarely outgrows it.
+size_t topk_ws(int n_rows, int64_t max_len = 0) {
+  size_t per = kTopkRowBytes;
+  if (max_len > 0 && topk_uses_workspace(n_rows, max_len)) {
+    const int64_t room = std::min<int64_t>(max_len / 16, int64_t(1) << 18);
+    if (room > kTopkCap) per += (size_t)(room - kTopkCap) * sizeof(uint64_t);
+  }
+  return (size_t)std::min(n_rows, kTopkPreferredRows) * per + kAlign;
 }
 
 size_t mla_ws(int n_rows, int cli, int64_t max_list) {
@@ -82,7 +90,7 @@ size_t mla_ws(int n_rows, int cli, int64_t max_list) {
 size_t forward_block_ws(const lsa_config* c, int R, int64_t max_len) {
   return align_up((size_t)R * max_len * sizeof(float)) + align_up((size_t)R * kTopkHistStride * sizeof(uint32_t)) +
          align_up((size_t)R * c->index_topk * sizeof(int32_t)) +
-         align_up((size_t)R * sizeof(int32_t)) + topk_ws(R) + mla_ws(R, c->cli_factor, c->index_topk);
+         align_up((size_t)R * sizeof(int32_t)) + topk_ws(R, max_len) + mla_ws(R, c->cli_factor, c->index_topk);
 }
 
 int prefill_block_rows(int n_rows, int64_t max_len) {
@@ -252,7 +260,7 @@ size_t lsa_workspace_size(const lsa_config* c, int32_t op, int32_t n_rows, int32
   const int64_t list = std::min<int64_t>(max_len, c->index_topk);
   switch (op) {
     case LSA_OP_TOPK:
-      return max_len <= c->index_topk ? kAlign : topk_ws(n_rows);
+      return max_len <= c->index_topk ? kAlign : topk_ws(n_rows, max_len);
     case LSA_OP_MLA_DECODE:
     case LSA_OP_MLA_PREFILL:
       return std::max(mla_ws(n_rows, 1, max_len), mla_ws(n_rows, 1, list)) + kAlign;
@@ -528,7 +536,7 @@ lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_
   int32_t* cnt_ws = reinterpret_cast<int32_t*>(p);
   p += align_up((size_t)R * sizeof(int32_t));
   void* topk_w = p;  // 256-byte aligned (every region above is a multiple of 256)
-  const size_t topk_bytes = topk_ws(R);
+  const size_t topk_bytes = topk_ws(R, max_len);
   p += topk_bytes;
   // Decode: the indexer builds the top-k's histogram while the scores are in
   // registers, which saves the top-k one pass over the scores and one launch.

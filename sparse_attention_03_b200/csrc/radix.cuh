@@ -59,15 +59,17 @@ __device__ void find_threshold(const uint32_t* h, uint32_t need, int& bin_out,
 // unique, so a radix select from the top, 11 bits a level, ends with exactly
 // `need` values v with (v >> (53 - decided)) >= prefix. It stops as soon as one
 // bin holds exactly what is still needed. for_each(f) must call f(v53, column)
-// for every candidate (each thread a share of them). Block-wide.
+// for every candidate (each thread a share of them); every candidate must carry
+// the top `decided0` bits `prefix0` (0 and 0 when nothing is decided yet).
+// Block-wide.
 template <int THREADS, class ForEach>
 __device__ void radix_levels(ForEach&& for_each, uint32_t need, uint32_t* h, int* s_bin, uint32_t* s_above,
-                             uint32_t* s_warp, uint64_t& prefix, int& decided) {
-  prefix = 0;
-  decided = 0;
-  const int widths[5] = {11, 11, 11, 11, 9};
-  for (int lvl = 0; lvl < 5; ++lvl) {
-    const int wdt = widths[lvl];
+                             uint32_t* s_warp, uint64_t& prefix, int& decided, uint64_t prefix0 = 0,
+                             int decided0 = 0) {
+  prefix = prefix0;
+  decided = decided0;
+  while (decided < 53) {
+    const int wdt = min(11, 53 - decided);
     const int shift = 53 - decided - wdt;
     for (int i = threadIdx.x; i < kBins; i += THREADS) h[i] = 0;
     __syncthreads();

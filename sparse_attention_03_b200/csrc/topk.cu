@@ -100,7 +100,7 @@ constexpr int kPerThread = kChunk / kHistThreads;  // 16 scores per thread
 static_assert(kPerThread == 2 * kUnroll, "two rounds of kUnroll loads per thread");
 
 __global__ void __launch_bounds__(kHistThreads, 4)
-    topk_select_kernel(TopkArgs a, int row0, HistCtl* hc, uint64_t* cand_all) {
+    topk_select_kernel(TopkArgs a, int row0, HistCtl* hc, uint64_t* cand_all, uint32_t cand_cap) {
   __shared__ uint32_t h[kBins];
   __shared__ uint64_t scand[kTopkCap];
   __shared__ int s_bin, s_last;
@@ -124,7 +124,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
   if (s >= e) return;
   const uint32_t n_chunks = (uint32_t)((g.hi - g.lo + kChunk - 1) / kChunk);
   HistCtl& w = hc[blockIdx.y];
-  uint64_t* __restrict__ cand = cand_all + (int64_t)blockIdx.y * kTopkCap;
+  uint64_t* __restrict__ cand = cand_all + (int64_t)blockIdx.y * cand_cap;
   // This chunk's scores are requested first; the histogram and the threshold
   // search overlap their latency.
   const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
@@ -196,7 +196,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
       if (ou < k_rem) mid[ou] = (int32_t)j;
       ++ou;
     } else if (kb == bin) {
-      if (oe < (uint32_t)kTopkCap)
+      if (oe < cand_cap)
         cand[oe] = ((uint64_t)score_key(sv[i]) << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
       ++oe;
     }
@@ -216,33 +216,98 @@ __global__ void __launch_bounds__(kHistThreads, 4)
     s_slot = 0;
   }
   const uint32_t n_cand = __ldcg(&ctl[1]);
-  const bool in_smem = n_cand <= (uint32_t)kTopkCap;
-  if (in_smem)
+  const uint32_t need0 = k_rem - above;
+  // Where the rest of the select runs: the threshold-bin candidates in shared
+  // memory (the common case); if they overflow it but fit the workspace, one
+  // more 11-bit digit of the key splits them first: the digits above the
+  // threshold digit go straight out and only the threshold digit's candidates
+  // are kept in shared memory; otherwise (very many equal keys) the row is
+  // rescanned for every level.
+  bool in_smem = n_cand <= (uint32_t)kTopkCap;
+  uint32_t n_sm = in_smem ? n_cand : 0, need = need0;
+  uint64_t pre0 = 0;
+  int dec0 = 0;
+  int32_t* __restrict__ dst = mid + above;
+  if (in_smem) {
     for (uint32_t i = tid; i < n_cand; i += kHistThreads) scand[i] = __ldcg(&cand[i]);
+  } else if (n_cand <= cand_cap) {
+    constexpr int kU = 4;
+    for (int i = tid; i < kBins; i += kHistThreads) h[i] = 0;
+    if (tid == 0) {
+      s_base_u = 0;
+      s_base_e = 0;
+    }
+    __syncthreads();
+    for (uint32_t b = warp * 32 * kU; b < n_cand; b += kHistThreads * kU) {
+      uint64_t c[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) c[u] = b + lane + 32 * u < n_cand ? __ldcg(&cand[b + lane + 32 * u]) : 0;
+#pragma unroll
+      for (int u = 0; u < kU; ++u)
+        if (b + lane + 32 * u < n_cand) atomicAdd(&h[(uint32_t)(c[u] >> 42) & (kBins - 1)], 1u);
+    }
+    __syncthreads();
+    int d1;
+    uint32_t above1;
+    find_threshold<kHistThreads>(h, need0, d1, above1, &s_bin, &s_above, s_warp);
+    const uint32_t below = (1u << lane) - 1u;
+    for (uint32_t b = warp * 32 * kU; b < n_cand; b += kHistThreads * kU) {
+      uint64_t c[kU];
+#pragma unroll
+      for (int u = 0; u < kU; ++u) c[u] = b + lane + 32 * u < n_cand ? __ldcg(&cand[b + lane + 32 * u]) : 0;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const bool ok = b + lane + 32 * u < n_cand;
+        const int dg = (int)((uint32_t)(c[u] >> 42) & (kBins - 1));
+        const uint32_t mu = __ballot_sync(0xffffffffu, ok && dg > d1);
+        const uint32_t me = __ballot_sync(0xffffffffu, ok && dg == d1);
+        uint32_t bu = 0, be = 0;
+        if (lane == 0) {
+          if (mu) bu = atomicAdd(&s_base_u, __popc(mu));
+          if (me) be = atomicAdd(&s_base_e, __popc(me));
+        }
+        bu = __shfl_sync(0xffffffffu, bu, 0) + __popc(mu & below);
+        be = __shfl_sync(0xffffffffu, be, 0) + __popc(me & below);
+        if (ok && dg > d1) {
+          if (bu < above1) dst[bu] = (int32_t)(0xFFFFFFFFu - (uint32_t)c[u]);
+        } else if (ok && dg == d1) {
+          if (be < (uint32_t)kTopkCap) scand[be] = c[u];
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t n2 = s_base_e;
+    if (n2 <= (uint32_t)kTopkCap) {
+      in_smem = true;
+      n_sm = n2;
+      pre0 = (uint64_t)d1;
+      dec0 = 11;
+      need = need0 - above1;
+      dst += above1;
+    }
+  }
   __syncthreads();
   auto for_each = [&](auto&& f) {
     if (in_smem) {
-      for (uint32_t i = tid; i < n_cand; i += kHistThreads) {
+      for (uint32_t i = tid; i < n_sm; i += kHistThreads) {
         const uint64_t c = scand[i];
         f(c & kLow53, (int64_t)(0xFFFFFFFFu - (uint32_t)c));
       }
-    } else {  // more equal-bin scores than the buffer holds: rescan the row
+    } else {  // more equal-key scores than the buffers hold: rescan the row
       for (int64_t j = g.lo + tid; j < g.hi; j += kHistThreads) {
         const uint32_t k2 = score_key(srow[j]);
         if ((int)(k2 >> 21) == bin) f((((uint64_t)k2 << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j)) & kLow53, j);
       }
     }
   };
-  const uint32_t need0 = k_rem - above;
   uint64_t prefix;
   int decided;
-  radix_levels<kHistThreads>(for_each, need0, h, &s_bin, &s_above, s_warp, prefix, decided);
-  int32_t* __restrict__ dst = mid + above;
+  radix_levels<kHistThreads>(for_each, need, h, &s_bin, &s_above, s_warp, prefix, decided, pre0, dec0);
   const int shb = 53 - decided;
   for_each([&](uint64_t v, int64_t j) {
     if ((v >> shb) >= prefix) {
       const uint32_t slot = atomicAdd(&s_slot, 1u);
-      if (slot < need0) dst[slot] = (int32_t)j;
+      if (slot < need) dst[slot] = (int32_t)j;
     }
   });
   // every CTA of the row has taken its ticket: the counters are free again
@@ -373,10 +438,81 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
     }
   }
   __syncthreads();
-  const uint32_t n_cand = s_nc;
-  const bool in_smem = n_cand <= (uint32_t)kRowCap;
-  uint32_t need = k_rem - above0;
-  const uint32_t need0 = need;
+  const uint32_t need0 = k_rem - above0;
+  uint32_t n_cand = s_nc, need = need0;
+  bool in_smem = n_cand <= (uint32_t)kRowCap;
+  uint64_t pre0 = 0;
+  int dec0 = 0;
+  int32_t* __restrict__ dst = mid + above0;
+  if (!in_smem) {
+    // The threshold bin outgrew shared memory: one more 11-bit digit of the
+    // key (key bits 20..10) splits it. A histogram pass and a collect pass over
+    // the row send the digits above the threshold digit straight out and keep
+    // the threshold digit's candidates in shared memory.
+    for (int i = tid; i < kBins; i += kRowThreads) h[i] = 0;
+    __syncthreads();
+    for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
+      float v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t j = base + lane + 32 * u;
+        v[u] = j < g.hi ? srow[j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const uint32_t key = score_key(v[u]);
+        if (base + lane + 32 * u < g.hi && (int)(key >> 21) == bin0) atomicAdd(&h[(key >> 10) & (kBins - 1)], 1u);
+      }
+    }
+    __syncthreads();
+    int d1;
+    uint32_t above1;
+    find_threshold<kRowThreads>(h, need0, d1, above1, &s_bin, &s_above, s_warp);
+    if (tid == 0) {
+      s_up = 0;
+      s_nc = 0;
+    }
+    __syncthreads();
+    const uint32_t below = (1u << lane) - 1u;
+    for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
+      float v[kUnroll];
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t j = base + lane + 32 * u;
+        v[u] = j < g.hi ? srow[j] : 0.f;
+      }
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int64_t j = base + lane + 32 * u;
+        const uint32_t key = score_key(v[u]);
+        const bool inb = j < g.hi && (int)(key >> 21) == bin0;
+        const int dg = (int)((key >> 10) & (kBins - 1));
+        const uint32_t mu = __ballot_sync(0xffffffffu, inb && dg > d1);
+        const uint32_t me = __ballot_sync(0xffffffffu, inb && dg == d1);
+        uint32_t bu = 0, be = 0;
+        if (lane == 0) {
+          if (mu) bu = atomicAdd(&s_up, __popc(mu));
+          if (me) be = atomicAdd(&s_nc, __popc(me));
+        }
+        bu = __shfl_sync(0xffffffffu, bu, 0) + __popc(mu & below);
+        be = __shfl_sync(0xffffffffu, be, 0) + __popc(me & below);
+        if (inb && dg > d1) {
+          if (bu < above1) dst[bu] = col(j);
+        } else if (inb && dg == d1) {
+          if (be < (uint32_t)kRowCap) cand[be] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+        }
+      }
+    }
+    __syncthreads();
+    if (s_nc <= (uint32_t)kRowCap) {
+      in_smem = true;
+      n_cand = s_nc;
+      pre0 = (uint64_t)d1;
+      dec0 = 11;
+      need = need0 - above1;
+      dst += above1;
+    }
+  }
 
   auto for_each = [&](auto&& f) {
     if (in_smem) {
@@ -384,7 +520,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
         const uint64_t c = cand[i];
         f(c & kLow53, (int64_t)(0xFFFFFFFFu - (uint32_t)c));
       }
-    } else {
+    } else {  // very many equal keys: rescan the row for every level
       for (int64_t j = g.lo + tid; j < g.hi; j += kRowThreads) {
         const uint32_t key = score_key(srow[j]);
         if ((int)(key >> 21) == bin0) {
@@ -396,13 +532,12 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   };
   uint64_t prefix;
   int decided;
-  radix_levels<kRowThreads>(for_each, need, h, &s_bin, &s_above, s_warp, prefix, decided);
-  int32_t* __restrict__ dst = mid + above0;
+  radix_levels<kRowThreads>(for_each, need, h, &s_bin, &s_above, s_warp, prefix, decided, pre0, dec0);
   const int sh = 53 - decided;
   for_each([&](uint64_t v, int64_t j) {
     if ((v >> sh) >= prefix) {
       const uint32_t slot = atomicAdd(&s_slot, 1u);
-      if (slot < need0) dst[slot] = col(j);
+      if (slot < need) dst[slot] = col(j);
     }
   });
 }
@@ -473,6 +608,10 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   const int64_t rows_fit = (int64_t)(a.ws_bytes / kTopkRowBytes);
   const int blk = (int)min64(min64(rows_fit, a.n_rows), 65535);
   uint64_t* cand = reinterpret_cast<uint64_t*>(hc + blk);
+  // candidates per row: all the workspace holds beyond the control blocks (at least kTopkCap)
+  const uint32_t cand_cap =
+      (uint32_t)min64((int64_t)((a.ws_bytes - (size_t)blk * sizeof(HistCtl)) / ((size_t)blk * sizeof(uint64_t))),
+                      int64_t(1) << 24);
   for (int row0 = 0; row0 < a.n_rows; row0 += blk) {
     const int nr = min(blk, a.n_rows - row0);
     cudaError_t e = cudaSuccess;
@@ -484,7 +623,7 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
       count_launches(1);
     }
     e = launch_pdl(topk_select_kernel, dim3((unsigned)chunks, (unsigned)nr), dim3(kHistThreads), 0, st, a, row0, hc,
-                   cand);
+                   cand, cand_cap);
     if (e != cudaSuccess) return e;
     count_launches(1);
     e = cudaGetLastError();

@@ -11,6 +11,8 @@ current stream, checks the device error flags and exits. Cases:
   topk_decode    lsa_topk on 16 rows x 131072 scores, with the indexer's histogram
   mla_decode     lsa_sparse_mla_decode, 16 rows x 2048 selected keys of 131072
   mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
+  decode_1m      lsa_forward (cli 2), 4 rows x 983040 keys (one long-context decode layer)
+  chunk_1m       lsa_forward (cli 2), a 4096-row prefill chunk at positions 983040.. (16 GB of scores)
   hier_decode    lsa_block_summaries of each row's newest block + lsa_hier_select (64-key blocks,
                  128 kept), 16 rows x 131072 keys
 """
@@ -93,6 +95,30 @@ def case_mla_prefill(reps):
     ws = lsa.workspace(cfg, lsa.OP_MLA_PREFILL, n_rows, 1, n_keys)
     for _ in range(reps):
         lsa.sparse_mla_prefill(cfg, wl.pos, wl.q_abs[0], wl.latent[0], idx, cnt, out, lse, ws)
+
+
+def case_decode_1m(reps):
+    cfg = lsa.LsaConfig()
+    lengths = np.full(4, 983040, dtype=np.int64)
+    wl = DeviceWorkload(0, 0, lengths)
+    outs = [torch.empty((4, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((4, 32), device="cuda") for _ in range(2)]
+    ws = lsa.workspace(cfg, lsa.OP_FORWARD_DECODE, 4, 4, 983040)
+    for _ in range(reps):
+        lsa.forward(cfg, 0, wl.seq_of_row, wl.pos, 983040, wl.q_idx, wl.w, wl.k_idx, wl.k_off, wl.q_abs, wl.latent,
+                    outs, lses, ws)
+
+
+def case_chunk_1m(reps):
+    cfg = lsa.LsaConfig()
+    n, q0 = 4096, 983040
+    wl = DeviceWorkload(0, 0, [q0 + n], n_rows=n, q_start=q0)
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((n, 32), device="cuda") for _ in range(2)]
+    ws = lsa.workspace(cfg, lsa.OP_FORWARD_PREFILL, n, 1, q0 + n)
+    for _ in range(reps):
+        lsa.forward(cfg, 1, None, wl.pos, q0 + n, wl.q_idx, wl.w, wl.k_idx, None, wl.q_abs, wl.latent, outs, lses,
+                    ws)
 
 
 def case_hier_decode(reps):

@@ -245,6 +245,45 @@ def test_topk_multi_cta_long_rows(L):
         np.testing.assert_array_equal(np.sort(idx[r, :n]), exp, err_msg=f"row {r}")
 
 
+def _dense_bin_rows(rng, pos, n_in_bin, exact=False):
+    # N(0,1) scores with n_in_bin middle columns in [96, 112), one bin of the
+    # first radix digit (sign, exponent and two mantissa bits), so the top of the
+    # selection lands in an overfull threshold bin; exact=True puts them all at 100.
+    rows = []
+    for p, m in zip(pos, n_in_bin):
+        v = rng.standard_normal(p + 1).astype(np.float32)
+        cols = rng.choice(np.arange(16, p + 1 - 1024), m, replace=False)
+        v[cols] = 100.0 if exact else rng.uniform(96.0, 112.0, m).astype(np.float32)
+        rows.append(v)
+    return rows
+
+
+@pytest.mark.parametrize("kernel", ["per_row", "multi_cta"])
+def test_topk_overfull_threshold_bin(L, kernel):
+    # The threshold bin holds more candidates than shared memory: one more key
+    # digit splits it (per-row kernel: over the row; multi-CTA kernel: over the
+    # candidates held in the workspace), and when the split digit still
+    # overflows (equal keys) the rescan path takes over. Exact sets.
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(31)
+    if kernel == "per_row":   # rows of at most 16384 columns
+        pos = np.array([15999, 12000, 16383, 9000], dtype=np.int64)
+        rows = _dense_bin_rows(rng, pos[:2], [6000, 10900]) + \
+            _dense_bin_rows(rng, pos[2:3], [7000], exact=True) + [np.full(pos[3] + 1, 1.5, dtype=np.float32)]
+    else:                     # few long rows: candidate room of max_len / 16 per row
+        pos = np.array([199999, 150000, 180000], dtype=np.int64)
+        rows = _dense_bin_rows(rng, pos[:2], [7000, 12000]) + _dense_bin_rows(rng, pos[2:], [8000], exact=True)
+    max_len = int(pos.max()) + 1
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, max_len)
+    assert st == L.LSA_OK
+    for r, p in enumerate(pos):
+        exp, dense = R.select_topk(R.mask_and_force(rows[r].astype(np.float64), int(p), max_len, ocfg), int(p), ocfg)
+        assert cnt[r] == cfg.index_topk and not dense
+        np.testing.assert_array_equal(np.sort(idx[r]), exp, err_msg=f"{kernel} row {r}")
+    assert L.device_error() == 0
+
+
 @pytest.mark.parametrize("streaming", [True, False])
 def test_topk_with_indexer_histogram(L, streaming):
     # the histogram lsa_index_scores emits gives lsa_topk the same selection as
@@ -680,6 +719,46 @@ def test_full_size_prefill_16k_sampled(L):
             eo, el = R.mla(qa, c, ocfg)
             assert_attention(bf16_host_f64(outs[z][r]), lses[z][r].cpu().numpy(), eo, el, check_lse=exact,
                              where=f"prefill row {r} sub {z}")
+
+
+def test_full_size_prefill_chunk_1m_sampled(L):
+    # The long-context workload's prefill chunk: 4096 new rows at positions
+    # 983040 .. 987135 against the whole 987136-key cache (every row sparse).
+    # The 16 GB score matrix, the tensor-core indexer over 33 TFLOP of causal
+    # pairs, the one-CTA-per-row top-k over 987136 columns and the prefill MLA
+    # gathering from a 1.1 GB latent cache, sampled rows against the oracle.
+    from sparse_attention_03_b200.device_inputs import DeviceWorkload
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    n, q0 = 4096, 983040
+    n_keys = q0 + n
+    wl = DeviceWorkload(0, 0, [n_keys], n_rows=n, q_start=q0)
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((n, 32), device="cuda") for _ in range(2)]
+    idx = torch.empty((n, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    ws = L.workspace(cfg, L.OP_FORWARD_PREFILL, n, 1, n_keys)
+    L.forward(cfg, 1, None, wl.pos, n_keys, wl.q_idx, wl.w, wl.k_idx, None, wl.q_abs, wl.latent, outs, lses, ws,
+              idx_out=idx, count_out=cnt)
+    assert L.device_error() == 0
+    idx, cnt = idx.cpu().numpy(), cnt.cpu().numpy()
+    del ws, wl
+    torch.cuda.empty_cache()
+    f = S.bf16_bits_to_f64
+    k = f(S.rms_rows_bf16(0, S.tid(0, S.K_IDX), 0, n_keys, 128))
+    for t in (0, 2049, n - 1):
+        p = q0 + t
+        q = f(S.normal_bf16(0, S.tid(0, S.Q_IDX), t * 4096, 4096)).reshape(32, 128)
+        w = S.normal_f32(0, S.tid(0, S.W), t * 32, 32, S.W_SIGMA).astype(np.float64)
+        s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, n_keys, ocfg)
+        exact = check_selection(idx[t], int(cnt[t]), s, p, ocfg, where=f"chunk row {t}")
+        sel, _ = R.select_topk(s, p, ocfg)
+        for z in range(2):
+            qa = f(S.normal_bf16(0, S.tid(0, S.q_abs_kind(z)), t * 32 * 576, 32 * 576)).reshape(32, 576)
+            c = f(S.normal_bf16_rows(0, S.tid(0, S.lat_kind(z)), sel, 576))
+            eo, el = R.mla(qa, c, ocfg)
+            assert_attention(bf16_host_f64(outs[z][t]), lses[z][t].cpu().numpy(), eo, el, check_lse=exact,
+                             where=f"chunk row {t} sub {z}")
 
 
 # --------------------------------------------------------------------------
