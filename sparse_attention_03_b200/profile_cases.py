@@ -13,6 +13,8 @@ current stream, checks the device error flags and exits. Cases:
   mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
   decode_1m      lsa_forward (cli 2), 4 rows x 983040 keys (one long-context decode layer)
   chunk_1m       lsa_forward (cli 2), a 4096-row prefill chunk at positions 983040.. (16 GB of scores)
+  prefill_16k    one prefill step of 16384 causal rows: lsa_index_scores, lsa_topk, then
+                 lsa_sparse_mla_prefill for two sub-blocks
   hier_decode    lsa_block_summaries of each row's newest block + lsa_hier_select (64-key blocks,
                  128 kept), 16 rows x 131072 keys
 """
@@ -119,6 +121,24 @@ def case_chunk_1m(reps):
     for _ in range(reps):
         lsa.forward(cfg, 1, None, wl.pos, q0 + n, wl.q_idx, wl.w, wl.k_idx, None, wl.q_abs, wl.latent, outs, lses,
                     ws)
+
+
+def case_prefill_16k(reps):
+    cfg = lsa.LsaConfig()
+    n = 16384
+    wl = DeviceWorkload(0, 0, [n], n_rows=n, q_start=0)
+    scores = torch.empty((n, n), device="cuda")
+    idx = torch.empty((n, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    tk_ws = lsa.workspace(cfg, lsa.OP_TOPK, n, 1, n)
+    mla_ws = lsa.workspace(cfg, lsa.OP_MLA_PREFILL, n, 1, n)
+    outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((n, 32), device="cuda") for _ in range(2)]
+    for _ in range(reps):
+        lsa.index_scores(cfg, None, wl.pos, wl.q_idx, wl.w, wl.k_idx, None, n, scores)
+        lsa.topk(cfg, wl.pos, n, scores, idx, cnt, tk_ws)
+        for z in range(2):
+            lsa.sparse_mla_prefill(cfg, wl.pos, wl.q_abs[z], wl.latent[z], idx, cnt, outs[z], lses[z], mla_ws)
 
 
 def case_hier_decode(reps):
