@@ -283,11 +283,23 @@ cudaError_t launch_index_prefill(const IndexArgs& a, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int n_blocks = (a.n_rows + kRowsPerBlock - 1) / kRowsPerBlock;
   const int64_t max_tiles = (a.max_len + kTileKeys - 1) / kTileKeys;
-  // Split the key range when there are too few row blocks to fill the SMs.
-  int64_t chunks = (4LL * sms + n_blocks - 1) / n_blocks;
-  chunks = max64(1, min64(chunks, max64(1, max_tiles / 32)));
-  const int tiles_per_cta = (int)((max_tiles + chunks - 1) / chunks);
-  chunks = (max_tiles + tiles_per_cta - 1) / tiles_per_cta;
+  // Split the key range when there are too few row blocks to fill the SMs: at
+  // least 4 CTAs per SM, at least 32 key tiles per CTA, and among the splits up
+  // to 4x that many the one whose CTA count best fills whole waves of one CTA
+  // per SM (row blocks that see every key take equal time).
+  const int64_t c_max_tiles = max64(1, max_tiles / 32);
+  const int64_t c_lo = max64(1, min64((4LL * sms + n_blocks - 1) / n_blocks, c_max_tiles));
+  int64_t chunks = c_lo, tiles_per_cta = (max_tiles + c_lo - 1) / c_lo;
+  double best = -1.0;
+  for (int64_t c = c_lo; c <= min64(4 * c_lo, c_max_tiles); ++c) {
+    const int64_t tpc = (max_tiles + c - 1) / c, cc = (max_tiles + tpc - 1) / tpc, n = cc * n_blocks;
+    const double eff = (double)n / (double)(((n + sms - 1) / sms) * sms);
+    if (eff > best + 1e-9) {
+      best = eff;
+      chunks = cc;
+      tiles_per_cta = tpc;
+    }
+  }
   PrefillParams p;
   p.w = a.w;
   p.pos = a.pos;
@@ -297,7 +309,7 @@ cudaError_t launch_index_prefill(const IndexArgs& a, cudaStream_t st) {
   p.n_rows = a.n_rows;
   p.n_init = a.n_init;
   p.n_loc = a.n_loc;
-  p.tiles_per_cta = tiles_per_cta;
+  p.tiles_per_cta = (int)tiles_per_cta;
   p.err = a.err;
   if (n_blocks > 65535) return cudaErrorInvalidValue;
   const cudaError_t e =

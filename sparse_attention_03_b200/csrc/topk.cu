@@ -363,6 +363,44 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   }
   const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
   const uint32_t k_rem = (uint32_t)(a.topk - a.n_init - a.n_loc);
+  // Streams the middle columns [lo, hi) in rounds of 8 values per lane:
+  // fn(v, jc) with jc(i) the column of v[i] (valid when lo <= jc(i) < hi). When
+  // the row is long and 16-byte aligned a warp loads 512 consecutive scores per step
+  // (four 16-byte loads per lane in flight, two rounds), else 256 (eight 4-byte
+  // loads per lane, one round). The 16-byte loads start at lo rounded down to 4
+  // and end at hi rounded up to 4, inside the row since ld is a multiple of 4.
+  const bool vec = g.hi - g.lo >= 32768 && (a.ld & 3) == 0 && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
+  auto stream_row = [&](auto&& fn) {
+    if (vec) {
+      for (int64_t base = (g.lo & ~int64_t(3)) + (int64_t)warp * 512; base < g.hi;
+           base += (int64_t)kRowThreads * 16) {
+        float4 q[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int64_t j4 = base + 128 * u + 4 * lane;
+          q[u] = j4 < g.hi ? *reinterpret_cast<const float4*>(srow + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          const float v[8] = {q[2 * hf].x,     q[2 * hf].y,     q[2 * hf].z,     q[2 * hf].w,
+                              q[2 * hf + 1].x, q[2 * hf + 1].y, q[2 * hf + 1].z, q[2 * hf + 1].w};
+          const int64_t j0 = base + 256 * hf + 4 * lane;
+          fn(v, [&](int i) -> int64_t { return j0 + 128 * (i >> 2) + (i & 3); });
+        }
+      }
+    } else {
+      for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
+        float v[kUnroll];
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const int64_t j = base + lane + 32 * u;
+          v[u] = j < g.hi ? srow[j] : 0.f;
+        }
+        fn(v, [&](int i) -> int64_t { return base + lane + 32 * i; });
+      }
+    }
+  };
+  auto valid = [&](int64_t j) { return j >= g.lo && j < g.hi; };
   int bin0 = 0;
   uint32_t above0 = 0;
   const uint32_t* hr = hist_in ? hist_in + (int64_t)r * kTopkHistStride : nullptr;
@@ -372,46 +410,38 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   } else {
     for (int i = tid; i < kBins; i += kRowThreads) h[i] = 0;
     __syncthreads();
-    for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
-      float v[kUnroll];
+    stream_row([&](const float(&v)[8], auto jc) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t j = base + lane + 32 * u;
-        v[u] = j < g.hi ? srow[j] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u)
-        if (base + lane + 32 * u < g.hi) atomicAdd(&h[score_key(v[u]) >> 21], 1u);
-    }
+      for (int u = 0; u < 8; ++u)
+        if (valid(jc(u))) atomicAdd(&h[score_key(v[u]) >> 21], 1u);
+    });
     __syncthreads();
   }
   find_threshold<kRowThreads>(h, k_rem, bin0, above0, &s_bin, &s_above, s_warp);
   __syncthreads();  // s_up / s_nc initialised
   int32_t* __restrict__ mid = out + a.n_init + a.n_loc;
+  const uint32_t below = (1u << lane) - 1u;
 
   // collect: higher bins straight out, the threshold bin into shared memory
-  for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
-    float v[kUnroll];
+  // (one pair of shared atomics per warp and round: the round's counts first).
+  // Only a few thousand of a row's scores reach the threshold bin: a round in
+  // which no lane of the warp has one costs one vote.
+  stream_row([&](const float(&v)[8], auto jc) {
+    uint32_t key[8], upm[8], eqm[8];
+    bool hit = false;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t j = base + lane + 32 * u;
-      v[u] = j < g.hi ? srow[j] : 0.f;
+    for (int u = 0; u < 8; ++u) {
+      key[u] = score_key(v[u]);
+      hit |= valid(jc(u)) && (int)(key[u] >> 21) >= bin0;
     }
-    // one pair of shared atomics per warp and round: the round's counts first
-    uint32_t key[kUnroll], upm[kUnroll], eqm[kUnroll];
-    int kb[kUnroll];
+    if (!__any_sync(0xffffffffu, hit)) return;
     uint32_t n_up = 0, n_eq = 0;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t j = base + lane + 32 * u;
-      key[u] = 0;
-      kb[u] = -1;
-      if (j < g.hi) {
-        key[u] = score_key(v[u]);
-        kb[u] = (int)(key[u] >> 21);
-      }
-      upm[u] = __ballot_sync(0xffffffffu, kb[u] > bin0);
-      eqm[u] = __ballot_sync(0xffffffffu, kb[u] == bin0);
+    for (int u = 0; u < 8; ++u) {
+      const bool ok = valid(jc(u));
+      const int kb = ok ? (int)(key[u] >> 21) : -1;
+      upm[u] = __ballot_sync(0xffffffffu, kb > bin0);
+      eqm[u] = __ballot_sync(0xffffffffu, kb == bin0);
       n_up += __popc(upm[u]);
       n_eq += __popc(eqm[u]);
     }
@@ -422,21 +452,20 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
     }
     b_up = __shfl_sync(0xffffffffu, b_up, 0);
     b_eq = __shfl_sync(0xffffffffu, b_eq, 0);
-    const uint32_t below = (1u << lane) - 1u;
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t j = base + lane + 32 * u;
-      if (kb[u] > bin0) {
+    for (int u = 0; u < 8; ++u) {
+      const int64_t j = jc(u);
+      if ((upm[u] >> lane) & 1u) {
         const uint32_t slot = b_up + __popc(upm[u] & below);
         if (slot < k_rem) mid[slot] = col(j);
-      } else if (kb[u] == bin0) {
+      } else if ((eqm[u] >> lane) & 1u) {
         const uint32_t slot = b_eq + __popc(eqm[u] & below);
         if (slot < (uint32_t)kRowCap) cand[slot] = ((uint64_t)key[u] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
       }
       b_up += __popc(upm[u]);
       b_eq += __popc(eqm[u]);
     }
-  }
+  });
   __syncthreads();
   const uint32_t need0 = k_rem - above0;
   uint32_t n_cand = s_nc, need = need0;
@@ -451,19 +480,13 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
     // the threshold digit's candidates in shared memory.
     for (int i = tid; i < kBins; i += kRowThreads) h[i] = 0;
     __syncthreads();
-    for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
-      float v[kUnroll];
+    stream_row([&](const float(&v)[8], auto jc) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t j = base + lane + 32 * u;
-        v[u] = j < g.hi ? srow[j] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
+      for (int u = 0; u < 8; ++u) {
         const uint32_t key = score_key(v[u]);
-        if (base + lane + 32 * u < g.hi && (int)(key >> 21) == bin0) atomicAdd(&h[(key >> 10) & (kBins - 1)], 1u);
+        if (valid(jc(u)) && (int)(key >> 21) == bin0) atomicAdd(&h[(key >> 10) & (kBins - 1)], 1u);
       }
-    }
+    });
     __syncthreads();
     int d1;
     uint32_t above1;
@@ -473,19 +496,12 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
       s_nc = 0;
     }
     __syncthreads();
-    const uint32_t below = (1u << lane) - 1u;
-    for (int64_t base = g.lo + warp * 32 * kUnroll; base < g.hi; base += kRowThreads * kUnroll) {
-      float v[kUnroll];
+    stream_row([&](const float(&v)[8], auto jc) {
 #pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t j = base + lane + 32 * u;
-        v[u] = j < g.hi ? srow[j] : 0.f;
-      }
-#pragma unroll
-      for (int u = 0; u < kUnroll; ++u) {
-        const int64_t j = base + lane + 32 * u;
+      for (int u = 0; u < 8; ++u) {
+        const int64_t j = jc(u);
         const uint32_t key = score_key(v[u]);
-        const bool inb = j < g.hi && (int)(key >> 21) == bin0;
+        const bool inb = valid(j) && (int)(key >> 21) == bin0;
         const int dg = (int)((key >> 10) & (kBins - 1));
         const uint32_t mu = __ballot_sync(0xffffffffu, inb && dg > d1);
         const uint32_t me = __ballot_sync(0xffffffffu, inb && dg == d1);
@@ -502,7 +518,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
           if (be < (uint32_t)kRowCap) cand[be] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
         }
       }
-    }
+    });
     __syncthreads();
     if (s_nc <= (uint32_t)kRowCap) {
       in_smem = true;

@@ -170,9 +170,10 @@ def test_index_scores_many_rows_grid_chunks(L, streaming):
 # Top-k on given fp32 scores: the decision is taken in fp32 on both sides, so
 # the selection must match the oracle's exactly, ties included.
 # --------------------------------------------------------------------------
-def _topk_case(L, cfg, s_rows, pos, max_len):
+def _topk_case(L, cfg, s_rows, pos, max_len, ld_pad=3):
+    # ld_pad 3: rows not 16-byte aligned (4-byte loads); 0 with max_len % 4 == 0: 16-byte loads
     n_rows = len(pos)
-    ld = max_len + 3
+    ld = max_len + ld_pad
     s = np.full((n_rows, ld), np.nan, dtype=np.float32)
     for r in range(n_rows):
         s[r, : pos[r] + 1] = s_rows[r][: pos[r] + 1]
@@ -258,8 +259,8 @@ def _dense_bin_rows(rng, pos, n_in_bin, exact=False):
     return rows
 
 
-@pytest.mark.parametrize("kernel", ["per_row", "multi_cta"])
-def test_topk_overfull_threshold_bin(L, kernel):
+@pytest.mark.parametrize("kernel,ld_pad", [("per_row", 3), ("per_row", 0), ("multi_cta", 3)])
+def test_topk_overfull_threshold_bin(L, kernel, ld_pad):
     # The threshold bin holds more candidates than shared memory: one more key
     # digit splits it (per-row kernel: over the row; multi-CTA kernel: over the
     # candidates held in the workspace), and when the split digit still
@@ -275,7 +276,7 @@ def test_topk_overfull_threshold_bin(L, kernel):
         pos = np.array([199999, 150000, 180000], dtype=np.int64)
         rows = _dense_bin_rows(rng, pos[:2], [7000, 12000]) + _dense_bin_rows(rng, pos[2:], [8000], exact=True)
     max_len = int(pos.max()) + 1
-    st, idx, cnt = _topk_case(L, cfg, rows, pos, max_len)
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, max_len, ld_pad)
     assert st == L.LSA_OK
     for r, p in enumerate(pos):
         exp, dense = R.select_topk(R.mask_and_force(rows[r].astype(np.float64), int(p), max_len, ocfg), int(p), ocfg)
