@@ -298,3 +298,38 @@ def hier_select(q, w, k_seq, k_blk, p, cfg: LsaConfig = PAGES, block: int = HIER
     s = mask_and_force(score_row(q, w, k_seq[: p + 1]), p, p + 1, cfg)[cand]
     order = np.lexsort((cand, -s))                 # score descending, then lower column
     return np.sort(cand[order[: cfg.index_topk]]).astype(np.int64), False, kept
+
+
+# --------------------------------------------------------------------------
+# The LoZA sparse pattern ("LongCat-Flash-Thinking-ZigZag架构深度剖析",
+# section "LoZA稀疏注意力机制" / "稀疏模式设计"): the attention matrix is split
+# into a Sink region (the start of the sequence), a Recent region (the latest
+# context) and a Chunked region (the middle, processed block by block). The
+# page names the regions and no sizes. Reading: a query at position p attends
+# to the keys j <= p with j < sink (Sink), p - j < recent (Recent), or
+# j // chunk == p // chunk (its own chunk of the middle: Chunked); the set is
+# static (no indexer) and attention over it is the same absorbed MLA.
+# --------------------------------------------------------------------------
+@dataclass(frozen=True)
+class LozaPattern:
+    """Region sizes of the LoZA pattern (not given by the page; defaults are the
+    LSA sink and local counts and a chunk of twice index_topk)."""
+
+    sink: int = 16
+    recent: int = 1024
+    chunk: int = 4096
+
+
+LOZA = LozaPattern()
+
+
+def loza_select(p: int, pat: LozaPattern = LOZA) -> np.ndarray:
+    """The keys a query at position p attends to, by the three region rules."""
+    j = np.arange(p + 1)
+    keep = (j < pat.sink) | (p - j < pat.recent) | (j // pat.chunk == p // pat.chunk)
+    return j[keep]
+
+
+def loza_row(q_abs: np.ndarray, latent: np.ndarray, p: int, pat: LozaPattern = LOZA, cfg: LsaConfig = PAGES):
+    """Absorbed MLA of one query row over its LoZA set (latent rows 0..p of its sequence)."""
+    return mla(q_abs, latent[loza_select(p, pat)], cfg)

@@ -527,3 +527,52 @@ def test_hier_kept_sets_nest_with_n_blocks():
         if prev is not None:
             assert set(prev) <= set(kept)
         prev = kept
+
+
+# --------------------------------------------------------------------------
+# LoZA pattern (sink / recent / own chunk)
+# --------------------------------------------------------------------------
+def test_loza_select_worked_examples():
+    # sink 2, recent 3, chunk 4, worked by hand from the three region rules
+    pat = R.LozaPattern(sink=2, recent=3, chunk=4)
+    expect = {0: [0], 3: [0, 1, 2, 3], 5: [0, 1, 3, 4, 5], 9: [0, 1, 7, 8, 9], 12: [0, 1, 10, 11, 12],
+              15: [0, 1, 12, 13, 14, 15], 17: [0, 1, 15, 16, 17]}
+    for p, keys in expect.items():
+        assert R.loza_select(p, pat).tolist() == keys, p
+
+
+@pytest.mark.parametrize("sink,recent,chunk", [(16, 1024, 4096), (2, 3, 4), (0, 1, 1), (5, 0, 7), (3, 9, 2),
+                                               (0, 0, 5), (40, 8, 16)])
+def test_loza_set_is_sink_plus_one_window(sink, recent, chunk):
+    # every LoZA set is [0, min(sink, p+1)) followed by one run ending at p that
+    # starts at the earlier of the recent window's and the chunk's first key
+    pat = R.LozaPattern(sink=sink, recent=recent, chunk=chunk)
+    for p in list(range(0, 70)) + [4095, 4096, 5119, 5120, 9000, 131071]:
+        s_end = min(sink, p + 1)
+        start = max(min(p - recent + 1, (p // chunk) * chunk), s_end)
+        keys = list(range(s_end)) + list(range(start, p + 1))
+        assert R.loza_select(p, pat).tolist() == keys, (sink, recent, chunk, p)
+
+
+def test_loza_covering_window_is_dense_attention():
+    rng = np.random.default_rng(41)
+    qa = rng.standard_normal((32, 576))
+    c = rng.standard_normal((300, 576))
+    for p in (0, 7, 120, 299):
+        for pat in (R.LozaPattern(sink=0, recent=p + 1, chunk=1), R.LozaPattern(sink=5, recent=1, chunk=512)):
+            o, lse = R.loza_row(qa, c, p, pat)
+            eo, el = R.dense_mla_row(qa, c, p)
+            np.testing.assert_allclose(o, eo, rtol=1e-12, atol=1e-12)
+            np.testing.assert_allclose(lse, el, rtol=1e-12, atol=1e-12)
+
+
+def test_loza_single_key_is_its_value_row():
+    # sink 0, recent 1, chunk 1: only the query's own key, whose softmax weight is 1
+    rng = np.random.default_rng(43)
+    qa = rng.standard_normal((32, 576))
+    c = rng.standard_normal((50, 576))
+    pat = R.LozaPattern(sink=0, recent=1, chunk=1)
+    for p in (0, 13, 49):
+        o, lse = R.loza_row(qa, c, p, pat)
+        np.testing.assert_array_equal(o, np.broadcast_to(c[p, :512], (32, 512)))
+        np.testing.assert_allclose(lse, PAGES.softmax_scale * (qa @ c[p]), rtol=1e-12)
