@@ -21,7 +21,9 @@ and the decode step with hierarchical indexing ("hier": per layer the newest
 block's summary, a coarse pass over 64-key block summaries keeping the sink /
 recent blocks and the 128 best others, the fine selection over their tokens,
 then both MLA sub-blocks; also the selection alone against the flat index pass
-and top-k), and the other workloads of the pages' configuration list as one
+and top-k), LoZA attention over the same decode workload ("loza": per layer both
+sub-blocks over each row's sink, recent window and own chunk, no indexer; with
+its HBM roofline), and the other workloads of the pages' configuration list as one
 lsa_forward layer each ("configs": single-token decode latency at 8192 cached
 keys with L2 flushed before every step, 64 sequences of 16K-32K cached keys,
 4 sequences at 983040, and a 4096-token prefill chunk against 983040).
@@ -380,6 +382,31 @@ def build_hier(D, device, block=64, n_blocks=128):
     D["hier_cfg"] = {"block": block, "n_blocks": n_blocks}
 
 
+LOZA_PATTERN = (16, 1024, 4096)  # sink, recent, chunk
+
+
+def build_loza(D, device):
+    """Per layer: both sub-blocks' LoZA attention (sink, recent window, own chunk)
+    over the same caches and queries as the decode step; no indexer."""
+    from sparse_attention_03_b200 import lsa
+    B, ctx, cfg = DECODE["batch"], D["ctx"], D["cfg"]
+    ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE, B, B, ctx, device=device)
+    D["loza_ws"] = ws
+    D["loza"] = [[lsa.loza_mla(cfg, LOZA_PATTERN, 0, l.seq_of_row, l.pos, l.k_off, ctx, l.q_abs[z], l.latent[z],
+                               D["out"][i, z], D["lse"][i, z], ws, bind=True) for z in range(2)]
+                 for i, l in enumerate(D["layers"])]
+    p = ctx - 1
+    s_end = min(LOZA_PATTERN[0], ctx)
+    w0 = max(min(p - LOZA_PATTERN[1] + 1, p // LOZA_PATTERN[2] * LOZA_PATTERN[2]), s_end)
+    D["loza_keys"] = s_end + ctx - w0
+
+
+def loza_step(D):
+    for calls in D["loza"]:
+        for call in calls:
+            call()
+
+
 def hier_step(D, select_only=False):
     """One decode step with hierarchical selection: per layer the newest block's
     summary, the two-stage selection, then both MLA sub-blocks on it."""
@@ -696,6 +723,16 @@ def gpu_arm(args):
     tfs = time_region(lambda s: flat_select_step(D), h_steps, world, device)
     assert lsa.device_error() == 0
 
+    # LoZA attention: the same two sub-blocks per layer over the static pattern
+    build_loza(D, device)
+    for _ in range(3):
+        loza_step(D)
+    lz_steps = max(5, args.steps // 2)
+    tl = time_region(lambda s: loza_step(D), lz_steps, world, device)
+    loza_value, _ = aggregate(B * nl * lz_steps, tl, world, device)
+    loza_keys = D["loza_keys"]
+    assert lsa.device_error() == 0
+
     D_hier_cfg = D["hier_cfg"]
     del D
     torch.cuda.empty_cache()
@@ -738,6 +775,15 @@ def gpu_arm(args):
                     "flat_select_us_per_layer": 1e6 * tfs / (h_steps * nl),
                     "config": {"workload": f"hier_decode_b16_ctx131072_14layers_block{hc['block']}"
                                            f"_keep{hc['n_blocks']}", **hc}}
+    lz_bytes = B * 2 * loza_keys * 1152 + B * 2 * (32 * 576 * 2 + 32 * 512 * 2)  # per layer: rows read, q in, out
+    lz_layer_s = tl / (lz_steps * nl)
+    line["loza"] = {"value": loza_value, "unit": "tokens/s/layer", "ms_per_step": 1e3 * tl / lz_steps,
+                    "config": {"workload": "loza_decode_b16_ctx131072_14layers_cli2",
+                               "pattern": dict(zip(("sink", "recent", "chunk"), LOZA_PATTERN)),
+                               "keys_per_row": loza_keys},
+                    "roofline": {"bound": "hbm", "achieved": lz_bytes / lz_layer_s / 1e9, "peak": peak,
+                                 "unit": "GB/s", "frac": lz_bytes / lz_layer_s / 1e9 / peak,
+                                 "peak_source": f"{psrc} hbm_gbs"}}
     if prefill:
         line["prefill"] = prefill
     if configs:

@@ -338,6 +338,38 @@ LSA_API lsa_status lsa_sparse_mla_prefill(const lsa_config* cfg, int32_t n_rows,
                                   float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * LoZA attention ("LongCat-Flash-Thinking-ZigZag架构深度剖析", section
+ * "LoZA稀疏注意力机制" / "稀疏模式设计": the attention matrix is split into a
+ * Sink region (the start of the sequence), a Recent region (the latest
+ * context) and a Chunked region (the middle, processed block by block)). The
+ * page gives no sizes; reading taken: a query at position p attends to the keys
+ * j <= p with j < sink, or p - j < recent, or j / chunk == p / chunk (its own
+ * chunk). The set is static, no indexer runs, and attention over it is the same
+ * absorbed MLA as lsa_sparse_mla_decode / _prefill (scale, layouts, outputs).
+ *
+ * mode 0 = decode: row r is a query of sequence seq_of_row[r] (NULL: r) at
+ *          position pos[r] (pos NULL: the sequence's last key); latent packed
+ *          by k_off like lsa_sparse_mla_decode; max_len >= every sequence's length.
+ * mode 1 = prefill: one sequence, latent bf16 [max_len, 576], k_off and
+ *          seq_of_row NULL, pos required (every pos[r] < max_len).
+ * q_abs bf16 [n_rows, 32, 576], out bf16 [n_rows, 32, 512], lse fp32
+ * [n_rows, 32] or NULL. Workspace optional (split-K partials), sized by
+ * lsa_workspace_size(LSA_OP_MLA_DECODE) (mode 0) or (LSA_OP_MLA_PREFILL)
+ * (mode 1) with the same n_rows and max_len. LSA_ERR_INVALID for a NULL
+ * pattern, sink < 0, recent < 0 or chunk < 1. A bad pos or seq_of_row entry
+ * sets LSA_DEVERR_POS / LSA_DEVERR_SEQ; that row attends to nothing.
+ */
+typedef struct lsa_loza_pattern {
+  int32_t sink;    /* keys at the start every query sees */
+  int32_t recent;  /* the query's latest keys, its own included */
+  int32_t chunk;   /* the query also sees every earlier key of its chunk [p/chunk*chunk, p] */
+} lsa_loza_pattern;
+LSA_API lsa_status lsa_loza_mla(const lsa_config* cfg, const lsa_loza_pattern* pattern, int32_t mode, int32_t n_rows,
+                                int32_t n_seq, const int32_t* seq_of_row, const int32_t* pos, const int64_t* k_off,
+                                int64_t max_len, const lsa_bf16* q_abs, const lsa_bf16* latent, lsa_bf16* out,
+                                float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
  * The whole layer: one index pass and top-k, then cli_factor attention
  * sub-blocks over the same selection ([Lite-Sparse] LSA section, cross-layer
  * index reuse: only the first sub-block owns an indexer; [LSA-2.0] 跨层索引).

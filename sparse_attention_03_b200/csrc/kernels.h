@@ -121,6 +121,10 @@ struct MlaArgs {
   // row's list starts with its n_init sink and n_loc local columns): the kernel
   // attends over those before it waits for the previous kernel in the stream.
   int forced_first = 0, n_init = 0, n_loc = 0;
+  // LoZA rows (no index list): each row attends to keys [0, loza_sink) and to
+  // the run from the earlier of its recent window's and its chunk's first key
+  // up to its own position.
+  int loza = 0, loza_sink = 0, loza_recent = 0, loza_chunk = 1;
   int64_t n_keys;            // prefill: rows in latent
   int64_t max_list;          // host bound on keys per row (sizes split-K)
   float scale;

@@ -458,6 +458,48 @@ lsa_status lsa_sparse_mla_prefill(const lsa_config* c, int32_t n_rows, const int
   return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
 }
 
+lsa_status lsa_loza_mla(const lsa_config* c, const lsa_loza_pattern* pat, int32_t mode, int32_t n_rows,
+                        int32_t n_seq, const int32_t* seq_of_row, const int32_t* pos, const int64_t* k_off,
+                        int64_t max_len, const lsa_bf16* q_abs, const lsa_bf16* latent, lsa_bf16* out, float* lse,
+                        void* ws, size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_loza_mla";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (!pat) return set_error(LSA_ERR_INVALID, "%s: pattern is NULL", fn);
+  if (pat->sink < 0 || pat->recent < 0 || pat->chunk < 1)
+    return set_error(LSA_ERR_INVALID, "%s: need sink >= 0, recent >= 0, chunk >= 1", fn);
+  if ((mode != 0 && mode != 1) || n_rows < 0 || n_seq < 1 || max_len < 1)
+    return set_error(LSA_ERR_INVALID, "%s: need mode 0/1, n_rows >= 0, n_seq >= 1, max_len >= 1", fn);
+  if (mode == 0 && !k_off) return set_error(LSA_ERR_INVALID, "%s: decode needs k_off", fn);
+  if (mode == 1 && (n_seq != 1 || k_off || seq_of_row))
+    return set_error(LSA_ERR_INVALID, "%s: prefill takes one sequence (k_off and seq_of_row NULL)", fn);
+  if (n_rows == 0) return LSA_OK;
+  if ((mode == 1 && !pos) || !q_abs || !latent || !out) return set_error(LSA_ERR_INVALID, "%s: NULL argument", fn);
+  if (!aligned16(q_abs) || !aligned16(latent) || !aligned16(out))
+    return set_error(LSA_ERR_INVALID, "%s: q_abs, latent and out must be 16-byte aligned", fn);
+  MlaArgs a = mla_args(c, 1, n_rows, mode == 0 ? 1 : 0);
+  a.q[0] = q_abs;
+  a.lat[0] = latent;
+  a.out[0] = out;
+  a.lse[0] = lse;
+  a.k_off = mode == 0 ? k_off : nullptr;
+  a.seq_of_row = mode == 0 ? seq_of_row : nullptr;
+  a.n_seq = n_seq;
+  a.pos = pos;
+  a.n_keys = max_len;
+  a.idx = nullptr;
+  a.count = nullptr;
+  a.loza = 1;
+  a.loza_sink = pat->sink;
+  a.loza_recent = pat->recent;
+  a.loza_chunk = pat->chunk;
+  // a row's set: at most the sink plus the longer of its window and its chunk
+  a.max_list = std::min<int64_t>(max_len, (int64_t)pat->sink + std::max<int64_t>(pat->recent, pat->chunk));
+  a.ws = ws;
+  a.ws_bytes = ws ? ws_bytes : 0;
+  return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
+}
+
 lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_t n_seq,
                        const int32_t* seq_of_row, const int32_t* pos, int64_t max_len,
                        const lsa_bf16* q_idx, const float* w, const lsa_bf16* k_idx,

@@ -235,8 +235,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     const RowGeom geo = row_geometry(a, r, false);
     const int nk = (int)max64(0, min64((int64_t)cap, geo.n_list - b0));
     // With an index list the split holds at most topk <= kMaxTopk keys (the
-    // launcher sizes the splits from topk); a dense row's keys are b0 + slot and
-    // need no list.
+    // launcher sizes the splits from topk); a dense row's keys are b0 + slot, a
+    // LoZA row's follow from its position (loza_key): neither needs a list.
     for (int c0 = 0; irow && c0 < nk; c0 += 32 * kChunk) {
       if (c0 > 0) {
 #pragma unroll
@@ -261,13 +261,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     __syncwarp();
     const int n_tiles = (nk + kTK - 1) / kTK;
     const uint16_t* __restrict__ latb = a.lat[z] + geo.kbase * kDLat;
+    const LozaSpan zs = a.loza ? loza_span(a, geo.nvis) : LozaSpan{0, 0};
     for (int base = 0; base < n_tiles; base += kStages) {
 #pragma unroll
       for (int i = 0; i < kStages; ++i) {
         const int tt = base + i;
         if (tt < n_tiles) {
           const int sl = tt * kTK + lane;
-          const int key = sl < nk ? (irow ? sm.list[sl] : (int)(b0 + sl)) : -1;
+          const int key = sl >= nk ? -1 : irow ? sm.list[sl] : (int)(a.loza ? loza_key(zs, b0 + sl) : b0 + sl);
           if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag);
           sm.keys[i][lane] = key;
           uint16_t* dst = &sm.k[i][lane * kSRow];

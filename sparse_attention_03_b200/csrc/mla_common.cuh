@@ -35,6 +35,23 @@ __device__ __forceinline__ int64_t known_key(const ListPlan& p, const MlaArgs& a
   return (p.dense || i < a.n_init) ? i : p.hi + (i - a.n_init);
 }
 
+// A LoZA row that sees nvis keys ("LongCat-Flash-Thinking-ZigZag架构深度剖析",
+// "稀疏模式设计": Sink, Recent and Chunked regions): its keys are [0, s_end) and
+// [w0, nvis), w0 the earlier of the recent window's and the own chunk's first
+// key (never inside the sink run). Slot i holds key i below s_end, else
+// w0 + (i - s_end).
+struct LozaSpan {
+  int64_t s_end, w0;
+};
+__device__ __forceinline__ LozaSpan loza_span(const MlaArgs& a, int64_t nvis) {
+  const int64_t p = nvis - 1;
+  LozaSpan z;
+  z.s_end = min64((int64_t)a.loza_sink, nvis);
+  z.w0 = max64(min64(p - a.loza_recent + 1, (p / a.loza_chunk) * a.loza_chunk), z.s_end);
+  return z;
+}
+__device__ __forceinline__ int64_t loza_key(const LozaSpan& z, int64_t i) { return i < z.s_end ? i : z.w0 + (i - z.s_end); }
+
 // Row geometry, with every out-of-range input clamped (and flagged by one thread).
 __device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool report) {
   RowGeom g{0, 0, 0};
@@ -64,6 +81,10 @@ __device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool re
     g.nvis = p1;
   }
   g.n_list = g.nvis;
+  if (a.loza && g.nvis > 0) {
+    const LozaSpan z = loza_span(a, g.nvis);
+    g.n_list = z.s_end + g.nvis - z.w0;
+  }
   if (a.idx) {
     int c = a.count[r];
     if (c < 0 || c > a.topk) {

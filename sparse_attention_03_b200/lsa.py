@@ -29,7 +29,7 @@ EXPORTS = (
     "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill", "lsa_forward", "lsa_last_error",
     "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16", "lsa_synth_normal_f32",
     "lsa_synth_rms_rows_bf16", "lsa_launch_count", "lsa_index_project", "lsa_block_summaries",
-    "lsa_hier_workspace_size", "lsa_hier_select", "lsa_sparse_mla_decode_topk",
+    "lsa_hier_workspace_size", "lsa_hier_select", "lsa_sparse_mla_decode_topk", "lsa_loza_mla",
 )
 HIER_BLOCK, HIER_BLOCKS = 64, 128
 
@@ -78,6 +78,8 @@ def load():
     lib.lsa_sparse_mla_decode.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]
     lib.lsa_sparse_mla_decode_topk.argtypes = lib.lsa_sparse_mla_decode.argtypes
     lib.lsa_sparse_mla_prefill.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
+    lib.lsa_loza_mla.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LozaPattern), _I32, _I32, _I32, _P, _P, _P,
+                                 _I64, _P, _P, _P, _P, _P, _SZ, _P]
     lib.lsa_forward.argtypes = [ctypes.POINTER(Config), _I32, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P,
                                 ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P), ctypes.POINTER(_P),
                                 _P, _P, _P, _SZ, _P]
@@ -99,7 +101,7 @@ def load():
     lib.lsa_synth_rms_rows_bf16.argtypes = [_P, _I64, _I32, _U64, _U64, _I64, _P]
     for name in ("lsa_index_scores", "lsa_topk", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
                  "lsa_forward", "lsa_index_project", "lsa_block_summaries", "lsa_hier_select", "lsa_device_error",
-                 "lsa_sparse_mla_decode_topk", "lsa_abi_version", "lsa_synth_normal_bf16",
+                 "lsa_sparse_mla_decode_topk", "lsa_loza_mla", "lsa_abi_version", "lsa_synth_normal_bf16",
                  "lsa_synth_normal_f32", "lsa_synth_rms_rows_bf16"):
         getattr(lib, name).restype = _I32
     _lib = lib
@@ -252,6 +254,25 @@ def sparse_mla_prefill(cfg, pos, q_abs, latent, idx, count, out, lse, ws, stream
         ctypes.byref(cfg._c()), pos.shape[0], _ptr(pos), _ptr(q_abs), _ptr(latent), latent.shape[0],
         _ptr(idx), _ptr(count), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
         _stream(stream)), bind=bind)
+
+
+class LozaPattern(ctypes.Structure):
+    """lsa_loza_pattern: sink keys, recent keys, chunk length."""
+    _fields_ = [("sink", _I32), ("recent", _I32), ("chunk", _I32)]
+
+
+def loza_mla(cfg, pattern, mode, seq_of_row, pos, k_off, max_len, q_abs, latent, out, lse, ws=None, stream=None,
+             bind=False):
+    """LoZA attention (sink, recent window, own chunk); pattern = (sink, recent, chunk)."""
+    for t, n in ((q_abs, "q_abs"), (latent, "latent"), (out, "out")):
+        _dt(t, torch.bfloat16, n)
+    _dt(lse, torch.float32, "lse")
+    pat = LozaPattern(*pattern)
+    n_seq = 1 if k_off is None else k_off.shape[0] - 1
+    return _invoke(load().lsa_loza_mla, (
+        ctypes.byref(cfg._c()), ctypes.byref(pat), int(mode), q_abs.shape[0], n_seq, _ptr(seq_of_row), _ptr(pos),
+        _ptr(k_off), int(max_len), _ptr(q_abs), _ptr(latent), _ptr(out), _ptr(lse), _ptr(ws),
+        0 if ws is None else ws.numel(), _stream(stream)), bind=bind, keep=(pat,))
 
 
 def index_project(cfg, seq_of_row, pos, k_off, max_len, c_q, hidden, wq_b, wk, wproj, k_norm_w, q_idx, w, k_cache,

@@ -142,3 +142,20 @@ def test_hier_validation(lib):
     assert lib.lsa_block_summaries(*summ(20)) == lsa.LSA_ERR_UNSUPPORTED
     assert lib.lsa_block_summaries(*summ(64, None)) == lsa.LSA_ERR_INVALID
     assert lsa.block_offsets([1, 64, 65, 0], 64) == [0, 1, 2, 4, 4]
+
+
+def test_loza_validation(lib):
+    c = lsa.LsaConfig().c()
+    f = _fake()
+
+    def call(pat, mode=0, k_off=f, n_seq=2, pos=f, seq=None):
+        return lib.lsa_loza_mla(ctypes.byref(c), None if pat is None else ctypes.byref(lsa.LozaPattern(*pat)), mode,
+                                3, n_seq, seq, pos, k_off, 100, f, f, f, None, None, 0, None)
+    assert call(None) == lsa.LSA_ERR_INVALID
+    assert call((16, 1024, 0)) == lsa.LSA_ERR_INVALID          # chunk < 1
+    assert call((-1, 1024, 64)) == lsa.LSA_ERR_INVALID         # sink < 0
+    assert call((16, -5, 64)) == lsa.LSA_ERR_INVALID           # recent < 0
+    assert call((16, 1024, 64), k_off=None) == lsa.LSA_ERR_INVALID            # decode needs k_off
+    assert call((16, 1024, 64), mode=1, n_seq=1) == lsa.LSA_ERR_INVALID       # prefill: k_off must be NULL
+    assert call((16, 1024, 64), mode=1, k_off=None, n_seq=1, pos=None) == lsa.LSA_ERR_INVALID  # prefill needs pos
+    assert call((16, 1024, 64), mode=2) == lsa.LSA_ERR_INVALID

@@ -418,6 +418,80 @@ def test_mla_rising_logits_rescale(L):
         assert_attention(bf16_host_f64(out)[0], lse.cpu().numpy()[0], eo, el)
 
 
+@pytest.mark.parametrize("pattern", [(16, 1024, 4096), (2, 3, 8), (0, 1, 1), (40, 100, 64), (5, 0, 300)])
+def test_loza_decode_varlen(L, pattern):
+    # LoZA rows of sequences whose lengths straddle the sink, the recent window and
+    # chunk boundaries; split-K with a workspace and one pass without
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    pat = R.LozaPattern(*pattern)
+    lengths = [1, 3, 16, 17, 300, 1024, 1025, 4095, 4096, 4097, 5121, 9000]
+    wl = S.Workload(51, 0, lengths, cli=1)
+    d = _upload(wl)
+    B, max_len = len(lengths), max(lengths)
+    f = S.bf16_bits_to_f64
+    exp = []
+    for b in range(B):
+        a, e = int(wl.k_off[b]), int(wl.k_off[b + 1])
+        exp.append(R.loza_row(f(wl.q_abs[0][b]), f(wl.latent[0][a:e]), int(wl.pos[b]), pat, ocfg))
+    out = torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 32), device="cuda")
+    for ws in (L.workspace(cfg, L.OP_MLA_DECODE, B, B, max_len), None):
+        out.fill_(float("nan"))
+        L.loza_mla(cfg, pattern, 0, d["seq_of_row"], d["pos"], d["k_off"], max_len, d["q_abs"][0], d["latent"][0],
+                   out, lse, ws)
+        assert L.device_error() == 0
+        o, l = bf16_host_f64(out), lse.cpu().numpy()
+        for b in range(B):
+            assert_attention(o[b], l[b], exp[b][0], exp[b][1], where=f"{pattern} len {lengths[b]} ws={ws is not None}")
+
+
+@pytest.mark.parametrize("pattern", [(16, 1024, 4096), (2, 3, 8), (16, 64, 256)])
+def test_loza_prefill_rows(L, pattern):
+    # a prefill chunk at an offset, rows crossing chunk boundaries
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    pat = R.LozaPattern(*pattern)
+    n_keys, n_rows = 5200, 300
+    wl = S.Workload(52, 0, [n_keys], n_rows=n_rows, q_start=n_keys - n_rows, cli=1)
+    d = _upload(wl)
+    out = torch.empty((n_rows, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((n_rows, 32), device="cuda")
+    ws = L.workspace(cfg, L.OP_MLA_PREFILL, n_rows, 1, n_keys)
+    L.loza_mla(cfg, pattern, 1, None, d["pos"], None, n_keys, d["q_abs"][0], d["latent"][0], out, lse, ws)
+    assert L.device_error() == 0
+    o, l = bf16_host_f64(out), lse.cpu().numpy()
+    f = S.bf16_bits_to_f64
+    c = f(wl.latent[0])
+    for r in (0, 1, 95, 96, 97, 150, 199, n_rows - 1):
+        eo, el = R.loza_row(f(wl.q_abs[0][r]), c, int(wl.pos[r]), pat, ocfg)
+        assert_attention(o[r], l[r], eo, el, where=f"{pattern} row {r}")
+
+
+def test_loza_decode_explicit_positions(L):
+    # rows that are not the last key of their sequence, in shuffled sequence order
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    pattern = (16, 256, 1024)
+    lengths = [3000, 5000, 1500]
+    wl = S.Workload(53, 0, lengths, cli=1)
+    d = _upload(wl)
+    seq = np.array([2, 0, 1, 1, 0], dtype=np.int32)
+    pos = np.array([1499, 1023, 4095, 2000, 17], dtype=np.int32)
+    q = S.normal_bf16(53, S.tid(9, S.Q_ABS0), 0, 5 * 32 * 576).reshape(5, 32, 576)
+    out = torch.empty((5, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((5, 32), device="cuda")
+    L.loza_mla(cfg, pattern, 0, i32_dev(seq), i32_dev(pos), d["k_off"], max(lengths), bf16_dev(q), d["latent"][0],
+               out, lse, L.workspace(cfg, L.OP_MLA_DECODE, 5, 3, max(lengths)))
+    assert L.device_error() == 0
+    o, l = bf16_host_f64(out), lse.cpu().numpy()
+    f = S.bf16_bits_to_f64
+    for r in range(5):
+        a, e = int(wl.k_off[seq[r]]), int(wl.k_off[seq[r] + 1])
+        eo, el = R.loza_row(f(q[r]), f(wl.latent[0][a:e]), int(pos[r]), R.LozaPattern(*pattern), ocfg)
+        assert_attention(o[r], l[r], eo, el, where=f"row {r}")
+
+
 def test_mla_decode_dense(L):
     cfg = L.LsaConfig(cli_factor=1)
     ocfg = oracle_cfg(cfg)
