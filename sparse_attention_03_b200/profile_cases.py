@@ -11,6 +11,7 @@ current stream, checks the device error flags and exits. Cases:
   topk_decode    lsa_topk on 16 rows x 131072 scores, with the indexer's histogram
   mla_decode     lsa_sparse_mla_decode, 16 rows x 2048 selected keys of 131072
   mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
+  decode_8k      lsa_forward (cli 2), 1 row x 8192 keys (single-token decode latency)
   decode_1m      lsa_forward (cli 2), 4 rows x 983040 keys (one long-context decode layer)
   chunk_1m       lsa_forward (cli 2), a 4096-row prefill chunk at positions 983040.. (16 GB of scores)
   prefill_16k    one prefill step of 16384 causal rows: lsa_index_scores, lsa_topk, then
@@ -97,6 +98,17 @@ def case_mla_prefill(reps):
     ws = lsa.workspace(cfg, lsa.OP_MLA_PREFILL, n_rows, 1, n_keys)
     for _ in range(reps):
         lsa.sparse_mla_prefill(cfg, wl.pos, wl.q_abs[0], wl.latent[0], idx, cnt, out, lse, ws)
+
+
+def case_decode_8k(reps):
+    cfg = lsa.LsaConfig()
+    wl = DeviceWorkload(0, 0, np.array([8192], dtype=np.int64))
+    outs = [torch.empty((1, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((1, 32), device="cuda") for _ in range(2)]
+    ws = lsa.workspace(cfg, lsa.OP_FORWARD_DECODE, 1, 1, 8192)
+    for _ in range(reps):
+        lsa.forward(cfg, 0, wl.seq_of_row, wl.pos, 8192, wl.q_idx, wl.w, wl.k_idx, wl.k_off, wl.q_abs, wl.latent,
+                    outs, lses, ws)
 
 
 def case_decode_1m(reps):
