@@ -71,7 +71,7 @@ struct TopkArgs {
   // the one-CTA-per-row kernel.
   uint32_t* zero_hist = nullptr;
 };
-constexpr int kTopkCap = 4096;                              // candidates kept per row
+constexpr int kTopkCap = 4096;                              // candidates per row: the base layout, and shared memory
 constexpr size_t kTopkRowBytes = 2048 * 4 + 32 + kTopkCap * 8;  // hist + ctl + candidates
 constexpr int kTopkHistStride = 2048 + 8;                   // words between rows' histograms
 

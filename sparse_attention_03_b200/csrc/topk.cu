@@ -17,8 +17,11 @@
 //   * few long rows: many CTAs per row. Each finds the threshold bin, places
 //     its chunk's columns with one block-wide prefix sum and one global atomic,
 //     and the last CTA of the row (an atomic ticket) finishes the select on the
-//     candidates. If the candidate buffer overflowed (many equal scores), that
-//     CTA rescans the row instead.
+//     candidates, which the workspace keeps (up to a sixteenth of the row).
+// When the threshold bin holds more candidates than shared memory, the next 11
+// key bits split it first (the digits above the threshold digit go straight
+// out), over the workspace's candidates or, in the one-CTA kernel, over the row;
+// only equal keys beyond that fall back to rescanning the row per level.
 // No kernel waits on another CTA.
 #include "common.cuh"
 #include "kernels.h"
