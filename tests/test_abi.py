@@ -56,6 +56,21 @@ def test_workspace_sizes(lib):
     assert lsa.workspace_size(bad, lsa.OP_TOPK, 4, 4, 100) == 0
 
 
+def test_topk_workspace_grows_with_long_rows(lib):
+    # few long rows (the multi-CTA select) keep up to a sixteenth of the row's
+    # length of threshold-bin candidates (8 bytes each), at least the base 4096,
+    # on top of the 8 KB histogram and control block of every row
+    cfg = lsa.LsaConfig()
+    base_row = 2056 * 4 + 4096 * 8                     # histogram + control, base candidates
+    for rows, n in ((4, 983040), (16, 131072), (16, 40000), (3, 2 ** 23)):
+        room = max(4096, min(n // 16, 2 ** 18))
+        per = base_row + (room - 4096) * 8
+        assert lsa.workspace_size(cfg, lsa.OP_TOPK, rows, rows, n) == rows * per + 256, (rows, n)
+    # many rows or short rows take the one-CTA-per-row kernel: no candidate room
+    assert lsa.workspace_size(cfg, lsa.OP_TOPK, 300, 300, 983040) == 300 * base_row + 256
+    assert lsa.workspace_size(cfg, lsa.OP_TOPK, 4, 4, 16384) == 4 * base_row + 256
+
+
 def _fake(n=1):
     return ctypes.c_void_p(0x10000 * n)  # aligned, never dereferenced by the host checks
 

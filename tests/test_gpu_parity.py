@@ -285,6 +285,30 @@ def test_topk_overfull_threshold_bin(L, kernel, ld_pad):
     assert L.device_error() == 0
 
 
+def test_topk_overfull_bin_with_minimal_workspace(L):
+    # a workspace of one base row block (4096 candidates per row) cannot hold the
+    # overfull bin: the multi-CTA select falls back to rescanning the row, rows
+    # one block at a time
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(37)
+    pos = np.array([99999, 70000], dtype=np.int64)
+    rows = _dense_bin_rows(rng, pos, [6000, 5000])
+    max_len = int(pos.max()) + 1
+    s = np.full((2, max_len), -np.inf, dtype=np.float32)
+    for r, p in enumerate(pos):
+        s[r, : p + 1] = rows[r]
+    ws = torch.empty(40992 + 256, dtype=torch.uint8, device="cuda")
+    idx = torch.empty((2, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((2,), dtype=torch.int32, device="cuda")
+    assert L.topk(cfg, i32_dev(pos), max_len, f32_dev(s), idx, cnt, ws) == L.LSA_OK
+    idx = idx.cpu().numpy()
+    for r, p in enumerate(pos):
+        exp, _ = R.select_topk(R.mask_and_force(s[r].astype(np.float64), int(p), max_len, ocfg), int(p), ocfg)
+        np.testing.assert_array_equal(np.sort(idx[r]), exp, err_msg=f"row {r}")
+    assert L.device_error() == 0
+
+
 @pytest.mark.parametrize("streaming", [True, False])
 def test_topk_with_indexer_histogram(L, streaming):
     # the histogram lsa_index_scores emits gives lsa_topk the same selection as
