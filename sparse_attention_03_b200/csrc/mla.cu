@@ -478,7 +478,9 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
 }
 
 // One CTA per (head, row, sub-block): 128 threads x 4 value dims, so that a
-// small decode batch still spreads the merge over many SMs.
+// small decode batch still spreads the merge over many SMs. Every thread issues
+// its partial-output loads before the split weights are known, so the two
+// reads overlap.
 __global__ void __launch_bounds__(128) mla_merge_kernel(MlaArgs a, Split sp, const float* part_o,
                                                         const float2* part_ml) {
   __shared__ float wgt[kMaxSplits];
@@ -487,6 +489,13 @@ __global__ void __launch_bounds__(128) mla_merge_kernel(MlaArgs a, Split sp, con
   pdl_trigger();  // the next MLA may start its forced columns; it waits for this grid before writing
   const int h = blockIdx.x, r = blockIdx.y, z = blockIdx.z, tid = threadIdx.x;
   const int64_t base = ((int64_t)z * a.n_rows + r) * sp.n_split;
+  const int e = tid * 4;
+  constexpr int kIn = 8;  // partial rows in flight per thread
+  float4 v[kIn];
+#pragma unroll
+  for (int i = 0; i < kIn; ++i)
+    v[i] = i < sp.n_split ? *reinterpret_cast<const float4*>(part_o + ((base + i) * kH + h) * kDV + e)
+                          : make_float4(0.f, 0.f, 0.f, 0.f);
   if (tid < 32) {
     const float2 ml = tid < sp.n_split ? part_ml[(base + tid) * kH + h] : make_float2(-INFINITY, 0.f);
     float M = ml.x;
@@ -503,16 +512,18 @@ __global__ void __launch_bounds__(128) mla_merge_kernel(MlaArgs a, Split sp, con
     }
   }
   __syncthreads();
-  const int e = tid * 4;
   float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int s = 0; s < sp.n_split; ++s) {
-    const float4 v = *reinterpret_cast<const float4*>(part_o + ((base + s) * kH + h) * kDV + e);
-    const float wv = wgt[s];
-    acc.x = fmaf(wv, v.x, acc.x);
-    acc.y = fmaf(wv, v.y, acc.y);
-    acc.z = fmaf(wv, v.z, acc.z);
-    acc.w = fmaf(wv, v.w, acc.w);
-  }
+  auto add = [&](const float4& x, float wv) {
+    acc.x = fmaf(wv, x.x, acc.x);
+    acc.y = fmaf(wv, x.y, acc.y);
+    acc.z = fmaf(wv, x.z, acc.z);
+    acc.w = fmaf(wv, x.w, acc.w);
+  };
+#pragma unroll
+  for (int i = 0; i < kIn; ++i)
+    if (i < sp.n_split) add(v[i], wgt[i]);
+  for (int s = kIn; s < sp.n_split; ++s)
+    add(*reinterpret_cast<const float4*>(part_o + ((base + s) * kH + h) * kDV + e), wgt[s]);
   const float il = inv_l;
   uint2 pk;
   pk.x = pack_bf16x2(acc.x * il, acc.y * il);
