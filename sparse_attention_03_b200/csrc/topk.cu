@@ -333,6 +333,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   __shared__ uint64_t cand[kRowCap];
   __shared__ int s_bin;
   __shared__ uint32_t s_above, s_warp[kRowThreads / 32], s_up, s_nc, s_slot;
+  __shared__ uint32_t s_wu[kRowThreads / 32], s_we[kRowThreads / 32];
   extern __shared__ int32_t s_map[];  // the row's column map (col_ld entries) when there is one
   pdl_wait();
   pdl_trigger();  // dependents may launch now; they wait for this grid before reading its outputs
@@ -366,6 +367,22 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   }
   const float* __restrict__ srow = a.scores + (int64_t)r * a.ld;
   const uint32_t k_rem = (uint32_t)(a.topk - a.n_init - a.n_loc);
+  // Short rows (at most 16 middle scores per thread): every score is requested
+  // at once, before the histogram and the threshold search, and the collect
+  // places each thread's scores with one block-wide prefix sum.
+  constexpr int kShort = 2 * kUnroll;
+  const bool short_row = g.hi - g.lo <= (int64_t)kRowThreads * kShort;
+  auto scol = [&](int i) -> int64_t {  // warp w, round q: columns lo + 4096 q + 256 w .. + 255
+    return g.lo + (int64_t)(i / kUnroll) * kRowThreads * kUnroll + warp * 32 * kUnroll + lane + 32 * (i % kUnroll);
+  };
+  float sv[kShort];
+  if (short_row) {
+#pragma unroll
+    for (int i = 0; i < kShort; ++i) {
+      const int64_t j = scol(i);
+      sv[i] = j < g.hi ? srow[j] : 0.f;
+    }
+  }
   // Streams the middle columns [lo, hi) in rounds of 8 values per lane:
   // fn(v, jc) with jc(i) the column of v[i] (valid when lo <= jc(i) < hi). When
   // the row is long and 16-byte aligned a warp loads 512 consecutive scores per step
@@ -413,11 +430,17 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   } else {
     for (int i = tid; i < kBins; i += kRowThreads) h[i] = 0;
     __syncthreads();
-    stream_row([&](const float(&v)[8], auto jc) {
+    if (short_row) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (valid(jc(u))) atomicAdd(&h[score_key(v[u]) >> 21], 1u);
-    });
+      for (int i = 0; i < kShort; ++i)
+        if (scol(i) < g.hi) atomicAdd(&h[score_key(sv[i]) >> 21], 1u);
+    } else {
+      stream_row([&](const float(&v)[8], auto jc) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u)
+          if (valid(jc(u))) atomicAdd(&h[score_key(v[u]) >> 21], 1u);
+      });
+    }
     __syncthreads();
   }
   find_threshold<kRowThreads>(h, k_rem, bin0, above0, &s_bin, &s_above, s_warp);
@@ -425,6 +448,51 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   int32_t* __restrict__ mid = out + a.n_init + a.n_loc;
   const uint32_t below = (1u << lane) - 1u;
 
+  if (short_row) {
+    // collect of a short row: each thread's counts above and in the threshold
+    // bin, exclusive prefix sums over the block, then every score to its place
+    uint32_t nu = 0, ne = 0;
+#pragma unroll
+    for (int i = 0; i < kShort; ++i) {
+      const int kb = scol(i) < g.hi ? (int)(score_key(sv[i]) >> 21) : -1;
+      nu += kb > bin0;
+      ne += kb == bin0;
+    }
+    uint32_t iu = nu, ie = ne;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const uint32_t yu = __shfl_up_sync(0xffffffffu, iu, off), ye = __shfl_up_sync(0xffffffffu, ie, off);
+      if (lane >= off) {
+        iu += yu;
+        ie += ye;
+      }
+    }
+    if (lane == 31) {
+      s_wu[warp] = iu;
+      s_we[warp] = ie;
+    }
+    __syncthreads();
+    uint32_t ou = iu - nu, oe = ie - ne;
+    for (int w2 = 0; w2 < warp; ++w2) {
+      ou += s_wu[w2];
+      oe += s_we[w2];
+    }
+    if (tid == kRowThreads - 1) s_nc = oe + ne;  // the last thread's prefix is the total
+#pragma unroll
+    for (int i = 0; i < kShort; ++i) {
+      const int64_t j = scol(i);
+      if (j >= g.hi) continue;
+      const uint32_t key = score_key(sv[i]);
+      const int kb = (int)(key >> 21);
+      if (kb > bin0) {
+        if (ou < k_rem) mid[ou] = col(j);
+        ++ou;
+      } else if (kb == bin0) {
+        if (oe < (uint32_t)kRowCap) cand[oe] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+        ++oe;
+      }
+    }
+  } else
   // collect: higher bins straight out, the threshold bin into shared memory
   // (one pair of shared atomics per warp and round: the round's counts first).
   // Only a few thousand of a row's scores reach the threshold bin: a round in
