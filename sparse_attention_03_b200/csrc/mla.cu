@@ -98,15 +98,22 @@ __device__ __forceinline__ void half_sync(int h) { asm volatile("bar.sync %0, 12
 __device__ __forceinline__ void stagger_arrive() { asm volatile("bar.arrive 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 __device__ __forceinline__ void stagger_wait() { asm volatile("bar.sync 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 
-// A split's tiles of a forced-first list: whole tiles of the known prefix
-// [0, K), then whole tiles of the selected part [K, L), each part shared evenly
-// by the splits (only each part's last tile of a row can be partly empty).
+// A split's tiles of a forced-first list: whole tiles of the known prefix,
+// then whole tiles of the rest read from the list, each part shared evenly by
+// the splits. The known prefix is the forced columns' whole tiles (a dense
+// row: its whole list); the forced columns left over in a part tile are read
+// from the list with the selected ones, which the top-k wrote in the same
+// order, so a sparse row of 2048 keys is 64 full tiles (1024 + 1024 keys), not
+// 65 with two part tiles. ub = the first slot read from the list.
 struct FfTiles {
   int kt0, kt, ut0, ut;
+  int64_t ub;
 };
 __device__ __forceinline__ FfTiles ff_tiles(const ListPlan& p, int s, int n) {
-  const int Kt = (int)((p.K + kTK - 1) / kTK), Ut = (int)((p.L - p.K + kTK - 1) / kTK);
+  const int Kt = (int)(p.dense ? (p.K + kTK - 1) / kTK : p.K / kTK);
   FfTiles f;
+  f.ub = min64((int64_t)Kt * kTK, p.L);
+  const int Ut = (int)((p.L - f.ub + kTK - 1) / kTK);
   f.kt0 = Kt * s / n;
   f.kt = Kt * (s + 1) / n - f.kt0;
   f.ut0 = Ut * s / n;
@@ -193,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
       bool listed[kBatch];
 #pragma unroll
       for (int j = 0; j < kBatch; ++j) {
-        const int64_t sl = lp.K + (int64_t)(ft.ut0 + u0 + j) * kTK + lane;
+        const int64_t sl = ft.ub + (int64_t)(ft.ut0 + u0 + j) * kTK + lane;
         listed[j] = u0 + j < ft.ut && sl < uend;
         key[j] = listed[j] ? __ldg(irow + sl) : -1;
       }
