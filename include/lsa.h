@@ -356,8 +356,9 @@ LSA_API lsa_status lsa_sparse_mla_prefill(const lsa_config* cfg, int32_t n_rows,
  * [n_rows, 32] or NULL. Workspace optional (split-K partials), sized by
  * lsa_workspace_size(LSA_OP_MLA_DECODE) (mode 0) or (LSA_OP_MLA_PREFILL)
  * (mode 1) with the same n_rows and max_len. LSA_ERR_INVALID for a NULL
- * pattern, sink < 0, recent < 0 or chunk < 1. A bad pos or seq_of_row entry
- * sets LSA_DEVERR_POS / LSA_DEVERR_SEQ; that row attends to nothing.
+ * pattern, sink < 0, recent < 0 or chunk < 1. A position outside its sequence
+ * sets LSA_DEVERR_POS and is clamped into it; a seq_of_row entry outside
+ * [0, n_seq) sets LSA_DEVERR_SEQ and that row attends to nothing (zero output).
  */
 typedef struct lsa_loza_pattern {
   int32_t sink;    /* keys at the start every query sees */
