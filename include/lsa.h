@@ -10,6 +10,8 @@
  *     "LSA（LongCat 稀疏注意力）", "预填充优化", "测试与验证".
  *   [LSA-2.0] "LongCat Sparse Attention技术深度解析：为什么它能提升100万上下文
  *     处理效率", sections "流式感知索引", "跨层索引", "模型架构配置".
+ *   "LongCat-Flash-Thinking-ZigZag架构深度剖析", section "LoZA稀疏注意力机制"
+ *     (lsa_loza_mla only).
  *
  * Conventions shared by every entry point
  * ---------------------------------------
