@@ -181,7 +181,8 @@ LSA_API lsa_status lsa_topk(const lsa_config* cfg, int32_t n_rows, const int32_t
  * stream operation, so a capture cannot contain one), serving loops that must
  * not pay the device-wide synchronisation cudaMalloc/cudaFree may cause, and
  * plugins whose host framework hands them only their input and output buffers.
- * The caller passes exactly the buffers of lsa_topk except the workspace.
+ * The caller passes the buffers of lsa_topk except the workspace and the
+ * optional topk_hist (this entry point always builds its own histogram).
  *
  * Scratch: a file-scope device array of LSA_TOPK_STATIC_MAX_ROWS x 40992 bytes
  * (2.5 MiB) inside the library; every GPU that loads the library keeps it
@@ -192,7 +193,8 @@ LSA_API lsa_status lsa_topk(const lsa_config* cfg, int32_t n_rows, const int32_t
  * zero; calls whose kernels may overlap on the GPU (other streams, other host
  * threads) race on it and must be serialised by the caller.
  * n_rows > LSA_TOPK_STATIC_MAX_ROWS returns LSA_ERR_INVALID (split the rows or
- * use lsa_topk). Statuses otherwise as lsa_topk.
+ * use lsa_topk). The configuration is checked as lsa_topk checks it; statuses
+ * otherwise as lsa_topk.
  */
 #define LSA_TOPK_STATIC_MAX_ROWS 64
 LSA_API lsa_status lsa_topk_static(const lsa_config* cfg, int32_t n_rows, const int32_t* pos,

@@ -18,10 +18,10 @@ method. Sources (web pages; cited by title and section):
   处理效率" (wmrh.cn). Sections used: "模型架构配置" (index_n_heads 32,
   index_head_dim 128, index_topk 2048, index_local_tokens 1024,
   index_init_tokens 16, cli_factor 2), "跨层索引" (one index pass serves
-  consecutive layers).
+  consecutive layers), "多token预测模块集成" (the MTP draft steps share one
+  index pass).
 
-Readings taken where the pages are silent or garbled (each is also listed in
-the design notes):
+Readings taken where the pages are silent or garbled:
 * The fallback comparison lost its operator in the scrape; it is read as
   "cached length <= index_topk", applied per query row.
 * No extra scale in the index score; any scale lives in w.
@@ -146,6 +146,36 @@ def lsa_row(q_idx, w, k_seq, p, q_abs_list, latent_list, cfg: LsaConfig = PAGES)
         s = mask_and_force(score_row(q_idx, w, k_seq[:n]), p, L, cfg)
         sel, dense = select_topk(s, p, cfg)
     outs = [mla(qa, lat[sel], cfg) for qa, lat in zip(q_abs_list, latent_list)]
+    return sel, dense, outs
+
+
+def mtp_round(q_idx, w, k_seq, p, q_abs_steps, latent, cfg: LsaConfig = PAGES):
+    """One round of multi-token-prediction drafting over one shared index pass.
+
+    [LSA-2.0] 多token预测模块集成: the method extends to a three-step MTP module
+    for speculative decoding, and all draft steps share a single index pass.
+    Reading (the page says only that the pass is shared): the indexer, forcing
+    and top-k (or the dense fallback) run once, for the first draft step's query
+    at position p. Draft step i (i = 0, 1, ...) has its query at position p + i;
+    by then the keys p+1 .. p+i (the earlier drafts' and its own) are in the
+    cache, and a query sees its own key, so step i attends over the shared
+    selection together with those keys. Nothing is dropped from the shared
+    selection (it is reused as it stands).
+
+    k_seq [L, 128] and latent [L, 576] hold the sequence's caches with keys
+    0 .. p + len(q_abs_steps) - 1 present. Returns (selected, dense,
+    [(o, lse) per step]).
+    """
+    n = p + 1
+    if n <= cfg.index_topk:
+        sel, dense = np.arange(n, dtype=np.int64), True      # the indexer is not run
+    else:
+        s = mask_and_force(score_row(q_idx, w, k_seq[:n]), p, k_seq.shape[0], cfg)
+        sel, dense = select_topk(s, p, cfg)
+    outs = []
+    for i, qa in enumerate(q_abs_steps):
+        keys = np.concatenate([sel, np.arange(p + 1, p + 1 + i, dtype=np.int64)])
+        outs.append(mla(qa, latent[keys], cfg))
     return sel, dense, outs
 
 

@@ -15,6 +15,9 @@ lsa_status set_error(lsa_status st, const char* fmt, ...);
 int* device_error_word();
 // Adds n to the process-wide launch counter (lsa_launch_count).
 void count_launches(int64_t n);
+// LSA_OK when the configuration is one the kernels implement; otherwise the
+// status (with its message recorded for lsa_last_error) naming the function.
+lsa_status check_cfg(const lsa_config* c, const char* fn);
 
 struct IndexArgs {
   const uint16_t* q_idx;   // [n_rows, 32, 128]

@@ -38,15 +38,6 @@ int* device_error_word() {
   return ptrs[dev];
 }
 
-namespace {
-
-constexpr size_t kAlign = 256;
-constexpr int kTopkPreferredRows = 4096;
-constexpr size_t kPrefillScoreBudget = size_t(4) << 30;  // bytes of scores per prefill block
-
-size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
-bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
-
 lsa_status check_cfg(const lsa_config* c, const char* fn) {
   if (!c) return set_error(LSA_ERR_INVALID, "%s: cfg is NULL", fn);
   if (c->index_n_heads != kHi || c->index_head_dim != kDi || c->n_heads != kH ||
@@ -64,6 +55,16 @@ lsa_status check_cfg(const lsa_config* c, const char* fn) {
     return set_error(LSA_ERR_INVALID, "%s: softmax_scale must be finite and > 0", fn);
   return LSA_OK;
 }
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kTopkPreferredRows = 4096;
+constexpr size_t kPrefillScoreBudget = size_t(4) << 30;  // bytes of scores per prefill block
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
 
 lsa_status cuda_status(cudaError_t e, const char* fn) {
   if (e == cudaSuccess) return LSA_OK;

@@ -13,6 +13,8 @@
 // until the process exits. Host code cannot use the array's name as a device
 // address, so the device address is looked up once per device with
 // cudaGetSymbolAddress on the first call made while that device is current.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,16 +26,18 @@ constexpr int kStaticRows = LSA_TOPK_STATIC_MAX_ROWS;
 static __device__ __align__(256) unsigned char g_topk_scratch[(size_t)kStaticRows * kTopkRowBytes];
 
 // Device address of g_topk_scratch on the current device (null on failure).
+// Host threads may make their first calls on a device at the same time: each
+// then looks the address up and stores the same value, through atomics.
 void* static_scratch() {
-  static void* addr[64] = {};
+  static std::atomic<void*> addr[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  if (!addr[dev]) {
-    void* p = nullptr;
+  void* p = addr[dev].load(std::memory_order_relaxed);
+  if (!p) {
     if (cudaGetSymbolAddress(&p, g_topk_scratch) != cudaSuccess) return nullptr;
-    addr[dev] = p;
+    addr[dev].store(p, std::memory_order_relaxed);
   }
-  return addr[dev];
+  return p;
 }
 
 }  // namespace
@@ -45,10 +49,8 @@ extern "C" lsa_status lsa_topk_static(const lsa_config* c, int32_t n_rows, const
                                       int64_t max_len, const float* scores, int64_t ld, int32_t* idx,
                                       int32_t* count, void* stream) {
   const char* fn = "lsa_topk_static";
-  if (!c) return set_error(LSA_ERR_INVALID, "%s: cfg is NULL", fn);
-  if (c->index_topk < 1 || c->index_topk > kMaxTopk || c->index_init_tokens < 0 ||
-      c->index_local_tokens < 0 || (int64_t)c->index_init_tokens + c->index_local_tokens >= c->index_topk)
-    return set_error(LSA_ERR_UNSUPPORTED, "%s: need 0 <= init, 0 <= local, init + local < topk <= 2048", fn);
+  const lsa_status cs = check_cfg(c, fn);  // the same configurations as lsa_topk
+  if (cs != LSA_OK) return cs;
   if (n_rows < 0 || max_len < 1 || ld < max_len)
     return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0 and 1 <= max_len <= ld", fn);
   if (n_rows > kStaticRows)

@@ -30,7 +30,9 @@ EXPORTS = (
     "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16", "lsa_synth_normal_f32",
     "lsa_synth_rms_rows_bf16", "lsa_launch_count", "lsa_index_project", "lsa_block_summaries",
     "lsa_hier_workspace_size", "lsa_hier_select", "lsa_sparse_mla_decode_topk", "lsa_loza_mla",
+    "lsa_topk_static",
 )
+TOPK_STATIC_MAX_ROWS = 64
 HIER_BLOCK, HIER_BLOCKS = 64, 128
 
 
@@ -75,6 +77,7 @@ def load():
     lib.lsa_index_scores.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _P, _P, _P, _P, _P, _I64, _P, _I64, _P,
                                      _P]
     lib.lsa_topk.argtypes = [ctypes.POINTER(Config), _I32, _P, _I64, _P, _I64, _P, _P, _P, _P, _SZ, _P]
+    lib.lsa_topk_static.argtypes = [ctypes.POINTER(Config), _I32, _P, _I64, _P, _I64, _P, _P, _P]
     lib.lsa_sparse_mla_decode.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]
     lib.lsa_sparse_mla_decode_topk.argtypes = lib.lsa_sparse_mla_decode.argtypes
     lib.lsa_sparse_mla_prefill.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
@@ -99,7 +102,7 @@ def load():
     lib.lsa_synth_normal_bf16.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
     lib.lsa_synth_normal_f32.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
     lib.lsa_synth_rms_rows_bf16.argtypes = [_P, _I64, _I32, _U64, _U64, _I64, _P]
-    for name in ("lsa_index_scores", "lsa_topk", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
+    for name in ("lsa_index_scores", "lsa_topk", "lsa_topk_static", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
                  "lsa_forward", "lsa_index_project", "lsa_block_summaries", "lsa_hier_select", "lsa_device_error",
                  "lsa_sparse_mla_decode_topk", "lsa_loza_mla", "lsa_abi_version", "lsa_synth_normal_bf16",
                  "lsa_synth_normal_f32", "lsa_synth_rms_rows_bf16"):
@@ -227,6 +230,16 @@ def topk(cfg, pos, max_len, scores, idx, count, ws, stream=None, bind=False, top
         ctypes.byref(cfg._c()), pos.shape[0], _ptr(pos), int(max_len), _ptr(scores), scores.shape[1],
         _ptr(topk_hist), _ptr(idx), _ptr(count), _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
         allow_dense=True, bind=bind)
+
+
+def topk_static(cfg, pos, max_len, scores, idx, count, stream=None, bind=False):
+    """topk without a workspace: the library's built-in scratch (at most
+    TOPK_STATIC_MAX_ROWS rows; calls that overlap on the GPU race on it)."""
+    _dt(scores, torch.float32, "scores"); _dt(pos, torch.int32, "pos")
+    _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
+    return _invoke(load().lsa_topk_static, (
+        ctypes.byref(cfg._c()), pos.shape[0], _ptr(pos), int(max_len), _ptr(scores), scores.shape[1],
+        _ptr(idx), _ptr(count), _stream(stream)), allow_dense=True, bind=bind)
 
 
 def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None, bind=False,

@@ -327,6 +327,83 @@ def test_tiny_config_whole_row():
 
 
 # --------------------------------------------------------------------------
+# MTP draft round: the draft steps share one index pass
+# ([LSA-2.0] 多token预测模块集成)
+# --------------------------------------------------------------------------
+def _tagged_latent(L):
+    # V[j] = e_j: with q = 0 the output is the mean of the attended keys' tags
+    c = np.zeros((L, 576))
+    c[np.arange(L), np.arange(L)] = 1.0
+    return c
+
+
+def test_mtp_round_hand_worked_tiny():
+    # Tiny config (topk 8, init 2, local 4), 15 cached keys, first draft step at
+    # p = 11 (12 visible keys > 8: sparse). One index head with weight 1 and
+    # q = e_0 makes score_j = max(k[j, 0], 0). Worked by hand: the forced columns
+    # are the sinks {0, 1} and the local window {8, 9, 10, 11}; of the middle
+    # columns 2..7 the two best are 3 (5.0) and 6 (4.0). Step 0 attends over
+    # that set; step 1 (query at 12) adds key 12; step 2 (query at 13) adds 12
+    # and 13. Key 14 is never attended (no draft has reached it).
+    L, p = 15, 11
+    q = np.zeros((32, 128)); q[0, 0] = 1.0
+    w = np.zeros(32); w[0] = 1.0
+    k = np.zeros((L, 128))
+    k[:, 0] = [0.1, 0.2, 0.3, 5.0, 0.5, 0.6, 4.0, 0.7, 9.0, 9.0, 9.0, 9.0, 9.0, 9.0, 9.0]
+    lat = _tagged_latent(L)
+    sel, dense, outs = R.mtp_round(q, w, k, p, [np.zeros((32, 576))] * 3, lat, TINY)
+    assert not dense
+    np.testing.assert_array_equal(sel, [0, 1, 3, 6, 8, 9, 10, 11])
+    sets = [[0, 1, 3, 6, 8, 9, 10, 11], [0, 1, 3, 6, 8, 9, 10, 11, 12], [0, 1, 3, 6, 8, 9, 10, 11, 12, 13]]
+    for i, keys in enumerate(sets):
+        expect = np.zeros(512)
+        expect[keys] = 1.0 / len(keys)
+        np.testing.assert_allclose(outs[i][0], np.tile(expect, (32, 1)), atol=1e-15)
+        np.testing.assert_allclose(outs[i][1], np.full(32, math.log(len(keys))), rtol=1e-14)
+
+
+def test_mtp_round_dense_steps_are_dense_attention():
+    # p + 1 <= topk: no selection; step i is plain softmax attention over keys
+    # 0 .. p+i, checked against torch's attention on those keys.
+    L, p = 140, 100
+    r = np.random.default_rng(3)
+    q, w, k = r.standard_normal((32, 128)), r.standard_normal(32), r.standard_normal((L, 128))
+    qs = [r.standard_normal((32, 576)) for _ in range(3)]
+    lat = r.standard_normal((L, 576))
+    sel, dense, outs = R.mtp_round(q, w, k, p, qs, lat, PAGES)
+    assert dense and np.array_equal(sel, np.arange(p + 1))
+    for i in range(3):
+        c = lat[: p + 1 + i]
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            torch.from_numpy(qs[i])[None, :, None, :], torch.from_numpy(c)[None, None].expand(1, 32, -1, -1),
+            torch.from_numpy(c[:, :512])[None, None].expand(1, 32, -1, -1), scale=PAGES.softmax_scale)
+        np.testing.assert_allclose(outs[i][0], ref[0, :, 0].numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_mtp_round_shares_the_first_steps_selection():
+    # pages' constants, sparse: every step reuses step 0's selection (made at p,
+    # forced window p-1023 .. p) and adds only its new keys; step 0 is the
+    # layer path's sub-block. A step that ran its own index pass would drop
+    # p-1023 .. p-1023+i from its window; one that skipped its new keys would
+    # miss p+1 .. p+i: the tagged values show both.
+    p, L = 3000, 3003
+    r = np.random.default_rng(4)
+    q, w, k = r.standard_normal((32, 128)), r.standard_normal(32) / math.sqrt(32), r.standard_normal((L, 128))
+    lat = np.zeros((L, 576))
+    lat[np.arange(L), np.arange(L) % 512] = 1.0
+    sel, dense, outs = R.mtp_round(q, w, k, p, [np.zeros((32, 576))] * 3, lat, PAGES)
+    sel0, _, outs0 = R.lsa_row(q, w, k[: p + 1], p, [np.zeros((32, 576))], [lat[: p + 1]], PAGES)
+    np.testing.assert_array_equal(sel, sel0)
+    np.testing.assert_array_equal(outs[0][0], outs0[0][0])
+    assert not dense and {p - 1023, p} <= set(sel.tolist()) and sel.max() == p
+    for i in range(3):
+        keys = np.concatenate([sel, np.arange(p + 1, p + 1 + i)])
+        expect = np.zeros(512)
+        np.add.at(expect, keys % 512, 1.0 / len(keys))
+        np.testing.assert_allclose(outs[i][0][0], expect, atol=1e-15)
+
+
+# --------------------------------------------------------------------------
 # Indexer projection (upstream of the path): RoPE, RMSNorm, the projections.
 # --------------------------------------------------------------------------
 def test_rope_closed_form_frequencies():
