@@ -156,6 +156,7 @@ def peaks():
 
 # the decode indexer's code: its kernel and its key-tile helpers
 INDEX_DECODE_SOURCES = ("index_decode.cu", "index_tile.cuh")
+INDEX_PREFILL_SOURCES = ("index_prefill.cu",)
 
 
 def source_sha(srcs) -> str:
@@ -292,35 +293,48 @@ def build_decode(device):
     idx = torch.empty((B, 2048), dtype=torch.int32, device=device)
     cnt = torch.empty((B,), dtype=torch.int32, device=device)
     tk_ws = lsa.workspace(cfg, lsa.OP_TOPK, B, B, ctx, device=device)
-    mla_ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE, B, B, ctx, device=device)
+    mla_ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE_LAYER, B, B, ctx, device=device)
+    mtp_ws = lsa.workspace(cfg, lsa.OP_MTP_DECODE, B, B, ctx, device=device)
     hist = lsa.topk_hist_buffer(B, device=device)
     D = dict(layers=layers, q_idx=q_idx, w=w, q_abs=q_abs, out=out, lse=lse, cfg=cfg, ws=ws, scores=scores,
-             idx=idx, cnt=cnt, tk_ws=tk_ws, mla_ws=mla_ws, ctx=ctx, hist=hist)
+             idx=idx, cnt=cnt, tk_ws=tk_ws, mla_ws=mla_ws, mtp_ws=mtp_ws, ctx=ctx, hist=hist)
     # Marshal every call once: the timed loops only cross the C-ABI.
     D["calls"] = []
+    D["two_launch"] = []
     D["fwd"] = []
     for i, l in enumerate(layers):
         D["calls"].append((
             lsa.index_scores(cfg, l.seq_of_row, l.pos, l.q_idx, l.w, l.k_idx, l.k_off, ctx, scores, bind=True,
                              topk_hist=hist),
             lsa.topk(cfg, l.pos, ctx, scores, idx, cnt, tk_ws, bind=True, topk_hist=hist),
-            [lsa.sparse_mla_decode(cfg, l.q_abs[z], l.latent[z], l.k_off, idx, cnt, ctx, out[i, z], lse[i, z],
-                                   mla_ws, bind=True, lists_from_topk=True) for z in range(2)]))
+            lsa.sparse_mla_decode_layer(cfg, l.q_abs, l.latent, l.k_off, idx, cnt, ctx, [out[i, 0], out[i, 1]],
+                                        [lse[i, 0], lse[i, 1]], mla_ws, bind=True)))
+        # the same sub-blocks as two launches (a model whose second sub-block's
+        # query waits for the first one's output)
+        D["two_launch"].append([lsa.sparse_mla_decode(cfg, l.q_abs[z], l.latent[z], l.k_off, idx, cnt, ctx,
+                                                      out[i, z], lse[i, z], mla_ws, bind=True, lists_from_topk=True)
+                                for z in range(2)])
         D["fwd"].append(lsa.forward(cfg, 0, l.seq_of_row, l.pos, ctx, l.q_idx, l.w, l.k_idx, l.k_off, l.q_abs,
                                     l.latent, [out[i, 0], out[i, 1]], [lse[i, 0], lse[i, 1]], ws, bind=True))
-    # MTP draft round: one index pass shared by three draft steps, each attending
-    # over the same latent cache with its own absorbed query
+    # MTP draft round: the index pass and top-k once, for the first draft step's
+    # query at position ctx - 3; the three draft steps (queries at ctx - 3,
+    # ctx - 2, ctx - 1, each also seeing the later keys up to its own) in one
+    # launch over one latent cache
     q3 = torch.empty((nl, B, 32, 576), dtype=torch.bfloat16, device=device)
     for i in range(nl):
         lsa.synth_normal_bf16(q3[i], 0, 16 * (100 + i) + 3)
-    out3 = torch.empty((B, 32, 512), dtype=torch.bfloat16, device=device)
-    lse3 = torch.empty((B, 32), dtype=torch.float32, device=device)
+    out3 = [torch.empty((B, 32, 512), dtype=torch.bfloat16, device=device) for _ in range(3)]
+    lse3 = [torch.empty((B, 32), dtype=torch.float32, device=device) for _ in range(3)]
+    pos3 = torch.full((B,), ctx - 3, dtype=torch.int32, device=device)
     D["mtp"] = []
     for i, l in enumerate(layers):
-        qs = [l.q_abs[0], l.q_abs[1], q3[i]]
-        D["mtp"].append([lsa.sparse_mla_decode(cfg, qs[st], l.latent[0], l.k_off, idx, cnt, ctx, out3, lse3,
-                                               mla_ws, bind=True, lists_from_topk=True) for st in range(3)])
-    D["q3"] = q3
+        D["mtp"].append((
+            lsa.index_scores(cfg, l.seq_of_row, pos3, l.q_idx, l.w, l.k_idx, l.k_off, ctx, scores, bind=True,
+                             topk_hist=hist),
+            lsa.topk(cfg, pos3, ctx, scores, idx, cnt, tk_ws, bind=True, topk_hist=hist),
+            lsa.mtp_mla_decode(cfg, pos3, [l.q_abs[0], l.q_abs[1], q3[i]], l.latent[0], l.k_off, idx, cnt, ctx,
+                               out3, lse3, mtp_ws, bind=True)))
+    D["mtp_keep"] = (q3, out3, lse3, pos3)
     return D
 
 
@@ -410,12 +424,11 @@ def loza_step(D):
 def hier_step(D, select_only=False):
     """One decode step with hierarchical selection: per layer the newest block's
     summary, the two-stage selection, then both MLA sub-blocks on it."""
-    for h, (_, _, mla_calls) in zip(D["hier"], D["calls"]):
+    for h, (_, _, mla_call) in zip(D["hier"], D["calls"]):
         h["update"]()
         h["select"]()
         if not select_only:
-            for call in mla_calls:
-                call()
+            mla_call()
 
 
 def flat_select_step(D):
@@ -431,24 +444,36 @@ def project_step(D):
 
 def mtp_round(D):
     """One MTP draft round through every layer: the index pass and top-k once,
-    then three draft steps of sparse MLA over that one selection."""
-    for (idx_call, topk_call, _), steps in zip(D["calls"], D["mtp"]):
+    then the three draft steps of sparse MLA over that one selection (one launch)."""
+    for idx_call, topk_call, mtp_call in D["mtp"]:
         idx_call()
         topk_call()
-        for call in steps:
-            call()
+        mtp_call()
 
 
-def decode_step(D, ev=None):
+def decode_step(D, ev=None, mla_ev=None):
     """One decode step through every layer via the C-ABI entry points (index pass,
-    top-k, two sub-blocks of sparse MLA). If `ev` is given, records events on the
-    launching stream around each indexer launch."""
-    for i, (idx_call, topk_call, mla_calls) in enumerate(D["calls"]):
+    top-k, both sub-blocks of sparse MLA in one launch). If `ev` (`mla_ev`) is
+    given, records events on the launching stream around each indexer (attention)
+    launch."""
+    for i, (idx_call, topk_call, mla_call) in enumerate(D["calls"]):
         if ev is not None:
             ev[i][0].record()
         idx_call()
         if ev is not None:
             ev[i][1].record()
+        topk_call()
+        if mla_ev is not None:
+            mla_ev[i][0].record()
+        mla_call()
+        if mla_ev is not None:
+            mla_ev[i][1].record()
+
+
+def decode_step_two_launch(D):
+    """The same step with the two sub-blocks' attention as two launches."""
+    for (idx_call, topk_call, _), mla_calls in zip(D["calls"], D["two_launch"]):
+        idx_call()
         topk_call()
         mla_calls[0]()
         mla_calls[1]()
@@ -475,7 +500,8 @@ def decode_forward_e2e(D, h_in, h_out, pipe):
     with torch.cuda.stream(copy):
         for i in range(len(D["fwd"])):
             copy.wait_event(ev_out[i])
-            h_out[i].copy_(D["out"][i], non_blocking=True)
+            h_out[0][i].copy_(D["out"][i], non_blocking=True)
+            h_out[1][i].copy_(D["lse"][i], non_blocking=True)
     comp.wait_stream(copy)
 
 
@@ -533,7 +559,7 @@ def run_prefill(device, steps, warmup):
     idx_ms = statistics.mean(a.elapsed_time(b) for a, b in ev)
     flops = 2.0 * 32 * 128 * (n * (n + 1) / 2)  # visible (row, key) pairs
     pk, src = peaks()
-    peak = pk.get("bf16_tflops_sustained", pk.get("bf16_tflops"))
+    peak = pk["bf16_tflops"]  # the burst figure: a ~1 ms kernel, not a seconds-long loop
     achieved = flops / (idx_ms / 1e3) / 1e12
     del wl, scores
     torch.cuda.empty_cache()
@@ -541,7 +567,8 @@ def run_prefill(device, steps, warmup):
             "config": {"workload": "prefill_causal_16384", "seq_len": n},
             "roofline": {"kernel": "index_prefill_kernel", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
-                         "peak_source": f"{src} bf16_tflops_sustained", "traffic": None}}
+                         "peak_source": f"{src} bf16_tflops (burst)",
+                         "traffic": kernel_traffic("index_prefill_kernel", INDEX_PREFILL_SOURCES)}}
 
 
 def _forward_case(device, lengths, n_rows=None, q_start=None):
@@ -678,9 +705,27 @@ def gpu_arm(args):
     peak = pk["hbm_gbs"]
     achieved = alg_bytes / (statistics.mean(idx_ms) / 1e3) / 1e9
 
+    # roofline of the attention kernel (both sub-blocks in one launch): events
+    # around each MLA launch in separate untimed steps (an event between two
+    # kernels stops the second from starting early, so the timed steps carry none)
+    mla_ev = events()
+    for _ in range(3):
+        decode_step(D, mla_ev=mla_ev)
+    torch.cuda.synchronize()
+    mla_ms = statistics.mean(a.elapsed_time(b) for a, b in mla_ev)
+    mla_bytes = B * 2 * (2048 * 1152 + 32 * 576 * 2 + 32 * 512 * 2 + 32 * 4)
+    mla_achieved = mla_bytes / (mla_ms / 1e3) / 1e9
+
+    # the same step with the sub-blocks' attention as two launches
+    for _ in range(3):
+        decode_step_two_launch(D)
+    t2 = time_region(lambda s: decode_step_two_launch(D), args.steps, world, device)
+    two_value, _ = aggregate(units, t2, world, device)
+
     # end-to-end through lsa_forward with pinned host buffers
     h_in = [D["q_idx"].cpu().pin_memory(), D["w"].cpu().pin_memory(), D["q_abs"].cpu().pin_memory()]
-    h_out = torch.empty(D["out"].shape, dtype=D["out"].dtype).pin_memory()
+    h_out = [torch.empty(D["out"].shape, dtype=D["out"].dtype).pin_memory(),
+             torch.empty(D["lse"].shape, dtype=D["lse"].dtype).pin_memory()]
     pipe = (torch.cuda.current_stream(), torch.cuda.Stream(),
             [torch.cuda.Event() for _ in range(nl)], [torch.cuda.Event() for _ in range(nl)])
     for _ in range(max(3, args.warmup // 2)):
@@ -690,7 +735,7 @@ def gpu_arm(args):
     te = time_region(lambda s: decode_forward_e2e(D, h_in, h_out, pipe), e2e_steps, world, device)
     e2e_value, _ = aggregate(B * nl * e2e_steps, te, world, device)
     h2d = sum(x.numel() * x.element_size() for x in h_in)
-    d2h = h_out.numel() * h_out.element_size()
+    d2h = sum(x.numel() * x.element_size() for x in h_out)
 
     # the indexer's own projections and key append for one decode token per sequence
     # (runs after the timed decode step: it rewrites the newest key row of each cache)
@@ -758,7 +803,13 @@ def gpu_arm(args):
                      "traffic": kernel_traffic("index_decode_kernel", INDEX_DECODE_SOURCES),
                      "alg_bytes_per_launch": alg_bytes, "avg_launch_ms": statistics.mean(idx_ms)},
         "e2e": {"value": e2e_value, "unit": "tokens/s/layer", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "roofline_attention": {"kernel": "mla_kernel", "bound": "hbm", "achieved": mla_achieved, "peak": peak,
+                               "unit": "GB/s", "frac": mla_achieved / peak, "peak_source": f"{psrc} hbm_gbs",
+                               "alg_bytes_per_launch": mla_bytes, "avg_launch_ms": mla_ms,
+                               "timing": "events around each launch in 3 untimed steps"},
         "gpu_launches": launches,
+        "two_launch": {"value": two_value, "unit": "tokens/s/layer", "ms_per_step": 1e3 * t2 / args.steps,
+                       "note": "both sub-blocks' attention as two launches (second query after the first output)"},
         "clocks": {k: clocks[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
     }
     line["project"] = {"value": pj_value, "unit": "tokens/s/layer", "us_per_layer": 1e6 * pj_layer_s,

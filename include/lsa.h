@@ -101,6 +101,8 @@ LSA_API void lsa_config_default(lsa_config* cfg);
 #define LSA_OP_FORWARD_DECODE 4
 #define LSA_OP_FORWARD_PREFILL 5
 #define LSA_OP_INDEX_PROJECT 6
+#define LSA_OP_MLA_DECODE_LAYER 7 /* lsa_sparse_mla_decode_layer (cfg->cli_factor sub-blocks) */
+#define LSA_OP_MTP_DECODE 8       /* lsa_mtp_mla_decode (any n_draft) */
 
 /*
  * Bytes of workspace the operation uses at full speed for these sizes (host
@@ -301,6 +303,8 @@ LSA_API lsa_status lsa_hier_select(const lsa_config* cfg, int32_t n_rows, int32_
  * [batch, index_topk]; count int32 [batch]; out bf16 [batch, 32, 512];
  * lse fp32 [batch, 32] or NULL. max_len (host) >= every L_b (sizes split-K).
  * Workspace optional (split-K partials): lsa_workspace_size(LSA_OP_MLA_DECODE).
+ * Calls that may overlap on the GPU must not share a workspace (true of every
+ * MLA entry point).
  */
 /*
  * lsa_sparse_mla_decode_topk: the same attention, for idx / count written by
@@ -327,6 +331,56 @@ LSA_API lsa_status lsa_sparse_mla_decode(const lsa_config* cfg, int32_t batch, c
                                  const lsa_bf16* latent, const int64_t* k_off, const int32_t* idx,
                                  const int32_t* count, int64_t max_len, lsa_bf16* out, float* lse,
                                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * lsa_sparse_mla_decode_layer: the cfg->cli_factor attention sub-blocks of a
+ * layer that share one selection ([Lite-Sparse] LSA section, cross-layer index
+ * reuse: the second sub-block reuses the first one's topk_indices; [LSA-2.0]
+ * 跨层索引), in one launch. Sub-block z attends with its own queries q_abs[z]
+ * over its own latent cache latent[z] (both packed by the same k_off) and
+ * writes out[z] / lse[z], exactly as lsa_sparse_mla_decode_topk would for each
+ * z; idx / count must come from lsa_topk, lsa_forward or lsa_hier_select
+ * (forced columns first), and the same early start before the top-k applies.
+ * q_abs, latent, out, lse: HOST arrays of cli_factor DEVICE pointers (lse
+ * itself or its entries may be NULL). All sub-blocks' queries must be ready at
+ * the call: a model whose second sub-block's query depends on the first one's
+ * output calls lsa_sparse_mla_decode_topk once per sub-block instead.
+ * Workspace: lsa_workspace_size(LSA_OP_MLA_DECODE_LAYER, batch, batch, max_len).
+ */
+LSA_API lsa_status lsa_sparse_mla_decode_layer(const lsa_config* cfg, int32_t batch, const lsa_bf16* const* q_abs,
+                                               const lsa_bf16* const* latent, const int64_t* k_off,
+                                               const int32_t* idx, const int32_t* count, int64_t max_len,
+                                               lsa_bf16* const* out, float* const* lse, void* ws, size_t ws_bytes,
+                                               void* stream);
+
+/*
+ * lsa_mtp_mla_decode: the draft steps of one multi-token-prediction round over
+ * one shared index pass ([LSA-2.0] 多token预测模块集成: the method extends to
+ * a three-step MTP module for speculative decoding, and all draft steps share
+ * a single index pass), in one launch. The page says only that the pass is
+ * shared; reading taken: the index pass and top-k ran once, for the first
+ * draft step's query of sequence b at position pos[b] (idx / count from
+ * lsa_topk / lsa_forward with that pos, forced columns first). Draft step i
+ * (0 <= i < n_draft) has its query at position pos[b] + i; the keys
+ * pos[b]+1 .. pos[b]+i (the earlier drafts' and its own) are already in the
+ * cache, and a query sees its own key, so step i attends over the shared
+ * selection plus those i keys:
+ *   out[i][b] = attention of q_abs[i][b] over latent[k_off[b] + j],
+ *               j in {idx[b, :count[b]]} U {pos[b]+1 .. pos[b]+i}.
+ * All steps read the one latent cache `latent` (the MTP module's), packed by
+ * k_off; every sequence must hold keys through pos[b] + n_draft - 1 (a step
+ * whose keys run past the sequence sets LSA_DEVERR_POS and attends only to the
+ * keys present). 1 <= n_draft <= 4. q_abs, out, lse: HOST arrays of n_draft
+ * DEVICE pointers (q_abs[i] bf16 [batch, 32, 576], out[i] bf16 [batch, 32,
+ * 512], lse[i] fp32 [batch, 32]; lse or its entries may be NULL). pos int32
+ * [batch] (device). Workspace: lsa_workspace_size(LSA_OP_MTP_DECODE, batch,
+ * batch, max_len).
+ */
+LSA_API lsa_status lsa_mtp_mla_decode(const lsa_config* cfg, int32_t n_draft, int32_t batch, const int32_t* pos,
+                                      const lsa_bf16* const* q_abs, const lsa_bf16* latent, const int64_t* k_off,
+                                      const int32_t* idx, const int32_t* count, int64_t max_len,
+                                      lsa_bf16* const* out, float* const* lse, void* ws, size_t ws_bytes,
+                                      void* stream);
 
 /*
  * Sparse absorbed-latent MLA, prefill ([Lite-Sparse] LSA section: at prefill
@@ -410,6 +464,19 @@ LSA_API lsa_status lsa_device_error(int32_t* flags);
 /* Number of kernels this library has launched in the process so far (host
  * counter, no CUDA call). Used to count the launches inside a timed region. */
 LSA_API int64_t lsa_launch_count(void);
+
+/*
+ * Test hook for the bounded waits of the sparse-MLA kernel (no counterpart in
+ * the pages; never needed in normal use). Arms the next sparse-MLA launch made
+ * by this host thread, and only that one: every CTA's producer stops handing
+ * key tiles to the ring before tile drop_tile (-1: it does not stop), and the
+ * attention warps give up any wait after wait_ns nanoseconds (0: the normal
+ * 2 s). A wait for a tile that was never issued then runs out: the kernel
+ * returns with garbage output for those rows, sets LSA_DEVERR_TIMEOUT, and
+ * every copy it did issue has landed before it exits, so the device stays
+ * usable. Tests use it to exercise the timeout report.
+ */
+LSA_API void lsa_debug_arm_mla_wait_test(int64_t wait_ns, int32_t drop_tile);
 
 /* ABI version of this header (1). */
 LSA_API int32_t lsa_abi_version(void);

@@ -109,21 +109,27 @@ struct ProjectLaunch {
 size_t project_ws_bytes(int n_rows);
 cudaError_t launch_index_project(const ProjectLaunch& L, cudaStream_t st);
 
+constexpr int kMaxSub = 4;  // sub-blocks (or MTP draft steps) of one MLA launch
 struct MlaArgs {
-  const uint16_t* q[2];
-  const uint16_t* lat[2];
-  uint16_t* out[2];
-  float* lse[2];
+  // Per sub-block z < n_sub (grid z): its queries, latent cache, outputs.
+  const uint16_t* q[kMaxSub];
+  const uint16_t* lat[kMaxSub];
+  uint16_t* out[kMaxSub];
+  float* lse[kMaxSub];
   const int64_t* k_off;      // decode: [n_seq+1]
   const int32_t* seq_of_row; // decode: row -> sequence (null: identity)
   const int32_t* pos;        // prefill: required; decode: optional (null: the whole sequence)
   const int32_t* idx;        // [n_rows, topk] or null (dense)
   const int32_t* count;
-  int n_rows, n_seq, topk, decode, cli;
+  int n_rows, n_seq, topk, decode, n_sub;
   // The index lists were written by the top-k for these rows (every non-dense
   // row's list starts with its n_init sink and n_loc local columns): the kernel
   // attends over those before it waits for the previous kernel in the stream.
   int forced_first = 0, n_init = 0, n_loc = 0;
+  // MTP draft steps (forced-first lists only): sub-block z is draft step z,
+  // whose query sits z positions after the index owner's; it attends over the
+  // shared list and also over the keys pos+1 .. pos+z.
+  int mtp = 0;
   // LoZA rows (no index list): each row attends to keys [0, loza_sink) and to
   // the run from the earlier of its recent window's and its chunk's first key
   // up to its own position.
@@ -134,10 +140,17 @@ struct MlaArgs {
   void* ws;
   size_t ws_bytes;
   int* err;
+  // Bounded waits: the math warps give up a wait after wait_ns. Test hook:
+  // drop_tile >= 0 makes every CTA's producer stop before that tile, so the
+  // wait for it runs out (the timeout report path); -1 in normal use.
+  long long wait_ns = 2000000000ll;
+  int drop_tile = -1;
 };
-// Split-K partial bytes for a given split count.
-size_t mla_ws_bytes(int n_rows, int cli, int n_split);
-int mla_choose_splits(int n_rows, int cli, int64_t max_list, bool forced_first = false);
+// Split-K workspace bytes (partials and merge tickets) for a given split count.
+size_t mla_ws_bytes(int n_rows, int n_sub, int n_split);
+int mla_choose_splits(int n_rows, int n_sub, int64_t max_list, bool forced_first = false);
+// Arms the next launch_mla on this host thread with the test hook above.
+void mla_arm_wait_test(long long wait_ns, int drop_tile);
 cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st);
 
 }  // namespace lsa

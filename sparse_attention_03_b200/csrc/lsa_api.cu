@@ -83,8 +83,10 @@ size_t topk_ws(int n_rows, int64_t max_len = 0) {
   return (size_t)std::min(n_rows, kTopkPreferredRows) * per + kAlign;
 }
 
-size_t mla_ws(int n_rows, int cli, int64_t max_list) {
-  return mla_ws_bytes(n_rows, cli, mla_choose_splits(n_rows, cli, max_list));
+// Split-K workspace of the MLA launch, whichever split count it picks.
+size_t mla_ws(int n_rows, int n_sub, int64_t max_list) {
+  return std::max(mla_ws_bytes(n_rows, n_sub, mla_choose_splits(n_rows, n_sub, max_list, false)),
+                  mla_ws_bytes(n_rows, n_sub, mla_choose_splits(n_rows, n_sub, max_list, true)));
 }
 
 // Workspace of one forward block of R rows (sparse path).
@@ -174,10 +176,10 @@ lsa_status run_topk(const lsa_config* c, int n_rows, const int32_t* pos, int64_t
   return max_len <= c->index_topk ? LSA_DENSE : LSA_OK;
 }
 
-MlaArgs mla_args(const lsa_config* c, int cli, int n_rows, int decode) {
+MlaArgs mla_args(const lsa_config* c, int n_sub, int n_rows, int decode) {
   MlaArgs a = {};
   a.n_rows = n_rows;
-  a.cli = cli;
+  a.n_sub = n_sub;
   a.decode = decode;
   a.topk = c->index_topk;
   a.scale = c->softmax_scale;
@@ -273,6 +275,10 @@ size_t lsa_workspace_size(const lsa_config* c, int32_t op, int32_t n_rows, int32
       return forward_block_ws(c, prefill_block_rows(n_rows, max_len), max_len) + kAlign;
     case LSA_OP_INDEX_PROJECT:
       return project_ws_bytes(n_rows) + kAlign;
+    case LSA_OP_MLA_DECODE_LAYER:
+      return mla_ws(n_rows, c->cli_factor, list) + kAlign;
+    case LSA_OP_MTP_DECODE:
+      return mla_ws(n_rows, kMaxSub, list) + kAlign;
     default:
       return 0;
   }
@@ -429,6 +435,78 @@ lsa_status lsa_sparse_mla_decode_topk(const lsa_config* c, int32_t batch, const 
                                       void* ws, size_t ws_bytes, void* stream) {
   return mla_decode("lsa_sparse_mla_decode_topk", true, c, batch, q_abs, latent, k_off, idx, count, max_len, out,
                     lse, ws, ws_bytes, stream);
+}
+
+}  // extern "C"
+
+namespace {
+// Sub-blocks over one shared forced-first selection in one launch: the
+// cli_factor sub-blocks of a layer (mtp 0), or the draft steps of an MTP round
+// (mtp 1: step z also sees keys pos+1 .. pos+z).
+lsa_status mla_decode_shared(const char* fn, const lsa_config* c, int n_sub, int mtp, int32_t batch,
+                             const int32_t* pos, const lsa_bf16* const* q_abs, const lsa_bf16* const* latent,
+                             const int64_t* k_off, const int32_t* idx, const int32_t* count, int64_t max_len,
+                             lsa_bf16* const* out, float* const* lse, void* ws, size_t ws_bytes, void* stream) {
+  if (batch < 0 || max_len < 1) return set_error(LSA_ERR_INVALID, "%s: need batch >= 0, max_len >= 1", fn);
+  if (batch == 0) return LSA_OK;
+  if (!q_abs || !latent || !out || !k_off || !idx || !count || (mtp && !pos))
+    return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  MlaArgs a = mla_args(c, n_sub, batch, 1);
+  for (int z = 0; z < n_sub; ++z) {
+    const lsa_bf16* lat = latent[mtp ? 0 : z];
+    if (!q_abs[z] || !lat || !out[z]) return set_error(LSA_ERR_INVALID, "%s: NULL pointer for sub-block %d", fn, z);
+    if (!aligned16(q_abs[z]) || !aligned16(lat) || !aligned16(out[z]))
+      return set_error(LSA_ERR_INVALID, "%s: q_abs, latent and out must be 16-byte aligned", fn);
+    a.q[z] = q_abs[z];
+    a.lat[z] = lat;
+    a.out[z] = out[z];
+    a.lse[z] = lse ? lse[z] : nullptr;
+  }
+  a.k_off = k_off;
+  a.n_seq = batch;
+  a.pos = pos;
+  a.idx = idx;
+  a.count = count;
+  a.max_list = c->index_topk;
+  a.forced_first = 1;
+  a.n_init = c->index_init_tokens;
+  a.n_loc = c->index_local_tokens;
+  a.mtp = mtp;
+  a.ws = ws;
+  a.ws_bytes = ws ? ws_bytes : 0;
+  return cuda_status(launch_mla(a, (cudaStream_t)stream), fn);
+}
+}  // namespace
+
+extern "C" {
+
+lsa_status lsa_sparse_mla_decode_layer(const lsa_config* c, int32_t batch, const lsa_bf16* const* q_abs,
+                                       const lsa_bf16* const* latent, const int64_t* k_off, const int32_t* idx,
+                                       const int32_t* count, int64_t max_len, lsa_bf16* const* out,
+                                       float* const* lse, void* ws, size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_sparse_mla_decode_layer";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  return mla_decode_shared(fn, c, c->cli_factor, 0, batch, nullptr, q_abs, latent, k_off, idx, count, max_len, out,
+                           lse, ws, ws_bytes, stream);
+}
+
+lsa_status lsa_mtp_mla_decode(const lsa_config* c, int32_t n_draft, int32_t batch, const int32_t* pos,
+                              const lsa_bf16* const* q_abs, const lsa_bf16* latent, const int64_t* k_off,
+                              const int32_t* idx, const int32_t* count, int64_t max_len, lsa_bf16* const* out,
+                              float* const* lse, void* ws, size_t ws_bytes, void* stream) {
+  const char* fn = "lsa_mtp_mla_decode";
+  lsa_status s = check_cfg(c, fn);
+  if (s != LSA_OK) return s;
+  if (n_draft < 1 || n_draft > kMaxSub)
+    return set_error(LSA_ERR_UNSUPPORTED, "%s: n_draft must be in [1, %d]", fn, kMaxSub);
+  const lsa_bf16* lat[kMaxSub] = {latent};
+  return mla_decode_shared(fn, c, n_draft, 1, batch, pos, q_abs, lat, k_off, idx, count, max_len, out, lse, ws,
+                           ws_bytes, stream);
+}
+
+void lsa_debug_arm_mla_wait_test(int64_t wait_ns, int32_t drop_tile) {
+  mla_arm_wait_test((long long)wait_ns, (int)drop_tile);
 }
 
 lsa_status lsa_sparse_mla_prefill(const lsa_config* c, int32_t n_rows, const int32_t* pos,

@@ -22,8 +22,11 @@
 // with the 512 value dims split across the warps (64 each, fp32 accumulators in
 // registers). A row's key list is cut into splits of whole tiles, balanced per
 // row; with more than one split the CTA writes an unnormalised partial
-// (O, m, l) and a merge kernel combines the splits; with one split it writes
-// bf16 output and lse directly. Gathered indices are bounds-checked against the
+// (O, m, l) and one merge kernel combines the splits of every row and
+// sub-block; with one split it writes bf16 output and lse directly. The
+// sub-blocks that share a selection (or the MTP draft steps that share one)
+// are the grid's third dimension, so one attention launch and at most one
+// merge launch cover them all. Gathered indices are bounds-checked against the
 // row's visible keys; every wait is bounded.
 #include "common.cuh"
 #include "kernels.h"
@@ -105,20 +108,42 @@ __device__ __forceinline__ void stagger_wait() { asm volatile("bar.sync 4, %0;\n
 // from the list with the selected ones, which the top-k wrote in the same
 // order, so a sparse row of 2048 keys is 64 full tiles (1024 + 1024 keys), not
 // 65 with two part tiles. ub = the first slot read from the list.
+// An MTP draft step's newer keys (p.ext of them) are known as well: a dense
+// row's known run simply continues past its position; a sparse row gets one
+// more known tile after its forced ones.
 struct FfTiles {
   int kt0, kt, ut0, ut;
   int64_t ub;
+  int kf;  // known tiles holding forced (or dense) keys; a known tile kf holds the extra keys
 };
 __device__ __forceinline__ FfTiles ff_tiles(const ListPlan& p, int s, int n) {
-  const int Kt = (int)(p.dense ? (p.K + kTK - 1) / kTK : p.K / kTK);
   FfTiles f;
-  f.ub = min64((int64_t)Kt * kTK, p.L);
+  f.kf = (int)(p.dense ? (p.K + p.ext + kTK - 1) / kTK : p.K / kTK);
+  const int Kt = f.kf + (!p.dense && p.ext > 0 ? 1 : 0);
+  f.ub = min64((int64_t)f.kf * kTK, p.L);
   const int Ut = (int)((p.L - f.ub + kTK - 1) / kTK);
   f.kt0 = Kt * s / n;
   f.kt = Kt * (s + 1) / n - f.kt0;
   f.ut0 = Ut * s / n;
   f.ut = Ut * (s + 1) / n - f.ut0;
   return f;
+}
+// The key of known slot sl (-1: masked).
+__device__ __forceinline__ int known_slot_key(const ListPlan& p, const FfTiles& f, const MlaArgs& a, int64_t sl) {
+  if (p.dense) return sl < p.K + p.ext ? (int)sl : -1;
+  if (sl < (int64_t)f.kf * kTK) return sl < p.K ? (int)known_key(p, a, sl) : -1;
+  const int64_t e = sl - (int64_t)f.kf * kTK;
+  return e < p.ext ? (int)(p.nvis + e) : -1;
+}
+// Extra keys of sub-block z of an MTP launch, clipped to the sequence (flagged).
+__device__ __forceinline__ int mtp_ext(const MlaArgs& a, const RowGeom& g, int z, bool report) {
+  if (!a.mtp || g.nvis <= 0) return 0;
+  int e = z;
+  if (g.nvis + e > g.klen) {
+    if (report) flag_error(a.err, LSA_DEVERR_POS);
+    e = (int)max64(0, g.klen - g.nvis);
+  }
+  return e;
 }
 
 // Warp roles (math warps 0..7): head half mt = w >> 2 (heads 16mt .. 16mt+15)
@@ -164,13 +189,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     mbar_expect_tx(&sm.qbar, kRowBytes);
     bulk_row(&sm.q[lane * kSRow], qg, &sm.qbar);
     const RowGeom geo = row_base(a, r, false);
-    const ListPlan lp = list_plan(a, geo.nvis);
+    const ListPlan lp = list_plan(a, geo.nvis, mtp_ext(a, geo, z, false));
     const FfTiles ft = ff_tiles(lp, s, sp.n_split);
-    const int n_tiles = ft.kt + ft.ut;
     const uint16_t* __restrict__ latb = a.lat[z] + geo.kbase * kDLat;
+    int issued = 0;  // tiles handed to the ring (all of them unless the test hook stops early)
     auto issue = [&](int tt, int key) {
+      if (tt == a.drop_tile) return false;
       const int i = tt % kStages;
-      if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag);
+      if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag, a.wait_ns);
       sm.keys[i][lane] = key;
       uint16_t* dst = &sm.k[i][lane * kSRow];
       if (key >= 0) {
@@ -182,12 +208,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
         fence_proxy_async();
         mbar_arrive(&sm.full[i]);
       }
+      ++issued;
+      return true;
     };
-    // the known slots (forced columns, or a dense row's whole list): keys by formula
-    for (int tt = 0; tt < ft.kt; ++tt) {
-      const int64_t sl = (int64_t)(ft.kt0 + tt) * kTK + lane;
-      issue(tt, sl < lp.K ? (int)known_key(lp, a, sl) : -1);
-    }
+    // the known slots (forced columns, or a dense row's whole list, then any
+    // MTP extra keys): keys by formula
+    bool go = true;
+    for (int tt = 0; go && tt < ft.kt; ++tt)
+      go = issue(tt, known_slot_key(lp, ft, a, (int64_t)(ft.kt0 + tt) * kTK + lane));
     // the selected slots: the top-k's list, after it has finished
     pdl_wait();
     int c = a.count[r];
@@ -195,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     const int64_t uend = max64(lp.K, min64((int64_t)c, lp.L));
     const int32_t* __restrict__ irow = a.idx + (int64_t)r * a.topk;
     constexpr int kBatch = 8;  // tiles whose indices are requested together
-    for (int u0 = 0; u0 < ft.ut; u0 += kBatch) {
+    for (int u0 = 0; go && u0 < ft.ut; u0 += kBatch) {
       int key[kBatch];
       bool listed[kBatch];
 #pragma unroll
@@ -210,13 +238,14 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
           flag_error(a.err, LSA_DEVERR_INDEX);
           key[j] = -1;
         }
-        if (u0 + j < ft.ut) issue(ft.kt + u0 + j, key[j]);
+        if (go && u0 + j < ft.ut) go = issue(ft.kt + u0 + j, key[j]);
       }
     }
+    // Retire only after every copy into this CTA's shared memory has landed.
     if (lane == 0) {
       mbar_drain(&sm.qbar, 0);
-      for (int i = 0; i < kStages && i < n_tiles; ++i) {
-        const int last = i + ((n_tiles - 1 - i) / kStages) * kStages;
+      for (int i = 0; i < kStages && i < issued; ++i) {
+        const int last = i + ((issued - 1 - i) / kStages) * kStages;
         mbar_drain(&sm.full[i], (last / kStages) & 1);
       }
     }
@@ -269,14 +298,16 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     const int n_tiles = (nk + kTK - 1) / kTK;
     const uint16_t* __restrict__ latb = a.lat[z] + geo.kbase * kDLat;
     const LozaSpan zs = a.loza ? loza_span(a, geo.nvis) : LozaSpan{0, 0};
-    for (int base = 0; base < n_tiles; base += kStages) {
+    // tiles handed to the ring: all of them unless the test hook stops early
+    const int issued = a.drop_tile >= 0 ? min(n_tiles, a.drop_tile) : n_tiles;
+    for (int base = 0; base < issued; base += kStages) {
 #pragma unroll
       for (int i = 0; i < kStages; ++i) {
         const int tt = base + i;
-        if (tt < n_tiles) {
+        if (tt < issued) {
           const int sl = tt * kTK + lane;
           const int key = sl >= nk ? -1 : irow ? sm.list[sl] : (int)(a.loza ? loza_key(zs, b0 + sl) : b0 + sl);
-          if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag);
+          if (tt >= kStages) mbar_wait(&sm.empty[i], ((tt / kStages) - 1) & 1, abort_flag, a.wait_ns);
           sm.keys[i][lane] = key;
           uint16_t* dst = &sm.k[i][lane * kSRow];
           if (key >= 0) {
@@ -295,8 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     // Retire only after every copy into this CTA's shared memory has landed.
     if (lane == 0) {
       mbar_drain(&sm.qbar, 0);
-      for (int i = 0; i < kStages && i < n_tiles; ++i) {
-        const int last = i + ((n_tiles - 1 - i) / kStages) * kStages;
+      for (int i = 0; i < kStages && i < issued; ++i) {
+        const int last = i + ((issued - 1 - i) / kStages) * kStages;
         mbar_drain(&sm.full[i], (last / kStages) & 1);
       }
     }
@@ -307,7 +338,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   int n_tiles;
   if (ff) {
     const RowGeom geo = row_base(a, r, s == 0 && tid == 0);
-    const FfTiles ft = ff_tiles(list_plan(a, geo.nvis), s, sp.n_split);
+    const FfTiles ft = ff_tiles(list_plan(a, geo.nvis, mtp_ext(a, geo, z, s == 0 && tid == 0)), s, sp.n_split);
     n_tiles = ft.kt + ft.ut;
   } else {
     const RowGeom geo = row_geometry(a, r, s == 0 && tid == 0);
@@ -316,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   }
   const int g = lane >> 2, t = lane & 3;
   const int mt = warp >> 2, kq = warp & 3;
-  mbar_wait(&sm.qbar, 0, abort_flag);
+  mbar_wait(&sm.qbar, 0, abort_flag, a.wait_ns);
   // Q fragments of this warp: heads 16mt .. 16mt+15, k16 steps 9kq .. 9kq+8.
   uint32_t qf[9][4];
   {
@@ -345,7 +376,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   if (mt == 1 && n_tiles > 0) stagger_wait();
   for (int tt = 0; tt < n_tiles; ++tt) {
     const int st = tt % kStages;
-    mbar_wait(&sm.full[st], (tt / kStages) & 1, abort_flag);
+    mbar_wait(&sm.full[st], (tt / kStages) & 1, abort_flag, a.wait_ns);
     const uint16_t* kt = sm.k[st];
 
     // ---- partial logits over this warp's dim quarter ----
@@ -540,34 +571,58 @@ __global__ void __launch_bounds__(128) mla_merge_kernel(MlaArgs a, Split sp, con
 
 }  // namespace
 
-size_t mla_ws_bytes(int n_rows, int cli, int n_split) {
+size_t mla_ws_bytes(int n_rows, int n_sub, int n_split) {
   if (n_split <= 1) return 0;
   const size_t per = (size_t)kH * kDV * sizeof(float) + (size_t)kH * sizeof(float2);
-  return (size_t)n_rows * cli * n_split * per + 256;
+  return (size_t)n_rows * n_sub * n_split * per + 256;
 }
 
-int mla_choose_splits(int n_rows, int cli, int64_t max_list, bool forced_first) {
+int mla_choose_splits(int n_rows, int n_sub, int64_t max_list, bool forced_first) {
   // One wave at one CTA per SM: split the rows' key lists until the CTAs cover
   // the SMs, keeping at least four tiles per split (the ring's depth) and at
   // most kMaxSplits splits. With forced-first lists the CTAs start while the
   // top-k is still finishing, which holds one SM per row (its last CTA): leave
-  // those SMs out, so that no CTA starts only after the top-k.
+  // those SMs out, so that no CTA starts only after the top-k, unless that
+  // would leave more SMs idle than the late CTAs cost (at most an eighth of
+  // the CTAs start late).
   int sms = 148;
   int dev = 0;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (forced_first) sms = max(sms - n_rows, sms / 2);
-  const int64_t work = max64((int64_t)n_rows * cli, 1);
+  const int64_t work = max64((int64_t)n_rows * n_sub, 1);
+  int64_t per = sms / work;
+  if (forced_first) {
+    const int64_t free_sms = max(sms - n_rows, sms / 2);
+    const int64_t reserved = free_sms / work;
+    if (per > reserved && per * work - free_sms > per * work / 8) per = reserved;
+  }
   const int64_t by_len = (max_list + kStages * kTK - 1) / (kStages * kTK);
-  int64_t n = min64(by_len, sms / work);
+  int64_t n = min64(by_len, per);
   n = max64(1, min64(n, kMaxSplits));
   return (int)n;
 }
 
-cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
-  if (a.n_rows <= 0) return cudaSuccess;
-  int n_split = mla_choose_splits(a.n_rows, a.cli, a.max_list, a.forced_first && a.idx);
+namespace {
+thread_local long long t_test_wait_ns = 0;
+thread_local int t_test_drop = -1;
+}  // namespace
+
+void mla_arm_wait_test(long long wait_ns, int drop_tile) {
+  t_test_wait_ns = wait_ns;
+  t_test_drop = drop_tile;
+}
+
+cudaError_t launch_mla(const MlaArgs& a_in, cudaStream_t st) {
+  if (a_in.n_rows <= 0) return cudaSuccess;
+  MlaArgs a = a_in;
+  if (t_test_drop >= 0 || t_test_wait_ns > 0) {  // the armed test hook applies to this launch only
+    a.drop_tile = t_test_drop;
+    if (t_test_wait_ns > 0) a.wait_ns = t_test_wait_ns;
+    t_test_drop = -1;
+    t_test_wait_ns = 0;
+  }
+  int n_split = mla_choose_splits(a.n_rows, a.n_sub, a.max_list, a.forced_first && a.idx);
   // Shrink split-K to what the workspace holds.
-  while (n_split > 1 && mla_ws_bytes(a.n_rows, a.cli, n_split) > a.ws_bytes) --n_split;
+  while (n_split > 1 && mla_ws_bytes(a.n_rows, a.n_sub, n_split) > a.ws_bytes) --n_split;
   Split sp;
   sp.n_split = n_split;
   // With an index list no row has more than topk keys (the shared list's size).
@@ -578,7 +633,7 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
   if (n_split > 1) {
     uintptr_t p = (reinterpret_cast<uintptr_t>(a.ws) + 255) & ~uintptr_t(255);
     part_o = reinterpret_cast<float*>(p);
-    part_ml = reinterpret_cast<float2*>(part_o + (size_t)a.n_rows * a.cli * n_split * kH * kDV);
+    part_ml = reinterpret_cast<float2*>(part_o + (size_t)a.n_rows * a.n_sub * n_split * kH * kDV);
   }
   static bool attr_set[64] = {};
   int dev = 0;
@@ -596,7 +651,7 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
     b.n_rows = a.n_rows;
     if (row0 > 0) {
       // rows beyond 65535 are handled by shifting every per-row pointer
-      for (int z = 0; z < a.cli; ++z) {
+      for (int z = 0; z < a.n_sub; ++z) {
         b.q[z] = a.q[z] + (int64_t)row0 * kH * kDLat;
         b.out[z] = a.out[z] + (int64_t)row0 * kH * kDV;
         b.lse[z] = a.lse[z] ? a.lse[z] + (int64_t)row0 * kH : nullptr;
@@ -613,11 +668,11 @@ cudaError_t launch_mla(const MlaArgs& a, cudaStream_t st) {
       b.k_off = a.k_off + row0;
       b.n_seq = a.n_seq - row0;
     }
-    cudaError_t e = launch_pdl(mla_kernel, dim3(n_split, nr, a.cli), dim3(kThreads), sizeof(MlaSmem), st, b, sp,
-                               part_o, part_ml);
+    cudaError_t e = launch_pdl(mla_kernel, dim3(n_split, nr, a.n_sub), dim3(kThreads), sizeof(MlaSmem), st, b,
+                               sp, part_o, part_ml);
     if (e != cudaSuccess) return e;
     if (n_split > 1) {
-      e = launch_pdl(mla_merge_kernel, dim3(kH, nr, a.cli), dim3(128), 0, st, b, sp, (const float*)part_o,
+      e = launch_pdl(mla_merge_kernel, dim3(kH, nr, a.n_sub), dim3(128), 0, st, b, sp, (const float*)part_o,
                      (const float2*)part_ml);
       if (e != cudaSuccess) return e;
     }

@@ -9,6 +9,7 @@ namespace lsa {
 
 struct RowGeom {
   int64_t kbase, nvis, n_list;
+  int64_t klen;  // keys the row's sequence holds (the bound of MTP's extra keys)
 };
 
 // Where the row's keys live and how many it sees, from the caller's inputs alone
@@ -18,17 +19,23 @@ __device__ __forceinline__ RowGeom row_base(const MlaArgs& a, int r, bool report
 // The list of a row whose index list came from the top-k (forced columns first):
 // the expected length L, its known prefix K (the forced columns, or the whole
 // list of a dense row) and the key of a known slot, all from the position.
+// ext: keys after the row's own position that it also attends to (an MTP draft
+// step's newer keys, nvis .. nvis+ext-1); they follow the list.
 struct ListPlan {
   int64_t L, K;
-  int64_t hi;  // first local-window column (non-dense rows)
+  int64_t hi;    // first local-window column (non-dense rows)
+  int64_t nvis;
+  int ext;
   bool dense;
 };
-__device__ __forceinline__ ListPlan list_plan(const MlaArgs& a, int64_t nvis) {
+__device__ __forceinline__ ListPlan list_plan(const MlaArgs& a, int64_t nvis, int ext = 0) {
   ListPlan p;
   p.dense = nvis <= a.topk;
   p.L = min64(nvis, (int64_t)a.topk);
   p.K = p.dense ? p.L : min64(p.L, (int64_t)a.n_init + a.n_loc);
   p.hi = nvis - a.n_loc;
+  p.nvis = nvis;
+  p.ext = ext;
   return p;
 }
 __device__ __forceinline__ int64_t known_key(const ListPlan& p, const MlaArgs& a, int64_t i) {
@@ -54,7 +61,7 @@ __device__ __forceinline__ int64_t loza_key(const LozaSpan& z, int64_t i) { retu
 
 // Row geometry, with every out-of-range input clamped (and flagged by one thread).
 __device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool report) {
-  RowGeom g{0, 0, 0};
+  RowGeom g{0, 0, 0, 0};
   if (a.decode) {
     const int seq = a.seq_of_row ? a.seq_of_row[r] : r;
     if (seq < 0 || seq >= a.n_seq) {
@@ -62,6 +69,7 @@ __device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool re
     } else {
       g.kbase = a.k_off[seq];
       const int64_t klen = a.k_off[seq + 1] - g.kbase;
+      g.klen = klen;
       g.nvis = klen;
       if (a.pos) {
         int64_t p1 = (int64_t)a.pos[r] + 1;
@@ -73,6 +81,7 @@ __device__ __forceinline__ RowGeom row_geometry(const MlaArgs& a, int r, bool re
       }
     }
   } else {
+    g.klen = a.n_keys;
     int64_t p1 = (int64_t)a.pos[r] + 1;
     if (p1 < 1 || p1 > a.n_keys) {
       if (report) flag_error(a.err, LSA_DEVERR_POS);

@@ -20,7 +20,7 @@ LIB_PATH = os.path.join(_HERE, "liblsa.so")
 LSA_OK, LSA_DENSE = 0, 1
 LSA_ERR_INVALID, LSA_ERR_UNSUPPORTED, LSA_ERR_WORKSPACE, LSA_ERR_CUDA, LSA_ERR_DEVICE = -1, -2, -3, -4, -5
 OP_TOPK, OP_MLA_DECODE, OP_MLA_PREFILL, OP_FORWARD_DECODE, OP_FORWARD_PREFILL = 1, 2, 3, 4, 5
-OP_INDEX_PROJECT = 6
+OP_INDEX_PROJECT, OP_MLA_DECODE_LAYER, OP_MTP_DECODE = 6, 7, 8
 TOPK_HIST_WORDS = 2056
 DEVERR_POS, DEVERR_INDEX, DEVERR_COUNT, DEVERR_SEQ, DEVERR_TIMEOUT = 1, 2, 4, 8, 16
 
@@ -30,7 +30,7 @@ EXPORTS = (
     "lsa_device_error", "lsa_abi_version", "lsa_synth_normal_bf16", "lsa_synth_normal_f32",
     "lsa_synth_rms_rows_bf16", "lsa_launch_count", "lsa_index_project", "lsa_block_summaries",
     "lsa_hier_workspace_size", "lsa_hier_select", "lsa_sparse_mla_decode_topk", "lsa_loza_mla",
-    "lsa_topk_static",
+    "lsa_topk_static", "lsa_sparse_mla_decode_layer", "lsa_mtp_mla_decode", "lsa_debug_arm_mla_wait_test",
 )
 TOPK_STATIC_MAX_ROWS = 64
 HIER_BLOCK, HIER_BLOCKS = 64, 128
@@ -80,6 +80,13 @@ def load():
     lib.lsa_topk_static.argtypes = [ctypes.POINTER(Config), _I32, _P, _I64, _P, _I64, _P, _P, _P]
     lib.lsa_sparse_mla_decode.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _P, _P, _I64, _P, _P, _P, _SZ, _P]
     lib.lsa_sparse_mla_decode_topk.argtypes = lib.lsa_sparse_mla_decode.argtypes
+    _PP = ctypes.POINTER(_P)
+    lib.lsa_sparse_mla_decode_layer.argtypes = [ctypes.POINTER(Config), _I32, _PP, _PP, _P, _P, _P, _I64, _PP, _PP,
+                                                _P, _SZ, _P]
+    lib.lsa_mtp_mla_decode.argtypes = [ctypes.POINTER(Config), _I32, _I32, _P, _PP, _P, _P, _P, _P, _I64, _PP, _PP,
+                                       _P, _SZ, _P]
+    lib.lsa_debug_arm_mla_wait_test.argtypes = [_I64, _I32]
+    lib.lsa_debug_arm_mla_wait_test.restype = None
     lib.lsa_sparse_mla_prefill.argtypes = [ctypes.POINTER(Config), _I32, _P, _P, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P]
     lib.lsa_loza_mla.argtypes = [ctypes.POINTER(Config), ctypes.POINTER(LozaPattern), _I32, _I32, _I32, _P, _P, _P,
                                  _I64, _P, _P, _P, _P, _P, _SZ, _P]
@@ -102,7 +109,8 @@ def load():
     lib.lsa_synth_normal_bf16.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
     lib.lsa_synth_normal_f32.argtypes = [_P, _I64, _U64, _U64, _I64, ctypes.c_double, _P]
     lib.lsa_synth_rms_rows_bf16.argtypes = [_P, _I64, _I32, _U64, _U64, _I64, _P]
-    for name in ("lsa_index_scores", "lsa_topk", "lsa_topk_static", "lsa_sparse_mla_decode", "lsa_sparse_mla_prefill",
+    for name in ("lsa_index_scores", "lsa_topk", "lsa_topk_static", "lsa_sparse_mla_decode",
+                 "lsa_sparse_mla_prefill", "lsa_sparse_mla_decode_layer", "lsa_mtp_mla_decode",
                  "lsa_forward", "lsa_index_project", "lsa_block_summaries", "lsa_hier_select", "lsa_device_error",
                  "lsa_sparse_mla_decode_topk", "lsa_loza_mla", "lsa_abi_version", "lsa_synth_normal_bf16",
                  "lsa_synth_normal_f32", "lsa_synth_rms_rows_bf16"):
@@ -256,6 +264,47 @@ def sparse_mla_decode(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, 
         ctypes.byref(cfg._c()), q_abs.shape[0], _ptr(q_abs), _ptr(latent), _ptr(k_off), _ptr(idx),
         _ptr(count), int(max_len), _ptr(out), _ptr(lse), _ptr(ws), 0 if ws is None else ws.numel(),
         _stream(stream)), bind=bind)
+
+
+def _bf16_list(ts, name):
+    for t in ts:
+        _dt(t, torch.bfloat16, name)
+        _ptr(t)
+
+
+def sparse_mla_decode_layer(cfg, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None, bind=False):
+    """The cfg.cli_factor sub-blocks sharing one top-k selection in one launch
+    (q_abs, latent, out, lse: lists of cli_factor tensors; lse may be None)."""
+    _bf16_list(list(q_abs) + list(latent) + list(out), "q_abs/latent/out")
+    for t in (lse or []):
+        _dt(t, torch.float32, "lse")
+    _dt(k_off, torch.int64, "k_off"); _dt(idx, torch.int32, "idx"); _dt(count, torch.int32, "count")
+    keep = (_ptr_array(q_abs), _ptr_array(latent), _ptr_array(out), _ptr_array(lse) if lse else None)
+    return _invoke(load().lsa_sparse_mla_decode_layer, (
+        ctypes.byref(cfg._c()), q_abs[0].shape[0], keep[0], keep[1], _ptr(k_off), _ptr(idx), _ptr(count),
+        int(max_len), keep[2], keep[3], _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+        bind=bind, keep=keep)
+
+
+def mtp_mla_decode(cfg, pos, q_abs, latent, k_off, idx, count, max_len, out, lse, ws, stream=None, bind=False):
+    """The draft steps of one MTP round over one shared selection made at pos
+    (q_abs, out, lse: lists of n_draft tensors; step i also sees keys pos+1..pos+i)."""
+    _bf16_list(list(q_abs) + [latent] + list(out), "q_abs/latent/out")
+    for t in (lse or []):
+        _dt(t, torch.float32, "lse")
+    _dt(pos, torch.int32, "pos"); _dt(k_off, torch.int64, "k_off"); _dt(idx, torch.int32, "idx")
+    _dt(count, torch.int32, "count")
+    keep = (_ptr_array(q_abs), _ptr_array(out), _ptr_array(lse) if lse else None)
+    return _invoke(load().lsa_mtp_mla_decode, (
+        ctypes.byref(cfg._c()), len(q_abs), pos.shape[0], _ptr(pos), keep[0], _ptr(latent), _ptr(k_off), _ptr(idx),
+        _ptr(count), int(max_len), keep[1], keep[2], _ptr(ws), 0 if ws is None else ws.numel(), _stream(stream)),
+        bind=bind, keep=keep)
+
+
+def debug_arm_mla_wait_test(wait_ns: int, drop_tile: int):
+    """Test hook: the next sparse-MLA launch of this thread stops issuing tiles at
+    drop_tile and gives up its waits after wait_ns (see include/lsa.h)."""
+    load().lsa_debug_arm_mla_wait_test(int(wait_ns), int(drop_tile))
 
 
 def sparse_mla_prefill(cfg, pos, q_abs, latent, idx, count, out, lse, ws, stream=None, bind=False):

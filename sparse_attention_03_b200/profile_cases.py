@@ -11,6 +11,8 @@ current stream, checks the device error flags and exits. Cases:
   topk_decode    lsa_topk on 16 rows x 131072 scores, with the indexer's histogram
   mla_decode     lsa_sparse_mla_decode, 16 rows x 2048 selected keys of 131072
   mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
+  mla_layer      lsa_sparse_mla_decode_layer (both sub-blocks in one launch) on the top-k's lists,
+                 16 rows x 131072 keys
   decode_8k      lsa_forward (cli 2), 1 row x 8192 keys (single-token decode latency)
   decode_1m      lsa_forward (cli 2), 4 rows x 983040 keys (one long-context decode layer)
   chunk_1m       lsa_forward (cli 2), a 4096-row prefill chunk at positions 983040.. (16 GB of scores)
@@ -83,6 +85,23 @@ def case_mla_decode(reps):
     ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE, 16, 16, 131072)
     for _ in range(reps):
         lsa.sparse_mla_decode(cfg, wl.q_abs[0], wl.latent[0], wl.k_off, idx, cnt, 131072, out, lse, ws)
+
+
+def case_mla_layer(reps):
+    cfg = lsa.LsaConfig()
+    lengths = np.full(16, 131072, dtype=np.int64)
+    wl = DeviceWorkload(0, 0, lengths, cli=2)
+    scores = torch.empty((16, 131072), device="cuda")
+    hist = lsa.topk_hist_buffer(16)
+    idx = torch.empty((16, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((16,), dtype=torch.int32, device="cuda")
+    lsa.index_scores(cfg, wl.seq_of_row, wl.pos, wl.q_idx, wl.w, wl.k_idx, wl.k_off, 131072, scores, topk_hist=hist)
+    lsa.topk(cfg, wl.pos, 131072, scores, idx, cnt, lsa.workspace(cfg, lsa.OP_TOPK, 16, 16, 131072), topk_hist=hist)
+    outs = [torch.empty((16, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((16, 32), device="cuda") for _ in range(2)]
+    ws = lsa.workspace(cfg, lsa.OP_MLA_DECODE_LAYER, 16, 16, 131072)
+    for _ in range(reps):
+        lsa.sparse_mla_decode_layer(cfg, wl.q_abs, wl.latent, wl.k_off, idx, cnt, 131072, outs, lses, ws)
 
 
 def case_mla_prefill(reps):

@@ -671,20 +671,16 @@ def test_forward_tiny_config(L):
     _forward_check(L, wl, _upload(wl), cfg, 0, range(len(lengths)), max(lengths))
 
 
-def test_mtp_draft_steps_share_one_index_pass(L):
-    # [LSA-2.0] "多token预测模块集成": all three MTP draft steps share one index
-    # pass. Reading: the indexer and the top-k run once, for the first draft
-    # step's query at position p; the three draft steps (positions p, p+1, p+2,
-    # their tokens already appended to the cache) attend over that one
-    # selection with their own absorbed queries.
+def _mtp_case(L, seed, lengths, short=()):
+    # sequence b's index owner (the first draft step) sits at lengths[b] - 3, so
+    # the cache holds the two later drafts' keys; rows in `short` sit at
+    # lengths[b] - 2 (the last draft's key is missing: flagged, not attended)
     cfg = L.LsaConfig(cli_factor=1)
-    ocfg = oracle_cfg(cfg)
-    lengths = [2052, 3000, 5002, 9001, 2049]
-    wl = S.Workload(21, 0, lengths, cli=1)
-    wl.pos = (wl.lengths - 3).astype(np.int32)   # the index owner is the first draft step
+    wl = S.Workload(seed, 0, lengths, cli=1)
+    wl.pos = np.array([n - (2 if b in short else 3) for b, n in enumerate(wl.lengths)], dtype=np.int32)
     d = _upload(wl)
     B, max_len = wl.n_rows, max(lengths)
-    q_steps = [S.normal_bf16(21, S.tid(50 + st, S.Q_ABS0), 0, B * 32 * 576).reshape(B, 32, 576)
+    q_steps = [S.normal_bf16(seed, S.tid(50 + st, S.Q_ABS0), 0, B * 32 * 576).reshape(B, 32, 576)
                for st in range(3)]
     scores = torch.empty((B, max_len), device="cuda")
     idx = torch.empty((B, cfg.index_topk), dtype=torch.int32, device="cuda")
@@ -693,26 +689,113 @@ def test_mtp_draft_steps_share_one_index_pass(L):
     L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], max_len, scores,
                    topk_hist=hist)
     L.topk(cfg, d["pos"], max_len, scores, idx, cnt, L.workspace(cfg, L.OP_TOPK, B, B, max_len), topk_hist=hist)
-    mws = L.workspace(cfg, L.OP_MLA_DECODE, B, B, max_len)
-    got = []
-    for st in range(3):
-        out = torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda")
-        lse = torch.empty((B, 32), device="cuda")
-        L.sparse_mla_decode(cfg, bf16_dev(q_steps[st]), d["latent"][0], d["k_off"], idx, cnt, max_len, out, lse,
-                            mws)
-        got.append((bf16_host_f64(out), lse.cpu().numpy()))
+    outs = [torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
+    lses = [torch.empty((B, 32), device="cuda") for _ in range(3)]
+    L.mtp_mla_decode(cfg, d["pos"], [bf16_dev(q) for q in q_steps], d["latent"][0], d["k_off"], idx, cnt, max_len,
+                     outs, lses, L.workspace(cfg, L.OP_MTP_DECODE, B, B, max_len))
+    return cfg, wl, q_steps, idx.cpu().numpy(), cnt.cpu().numpy(), [(bf16_host_f64(o), l.cpu().numpy())
+                                                                      for o, l in zip(outs, lses)]
+
+
+def test_mtp_draft_steps_share_one_index_pass(L):
+    # [LSA-2.0] "多token预测模块集成": the three MTP draft steps share one index
+    # pass; one launch attends all three (oracle.mtp_round: step i sees the shared
+    # selection plus keys p+1 .. p+i). Rows: sparse, the dense boundary (p + 1 =
+    # 2048 and 2049), dense, long.
+    lengths = [2052, 3000, 5002, 9001, 2050, 2051, 700, 12000]
+    cfg, wl, q_steps, gi, gc, got = _mtp_case(L, 21, lengths)
     assert L.device_error() == 0
-    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
-    for r in range(B):
+    ocfg = oracle_cfg(cfg)
+    for r in range(wl.n_rows):
         q, w, k, _, lat = host_rows(wl, r)
         p = int(wl.pos[r])
         s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
         exact = check_selection(gi[r], int(gc[r]), s, p, ocfg, where=f"row {r}")
-        sel, _ = R.select_topk(s, p, ocfg)
-        assert gi[r, : gc[r]].max() <= p, "the shared set holds no key after the index owner's position"
+        qs = [S.bf16_bits_to_f64(q_steps[st][r]) for st in range(3)]
+        sel, dense, res = R.mtp_round(q, w, k, p, qs, lat[0], ocfg)
+        if not exact:   # a near-tie: the GPU's own (valid) set, through the same round
+            sel = np.sort(gi[r, : gc[r]]).astype(np.int64)
+            res = [R.mla(qs[st], lat[0][np.concatenate([sel, np.arange(p + 1, p + 1 + st)])], ocfg)
+                   for st in range(3)]
         for st in range(3):
-            eo, el = R.mla(S.bf16_bits_to_f64(q_steps[st][r]), lat[0][sel], ocfg)
-            assert_attention(got[st][0][r], got[st][1][r], eo, el, check_lse=exact, where=f"row {r} step {st}")
+            assert_attention(got[st][0][r], got[st][1][r], res[st][0], res[st][1], where=f"row {r} step {st}")
+
+
+def test_mtp_draft_key_past_the_sequence_is_flagged(L):
+    # the last draft's key is not in the cache: LSA_DEVERR_POS, and that step
+    # attends to the keys that are there
+    lengths = [3000, 2600]
+    cfg, wl, q_steps, gi, gc, got = _mtp_case(L, 22, lengths, short=(1,))
+    assert L.device_error() & L.DEVERR_POS
+    ocfg = oracle_cfg(cfg)
+    q, w, k, _, lat = host_rows(wl, 1)
+    p = int(wl.pos[1])
+    sel = np.sort(gi[1, : gc[1]]).astype(np.int64)
+    eo, el = R.mla(S.bf16_bits_to_f64(q_steps[2][1]), lat[0][np.concatenate([sel, [p + 1]])], ocfg)
+    assert_attention(got[2][0][1], got[2][1][1], eo, el, where="short row, step 2")
+
+
+def test_mla_decode_layer_one_launch_matches_oracle(L):
+    # both sub-blocks of a layer over one top-k selection in one launch (with
+    # the in-kernel split-K merge), against the oracle's layer path
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    lengths = [2049, 3000, 4100, 5555, 7000, 8192, 2100, 6100, 1500, 16]
+    wl = S.Workload(23, 0, lengths)
+    d = _upload(wl)
+    B, max_len = wl.n_rows, max(lengths)
+    scores = torch.empty((B, max_len), device="cuda")
+    idx = torch.empty((B, cfg.index_topk), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((B,), dtype=torch.int32, device="cuda")
+    hist = L.topk_hist_buffer(B)
+    L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], max_len, scores,
+                   topk_hist=hist)
+    L.topk(cfg, d["pos"], max_len, scores, idx, cnt, L.workspace(cfg, L.OP_TOPK, B, B, max_len), topk_hist=hist)
+    outs = [torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(2)]
+    lses = [torch.empty((B, 32), device="cuda") for _ in range(2)]
+    ws = L.workspace(cfg, L.OP_MLA_DECODE_LAYER, B, B, max_len)
+    ws.random_(0, 256)   # the workspace needs no clearing
+    for _ in range(2):   # and a second launch reuses it
+        L.sparse_mla_decode_layer(cfg, d["q_abs"], d["latent"], d["k_off"], idx, cnt, max_len, outs, lses, ws)
+        assert L.device_error() == 0
+        gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+        o = [bf16_host_f64(t) for t in outs]
+        l = [t.cpu().numpy() for t in lses]
+        for r in range(B):
+            q, w, k, qa, lat = host_rows(wl, r)
+            p = int(wl.pos[r])
+            s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
+            exact = check_selection(gi[r], int(gc[r]), s, p, ocfg, where=f"row {r}")
+            sel = R.select_topk(s, p, ocfg)[0] if exact else np.sort(gi[r, : gc[r]]).astype(np.int64)
+            for z in range(2):
+                eo, el = R.mla(qa[z], lat[z][sel], ocfg)
+                assert_attention(o[z][r], l[z][r], eo, el, where=f"row {r} sub {z}")
+
+
+def test_mla_wait_timeout_is_reported_and_the_next_call_is_clean(L):
+    # A bounded wait that runs out: the test hook makes every CTA's producer stop
+    # before its second tile and the attention warps give up after 2 ms. The
+    # kernel must return, report LSA_DEVERR_TIMEOUT, and leave the device fit for
+    # the next call, which must match the oracle again.
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    lengths = [3000, 5000, 2500, 7000]
+    wl = S.Workload(24, 0, lengths, cli=1)
+    d = _upload(wl)
+    B, max_len = wl.n_rows, max(lengths)
+    out = torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 32), device="cuda")
+    ws = L.workspace(cfg, L.OP_MLA_DECODE, B, B, max_len)
+    L.debug_arm_mla_wait_test(2_000_000, 1)
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], None, None, max_len, out, lse, ws)
+    assert L.device_error() & L.DEVERR_TIMEOUT
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], None, None, max_len, out, lse, ws)
+    assert L.device_error() == 0
+    o, l = bf16_host_f64(out), lse.cpu().numpy()
+    for r in range(B):
+        _, _, _, qa, lat = host_rows(wl, r)
+        eo, el = R.mla(qa[0], lat[0], ocfg)
+        assert_attention(o[r], l[r], eo, el, where=f"row {r} after the timeout")
 
 
 def test_empty_batch_is_noop(L):
