@@ -101,50 +101,6 @@ __device__ __forceinline__ void half_sync(int h) { asm volatile("bar.sync %0, 12
 __device__ __forceinline__ void stagger_arrive() { asm volatile("bar.arrive 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 __device__ __forceinline__ void stagger_wait() { asm volatile("bar.sync 4, %0;\n" ::"n"(kMathThreads) : "memory"); }
 
-// A split's tiles of a forced-first list: whole tiles of the known prefix,
-// then whole tiles of the rest read from the list, each part shared evenly by
-// the splits. The known prefix is the forced columns' whole tiles (a dense
-// row: its whole list); the forced columns left over in a part tile are read
-// from the list with the selected ones, which the top-k wrote in the same
-// order, so a sparse row of 2048 keys is 64 full tiles (1024 + 1024 keys), not
-// 65 with two part tiles. ub = the first slot read from the list.
-// An MTP draft step's newer keys (p.ext of them) are known as well: a dense
-// row's known run simply continues past its position; a sparse row gets one
-// more known tile after its forced ones.
-struct FfTiles {
-  int kt0, kt, ut0, ut;
-  int64_t ub;
-  int kf;  // known tiles holding forced (or dense) keys; a known tile kf holds the extra keys
-};
-__device__ __forceinline__ FfTiles ff_tiles(const ListPlan& p, int s, int n) {
-  FfTiles f;
-  f.kf = (int)(p.dense ? (p.K + p.ext + kTK - 1) / kTK : p.K / kTK);
-  const int Kt = f.kf + (!p.dense && p.ext > 0 ? 1 : 0);
-  f.ub = min64((int64_t)f.kf * kTK, p.L);
-  const int Ut = (int)((p.L - f.ub + kTK - 1) / kTK);
-  f.kt0 = Kt * s / n;
-  f.kt = Kt * (s + 1) / n - f.kt0;
-  f.ut0 = Ut * s / n;
-  f.ut = Ut * (s + 1) / n - f.ut0;
-  return f;
-}
-// The key of known slot sl (-1: masked).
-__device__ __forceinline__ int known_slot_key(const ListPlan& p, const FfTiles& f, const MlaArgs& a, int64_t sl) {
-  if (p.dense) return sl < p.K + p.ext ? (int)sl : -1;
-  if (sl < (int64_t)f.kf * kTK) return sl < p.K ? (int)known_key(p, a, sl) : -1;
-  const int64_t e = sl - (int64_t)f.kf * kTK;
-  return e < p.ext ? (int)(p.nvis + e) : -1;
-}
-// Extra keys of sub-block z of an MTP launch, clipped to the sequence (flagged).
-__device__ __forceinline__ int mtp_ext(const MlaArgs& a, const RowGeom& g, int z, bool report) {
-  if (!a.mtp || g.nvis <= 0) return 0;
-  int e = z;
-  if (g.nvis + e > g.klen) {
-    if (report) flag_error(a.err, LSA_DEVERR_POS);
-    e = (int)max64(0, g.klen - g.nvis);
-  }
-  return e;
-}
 
 // Warp roles (math warps 0..7): head half mt = w >> 2 (heads 16mt .. 16mt+15)
 // and quarter kq = w & 3, so each SM sub-partition runs one warp of each half
@@ -190,7 +146,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     bulk_row(&sm.q[lane * kSRow], qg, &sm.qbar);
     const RowGeom geo = row_base(a, r, false);
     const ListPlan lp = list_plan(a, geo.nvis, mtp_ext(a, geo, z, false));
-    const FfTiles ft = ff_tiles(lp, s, sp.n_split);
+    const FfTiles ft = ff_tiles<kTK>(lp, s, sp.n_split);
     const uint16_t* __restrict__ latb = a.lat[z] + geo.kbase * kDLat;
     int issued = 0;  // tiles handed to the ring (all of them unless the test hook stops early)
     auto issue = [&](int tt, int key) {
@@ -215,7 +171,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
     // MTP extra keys): keys by formula
     bool go = true;
     for (int tt = 0; go && tt < ft.kt; ++tt)
-      go = issue(tt, known_slot_key(lp, ft, a, (int64_t)(ft.kt0 + tt) * kTK + lane));
+      go = issue(tt, known_slot_key<kTK>(lp, ft, a, (int64_t)(ft.kt0 + tt) * kTK + lane));
     // the selected slots: the top-k's list, after it has finished
     pdl_wait();
     int c = a.count[r];
@@ -338,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1) mla_kernel(MlaArgs a, Split sp, f
   int n_tiles;
   if (ff) {
     const RowGeom geo = row_base(a, r, s == 0 && tid == 0);
-    const FfTiles ft = ff_tiles(list_plan(a, geo.nvis, mtp_ext(a, geo, z, s == 0 && tid == 0)), s, sp.n_split);
+    const FfTiles ft = ff_tiles<kTK>(list_plan(a, geo.nvis, mtp_ext(a, geo, z, s == 0 && tid == 0)), s, sp.n_split);
     n_tiles = ft.kt + ft.ut;
   } else {
     const RowGeom geo = row_geometry(a, r, s == 0 && tid == 0);

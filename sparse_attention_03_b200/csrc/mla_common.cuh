@@ -42,6 +42,53 @@ __device__ __forceinline__ int64_t known_key(const ListPlan& p, const MlaArgs& a
   return (p.dense || i < a.n_init) ? i : p.hi + (i - a.n_init);
 }
 
+// A split's tiles (kTK keys each) of a forced-first list: whole tiles of the known prefix,
+// then whole tiles of the rest read from the list, each part shared evenly by
+// the splits. The known prefix is the forced columns' whole tiles (a dense
+// row: its whole list); the forced columns left over in a part tile are read
+// from the list with the selected ones, which the top-k wrote in the same
+// order, so a sparse row of 2048 keys is 64 full tiles (1024 + 1024 keys), not
+// 65 with two part tiles. ub = the first slot read from the list.
+// An MTP draft step's newer keys (p.ext of them) are known as well: a dense
+// row's known run simply continues past its position; a sparse row gets one
+// more known tile after its forced ones.
+struct FfTiles {
+  int kt0, kt, ut0, ut;
+  int64_t ub;
+  int kf;  // known tiles holding forced (or dense) keys; a known tile kf holds the extra keys
+};
+template <int kTK>
+__device__ __forceinline__ FfTiles ff_tiles(const ListPlan& p, int s, int n) {
+  FfTiles f;
+  f.kf = (int)(p.dense ? (p.K + p.ext + kTK - 1) / kTK : p.K / kTK);
+  const int Kt = f.kf + (!p.dense && p.ext > 0 ? 1 : 0);
+  f.ub = min64((int64_t)f.kf * kTK, p.L);
+  const int Ut = (int)((p.L - f.ub + kTK - 1) / kTK);
+  f.kt0 = Kt * s / n;
+  f.kt = Kt * (s + 1) / n - f.kt0;
+  f.ut0 = Ut * s / n;
+  f.ut = Ut * (s + 1) / n - f.ut0;
+  return f;
+}
+// The key of known slot sl (-1: masked).
+template <int kTK>
+__device__ __forceinline__ int known_slot_key(const ListPlan& p, const FfTiles& f, const MlaArgs& a, int64_t sl) {
+  if (p.dense) return sl < p.K + p.ext ? (int)sl : -1;
+  if (sl < (int64_t)f.kf * kTK) return sl < p.K ? (int)known_key(p, a, sl) : -1;
+  const int64_t e = sl - (int64_t)f.kf * kTK;
+  return e < p.ext ? (int)(p.nvis + e) : -1;
+}
+// Extra keys of sub-block z of an MTP launch, clipped to the sequence (flagged).
+__device__ __forceinline__ int mtp_ext(const MlaArgs& a, const RowGeom& g, int z, bool report) {
+  if (!a.mtp || g.nvis <= 0) return 0;
+  int e = z;
+  if (g.nvis + e > g.klen) {
+    if (report) flag_error(a.err, LSA_DEVERR_POS);
+    e = (int)max64(0, g.klen - g.nvis);
+  }
+  return e;
+}
+
 // A LoZA row that sees nvis keys ("LongCat-Flash-Thinking-ZigZag架构深度剖析",
 // "稀疏模式设计": Sink, Recent and Chunked regions): its keys are [0, s_end) and
 // [w0, nvis), w0 the earlier of the recent window's and the own chunk's first

@@ -772,6 +772,39 @@ def test_mla_decode_layer_one_launch_matches_oracle(L):
                 assert_attention(o[z][r], l[z][r], eo, el, where=f"row {r} sub {z}")
 
 
+def test_mla_topk_lists_wait_timeout_is_reported_and_the_next_call_is_clean(L):
+    # the same for the attention over the top-k's lists (the tensor-core kernel):
+    # every CTA's gather stops before its second tile, the waits give up after
+    # 2 ms, the kernel still frees its tensor memory and returns
+    cfg = L.LsaConfig(cli_factor=1)
+    ocfg = oracle_cfg(cfg)
+    lengths = [3000, 5000, 2500, 7000, 1500]
+    wl = S.Workload(25, 0, lengths, cli=1)
+    d = _upload(wl)
+    B, max_len = wl.n_rows, max(lengths)
+    idx, cnt = _topk_lists(L, cfg, wl, d, max_len)
+    out = torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, 32), device="cuda")
+    ws = L.workspace(cfg, L.OP_MLA_DECODE, B, B, max_len)
+    L.debug_arm_mla_wait_test(2_000_000, 1)
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], idx, cnt, max_len, out, lse, ws,
+                        lists_from_topk=True)
+    assert L.device_error() & L.DEVERR_TIMEOUT
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], idx, cnt, max_len, out, lse, ws,
+                        lists_from_topk=True)
+    assert L.device_error() == 0
+    o, l = bf16_host_f64(out), lse.cpu().numpy()
+    gi, gc = idx.cpu().numpy(), cnt.cpu().numpy()
+    for r in range(B):
+        q, w, k, qa, lat = host_rows(wl, r)
+        p = int(wl.pos[r])
+        s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
+        exact = check_selection(gi[r], int(gc[r]), s, p, ocfg, where=f"row {r}")
+        sel = R.select_topk(s, p, ocfg)[0] if exact else np.sort(gi[r, : gc[r]]).astype(np.int64)
+        eo, el = R.mla(qa[0], lat[0][sel], ocfg)
+        assert_attention(o[r], l[r], eo, el, where=f"row {r} after the timeout")
+
+
 def test_mla_wait_timeout_is_reported_and_the_next_call_is_clean(L):
     # A bounded wait that runs out: the test hook makes every CTA's producer stop
     # before its second tile and the attention warps give up after 2 ms. The
