@@ -7,14 +7,14 @@ namespace lsa {
 
 constexpr int kBins = 2048;  // 11-bit digits
 
-// For a histogram h[0..2048) and a budget `need`, finds the bin d such that
+// For a histogram h[0..BINS) and a budget `need`, finds the bin d such that
 // (count in bins above d) < need <= (count in bins >= d). Block-wide; every
 // thread returns the same answer.
-template <int THREADS>
+template <int THREADS, int BINS = kBins>
 __device__ void find_threshold(const uint32_t* h, uint32_t need, int& bin_out,
                                uint32_t& above_out, int* s_bin, uint32_t* s_above,
                                uint32_t* s_warp) {
-  constexpr int PER = kBins / THREADS;
+  constexpr int PER = BINS / THREADS;
   constexpr int WARPS = THREADS / 32;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   if (tid == 0) {

@@ -421,9 +421,117 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
     }
   };
   auto valid = [&](int64_t j) { return j >= g.lo && j < g.hi; };
+  const uint32_t below = (1u << lane) - 1u;
+  const uint32_t* hr = hist_in ? hist_in + (int64_t)r * kTopkHistStride : nullptr;
+  __syncthreads();  // s_up / s_nc / s_slot initialised
+
+  // Long rows without a histogram: a sample sets a bound, one pass collects every
+  // score above it, and the selection finishes on those candidates in shared
+  // memory. The sample is 64 runs of 256 consecutive middle columns spread over
+  // the row; its histogram of the top 13 key bits (a sixteenth of an octave a
+  // bin) gives the bound that about twice the budget's share of the sample
+  // passes. If at least the budget and at most kRowCap scores pass it, the
+  // selection is exact among them (the budget's best all pass); otherwise the
+  // two-pass path below runs as if nothing had happened. One pass over the row
+  // (plus the sample) instead of two.
+  if (!hr && !short_row && !a.col_map && g.hi - g.lo >= 65536) {
+    constexpr int kSegs = 64, kSegLen = 256, kSBins = 8192;
+    uint32_t* hs = reinterpret_cast<uint32_t*>(cand);  // the candidate buffer, free until the collect
+    for (int i = tid; i < kSBins; i += kRowThreads) hs[i] = 0;
+    __syncthreads();
+    const int64_t span = g.hi - g.lo - kSegLen;
+    for (int sg = warp; sg < kSegs; sg += kRowThreads / 32) {
+      const int64_t s0 = g.lo + span * sg / (kSegs - 1);
+      float v[kSegLen / 32];
+#pragma unroll
+      for (int u = 0; u < kSegLen / 32; ++u) v[u] = srow[s0 + lane + 32 * u];
+#pragma unroll
+      for (int u = 0; u < kSegLen / 32; ++u) atomicAdd(&hs[score_key(v[u]) >> 19], 1u);
+    }
+    __syncthreads();
+    const uint32_t target =
+        (uint32_t)(2.0 * k_rem * (double)(kSegs * kSegLen) / (double)(g.hi - g.lo)) + 16u;
+    int b13;
+    uint32_t a13;
+    find_threshold<kRowThreads, kSBins>(hs, target, b13, a13, &s_bin, &s_above, s_warp);
+    // every middle score at or above the bound into shared memory. The bound as
+    // a float: the lowest value whose key has top 13 bits b13 (score_key is
+    // monotonic), so most rounds cost one compare per score and one vote; the
+    // forced columns the 16-byte loads also cover (+inf) only reach the exact
+    // test below.
+    const uint32_t kmin = (uint32_t)b13 << 19;
+    const float tb = __uint_as_float((kmin & 0x80000000u) ? (kmin & 0x7FFFFFFFu) : ~kmin);
+    stream_row([&](const float(&v)[8], auto jc) {
+      bool hit = false;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) hit |= v[u] >= tb;
+      if (!__any_sync(0xffffffffu, hit)) return;  // most rounds: one vote
+      uint32_t key[8], m[8];
+      uint32_t n = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        key[u] = score_key(v[u]);
+        m[u] = __ballot_sync(0xffffffffu, valid(jc(u)) && (int)(key[u] >> 19) >= b13);
+        n += __popc(m[u]);
+      }
+      uint32_t b = 0;
+      if (lane == 0) b = atomicAdd(&s_nc, n);
+      b = __shfl_sync(0xffffffffu, b, 0);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if ((m[u] >> lane) & 1u) {
+          const uint32_t slot = b + __popc(m[u] & below);
+          if (slot < (uint32_t)kRowCap)
+            cand[slot] = ((uint64_t)key[u] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)jc(u));
+        }
+        b += __popc(m[u]);
+      }
+    });
+    __syncthreads();
+    const uint32_t n_c = s_nc;
+    if (n_c >= k_rem && n_c <= (uint32_t)kRowCap) {
+      // the candidates' top 11 bits: the threshold bin among them
+      for (int i = tid; i < kBins; i += kRowThreads) h[i] = 0;
+      __syncthreads();
+      for (uint32_t i = tid; i < n_c; i += kRowThreads) atomicAdd(&h[(uint32_t)(cand[i] >> 53)], 1u);
+      __syncthreads();
+      int bt;
+      uint32_t at;
+      find_threshold<kRowThreads>(h, k_rem, bt, at, &s_bin, &s_above, s_warp);
+      int32_t* __restrict__ mid = out + a.n_init + a.n_loc;
+      for (uint32_t i = tid; i < n_c; i += kRowThreads) {
+        const uint64_t c = cand[i];
+        if ((int)(c >> 53) > bt) {
+          const uint32_t slot = atomicAdd(&s_up, 1u);
+          if (slot < at) mid[slot] = (int32_t)(0xFFFFFFFFu - (uint32_t)c);
+        }
+      }
+      auto for_bin = [&](auto&& f) {
+        for (uint32_t i = tid; i < n_c; i += kRowThreads) {
+          const uint64_t c = cand[i];
+          if ((int)(c >> 53) == bt) f(c & kLow53, (int64_t)(0xFFFFFFFFu - (uint32_t)c));
+        }
+      };
+      uint64_t prefix;
+      int decided;
+      const uint32_t need = k_rem - at;
+      radix_levels<kRowThreads>(for_bin, need, h, &s_bin, &s_above, s_warp, prefix, decided);
+      const int shb = 53 - decided;
+      int32_t* __restrict__ dst = mid + at;
+      for_bin([&](uint64_t v, int64_t j) {
+        if ((v >> shb) >= prefix) {
+          const uint32_t slot = atomicAdd(&s_slot, 1u);
+          if (slot < need) dst[slot] = (int32_t)j;
+        }
+      });
+      return;
+    }
+    __syncthreads();
+    if (tid == 0) s_nc = 0;  // the bound missed: the exact two-pass path
+  }
+
   int bin0 = 0;
   uint32_t above0 = 0;
-  const uint32_t* hr = hist_in ? hist_in + (int64_t)r * kTopkHistStride : nullptr;
   if (hr) {
     for (int i = tid; i < kBins; i += kRowThreads) h[i] = hr[i];
     __syncthreads();
@@ -446,7 +554,6 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   find_threshold<kRowThreads>(h, k_rem, bin0, above0, &s_bin, &s_above, s_warp);
   __syncthreads();  // s_up / s_nc initialised
   int32_t* __restrict__ mid = out + a.n_init + a.n_loc;
-  const uint32_t below = (1u << lane) - 1u;
 
   if (short_row) {
     // collect of a short row: each thread's counts above and in the threshold
@@ -492,20 +599,21 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
         ++oe;
       }
     }
-  } else
+  } else {
   // collect: higher bins straight out, the threshold bin into shared memory
   // (one pair of shared atomics per warp and round: the round's counts first).
   // Only a few thousand of a row's scores reach the threshold bin: a round in
   // which no lane of the warp has one costs one vote.
+  const uint32_t kmin0 = (uint32_t)bin0 << 21;  // the threshold bin's lowest value as a float (see above)
+  const float tb0 = __uint_as_float((kmin0 & 0x80000000u) ? (kmin0 & 0x7FFFFFFFu) : ~kmin0);
   stream_row([&](const float(&v)[8], auto jc) {
     uint32_t key[8], upm[8], eqm[8];
     bool hit = false;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      key[u] = score_key(v[u]);
-      hit |= valid(jc(u)) && (int)(key[u] >> 21) >= bin0;
-    }
+    for (int u = 0; u < 8; ++u) hit |= v[u] >= tb0;
     if (!__any_sync(0xffffffffu, hit)) return;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) key[u] = score_key(v[u]);
     uint32_t n_up = 0, n_eq = 0;
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
@@ -537,6 +645,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
       b_eq += __popc(eqm[u]);
     }
   });
+  }
   __syncthreads();
   const uint32_t need0 = k_rem - above0;
   uint32_t n_cand = s_nc, need = need0;

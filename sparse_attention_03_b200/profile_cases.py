@@ -9,6 +9,7 @@ current stream, checks the device error flags and exits. Cases:
   index_decode   lsa_index_scores with the top-k histogram, 16 rows x 131072 keys (one 128K decode layer)
   index_prefill  lsa_index_scores, 16384 causal rows over 16384 keys
   topk_decode    lsa_topk on 16 rows x 131072 scores, with the indexer's histogram
+  topk_rows      lsa_topk on 512 rows x 500000 random scores (the one-CTA-per-row kernel, long rows)
   mla_decode     lsa_sparse_mla_decode, 16 rows x 2048 selected keys of 131072
   mla_prefill    lsa_sparse_mla_prefill, 4096 rows x 2048 selected keys of 16384
   mla_layer      lsa_sparse_mla_decode_layer (both sub-blocks in one launch) on the top-k's lists,
@@ -71,6 +72,19 @@ def case_topk_decode(reps):
     ws = lsa.workspace(cfg, lsa.OP_TOPK, 16, 16, 131072)
     for _ in range(reps):
         lsa.topk(cfg, wl.pos, 131072, scores, idx, cnt, ws, topk_hist=hist)
+
+
+def case_topk_rows(reps):
+    cfg = lsa.LsaConfig()
+    n, L = 512, 500000
+    scores = torch.empty((n, L), device="cuda")
+    lsa.synth_normal_f32(scores, 0, 7)
+    pos = torch.full((n,), L - 1, dtype=torch.int32, device="cuda")
+    idx = torch.empty((n, 2048), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((n,), dtype=torch.int32, device="cuda")
+    ws = lsa.workspace(cfg, lsa.OP_TOPK, n, n, L)
+    for _ in range(reps):
+        lsa.topk(cfg, pos, L, scores, idx, cnt, ws)
 
 
 def case_mla_decode(reps):

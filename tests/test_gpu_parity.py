@@ -213,6 +213,50 @@ def test_topk_exact_on_fp32_scores(L):
             np.testing.assert_array_equal(np.sort(idx[r]), exp, err_msg=f"row {r}")
 
 
+@pytest.mark.parametrize("ld_pad", [0, 3])
+def test_topk_many_long_rows_sampled_bound(L, ld_pad):
+    # 256+ rows longer than 65536 middle columns take the one-CTA kernel's
+    # sampled-bound path: a sample of the row sets a bound, one pass collects the
+    # scores above it, the select finishes on them. Rows where the bound admits
+    # too few (the best scores hidden between the sample runs) or too many (heavy
+    # ties, all equal, an overfull bin) fall back to the exact two-pass path.
+    # Exact sets against the oracle either way.
+    cfg = L.LsaConfig()
+    ocfg = oracle_cfg(cfg)
+    rng = np.random.default_rng(41 + ld_pad)
+    n = 264
+    pos = rng.integers(70000, 160000, n).astype(np.int64)
+    if ld_pad == 0:
+        pos -= (pos + 1) % 4          # 16-byte loads need max_len % 4 == 0 too
+        pos = np.maximum(pos, 70000 - 1)
+    rows = []
+    for r, p in enumerate(pos):
+        v = rng.standard_normal(p + 1).astype(np.float32)
+        kind = r % 8
+        if kind == 1:
+            v = np.round(v * 2).astype(np.float32)                    # heavy ties: too many pass
+        elif kind == 2:
+            v[:] = 0.75                                               # all equal
+        elif kind == 3:                                               # the best 1500 in one gap of the sample
+            span = (p + 1 - 1024 - 16) - 256
+            gap0 = 16 + span // 63 + 300
+            v[gap0:gap0 + 1500] = 50.0 + rng.random(1500).astype(np.float32)
+        elif kind == 4:                                               # an overfull bin
+            cols = rng.choice(np.arange(16, p + 1 - 1024), 6000, replace=False)
+            v[cols] = rng.uniform(96.0, 112.0, 6000).astype(np.float32)
+        elif kind == 5:
+            v *= 1e-3                                                 # tiny scores
+        rows.append(v)
+    max_len = int(pos.max()) + 1 + (3 - int(pos.max()) % 4 if ld_pad == 0 else 0)
+    st, idx, cnt = _topk_case(L, cfg, rows, pos, max_len, ld_pad)
+    assert st == L.LSA_OK
+    assert L.device_error() == 0
+    for r, p in enumerate(pos):
+        exp, dense = R.select_topk(R.mask_and_force(rows[r].astype(np.float64), int(p), max_len, ocfg), int(p), ocfg)
+        assert cnt[r] == cfg.index_topk and not dense
+        np.testing.assert_array_equal(np.sort(idx[r]), exp, err_msg=f"row {r} (kind {r % 8})")
+
+
 def test_topk_all_equal_overflow_path(L):
     # all-equal scores overflow the candidate buffer and take the rescan path;
     # ties go to the lowest indices.
