@@ -327,7 +327,12 @@ __global__ void __launch_bounds__(kHistThreads, 4)
 // instead of three; the multi-CTA kernels above serve few, very long rows.
 constexpr int kRowThreads = 512;
 constexpr int kRowCap = 4608;  // 36 KB of candidates: static shared memory stays under 48 KB
+constexpr int64_t kSampledMin = 65536;  // middle columns from which a row takes the sampled bound
 
+// kSampled: the instance for long rows without a histogram (below), launched
+// only when some row is long enough to use it; the other instance is compiled
+// without that path.
+template <bool kSampled>
 __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, int row0, const uint32_t* hist_in) {
   __shared__ uint32_t h[kBins];
   __shared__ uint64_t cand[kRowCap];
@@ -423,7 +428,6 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   auto valid = [&](int64_t j) { return j >= g.lo && j < g.hi; };
   const uint32_t below = (1u << lane) - 1u;
   const uint32_t* hr = hist_in ? hist_in + (int64_t)r * kTopkHistStride : nullptr;
-  __syncthreads();  // s_up / s_nc / s_slot initialised
 
   // Long rows without a histogram: a sample sets a bound, one pass collects every
   // score above it, and the selection finishes on those candidates in shared
@@ -434,7 +438,8 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   // selection is exact among them (the budget's best all pass); otherwise the
   // two-pass path below runs as if nothing had happened. One pass over the row
   // (plus the sample) instead of two.
-  if (!hr && !short_row && !a.col_map && g.hi - g.lo >= 65536) {
+  if constexpr (kSampled) if (!hr && !short_row && !a.col_map && g.hi - g.lo >= kSampledMin) {
+    __syncthreads();  // s_up / s_nc / s_slot initialised
     constexpr int kSegs = 64, kSegLen = 256, kSBins = 8192;
     uint32_t* hs = reinterpret_cast<uint32_t*>(cand);  // the candidate buffer, free until the collect
     for (int i = tid; i < kSBins; i += kRowThreads) hs[i] = 0;
@@ -761,7 +766,7 @@ static size_t row_map_smem(const TopkArgs& a) {
   if (!a.col_map) return 0;
   static bool attr_set = false;  // benign race: every caller sets the same value
   if (!attr_set) {
-    cudaFuncSetAttribute(topk_row_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 2048 * 4);
+    cudaFuncSetAttribute(topk_row_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, 2048 * 4);
     attr_set = true;
   }
   return (size_t)a.col_ld * sizeof(int32_t);
@@ -771,8 +776,8 @@ cudaError_t launch_topk_dense(const TopkArgs& a, cudaStream_t st) {
   // every row is dense: the per-row kernel writes 0..n-1 and the count
   for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
     const int nr = min(65535, a.n_rows - row0);
-    const cudaError_t e =
-        launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), row_map_smem(a), st, a, row0, (const uint32_t*)nullptr);
+    const cudaError_t e = launch_pdl(topk_row_kernel<false>, dim3(nr), dim3(kRowThreads), row_map_smem(a), st, a,
+                                     row0, (const uint32_t*)nullptr);
     if (e != cudaSuccess) return e;
     count_launches(1);
   }
@@ -792,10 +797,14 @@ cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st) {
   const bool per_row = !topk_uses_workspace(a.n_rows, a.max_len) || a.col_map != nullptr || a.zero_hist != nullptr;
   if (per_row) {
     const uint32_t* hist_in = a.hist_ext;
+    // some row may take the sampled bound: no histogram given, long enough, no column map
+    const bool sampled = !hist_in && !a.col_map && a.max_len - a.n_init - a.n_loc >= kSampledMin;
     for (int row0 = 0; row0 < a.n_rows; row0 += 65535) {
       const int nr = min(65535, a.n_rows - row0);
       const cudaError_t e =
-          launch_pdl(topk_row_kernel, dim3(nr), dim3(kRowThreads), row_map_smem(a), st, a, row0, hist_in);
+          sampled ? launch_pdl(topk_row_kernel<true>, dim3(nr), dim3(kRowThreads), 0, st, a, row0, hist_in)
+                  : launch_pdl(topk_row_kernel<false>, dim3(nr), dim3(kRowThreads), row_map_smem(a), st, a, row0,
+                               hist_in);
       if (e != cudaSuccess) return e;
       count_launches(1);
     }
