@@ -156,7 +156,7 @@ def peaks():
 
 # the decode indexer's code: its kernel and its key-tile helpers
 INDEX_DECODE_SOURCES = ("index_decode.cu", "index_tile.cuh")
-INDEX_PREFILL_SOURCES = ("index_prefill.cu",)
+INDEX_PREFILL_SOURCES = ("index_prefill.cu", "tc.cuh")
 
 
 def source_sha(srcs) -> str:
