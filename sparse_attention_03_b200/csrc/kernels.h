@@ -77,6 +77,10 @@ struct TopkArgs {
 constexpr int kTopkCap = 4096;                              // candidates per row: the base layout, and shared memory
 constexpr size_t kTopkRowBytes = 2048 * 4 + 32 + kTopkCap * 8;  // hist + ctl + candidates
 constexpr int kTopkHistStride = 2048 + 8;                   // words between rows' histograms
+// Rows with at most this many middle columns are "short" for the one-CTA
+// top-k: every score sits in registers, so a histogram built elsewhere saves
+// that kernel nothing.
+constexpr int64_t kTopkShortMid = 8192;
 
 cudaError_t launch_topk(const TopkArgs& a, cudaStream_t st);
 // Clears n_words 32-bit words on the stream with a kernel (keeps the launch chain).

@@ -660,8 +660,11 @@ lsa_status lsa_forward(const lsa_config* c, int32_t mode, int32_t n_rows, int32_
   const size_t topk_bytes = topk_ws(R, max_len);
   p += topk_bytes;
   // Decode: the indexer builds the top-k's histogram while the scores are in
-  // registers, which saves the top-k one pass over the scores and one launch.
-  const bool fuse_hist = mode == 0;
+  // registers, which saves the top-k one pass over the scores and one launch;
+  // not for rows short enough that the top-k holds all their scores anyway
+  // (there it would only add the histogram's zeroing launch).
+  const bool fuse_hist =
+      mode == 0 && max_len - c->index_init_tokens - c->index_local_tokens > kTopkShortMid;
   void* mla_w = p;
   const size_t mla_bytes = mla_ws(R, cli, c->index_topk);
 

@@ -376,6 +376,7 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   // at once, before the histogram and the threshold search, and the collect
   // places each thread's scores with one block-wide prefix sum.
   constexpr int kShort = 2 * kUnroll;
+  static_assert((int64_t)kRowThreads * kShort == kTopkShortMid, "short rows as the launcher sees them");
   const bool short_row = g.hi - g.lo <= (int64_t)kRowThreads * kShort;
   auto scol = [&](int i) -> int64_t {  // warp w, round q: columns lo + 4096 q + 256 w .. + 255
     return g.lo + (int64_t)(i / kUnroll) * kRowThreads * kUnroll + warp * 32 * kUnroll + lane + 32 * (i % kUnroll);
