@@ -174,3 +174,38 @@ def test_loza_validation(lib):
     assert call((16, 1024, 64), mode=1, n_seq=1) == lsa.LSA_ERR_INVALID       # prefill: k_off must be NULL
     assert call((16, 1024, 64), mode=1, k_off=None, n_seq=1, pos=None) == lsa.LSA_ERR_INVALID  # prefill needs pos
     assert call((16, 1024, 64), mode=2) == lsa.LSA_ERR_INVALID
+
+
+def test_layer_and_mtp_attention_validation(lib):
+    c = lsa.LsaConfig().c()
+    f = _fake()
+    arr = (ctypes.c_void_p * 4)(0x10000, 0x20000, 0x30000, 0x40000)
+    bad = (ctypes.c_void_p * 2)(0x10000, 0x10002)              # the second pointer misaligned
+    # both sub-blocks over one selection: NULL index list, NULL offsets, a misaligned sub-block pointer
+    layer = lambda q, idx=f, k_off=f: lib.lsa_sparse_mla_decode_layer(ctypes.byref(c), 2, q, arr, k_off, idx, f,
+                                                                       10, arr, None, None, 0, None)
+    assert layer(arr, idx=None) == lsa.LSA_ERR_INVALID
+    assert layer(arr, k_off=None) == lsa.LSA_ERR_INVALID
+    assert layer(bad) == lsa.LSA_ERR_INVALID
+    assert lib.lsa_sparse_mla_decode_layer(ctypes.byref(c), 0, None, None, None, None, None, 10, None, None, None,
+                                           0, None) == lsa.LSA_OK
+    # MTP: 1 <= n_draft <= 4, positions required
+    mtp = lambda n, pos=f: lib.lsa_mtp_mla_decode(ctypes.byref(c), n, 2, pos, arr, f, f, f, f, 10, arr, None,
+                                                  None, 0, None)
+    assert mtp(0) == lsa.LSA_ERR_UNSUPPORTED
+    assert mtp(5) == lsa.LSA_ERR_UNSUPPORTED
+    assert b"n_draft" in lib.lsa_last_error()
+    assert mtp(3, pos=None) == lsa.LSA_ERR_INVALID
+    # split-K partials: fp32 [32 x 512] + (m, l) per head, for every (row, sub-block, split)
+    cfg = lsa.LsaConfig()
+    part = 32 * 512 * 4 + 32 * 8
+    layer_ws = lsa.workspace_size(cfg, lsa.OP_MLA_DECODE_LAYER, 16, 16, 131072)
+    assert layer_ws >= 16 * 2 * 2 * part                       # both sub-blocks, at least two splits each
+    assert lsa.workspace_size(cfg, lsa.OP_MTP_DECODE, 16, 16, 131072) >= layer_ws   # sized for up to 4 steps
+
+
+def test_wait_test_hook_is_one_shot_and_host_only(lib):
+    # arming the hook touches no device; it applies to the next launch of the
+    # thread only (consumed there), so arming twice before any launch is harmless
+    lib.lsa_debug_arm_mla_wait_test(1000, 1)
+    lib.lsa_debug_arm_mla_wait_test(0, -1)
