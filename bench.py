@@ -479,30 +479,53 @@ def decode_step_two_launch(D):
         mla_calls[1]()
 
 
-def decode_forward_e2e(D, h_in, h_out, pipe):
-    """One step through lsa_forward with every layer's inputs copied from pinned
-    host memory and its outputs copied back. The copies run on a second stream:
-    layer l+1's inputs travel while layer l computes, layer l's outputs while
-    layer l+1 computes."""
+def build_e2e_sets(D, device):
+    """Two sets of per-step device buffers (queries in, attention out) with
+    lsa_forward bound to each, so that one step's host copies travel while the
+    other set computes."""
     import torch
-    comp, copy, ev_in, ev_out = pipe
-    with torch.cuda.stream(copy):
-        copy.wait_stream(comp)  # the previous step's readers of these buffers are done
-        for i in range(len(D["fwd"])):
-            D["q_idx"][i].copy_(h_in[0][i], non_blocking=True)
-            D["w"][i].copy_(h_in[1][i], non_blocking=True)
-            D["q_abs"][i].copy_(h_in[2][i], non_blocking=True)
-            ev_in[i].record(copy)
-    for i, call in enumerate(D["fwd"]):
-        comp.wait_event(ev_in[i])
+    from sparse_attention_03_b200 import lsa
+    sets = [dict(q_idx=D["q_idx"], w=D["w"], q_abs=D["q_abs"], out=D["out"], lse=D["lse"], fwd=D["fwd"])]
+    qi, w, qa = D["q_idx"].clone(), D["w"].clone(), D["q_abs"].clone()
+    out, lse = torch.empty_like(D["out"]), torch.empty_like(D["lse"])
+    fwd = [lsa.forward(D["cfg"], 0, l.seq_of_row, l.pos, D["ctx"], qi[i], w[i], l.k_idx, l.k_off, [qa[i, 0], qa[i, 1]],
+                       l.latent, [out[i, 0], out[i, 1]], [lse[i, 0], lse[i, 1]], D["ws"], bind=True)
+           for i, l in enumerate(D["layers"])]
+    sets.append(dict(q_idx=qi, w=w, q_abs=qa, out=out, lse=lse, fwd=fwd))
+    return sets
+
+
+def decode_forward_e2e(sets, s, h_in, h_out, pipe, last=False):
+    """Step s through lsa_forward (every layer), its inputs copied from pinned
+    host memory and its outputs (attention output and lse of every layer)
+    copied back. Steps alternate between two sets of device buffers: step s's
+    input copy (one stream) runs while step s-1 computes, and its output copy
+    (another stream) while step s+1 computes; the compute stream waits for
+    those copies once per step, so the layers' kernels stay back to back. With
+    last=True the compute stream also waits for this step's output copy, which
+    ends the timed region after every copy of every step."""
+    import torch
+    comp, h2d, d2h, evs = pipe
+    X, ev = sets[s % 2], evs[s % 2]
+    with torch.cuda.stream(h2d):
+        h2d.wait_event(ev["done"])              # this set's previous step has read its inputs
+        X["q_idx"].copy_(h_in[0], non_blocking=True)
+        X["w"].copy_(h_in[1], non_blocking=True)
+        X["q_abs"].copy_(h_in[2], non_blocking=True)
+        ev["in"].record(h2d)
+    comp.wait_event(ev["in"])
+    comp.wait_event(ev["out"])                  # this set's previous outputs have been copied out
+    for call in X["fwd"]:
         call()
-        ev_out[i].record(comp)
-    with torch.cuda.stream(copy):
-        for i in range(len(D["fwd"])):
-            copy.wait_event(ev_out[i])
-            h_out[0][i].copy_(D["out"][i], non_blocking=True)
-            h_out[1][i].copy_(D["lse"][i], non_blocking=True)
-    comp.wait_stream(copy)
+    ev["done"].record(comp)
+    with torch.cuda.stream(d2h):
+        d2h.wait_event(ev["done"])
+        h_out[0].copy_(X["out"], non_blocking=True)
+        h_out[1].copy_(X["lse"], non_blocking=True)
+        ev["out"].record(d2h)
+    if last:
+        comp.wait_stream(d2h)
+        comp.wait_stream(h2d)
 
 
 def time_region(fn, steps, world, device):
@@ -726,13 +749,16 @@ def gpu_arm(args):
     h_in = [D["q_idx"].cpu().pin_memory(), D["w"].cpu().pin_memory(), D["q_abs"].cpu().pin_memory()]
     h_out = [torch.empty(D["out"].shape, dtype=D["out"].dtype).pin_memory(),
              torch.empty(D["lse"].shape, dtype=D["lse"].dtype).pin_memory()]
-    pipe = (torch.cuda.current_stream(), torch.cuda.Stream(),
-            [torch.cuda.Event() for _ in range(nl)], [torch.cuda.Event() for _ in range(nl)])
-    for _ in range(max(3, args.warmup // 2)):
-        decode_forward_e2e(D, h_in, h_out, pipe)
+    sets = build_e2e_sets(D, device)
+    pipe = (torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream(),
+            [dict(**{k: torch.cuda.Event() for k in ("in", "done", "out")}) for _ in range(2)])
+    n_warm = max(3, args.warmup // 2)
+    for w_ in range(n_warm):
+        decode_forward_e2e(sets, w_, h_in, h_out, pipe, last=w_ == n_warm - 1)
     torch.cuda.synchronize()
     e2e_steps = max(5, args.steps // 2)
-    te = time_region(lambda s: decode_forward_e2e(D, h_in, h_out, pipe), e2e_steps, world, device)
+    te = time_region(lambda s: decode_forward_e2e(sets, s, h_in, h_out, pipe, last=s == e2e_steps - 1), e2e_steps,
+                     world, device)
     e2e_value, _ = aggregate(B * nl * e2e_steps, te, world, device)
     h2d = sum(x.numel() * x.element_size() for x in h_in)
     d2h = sum(x.numel() * x.element_size() for x in h_out)
