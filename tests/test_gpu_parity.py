@@ -715,17 +715,17 @@ def test_forward_tiny_config(L):
     _forward_check(L, wl, _upload(wl), cfg, 0, range(len(lengths)), max(lengths))
 
 
-def _mtp_case(L, seed, lengths, short=()):
-    # sequence b's index owner (the first draft step) sits at lengths[b] - 3, so
-    # the cache holds the two later drafts' keys; rows in `short` sit at
-    # lengths[b] - 2 (the last draft's key is missing: flagged, not attended)
+def _mtp_case(L, seed, lengths, short=(), n_draft=3):
+    # sequence b's index owner (the first draft step) sits at lengths[b] - n_draft,
+    # so the cache holds the later drafts' keys; rows in `short` sit one position
+    # later (the last draft's key is missing: flagged, not attended)
     cfg = L.LsaConfig(cli_factor=1)
     wl = S.Workload(seed, 0, lengths, cli=1)
-    wl.pos = np.array([n - (2 if b in short else 3) for b, n in enumerate(wl.lengths)], dtype=np.int32)
+    wl.pos = np.array([n - n_draft + (1 if b in short else 0) for b, n in enumerate(wl.lengths)], dtype=np.int32)
     d = _upload(wl)
     B, max_len = wl.n_rows, max(lengths)
     q_steps = [S.normal_bf16(seed, S.tid(50 + st, S.Q_ABS0), 0, B * 32 * 576).reshape(B, 32, 576)
-               for st in range(3)]
+               for st in range(n_draft)]
     scores = torch.empty((B, max_len), device="cuda")
     idx = torch.empty((B, cfg.index_topk), dtype=torch.int32, device="cuda")
     cnt = torch.empty((B,), dtype=torch.int32, device="cuda")
@@ -733,8 +733,8 @@ def _mtp_case(L, seed, lengths, short=()):
     L.index_scores(cfg, d["seq_of_row"], d["pos"], d["q_idx"], d["w"], d["k_idx"], d["k_off"], max_len, scores,
                    topk_hist=hist)
     L.topk(cfg, d["pos"], max_len, scores, idx, cnt, L.workspace(cfg, L.OP_TOPK, B, B, max_len), topk_hist=hist)
-    outs = [torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(3)]
-    lses = [torch.empty((B, 32), device="cuda") for _ in range(3)]
+    outs = [torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda") for _ in range(n_draft)]
+    lses = [torch.empty((B, 32), device="cuda") for _ in range(n_draft)]
     L.mtp_mla_decode(cfg, d["pos"], [bf16_dev(q) for q in q_steps], d["latent"][0], d["k_off"], idx, cnt, max_len,
                      outs, lses, L.workspace(cfg, L.OP_MTP_DECODE, B, B, max_len))
     return cfg, wl, q_steps, idx.cpu().numpy(), cnt.cpu().numpy(), [(bf16_host_f64(o), l.cpu().numpy())
@@ -763,6 +763,48 @@ def test_mtp_draft_steps_share_one_index_pass(L):
                    for st in range(3)]
         for st in range(3):
             assert_attention(got[st][0][r], got[st][1][r], res[st][0], res[st][1], where=f"row {r} step {st}")
+
+
+@pytest.mark.parametrize("n_draft", [1, 2, 4])
+def test_mtp_other_draft_counts(L, n_draft):
+    # one draft step is the plain layer path over the selection; four is the
+    # entry point's limit (three newer keys for the last step)
+    lengths = [2600, 2049 + n_draft - 1, 5000, 1500]
+    cfg, wl, q_steps, gi, gc, got = _mtp_case(L, 30 + n_draft, lengths, n_draft=n_draft)
+    assert L.device_error() == 0
+    ocfg = oracle_cfg(cfg)
+    for r in range(wl.n_rows):
+        q, w, k, _, lat = host_rows(wl, r)
+        p = int(wl.pos[r])
+        s = R.mask_and_force(R.score_row(q, w, k[: p + 1]), p, k.shape[0], ocfg)
+        exact = check_selection(gi[r], int(gc[r]), s, p, ocfg, where=f"row {r}")
+        qs = [S.bf16_bits_to_f64(q_steps[st][r]) for st in range(n_draft)]
+        sel, _, res = R.mtp_round(q, w, k, p, qs, lat[0], ocfg)
+        if not exact:
+            sel = np.sort(gi[r, : gc[r]]).astype(np.int64)
+            res = [R.mla(qs[st], lat[0][np.concatenate([sel, np.arange(p + 1, p + 1 + st)])], ocfg)
+                   for st in range(n_draft)]
+        for st in range(n_draft):
+            assert_attention(got[st][0][r], got[st][1][r], res[st][0], res[st][1], where=f"row {r} step {st}")
+
+
+def test_mla_decode_layer_single_sub_block_equals_topk_call(L):
+    # with cli_factor 1 the layer call is lsa_sparse_mla_decode_topk: the same kernel
+    # and split, so the same bits
+    cfg = L.LsaConfig(cli_factor=1)
+    lengths = [3000, 2048, 7000, 12]
+    wl = S.Workload(26, 0, lengths, cli=1)
+    d = _upload(wl)
+    B, max_len = wl.n_rows, max(lengths)
+    idx, cnt = _topk_lists(L, cfg, wl, d, max_len)
+    ws = L.workspace(cfg, L.OP_MLA_DECODE_LAYER, B, B, max_len)
+    o1, l1 = torch.empty((B, 32, 512), dtype=torch.bfloat16, device="cuda"), torch.empty((B, 32), device="cuda")
+    o2, l2 = torch.empty_like(o1), torch.empty_like(l1)
+    L.sparse_mla_decode_layer(cfg, d["q_abs"], d["latent"], d["k_off"], idx, cnt, max_len, [o1], [l1], ws)
+    L.sparse_mla_decode(cfg, d["q_abs"][0], d["latent"][0], d["k_off"], idx, cnt, max_len, o2, l2, ws,
+                        lists_from_topk=True)
+    assert L.device_error() == 0
+    assert torch.equal(o1.view(torch.int16), o2.view(torch.int16)) and torch.equal(l1, l2)
 
 
 def test_mtp_draft_key_past_the_sequence_is_flagged(L):
