@@ -396,15 +396,21 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
   // loads per lane, one round). The 16-byte loads start at lo rounded down to 4
   // and end at hi rounded up to 4, inside the row since ld is a multiple of 4.
   const bool vec = g.hi - g.lo >= 32768 && (a.ld & 3) == 0 && (reinterpret_cast<uintptr_t>(srow) & 15u) == 0;
+  const int64_t hi4 = (g.hi + 3) & ~int64_t(3);  // a load at j4 (a multiple of 4) is below hi iff j4 < hi4
   auto stream_row = [&](auto&& fn) {
     if (vec) {
       for (int64_t base = (g.lo & ~int64_t(3)) + (int64_t)warp * 512; base < g.hi;
            base += (int64_t)kRowThreads * 16) {
         float4 q[4];
+        if (kSampled && base + 512 <= hi4) {  // every load of the step below hi: no per-load test
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int64_t j4 = base + 128 * u + 4 * lane;
-          q[u] = j4 < g.hi ? *reinterpret_cast<const float4*>(srow + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          for (int u = 0; u < 4; ++u) q[u] = *reinterpret_cast<const float4*>(srow + base + 128 * u + 4 * lane);
+        } else {
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int64_t j4 = base + 128 * u + 4 * lane;
+            q[u] = j4 < g.hi ? *reinterpret_cast<const float4*>(srow + j4) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
         }
 #pragma unroll
         for (int hf = 0; hf < 2; ++hf) {
@@ -467,30 +473,26 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
     // test below.
     const uint32_t kmin = (uint32_t)b13 << 19;
     const float tb = __uint_as_float((kmin & 0x80000000u) ? (kmin & 0x7FFFFFFFu) : ~kmin);
+    // About twice the budget's share of the scores passes, so a 256-score
+    // round holds a passing score more often than not: each of the 8 values
+    // then takes its own vote, and only a value with a passing lane pays for
+    // the key, the range test and the append.
     stream_row([&](const float(&v)[8], auto jc) {
-      bool hit = false;
+      float mx = v[0];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) hit |= v[u] >= tb;
-      if (!__any_sync(0xffffffffu, hit)) return;  // most rounds: one vote
-      uint32_t key[8], m[8];
-      uint32_t n = 0;
+      for (int u = 1; u < 8; ++u) mx = fmaxf(mx, v[u]);
+      if (!__any_sync(0xffffffffu, mx >= tb)) return;  // rounds without a passing score: one vote
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        key[u] = score_key(v[u]);
-        m[u] = __ballot_sync(0xffffffffu, valid(jc(u)) && (int)(key[u] >> 19) >= b13);
-        n += __popc(m[u]);
-      }
-      uint32_t b = 0;
-      if (lane == 0) b = atomicAdd(&s_nc, n);
-      b = __shfl_sync(0xffffffffu, b, 0);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if ((m[u] >> lane) & 1u) {
-          const uint32_t slot = b + __popc(m[u] & below);
-          if (slot < (uint32_t)kRowCap)
-            cand[slot] = ((uint64_t)key[u] << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)jc(u));
-        }
-        b += __popc(m[u]);
+        if (!__any_sync(0xffffffffu, v[u] >= tb)) continue;
+        const uint32_t key = score_key(v[u]);
+        const bool take = v[u] >= tb && valid(jc(u)) && (int)(key >> 19) >= b13;
+        const uint32_t m = __ballot_sync(0xffffffffu, take);
+        if (m == 0) continue;
+        uint32_t b = 0;
+        if (lane == 0) b = atomicAdd(&s_nc, (uint32_t)__popc(m));
+        b = __shfl_sync(0xffffffffu, b, 0) + __popc(m & below);
+        if (take && b < (uint32_t)kRowCap) cand[b] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)jc(u));
       }
     });
     __syncthreads();
