@@ -246,6 +246,11 @@ def test_topk_many_long_rows_sampled_bound(L, ld_pad):
             v[cols] = rng.uniform(96.0, 112.0, 6000).astype(np.float32)
         elif kind == 5:
             v *= 1e-3                                                 # tiny scores
+        elif kind == 6:                                               # 600 large scores all inside the sample
+            n_mid = (p + 1 - 1024) - 16                               # runs: the bound lands among them and
+            for sg in range(60):                                      # admits fewer than the budget
+                s0 = 16 + (n_mid - 256) * sg // 63
+                v[s0 + 7:s0 + 247:24] = 50.0 + rng.random(10).astype(np.float32)
         rows.append(v)
     max_len = int(pos.max()) + 1 + (3 - int(pos.max()) % 4 if ld_pad == 0 else 0)
     st, idx, cnt = _topk_case(L, cfg, rows, pos, max_len, ld_pad)
