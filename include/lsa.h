@@ -485,9 +485,10 @@ LSA_API int32_t lsa_abi_version(void);
  * Synthetic inputs (tests and benchmarks; not part of the attention path).
  * Counter-based SplitMix64 (Steele, Lea, Flood, OOPSLA 2014): the stream of
  * tensor `tid` under `seed` starts at key = mix64(seed ^ tid*0xD1B54A32D192ED03)
- * and element i is mix64(key + (i+1)*0x9E3779B97F4A7C15). A normal draw is
- * (sum of the four 16-bit fields - 131070) * fp32(sigma/sqrt((2^32-1)/3)),
- * one fp32 multiply; bf16 outputs round to nearest even. Elements
+ * and element i is mix64(key + (i+1)*0x9E3779B97F4A7C15). Normal element i is
+ * (sum of the eight 16-bit fields of stream elements 2i and 2i+1 - 262140)
+ * * fp32(sigma/sqrt(2*(2^32-1)/3)), one fp32 multiply (tails at about 4.9
+ * sigma); bf16 outputs round to nearest even. Elements
  * first .. first+n-1 are written to dst[0 .. n-1].
  * lsa_synth_rms_rows_bf16 draws n_rows rows of d values, rounds them to bf16,
  * divides each row by sqrt(sum x^2 / d + 1e-6) in fp64, then rounds to fp32

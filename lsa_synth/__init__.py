@@ -14,12 +14,14 @@ Definition of the generator
   ``tid`` under ``seed`` starts from the state
   ``key = mix64(seed ^ (tid * 0xD1B54A32D192ED03))`` and element ``i`` is the
   (i+1)-th SplitMix64 output from that state: ``mix64(key + (i+1) * GOLDEN)``.
-* Approximate N(0, sigma^2): the four 16-bit fields of the 64-bit word are
-  summed (Irwin-Hall, 4 terms), centred by subtracting 131070 and multiplied
-  by one fp32 constant ``c = fp32(sigma / sqrt((65536^2 - 1) / 3))``. The
-  centred sum is an integer below 2^18, exact in fp32, so the product is one
-  correctly rounded fp32 multiply on any IEEE machine. Tails end at about
-  3.46 sigma.
+* Approximate N(0, sigma^2): normal element ``i`` takes the stream's words
+  ``2i`` and ``2i+1`` (outputs 2i+1 and 2i+2 from the key); their eight 16-bit
+  fields are summed (Irwin-Hall, 8 terms), centred by subtracting 262140 and
+  multiplied by one fp32 constant ``c = fp32(sigma / sqrt(2 (65536^2 - 1) / 3))``.
+  The centred sum is an integer of magnitude at most 262140 < 2^18, exact in
+  fp32, so the product is one correctly rounded fp32 multiply on any IEEE
+  machine. Tails end at about 4.90 sigma (a true normal passes that once in
+  about a million draws).
 * bf16 values are the fp32 value rounded to nearest even.
 * RMS-normalised rows (the index keys): the row is first rounded to bf16,
   then ``y = x / sqrt(sum(x^2)/d + 1e-6)``, evaluated in fp64 (the sum of the
@@ -34,8 +36,9 @@ GOLDEN = 0x9E3779B97F4A7C15
 TID_MUL = 0xD1B54A32D192ED03
 M1 = 0xBF58476D1CE4E5B9
 M2 = 0x94D049BB133111EB
-IH_VAR = (65536.0 * 65536.0 - 1.0) / 3.0  # variance of a sum of 4 uniform 16-bit ints
-IH_CENTRE = 131070
+IH_TERMS = 8
+IH_VAR = 2.0 * (65536.0 * 65536.0 - 1.0) / 3.0  # variance of a sum of 8 uniform 16-bit ints
+IH_CENTRE = 262140  # their mean, 8 * 65535 / 2
 
 _U = np.uint64
 
@@ -77,15 +80,20 @@ def hash_at(seed: int, tid: int, index: np.ndarray) -> np.ndarray:
     return mix64(z)
 
 
-def _irwin_hall(h: np.ndarray, sigma: float) -> np.ndarray:
+def _fields16(h: np.ndarray) -> np.ndarray:
     m = _U(0xFFFF)
-    s = (h & m) + ((h >> _U(16)) & m) + ((h >> _U(32)) & m) + ((h >> _U(48)) & m)
-    centred = s.astype(np.int64) - IH_CENTRE
+    return (h & m) + ((h >> _U(16)) & m) + ((h >> _U(32)) & m) + ((h >> _U(48)) & m)
+
+
+def _irwin_hall(h0: np.ndarray, h1: np.ndarray, sigma: float) -> np.ndarray:
+    """Normal values from the two words of each element."""
+    centred = (_fields16(h0) + _fields16(h1)).astype(np.int64) - IH_CENTRE
     return centred.astype(np.float32) * normal_scale(sigma)
 
 
 def normal_f32_at(seed: int, tid: int, index: np.ndarray, sigma: float = 1.0) -> np.ndarray:
-    return _irwin_hall(hash_at(seed, tid, index), sigma)
+    i2 = 2 * np.asarray(index, dtype=np.int64)
+    return _irwin_hall(hash_at(seed, tid, i2), hash_at(seed, tid, i2 + 1), sigma)
 
 
 def normal_bf16_rows(seed: int, tid: int, rows: np.ndarray, d: int) -> np.ndarray:
@@ -96,7 +104,8 @@ def normal_bf16_rows(seed: int, tid: int, rows: np.ndarray, d: int) -> np.ndarra
 
 
 def normal_f32(seed: int, tid: int, first: int, n: int, sigma: float = 1.0) -> np.ndarray:
-    return _irwin_hall(hash_range(seed, tid, first, n), sigma)
+    h = hash_range(seed, tid, 2 * first, 2 * n)
+    return _irwin_hall(h[0::2], h[1::2], sigma)
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:

@@ -3,9 +3,10 @@
 // Counter-based SplitMix64 (Steele, Lea and Flood, "Fast splittable
 // pseudorandom number generators", OOPSLA 2014): element i of the stream of
 // tensor `tid` under `seed` is mix64(key + (i+1) * 0x9E3779B97F4A7C15) with
-// key = mix64(seed ^ tid * 0xD1B54A32D192ED03). A normal draw sums the four
-// 16-bit fields (Irwin-Hall), centres the integer sum and multiplies it by one
-// fp32 constant; every step is exact or a single correctly rounded operation,
+// key = mix64(seed ^ tid * 0xD1B54A32D192ED03). Normal element i sums the
+// eight 16-bit fields of the stream's elements 2i and 2i+1 (Irwin-Hall, tails
+// at about 4.9 sigma), centres the integer sum and multiplies it by one fp32
+// constant; every step is exact or a single correctly rounded operation,
 // so a host implementation of the same definition reproduces each value bit for
 // bit.
 #include <math.h>
@@ -25,10 +26,14 @@ __host__ __device__ __forceinline__ uint64_t mix64(uint64_t z) {
   return z ^ (z >> 31);
 }
 
+__device__ __forceinline__ int fields16(uint64_t h) {
+  return (int)(h & 0xFFFF) + (int)((h >> 16) & 0xFFFF) + (int)((h >> 32) & 0xFFFF) + (int)((h >> 48) & 0xFFFF);
+}
+
 __device__ __forceinline__ float normal_at(uint64_t key, int64_t i, float c) {
-  const uint64_t h = mix64(key + (uint64_t)(i + 1) * kGolden);
-  const int s = (int)(h & 0xFFFF) + (int)((h >> 16) & 0xFFFF) + (int)((h >> 32) & 0xFFFF) +
-                (int)((h >> 48) & 0xFFFF) - 131070;
+  const uint64_t h0 = mix64(key + (uint64_t)(2 * i + 1) * kGolden);
+  const uint64_t h1 = mix64(key + (uint64_t)(2 * i + 2) * kGolden);
+  const int s = fields16(h0) + fields16(h1) - 262140;  // |s| <= 262140: exact in fp32
   return __fmul_rn((float)s, c);
 }
 
@@ -71,7 +76,7 @@ __global__ void synth_rms_rows_kernel(uint16_t* dst, int64_t n_rows, int d, uint
 uint64_t stream_key(uint64_t seed, uint64_t tid) { return mix64(seed ^ (tid * kTidMul)); }
 
 float normal_scale(double sigma) {
-  return (float)(sigma / sqrt((65536.0 * 65536.0 - 1.0) / 3.0));
+  return (float)(sigma / sqrt(2.0 * (65536.0 * 65536.0 - 1.0) / 3.0));
 }
 
 int grid_for(int64_t n, int threads) {

@@ -1293,17 +1293,17 @@ def _hier_check(L, cfg, seed, lengths, rows, block, n_blocks, min_exact):
 def test_hier_select_decode_varlen(L):
     lengths = [3000, 5000, 777, 20000, 2049, 2048, 40000]
     rows = [(s, n - 1) for s, n in enumerate(lengths)]
-    _hier_check(L, L.LsaConfig(), 5, lengths, rows, 64, 32, min_exact=6)   # one fine-stage near-tie
+    _hier_check(L, L.LsaConfig(), 5, lengths, rows, 64, 32, min_exact=5)   # two rows with a near-tie
 
 
 def test_hier_select_prefill_rows(L):
     # 200 rows of one sequence at consecutive positions (prefill shape)
     rows = [(0, 11800 + t) for t in range(200)]
-    # (of the 200 rows, 111 have no near-tie at either stage's boundary in the oracle)
-    _hier_check(L, L.LsaConfig(), 6, [12000], rows, 32, 80, min_exact=111)
+    # (of the 200 rows, 105 have no near-tie at either stage's boundary in the oracle)
+    _hier_check(L, L.LsaConfig(), 6, [12000], rows, 32, 80, min_exact=105)
 
 
-@pytest.mark.parametrize("block,n_blocks,n_exact", [(16, 256, 1), (128, 16, 3), (1024, 2, 3)])
+@pytest.mark.parametrize("block,n_blocks,n_exact", [(16, 256, 3), (128, 16, 2), (1024, 2, 2)])
 def test_hier_select_block_sizes(L, block, n_blocks, n_exact):
     # n_exact: rows without a near-tie at either boundary in the oracle
     lengths = [6000, 15000, 2500]
@@ -1353,7 +1353,7 @@ def test_hier_all_dense_status(L):
 def test_full_size_hier_sampled(L, name, batch, lo, hi, sample, n_exact):
     # the bench's hierarchical configuration (64-key blocks, 128 kept) at full
     # size; sampled rows re-drawn on the host and checked against the oracle.
-    # n_exact: sampled rows with no near-tie at either boundary (128K rows 0, 13,
+    # n_exact: sampled rows with no near-tie at either boundary (128K rows 0, 9,
     # 14); the others are checked by validity, kept blocks and score sums
     from sparse_attention_03_b200.device_inputs import DeviceWorkload
     cfg = L.LsaConfig()

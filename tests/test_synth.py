@@ -41,17 +41,24 @@ def test_normal_moments():
     x = S.normal_f32(0, 3, 0, 1 << 20).astype(np.float64)
     assert abs(x.mean()) < 5e-3
     assert abs(x.var() - 1.0) < 5e-3
-    assert np.abs(x).max() <= 3.47
+    # 8-term Irwin-Hall: bounded at 4.90 sigma, but well past the 4-term 3.46
+    assert np.abs(x).max() <= 4.90
+    assert (np.abs(x) > 3.5).sum() > 100
     y = S.normal_f32(0, 4, 0, 1 << 18, sigma=S.W_SIGMA).astype(np.float64)
     assert abs(y.var() * 32 - 1.0) < 1e-2
 
 
 def test_normal_is_one_fp32_multiply():
-    h = S.hash_range(9, 1, 0, 50)
+    # element i: the 16-bit fields of stream words 2i and 2i+1, summed, centred
+    h = S.hash_range(9, 1, 0, 100)
     m = np.uint64(0xFFFF)
-    s = sum(((h >> np.uint64(16 * q)) & m).astype(np.int64) for q in range(4)) - 131070
-    expect = np.float32(s.astype(np.float32)) * S.normal_scale(1.0)
+    f = sum(((h >> np.uint64(16 * q)) & m).astype(np.int64) for q in range(4))
+    s = f[0::2] + f[1::2] - 4 * 65535
+    scale = np.float32(1.0 / np.sqrt(8 * (65536.0 ** 2 - 1) / 12))
+    expect = np.float32(s.astype(np.float32)) * scale
     np.testing.assert_array_equal(S.normal_f32(9, 1, 0, 50), expect)
+    np.testing.assert_array_equal(S.normal_f32_at(9, 1, np.array([7, 3, 49])), expect[[7, 3, 49]])
+    np.testing.assert_array_equal(S.normal_f32(9, 1, 20, 5), expect[20:25])
 
 
 def test_rms_rows():
