@@ -594,13 +594,13 @@ def run_prefill(device, steps, warmup):
                          "traffic": kernel_traffic("index_prefill_kernel", INDEX_PREFILL_SOURCES)}}
 
 
-def _forward_case(device, lengths, n_rows=None, q_start=None):
+def _forward_case(device, lengths, n_rows=None, q_start=None, layer=300):
     """One layer's lsa_forward call (cli 2) on device-drawn inputs, bound once."""
     import torch
     from sparse_attention_03_b200 import lsa
     from sparse_attention_03_b200.device_inputs import DeviceWorkload
     cfg = lsa.LsaConfig()
-    wl = DeviceWorkload(0, 300, lengths, n_rows=n_rows, q_start=q_start, device=device)
+    wl = DeviceWorkload(0, layer, lengths, n_rows=n_rows, q_start=q_start, device=device)
     n, max_len = wl.n_rows, wl.max_len
     mode = 0 if n_rows is None else 1
     outs = [torch.empty((n, 32, 512), dtype=torch.bfloat16, device=device) for _ in range(2)]
@@ -617,7 +617,9 @@ def run_configs(device, steps):
     """The other workloads of the pages' configuration list, one lsa_forward layer
     (one index pass, top-k, two sub-blocks) per step: single-token latency at
     8192 cached keys (caches fit in L2, so L2 is flushed before every step and
-    each step is event-timed alone), the 64-sequence varlen decode, and the
+    each step is event-timed alone; and, as inside a model's forward, 14 such
+    layers back to back, whose caches together exceed L2), the 64-sequence
+    varlen decode, and the
     long-context pair (4 sequences at 983040 cached keys; a 4096-token prefill
     chunk against the 983040-token cache)."""
     import torch
@@ -647,6 +649,14 @@ def run_configs(device, steps):
             call()
         t = time_region(lambda s: call(), n_steps, 1, device)
         return units * n_steps / t, 1e3 * t / n_steps
+
+    # the same single-token layer, 14 layers (each with its own caches) per step
+    cases = [_forward_case(device, [8192], layer=300 + i) for i in range(14)]
+    v, ms = timed(lambda: [c() for c, _ in cases], 14, steps)
+    res["decode_b1_ctx8192_14layers"] = {"value": v, "unit": "tokens/s/layer", "us_per_layer": 1e3 * ms / 14,
+                                         "l2": "14 layers' caches (0.30 GB) per step, no flush"}
+    del cases
+    torch.cuda.empty_cache()
 
     # decode, batch 64, cached lengths uniform in [16384, 32768]
     lengths = S.decode_lengths(0, 64, 16384, 32768)

@@ -593,19 +593,17 @@ __global__ void __launch_bounds__(kRowThreads, 2) topk_row_kernel(TopkArgs a, in
       oe += s_we[w2];
     }
     if (tid == kRowThreads - 1) s_nc = oe + ne;  // the last thread's prefix is the total
+    // branch-free (predicated stores): one straight run of code for all 16
 #pragma unroll
     for (int i = 0; i < kShort; ++i) {
       const int64_t j = scol(i);
-      if (j >= g.hi) continue;
       const uint32_t key = score_key(sv[i]);
-      const int kb = (int)(key >> 21);
-      if (kb > bin0) {
-        if (ou < k_rem) mid[ou] = col(j);
-        ++ou;
-      } else if (kb == bin0) {
-        if (oe < (uint32_t)kRowCap) cand[oe] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
-        ++oe;
-      }
+      const int kb = j < g.hi ? (int)(key >> 21) : -1;
+      const bool up = kb > bin0, eq = kb == bin0;
+      if (up && ou < k_rem) mid[ou] = col(j);
+      if (eq && oe < (uint32_t)kRowCap) cand[oe] = ((uint64_t)key << 32) | (uint64_t)(0xFFFFFFFFu - (uint32_t)j);
+      ou += up;
+      oe += eq;
     }
   } else {
   // collect: higher bins straight out, the threshold bin into shared memory
