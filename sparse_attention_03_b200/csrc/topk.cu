@@ -13,7 +13,11 @@
 // of the top 11 key bits, built by the decode indexer while the scores are in
 // registers, or here. Two kernel shapes:
 //   * many or short rows: one CTA per row does everything, with the
-//     threshold-bin candidates in shared memory;
+//     threshold-bin candidates in shared memory. A short row's scores sit in
+//     registers; a long row without a histogram (a prefill block) is read once:
+//     a sample of the row sets a bound, one pass keeps every score above it in
+//     shared memory, and the select finishes there, with the exact two-pass
+//     path as the fallback when the bound admits too few or too many;
 //   * few long rows: many CTAs per row. Each finds the threshold bin, places
 //     its chunk's columns with one block-wide prefix sum and one global atomic,
 //     and the last CTA of the row (an atomic ticket) finishes the select on the
