@@ -133,8 +133,8 @@ LSA_API size_t lsa_workspace_size(const lsa_config* cfg, int32_t op, int32_t n_r
  * seq_of_row int32 [n_rows] or NULL (every row in sequence 0)
  * pos     int32 [n_rows]             scores fp32 [n_rows, ld], ld >= max_len
  * max_len host bound: every pos[r] < max_len.
- * topk_hist: optional uint32 [n_rows, LSA_TOPK_HIST_WORDS] (device). When not
- *   NULL it receives the first radix pass of the selection (a histogram of the
+ * topk_hist: optional uint32 [n_rows, LSA_TOPK_HIST_WORDS] (device, 16-byte
+ *   aligned). When not NULL it receives the first radix pass of the selection (a histogram of the
  *   top 11 bits of the order-preserving key of every middle-column score of
  *   rows with more than index_topk visible keys), built from the scores while
  *   they are still in registers; pass it to lsa_topk with the same scores.
@@ -163,10 +163,11 @@ LSA_API lsa_status lsa_index_scores(const lsa_config* cfg, int32_t n_rows, int32
  * max_len (host): every pos[r] < max_len. Returns LSA_DENSE when
  * max_len <= index_topk (every row dense; idx/count still written).
  * topk_hist: NULL, or the histogram lsa_index_scores wrote for these scores
- *   (saves one pass over the scores). Rows longer than 16384 columns (fewer
- *   than 256 rows) also keep their counters in its 8 words after each row's
- *   bins: they must be zero on entry, as lsa_index_scores leaves them, and are
- *   zero again on return.
+ *   (saves one pass over the scores; 16-byte aligned, else LSA_ERR_INVALID).
+ *   Rows longer than 16384 columns (fewer than 256 rows) also keep their
+ *   counters in its 8 words after each row's bins (one of them a 64-bit
+ *   counter): they must be zero on entry, as lsa_index_scores leaves them, and
+ *   are zero again on return.
  * Workspace: lsa_workspace_size(LSA_OP_TOPK, ...). Only fewer than 256 rows
  * longer than 16384 columns use it (then processed in blocks that fit,
  * minimum one row of 40992 B); otherwise ws may be NULL.

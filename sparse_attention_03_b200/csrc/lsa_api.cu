@@ -314,6 +314,8 @@ lsa_status lsa_index_scores(const lsa_config* c, int32_t n_rows, int32_t n_seq,
     return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
   if (!aligned16(q_idx) || !aligned16(k_idx))
     return set_error(LSA_ERR_INVALID, "%s: q_idx and k_idx must be 16-byte aligned", fn);
+  if (topk_hist && !aligned16(topk_hist))
+    return set_error(LSA_ERR_INVALID, "%s: topk_hist must be 16-byte aligned", fn);
   return run_index_scores(c, n_rows, n_seq, seq_of_row, 0, pos, q_idx, w, k_idx, k_off, max_len,
                           scores, ld, (cudaStream_t)stream, topk_hist);
 }
@@ -328,6 +330,8 @@ lsa_status lsa_topk(const lsa_config* c, int32_t n_rows, const int32_t* pos, int
     return set_error(LSA_ERR_INVALID, "%s: need n_rows >= 0 and 1 <= max_len <= ld", fn);
   if (n_rows == 0) return max_len <= c->index_topk ? LSA_DENSE : LSA_OK;
   if (!pos || !scores || !idx || !count) return set_error(LSA_ERR_INVALID, "%s: NULL array argument", fn);
+  if (topk_hist && !aligned16(topk_hist))
+    return set_error(LSA_ERR_INVALID, "%s: topk_hist must be 16-byte aligned", fn);
   if (max_len > c->index_topk && !ws && topk_uses_workspace(n_rows, max_len))
     return set_error(LSA_ERR_WORKSPACE, "%s: workspace is NULL", fn);
   return run_topk(c, n_rows, pos, max_len, scores, ld, idx, count, ws, ws_bytes, (cudaStream_t)stream,

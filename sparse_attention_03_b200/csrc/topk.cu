@@ -43,7 +43,10 @@ constexpr uint64_t kLow53 = (1ull << 53) - 1;
 // Per-row workspace: a zeroed histogram/control block, then the candidates.
 struct HistCtl {
   uint32_t hist[kBins];
-  uint32_t ctl[8];  // 0: emitted above, 1: candidates, 2: threshold bin, 3: count above it
+  // 0: emitted above; 4 and 5, one 64-bit counter: the threshold-bin candidates
+  // (low word) and the CTAs that have finished (high word), so that the last
+  // CTA's ticket also returns the candidate count
+  uint32_t ctl[8];
 };
 static_assert(sizeof(HistCtl) + kTopkCap * sizeof(uint64_t) == kTopkRowBytes, "workspace layout");
 
@@ -112,7 +115,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
   __shared__ uint64_t scand[kTopkCap];
   __shared__ int s_bin, s_last;
   __shared__ uint32_t s_above, s_warp[kHistThreads / 32], s_wu[kHistThreads / 32], s_we[kHistThreads / 32];
-  __shared__ uint32_t s_base_u, s_base_e, s_slot;
+  __shared__ uint32_t s_base_u, s_base_e, s_slot, s_ncand;
   pdl_wait();
   pdl_trigger();  // dependents may launch now; they wait for this grid before reading its outputs
   const int r = row0 + blockIdx.y;
@@ -189,7 +192,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
       te += a_e;
     }
     s_base_u = tu ? atomicAdd(&ctl[0], tu) : 0u;
-    s_base_e = te ? atomicAdd(&ctl[1], te) : 0u;
+    s_base_e = te ? (uint32_t)atomicAdd(reinterpret_cast<unsigned long long*>(&ctl[4]), (unsigned long long)te) : 0u;
   }
   __syncthreads();
   uint32_t ou = s_base_u + s_wu[warp] + iu - nu;
@@ -212,7 +215,11 @@ __global__ void __launch_bounds__(kHistThreads, 4)
   // ---- the last CTA of the row finishes it ----
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_last = atomicAdd(&ctl[4], 1u) == n_chunks - 1;
+  if (tid == 0) {
+    const unsigned long long t = atomicAdd(reinterpret_cast<unsigned long long*>(&ctl[4]), 1ull << 32);
+    s_last = (uint32_t)(t >> 32) == n_chunks - 1;
+    s_ncand = (uint32_t)t;  // every CTA reserved its candidates before its ticket
+  }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
@@ -222,7 +229,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
     a.count[r] = a.topk;
     s_slot = 0;
   }
-  const uint32_t n_cand = __ldcg(&ctl[1]);
+  const uint32_t n_cand = s_ncand;
   const uint32_t need0 = k_rem - above;
   // Where the rest of the select runs: the threshold-bin candidates in shared
   // memory (the common case); if they overflow it but fit the workspace, one
@@ -320,8 +327,7 @@ __global__ void __launch_bounds__(kHistThreads, 4)
   // every CTA of the row has taken its ticket: the counters are free again
   if (tid == 0) {
     ctl[0] = 0;
-    ctl[1] = 0;
-    ctl[4] = 0;
+    *reinterpret_cast<unsigned long long*>(&ctl[4]) = 0ull;
   }
 }
 

@@ -101,6 +101,11 @@ def test_rejects_bad_arguments(lib):
     # top-k without a workspace on few long rows (the multi-CTA path)
     assert lib.lsa_topk(ctypes.byref(c), 4, _fake(), 90000, _fake(), 90000, None, _fake(), _fake(), None, 0,
                         None) == lsa.LSA_ERR_WORKSPACE
+    # a histogram buffer off the 16-byte grid (its per-row counters include a 64-bit one)
+    assert lib.lsa_index_scores(ctypes.byref(c), 4, 1, None, _fake(), _fake(), _fake(), _fake(), None, 100,
+                                _fake(), 100, ctypes.c_void_p(0x10004), None) == lsa.LSA_ERR_INVALID
+    assert lib.lsa_topk(ctypes.byref(c), 4, _fake(), 90000, _fake(), 90000, ctypes.c_void_p(0x10004), _fake(),
+                        _fake(), _fake(), 10 ** 7, None) == lsa.LSA_ERR_INVALID
     # decode MLA without offsets
     assert lib.lsa_sparse_mla_decode(ctypes.byref(c), 2, _fake(), _fake(), None, None, None, 10, _fake(),
                                      None, None, 0, None) == lsa.LSA_ERR_INVALID
