@@ -16,7 +16,10 @@
 // 32 consecutive columns = the 32 heads of one token), apply ReLU and the head
 // weights in registers, mask/force and store one fp32 score per (token, key);
 // a warp's 32 lanes are 32 consecutive keys, so each store is a 128-byte line.
-// While the epilogue drains one accumulator the tensor core fills the other.
+// A warp loads its 4 tokens x 32 heads of an accumulator in one round (one
+// wait) and releases the accumulator before the math and the stores, so the
+// tensor core refills it while the epilogue finishes; while the epilogue drains
+// one accumulator the tensor core fills the other.
 // Warp 0 issues TMA, warp 1 allocates tensor memory and issues MMAs, warps 2-9
 // run the epilogue. Every mbarrier wait is bounded: on timeout the CTA raises an
 // error flag, stops, and still frees its tensor memory.
@@ -195,20 +198,25 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) ok = mbar_wait(&sm.tfull[hb], i & 1, abort_flag) ? 1 : 0;
         if (!__shfl_sync(0xffffffffu, ok, 0)) goto done;
         tc_fence_after();
-#pragma unroll 1
+        // this warp's 4 tokens x 32 heads in one round of loads; the
+        // accumulator goes back to the MMA issuer before the math and stores
+        float acc[4][32];
+        tmem_ld32_x4(tmem + lane_addr + hb * 256 + tok_half * 4 * 32, 32, acc);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.tempty[hb]);
+#pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int tok = hb * 8 + tok_half * 4 + u;
-          float acc[32];
-          tmem_ld32(tmem + lane_addr + hb * 256 + (tok - hb * 8) * 32, acc);
           float s = 0.f;
           const float4* wv = reinterpret_cast<const float4*>(sm.w[tok]);
 #pragma unroll
           for (int h4 = 0; h4 < 8; ++h4) {
             const float4 ww = wv[h4];
-            s = fmaf(ww.x, fmaxf(acc[4 * h4 + 0], 0.f), s);
-            s = fmaf(ww.y, fmaxf(acc[4 * h4 + 1], 0.f), s);
-            s = fmaf(ww.z, fmaxf(acc[4 * h4 + 2], 0.f), s);
-            s = fmaf(ww.w, fmaxf(acc[4 * h4 + 3], 0.f), s);
+            s = fmaf(ww.x, fmaxf(acc[u][4 * h4 + 0], 0.f), s);
+            s = fmaf(ww.y, fmaxf(acc[u][4 * h4 + 1], 0.f), s);
+            s = fmaf(ww.z, fmaxf(acc[u][4 * h4 + 2], 0.f), s);
+            s = fmaf(ww.w, fmaxf(acc[u][4 * h4 + 3], 0.f), s);
           }
           const int p = sm.pos[tok];
           if (j <= p && j < prm.max_len) {
@@ -216,9 +224,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             prm.scores[(int64_t)(row0 + tok) * prm.ld + j] = forced ? INFINITY : s;
           }
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sm.tempty[hb]);
       }
     }
   }

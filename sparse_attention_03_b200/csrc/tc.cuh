@@ -87,6 +87,29 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
 }
 
 
+// Four 32-column loads (columns taddr + q * col_stride, q = 0..3) issued back
+// to back and one wait: the load latency is paid once for 128 values.
+__device__ __forceinline__ void tmem_ld32_x4(uint32_t taddr, uint32_t col_stride, float (&v)[4][32]) {
+  uint32_t r[4][32];
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+        : "=r"(r[q][0]), "=r"(r[q][1]), "=r"(r[q][2]), "=r"(r[q][3]), "=r"(r[q][4]), "=r"(r[q][5]),
+          "=r"(r[q][6]), "=r"(r[q][7]), "=r"(r[q][8]), "=r"(r[q][9]), "=r"(r[q][10]), "=r"(r[q][11]),
+          "=r"(r[q][12]), "=r"(r[q][13]), "=r"(r[q][14]), "=r"(r[q][15]), "=r"(r[q][16]), "=r"(r[q][17]),
+          "=r"(r[q][18]), "=r"(r[q][19]), "=r"(r[q][20]), "=r"(r[q][21]), "=r"(r[q][22]), "=r"(r[q][23]),
+          "=r"(r[q][24]), "=r"(r[q][25]), "=r"(r[q][26]), "=r"(r[q][27]), "=r"(r[q][28]), "=r"(r[q][29]),
+          "=r"(r[q][30]), "=r"(r[q][31])
+        : "r"(taddr + q * col_stride));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" ::: "memory");
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[q][i] = __uint_as_float(r[q][i]);
+}
+
 __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
                                          uint32_t acc) {
   asm volatile(
