@@ -60,3 +60,29 @@ def test_reference_arm_only_rank0_works(monkeypatch):
     with redirect_stdout(buf):
         bench.reference_arm(argparse.Namespace(steps=1, warmup=3, gpus=2))
     assert buf.getvalue() == ""
+
+
+def test_reference_arm_line_contract(monkeypatch):
+    # rank 0 of a one-process run: one JSON line with the contract's keys, the
+    # oracle timed on this host's cores, no host<->device bytes
+    import json
+    sys.path.insert(0, ROOT)
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    buf = io.StringIO()
+    with redirect_stdout(buf):
+        bench.reference_arm(argparse.Namespace(steps=1, warmup=3, gpus=1))
+    lines = [x for x in buf.getvalue().splitlines() if x.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    for k in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+              "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert k in d, k
+    assert d["impl"] == "reference" and d["n_gpus"] == 1 and d["steps"] == 1 and d["warmup"] >= 3
+    assert d["value"] > 0 and d["higher_is_better"] is True and d["vs_baseline"] is None
+    assert d["config"]["workload"] == "decode_b16_ctx131072_14layers_cli2"
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["value"] == d["value"] and cb["sample"]
+    assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["e2e"]["d2h_bytes_per_step"] == 0
+    assert d["e2e"]["value"] == d["value"] and d["e2e"]["unit"] == d["unit"]
